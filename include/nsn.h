@@ -1,0 +1,203 @@
+/*
+ * nsn.h -- C ABI of the NSNQuant KV-cache hot path on B200 (sm_100a).
+ *
+ * The method (sources named by page title and section):
+ *   [TS] "NSNQuant: A Double Normalization Approach for Calibration-Free Low-Bit
+ *        Vector Quantization of KV Cache", technical summary (gist.science):
+ *        Metodologia 1 (Normalize-Shift-Normalize), 2 (Hadamard transform),
+ *        3 (vector quantization, codebook from k-means on randn, adaptive scale),
+ *        4 (KIVI-style residual window; attention scores that fold in s1, s2, o;
+ *        custom CUDA kernels for Hadamard, VQ and dequantization).
+ *   [GH] "NSNQuant" repository README: Overview; Codebook tuning (--abs 2-bit
+ *        codebook over absolute values, 1-bit codebook).
+ *
+ * Every token vector x (head_dim 128) of K or V is rotated, y = H x (orthonormal
+ * Sylvester Hadamard, natural order), then NSN is applied per block of 128
+ * tokens of one (batch, kv-head):
+ *   s1 = ||y||/sqrt(d), n1 = y/s1;  o = mean over the block of n1;  z = n1 - o;
+ *   s2 = ||z||/sqrt(d), u = z/s2.
+ * u is split into 16 sub-vectors of 8; each gets the nearest codeword (squared
+ * Euclidean, ties to the lowest index) of one 256 x 8 codebook:
+ *   1-bit mode: code over the signed codebook C;
+ *   2-bit mode: 8 sign bits (bit i set iff u_i < 0) + code over |u| against an
+ *               absolute-value codebook A (entries >= 0).
+ * Adaptive scale (flag): alpha = ||u||^2 / (u . u_hat) (1 if u . u_hat <= 0) is
+ * folded into the stored s2.  The token is reconstructed as
+ *   x_hat = H^T ((u_hat * s2 + o) * s1).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are caller-owned.  The library never allocates or frees memory.
+ *   - Device pointers must be 16-byte aligned; row strides are in ELEMENTS and
+ *     must keep every 128-element row 16-byte aligned.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t passed as
+ *     void*; NULL = legacy default stream).  No call synchronizes.
+ *   - Arguments are validated on the host before any launch; an invalid call
+ *     returns an error code and launches nothing (the cache is untouched).
+ *     A failed launch returns NSN_ERR_CUDA.
+ *   - fp16 values are stored as IEEE binary16 bit patterns (uint16_t).
+ */
+#ifndef NSN_H_
+#define NSN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NSN_HEAD_DIM 128 /* d */
+#define NSN_SUB_DIM 8    /* sub-vector length */
+#define NSN_N_SUB 16     /* sub-vectors per token */
+#define NSN_N_CODES 256  /* codebook entries (8-bit code) */
+#define NSN_BLOCK 128    /* tokens per NSN block (channel-mean scope) */
+#define NSN_MAX_GQA 8    /* query heads per kv-head supported by decode */
+
+typedef enum {
+  NSN_OK = 0,
+  NSN_ERR_INVALID_ARG = 1, /* null pointer, bad size, stride or alignment */
+  NSN_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. window not in {0,128}) */
+  NSN_ERR_WORKSPACE = 3,   /* decode workspace too small */
+  NSN_ERR_CUDA = 4,        /* a CUDA launch failed; see nsn_last_cuda_error() */
+  NSN_ERR_STATE = 5        /* the cache is in a state the call cannot use */
+} nsn_status;
+
+typedef enum { NSN_MODE_1BIT = 1, NSN_MODE_2BIT = 2 } nsn_mode;
+
+typedef enum { NSN_DTYPE_F32 = 0, NSN_DTYPE_BF16 = 1, NSN_DTYPE_F16 = 2 } nsn_dtype;
+
+/*
+ * Compressed cache of one tensor (K or V) of one layer.  All pointers are
+ * device pointers owned by the caller.  Layout (row-major, per (b, h) contiguous):
+ *   codes    uint8  [batch][n_kv_heads][capacity][16]   code of sub-vector s at byte s
+ *   signs    uint8  [batch][n_kv_heads][capacity][16]   2-bit mode only (NULL in 1-bit):
+ *                                                       byte s, bit i = sign of u[8s+i]
+ *   norms    fp16   [batch][n_kv_heads][capacity][2]    (s1, alpha*s2) per token
+ *   means    fp16   [batch][n_kv_heads][capacity/128][128]   o of each block (rotated domain)
+ *   window   fp16   [batch][n_kv_heads][window][128]    residual tokens, original domain
+ *   n_quant  int32  [batch][n_kv_heads]                 quantized tokens (multiple of 128
+ *                                                       when window > 0)
+ *   n_window int32  [batch][n_kv_heads]                 tokens in the residual window
+ *   status   int32  [1] or NULL                         device error bits, OR-ed by kernels:
+ *                                                       1 = capacity overflow on flush
+ * capacity must be a positive multiple of 128.  window must be 0 (quantize every
+ * token, no append) or 128 (KIVI-style residual of one block).
+ */
+typedef struct {
+  int32_t batch;
+  int32_t n_kv_heads;
+  int32_t capacity;
+  int32_t window;
+  int32_t mode;         /* nsn_mode */
+  int32_t scale_adjust; /* 1: fold the adaptive scale into the stored s2 */
+  uint8_t* codes;
+  uint8_t* signs;
+  uint16_t* norms;
+  uint16_t* means;
+  uint16_t* window_buf;
+  int32_t* n_quant;
+  int32_t* n_window;
+  int32_t* status;
+} nsn_cache;
+
+/* Byte sizes of the buffers of an nsn_cache with the given shape. */
+typedef struct {
+  size_t codes, signs, norms, means, window_buf, n_quant, n_window;
+} nsn_cache_sizes;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int nsn_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* nsn_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* nsn_last_cuda_error(void);
+
+/*
+ * Fills *out with the byte size of each cache buffer.  signs is 0 in 1-bit mode,
+ * window_buf is 0 when window == 0.  Returns NSN_ERR_INVALID_ARG on a bad shape.
+ */
+nsn_status nsn_cache_buffer_sizes(int batch, int n_kv_heads, int capacity, int window, int mode,
+                                  nsn_cache_sizes* out);
+
+/*
+ * Builds the codebook on the HOST (no GPU use).  [TS] Metodologia 3: k-means on
+ * synthetic standard-normal samples; [GH] Codebook tuning: --abs builds it over
+ * absolute values.
+ *   seed       stream seed.  Samples are standard normals from Philox4x64-10 (Salmon
+ *              et al., SC'11) with key (seed, 0x4E534E51) and counter (j,0,0,0) for
+ *              block j; each 64-bit word w -> u = ((w >> 12) + 0.5) * 2^-52; the pairs
+ *              (u0,u1), (u2,u3) -> Box-Muller normals (r cos 2 pi u_b, r sin 2 pi u_b),
+ *              r = sqrt(-2 ln u_a).  Normal i*dim + c is component c of sample i.
+ *   n_samples  >= n_codes.   n_codes, dim > 0.   abs_mode: 1 = use |samples|.
+ *   iters      Lloyd iterations (>= 0) from the first n_codes samples as initial
+ *              centroids; ties go to the lowest centroid; empty clusters keep theirs.
+ *   out        host float[n_codes * dim], row-major; every value is rounded to the
+ *              nearest fp16-representable number (so the fp32 quantizer and the fp16
+ *              decode read identical codewords).
+ */
+nsn_status nsn_build_codebook_host(uint64_t seed, int n_samples, int n_codes, int dim,
+                                   int abs_mode, int iters, float* out);
+
+/*
+ * Prefill: quantizes n_tokens tokens of every (b, h) of x into a FRESH cache
+ * (counters are overwritten).  [TS] Metodologia 1-3 (+ 4 for the residual split).
+ *   x          device, dtype element type, token (b, t, h) row at
+ *              x + b*stride_b + t*stride_t + h*stride_h (elements), 128 contiguous values.
+ *   n_tokens   L >= 0, same for every batch row.  With window 128 the first
+ *              Q = 128*floor((L-1)/128) tokens are quantized in blocks of 128 and the
+ *              remaining L-Q (1..128) are copied (as fp16) to the window; with
+ *              window 0 all L are quantized (the last block may be partial).
+ *              Requires Q <= capacity.
+ *   codebook   device float[256*8] (signed codebook in 1-bit, absolute in 2-bit).
+ * Stored values: codes/signs bit-exact to the definition (fp32 search with an exact
+ * fp64 re-check of near ties), s1, alpha*s2 and o rounded to fp16.
+ */
+nsn_status nsn_quantize_kv(nsn_cache* cache, const void* x, int dtype, int64_t stride_b,
+                           int64_t stride_t, int64_t stride_h, int n_tokens,
+                           const float* codebook, void* stream);
+
+/*
+ * Decode-time append of one new token per (b, h) to K and V ([TS] Metodologia 4,
+ * residual: when the window is full it is flushed -- quantized as one block and
+ * appended -- and emptied).  For every (b, h) of each cache: if n_window == 128 the
+ * window is quantized into block n_quant/128 (n_quant += 128, n_window = 0; if that
+ * block does not fit in capacity the token is not appended and status bit 1 is set);
+ * then the new token is stored (as fp16) at window[n_window] and n_window += 1.
+ *   k_new, v_new  device [b][h][128] rows at base + b*stride_b + h*stride_h (elements).
+ *   cb_k, cb_v    device float[256*8] codebooks of the K and V caches.
+ * Both caches must have window == 128 and the same batch / n_kv_heads.
+ */
+nsn_status nsn_append_residual(nsn_cache* k_cache, nsn_cache* v_cache, const void* k_new,
+                               const void* v_new, int dtype, int64_t stride_b, int64_t stride_h,
+                               const float* cb_k, const float* cb_v, void* stream);
+
+/*
+ * Workspace bytes that nsn_decode_attention needs for these caches and n_q_heads.
+ */
+size_t nsn_decode_workspace_bytes(const nsn_cache* k_cache, int n_q_heads);
+
+/*
+ * Decode attention of one query token per (b, q-head) over the compressed cache
+ * followed by the residual window ([TS] Metodologia 4: scores with s1, s2, o folded
+ * in).  q-head j uses kv-head j / (n_q_heads / n_kv_heads).
+ *   q              device dtype [b][n_q_heads][128], row at q + b*q_stride_b + j*q_stride_h.
+ *   n_q_heads      multiple of n_kv_heads, n_q_heads / n_kv_heads <= 8.
+ *   softmax_scale  score = softmax_scale * q . k (1/sqrt(128) for standard attention).
+ *   cb_k, cb_v     device float[256*8] codebooks; decode reads them rounded to fp16.
+ *   out            device float [b][n_q_heads][128].  A (b, h) with no tokens at all
+ *                  yields zeros.
+ *   workspace      device, >= nsn_decode_workspace_bytes() bytes, 256-byte aligned.
+ */
+nsn_status nsn_decode_attention(const nsn_cache* k_cache, const nsn_cache* v_cache,
+                                const void* q, int dtype, int n_q_heads, int64_t q_stride_b,
+                                int64_t q_stride_h, float softmax_scale, const float* cb_k,
+                                const float* cb_v, float* out, void* workspace, size_t ws_bytes,
+                                void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSN_H_ */

@@ -1,0 +1,119 @@
+"""Plain CPU oracle of the codebook construction.  TEST INFRASTRUCTURE ONLY.
+
+The pages build the single global codebook by k-means on synthetic standard
+normal samples (torch.randn) -- "NSNQuant ... technical summary", Metodologia 3
+"Codebook: construccion" -- and the 2-bit variant on absolute values
+("NSNQuant" README, "Codebook tuning": ``--abs``).  The fine-tuning for cosine
+distance that the pages mention afterwards is not part of this path.
+
+The seeded standard-normal samples come from a counter-based generator that
+each side implements from its published definition:
+  * Philox4x64-10: J. Salmon, M. Moraes, R. Dror, D. Shaw, "Parallel Random
+    Numbers: As Easy as 1, 2, 3", SC'11 (round function, multipliers and Weyl
+    key increments as defined there).
+  * Box-Muller: G. Box, M. Muller, "A Note on the Generation of Random Normal
+    Deviates", Ann. Math. Statist. 29 (1958).
+Stream layout (a reading; documented in the C header as well): key =
+(seed, 0x4E534E51), counter = (j, 0, 0, 0) for block j; the block's four
+64-bit words w0..w3 become uniforms u = ((w >> 12) + 0.5) * 2^-52 and the pairs
+(u0, u1), (u2, u3) give normals (r cos(2 pi u_b), r sin(2 pi u_b)) with
+r = sqrt(-2 ln u_a).  Normal number i*dim + c is component c of sample i.
+
+k-means (a reading of "K-Means on randn"): Lloyd iterations, initial centroids =
+the first K samples, nearest centroid by squared Euclidean distance with ties to
+the lowest index, empty clusters keep their centroid, a fixed iteration count;
+the result is rounded to fp16-representable values so that the fp32 quantizer
+and the fp16 decode read identical codewords.
+
+Pinned by tests/test_oracle_codebook.py against numpy's own Philox bit
+generator, the moments and a Kolmogorov-Smirnov test of the normal stream, scipy's
+Lloyd iteration (kmeans2 from the same initial centroids) and k-means fixed-point
+properties.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+_MASK64 = (1 << 64) - 1
+PHILOX_M0 = 0xD2E7470EE14C6C93
+PHILOX_M1 = 0xCA5A826395121157
+PHILOX_W0 = 0x9E3779B97F4A7C15
+PHILOX_W1 = 0xBB67AE8584CAA73B
+STREAM_KEY1 = 0x4E534E51
+
+
+def philox4x64_10(counter, key):
+    """One Philox4x64 block with 10 rounds (python ints, exact)."""
+    x0, x1, x2, x3 = (int(c) & _MASK64 for c in counter)
+    k0, k1 = (int(k) & _MASK64 for k in key)
+    for _ in range(10):
+        p0 = PHILOX_M0 * x0
+        p1 = PHILOX_M1 * x2
+        hi0, lo0 = p0 >> 64, p0 & _MASK64
+        hi1, lo1 = p1 >> 64, p1 & _MASK64
+        x0, x1, x2, x3 = (hi1 ^ x1 ^ k0), lo1, (hi0 ^ x3 ^ k1), lo0
+        k0 = (k0 + PHILOX_W0) & _MASK64
+        k1 = (k1 + PHILOX_W1) & _MASK64
+    return x0, x1, x2, x3
+
+
+def uniform_open(word: int) -> float:
+    """Map a 64-bit word to a double in the open interval (0, 1).
+
+    The top 52 bits plus one half, times 2^-52: exact, in [2^-53, 1 - 2^-53].
+    """
+    return ((word >> 12) + 0.5) * (2.0 ** -52)
+
+
+def normal_stream(seed: int, count: int) -> np.ndarray:
+    """The first `count` standard normals of the stream for `seed`."""
+    out = np.empty(count)
+    key = (seed & _MASK64, STREAM_KEY1)
+    nblocks = (count + 3) // 4
+    for j in range(nblocks):
+        w = philox4x64_10((j, 0, 0, 0), key)
+        u = [uniform_open(x) for x in w]
+        zs = []
+        for a, b in ((u[0], u[1]), (u[2], u[3])):
+            r = math.sqrt(-2.0 * math.log(a))
+            zs.append(r * math.cos(2.0 * math.pi * b))
+            zs.append(r * math.sin(2.0 * math.pi * b))
+        for t in range(4):
+            i = 4 * j + t
+            if i < count:
+                out[i] = zs[t]
+    return out
+
+
+def normal_samples(seed: int, n_samples: int, dim: int, abs_mode: bool) -> np.ndarray:
+    """[n_samples, dim] standard normals (absolute values in abs mode)."""
+    z = normal_stream(seed, n_samples * dim).reshape(n_samples, dim)
+    return np.abs(z) if abs_mode else z
+
+
+def kmeans(samples: np.ndarray, n_codes: int, iters: int) -> np.ndarray:
+    """Lloyd's k-means in fp64 (see module docstring for the readings)."""
+    x = np.asarray(samples, dtype=np.float64)
+    if x.shape[0] < n_codes:
+        raise ValueError("need at least n_codes samples")
+    cent = x[:n_codes].copy()
+    for _ in range(iters):
+        diff_sq = np.empty((x.shape[0], n_codes))
+        for a in range(0, x.shape[0], 4096):
+            diff = x[a:a + 4096, None, :] - cent[None, :, :]
+            diff_sq[a:a + 4096] = np.sum(diff * diff, axis=2)
+        label = np.argmin(diff_sq, axis=1)
+        for k in range(n_codes):
+            members = x[label == k]
+            if members.shape[0] > 0:
+                cent[k] = members.sum(axis=0) / members.shape[0]
+    return cent
+
+
+def build_codebook(seed: int, n_samples: int, n_codes: int, dim: int,
+                   abs_mode: bool, iters: int) -> np.ndarray:
+    """Codebook [n_codes, dim] as fp16-representable values (returned fp64)."""
+    cent = kmeans(normal_samples(seed, n_samples, dim, abs_mode), n_codes, iters)
+    return cent.astype(np.float16).astype(np.float64)
