@@ -1,0 +1,432 @@
+"""Benchmark of the NSNQuant KV hot path on B200.
+
+Default workload (one GPU): the decode-throughput layer -- batch 16, 32 query /
+8 KV heads, head_dim 128, 32768-token context per sequence quantized to 2-bit K
+and V with a 128-token fp16 residual window.  One timed step = one decode step
+of the whole batch: append one new K/V token per (sequence, kv-head) (flushing
+the full window through the quantizer on the first step) + decode attention of
+all 32 query heads.  `value` = generated tokens/s = batch * steps / time.
+
+The same JSON line also carries the compressed-KV GB/s, the roofline of the
+decode call, the prefill quantizer's throughput (tokens/s) with its own ALU
+roofline, an end-to-end number through the public API with host buffers, the
+SM clocks seen during the timed region, and the CPU oracle baseline.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torchrun; each rank runs an
+independent replica (the path shards by sequence; no collective is needed).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn tokens/s & compressed-KV GB/s vs HBM peak; quantize tokens/s"
+WORKLOAD = dict(config=3, name="decode-b16-32k-2bit", batch=16, n_kv_heads=8, n_q_heads=32, seq=32768,
+                mode_k=2, mode_v=2, window=128)
+BYTES_PER_TOKEN = {1: 16 + 4, 2: 16 + 16 + 4}   # codes (+ signs) + (s1, s2) per token-head
+MEAN_BYTES_PER_BLOCK = 128 * 2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+
+
+# ---------------------------------------------------------------------------
+# clocks sampler (nvidia-smi during the timed region)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id, self.proc, self.lines = gpu_id, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (test infrastructure; the only other place bench runs oracle/)
+# ---------------------------------------------------------------------------
+def oracle_decode_sample(budget_s: float, seed: int = 0):
+    """Times the oracle's decode attention for sampled (b, kv-head) sequences of
+    the workload shape (random compressed contents, 2-bit K/V, full window).
+    Returns (seconds per (b, kv-head), sequences timed, threads)."""
+    from calibration_free_vector_b200 import synthetic
+    from oracle import nsn_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    W = WORKLOAD
+    nq = W["seq"] - 128
+    g = W["n_q_heads"] // W["n_kv_heads"]
+    cbk = np.abs(np.random.RandomState(seed).normal(size=(256, 8)))
+    rs = np.random.RandomState(seed + 1)
+    times, n = [], 0
+    t_start = time.perf_counter()
+    while True:
+        kc = synthetic.random_cache_contents(seed + 10 * n, nq, 128, W["mode_k"])
+        vc = synthetic.random_cache_contents(seed + 10 * n + 5, nq, 128, W["mode_v"])
+        f = lambda c: {"codes": c["codes"].astype(np.int64), "signs": c["signs"],  # noqa: E731
+                       "s1": c["s1"].astype(np.float64), "s2": c["s2"].astype(np.float64),
+                       "o": c["o"].astype(np.float64)}
+        q = rs.normal(size=(g, 128))
+        t0 = time.perf_counter()
+        orc.decode_attention(q, f(kc), f(vc), kc["window"].astype(np.float64), vc["window"].astype(np.float64),
+                             cbk, cbk, W["mode_k"], W["mode_v"], 1 / math.sqrt(128))
+        times.append(time.perf_counter() - t0)
+        n += 1
+        if time.perf_counter() - t_start > budget_s or n >= 64:
+            break
+    return float(np.mean(times)), n, threads
+
+
+def oracle_quantize_sample(budget_s: float, seed: int = 0):
+    """Times the oracle quantizing sampled 128-token blocks of the workload's K
+    (2-bit).  Returns (seconds per block, blocks timed)."""
+    import torch
+    from calibration_free_vector_b200 import synthetic
+    from oracle import nsn_oracle as orc
+    cb = np.abs(np.random.RandomState(seed).normal(size=(256, 8)))
+    x = synthetic.KVRecipe(seed, 1).tokens(1, 128 * 8, torch.bfloat16, "cpu").float().numpy()[0, :, 0]
+    times = []
+    t_start = time.perf_counter()
+    for i in range(8):
+        t0 = time.perf_counter()
+        orc.quantize_block(x[128 * i:128 * (i + 1)].astype(np.float64), cb, 2)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_start > budget_s:
+            break
+    return float(np.mean(times)), len(times)
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle on the host cores, same metric/unit."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    W = WORKLOAD
+    per_seq = []
+    for _ in range(args.warmup):
+        oracle_decode_sample(0.0, seed=99)
+    threads = 1
+    per_step_budget = min(5.0, 100.0 / max(1, args.steps))
+    for s in range(args.steps):
+        t, n, threads = oracle_decode_sample(per_step_budget, seed=s)
+        per_seq.append(t)
+    step_s = float(np.mean(per_seq)) * W["batch"] * W["n_kv_heads"]
+    value = W["batch"] / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": W["name"], "batch": W["batch"], "seq_len": W["seq"], "n_q_heads": W["n_q_heads"],
+                   "n_kv_heads": W["n_kv_heads"], "mode_k": W["mode_k"], "mode_v": W["mode_v"],
+                   "window": W["window"], "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: oracle decode attention of >=1 sampled (batch, kv-head) "
+                                   f"sequence ({W['seq'] - 128} quantized + 128 window tokens, 4 q-heads), "
+                                   f"scaled to {W['batch']}x{W['n_kv_heads']} sequences"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from calibration_free_vector_b200 import nsn, synthetic
+    from calibration_free_vector_b200.build import build
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    nsn.load()
+
+    W = WORKLOAD
+    B, H, HQ, T = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["seq"]
+    g = HQ // H
+    K, WU = args.steps, args.warmup
+    e2e_steps = max(4, K // 2)
+    total_steps = WU + K + e2e_steps
+    cap = ((T + K + e2e_steps + 255) // 128) * 128
+
+    # codebooks from the host builder (k-means on seeded randn)
+    cbk_np = nsn.nsn_build_codebook_host(0x4E534E02, 65536, 256, 8, W["mode_k"] == 2, 20)
+    cbv_np = nsn.nsn_build_codebook_host(0x4E534E02 if W["mode_v"] == 2 else 0x4E534E01, 65536, 256, 8,
+                                         W["mode_v"] == 2, 20)
+    cbk, cbv = torch.from_numpy(cbk_np).to(dev), torch.from_numpy(cbv_np).to(dev)
+
+    rk = synthetic.KVRecipe(synthetic.config_seed(3, "k") + 7 * rank, H)
+    rv = synthetic.KVRecipe(synthetic.config_seed(3, "v") + 7 * rank, H)
+    kc = nsn.Cache(B, H, cap, W["window"], W["mode_k"], device=dev)
+    vc = nsn.Cache(B, H, cap, W["window"], W["mode_v"], device=dev)
+    stream = torch.cuda.current_stream()
+
+    # ---- prefill (quantizer throughput is measured here) ----
+    xk = rk.tokens(B, T, torch.bfloat16, dev, stream_id=0)
+    xv = rv.tokens(B, T, torch.bfloat16, dev, stream_id=0)
+    q_tokens = 128 * ((T - 1) // 128)
+    quant_ms = []
+    for rep in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        nsn.nsn_quantize_kv(kc, xk, cbk)
+        nsn.nsn_quantize_kv(vc, xv, cbv)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        quant_ms.append(e0.elapsed_time(e1))
+    quant_ms_best = min(quant_ms[1:])
+    new_k = rk.tokens(B, total_steps, torch.bfloat16, dev, stream_id=1)
+    new_v = rv.tokens(B, total_steps, torch.bfloat16, dev, stream_id=1)
+    qs = torch.stack([synthetic.queries(synthetic.config_seed(3, "q") + s, B, HQ, torch.bfloat16, dev)
+                      for s in range(total_steps)])
+    del xk, xv
+    out = torch.empty((B, HQ, 128), dtype=torch.float32, device=dev)
+    ws = nsn.decode_workspace(kc, HQ, dev)
+    scale = 1.0 / math.sqrt(128)
+
+    def step(s):
+        nsn.nsn_append_residual(kc, vc, new_k[s], new_v[s], cbk, cbv)
+        nsn.nsn_decode_attention(kc, vc, qs[s], scale, cbk, cbv, out, ws)
+
+    for s in range(WU):
+        step(s)
+    # Re-prefill so that the timed steps start from the workload's state: a full
+    # residual window, which the first timed append flushes (then one flush per
+    # 128 steps, as in the 64-step decode-throughput run).
+    nsn.nsn_quantize_kv(kc, rk.tokens(B, T, torch.bfloat16, dev, stream_id=0), cbk)
+    nsn.nsn_quantize_kv(vc, rv.tokens(B, T, torch.bfloat16, dev, stream_id=0), cbv)
+    torch.cuda.synchronize()
+
+    # ---- timed region ----
+    gpu_id = getattr(torch.cuda.get_device_properties(dev), "pci_bus_id", None) or str(local_rank)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(K):
+        s = WU + i
+        nsn.nsn_append_residual(kc, vc, new_k[s], new_v[s], cbk, cbv)
+        ev[i][0].record(stream)
+        nsn.nsn_decode_attention(kc, vc, qs[s], scale, cbk, cbv, out, ws)
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    # keep the same load for ~1 s more so that the clock sampler sees it
+    soak_end = time.perf_counter() + 1.0
+    while time.perf_counter() < soak_end:
+        for _ in range(20):
+            nsn.nsn_decode_attention(kc, vc, qs[WU + K - 1], scale, cbk, cbv, out, ws)
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    clocks["window"] = "timed region + 1 s of the same decode call right after it"
+
+    ms = t0.elapsed_time(t1)
+    decode_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_per_step = ms / K
+
+    # ---- algorithmic bytes of one decode call ----
+    nq = int(kc.n_quant[0, 0].item())
+    nw = int(kc.n_window[0, 0].item())
+    seqs = B * H
+    per_tok = BYTES_PER_TOKEN[W["mode_k"]] + BYTES_PER_TOKEN[W["mode_v"]]
+    compressed = seqs * (nq * per_tok + 2 * (nq // 128) * MEAN_BYTES_PER_BLOCK)
+    window_bytes = seqs * 2 * nw * 128 * 2
+    io_bytes = B * HQ * 128 * (2 + 4)
+    decode_bytes = compressed + window_bytes + io_bytes
+    dec_avg_ms = float(np.mean(decode_ms))
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers ----
+    pin_k = new_k.cpu().pin_memory()
+    pin_v = new_v.cpu().pin_memory()
+    pin_q = qs.cpu().pin_memory()
+    host_out = torch.empty((B, HQ, 128), dtype=torch.float32).pin_memory()
+    dk = torch.empty_like(new_k[0])
+    dv = torch.empty_like(new_v[0])
+    dq = torch.empty_like(qs[0])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        s = WU + K + i
+        dk.copy_(pin_k[s], non_blocking=True)
+        dv.copy_(pin_v[s], non_blocking=True)
+        dq.copy_(pin_q[s], non_blocking=True)
+        nsn.nsn_append_residual(kc, vc, dk, dv, cbk, cbv)
+        nsn.nsn_decode_attention(kc, vc, dq, scale, cbk, cbv, out, ws)
+        host_out.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = (dk.numel() + dv.numel() + dq.numel()) * 2
+    d2h = host_out.numel() * 4
+
+    status = int(kc.status.item()) | int(vc.status.item())
+
+    # ---- quantizer roofline (ALU-bound exhaustive search) ----
+    qtoken_heads = 2 * B * H * q_tokens
+    q_bytes = B * H * q_tokens * (2 * 256 + (BYTES_PER_TOKEN[W["mode_k"]] + BYTES_PER_TOKEN[W["mode_v"]])) \
+        + 2 * B * H * (q_tokens // 128) * MEAN_BYTES_PER_BLOCK
+    fma_per_th = 16 * 256 * 8
+    alu_peak = 148 * 128 * 1.965e9 / 1e12   # FP32 FMA lanes x max SM clock, in T FMA/s
+    q_ach = qtoken_heads * fma_per_th / (quant_ms_best * 1e-3) / 1e12
+
+    if rank == 0:
+        cpu_t, cpu_n, cpu_threads = oracle_decode_sample(float(os.environ.get("NSN_CPU_BUDGET_S", "15")))
+        cpu_step = cpu_t * B * H
+        cq_t, cq_n = oracle_quantize_sample(8.0)
+        line = {
+            "metric": METRIC,
+            "value": world * B * K / (ms * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world, "steps": K, "warmup": WU, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": W["name"], "batch": B, "seq_len": T, "n_q_heads": HQ, "n_kv_heads": H,
+                       "head_dim": 128, "mode_k": W["mode_k"], "mode_v": W["mode_v"], "window": W["window"],
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "l2": f"inputs larger than L2 (compressed cache {compressed / 1e6:.0f} MB per step)"},
+            "compressed_kv_gbs": decode_bytes / (ms_per_step * 1e-3) / 1e9,
+            "decode_call_ms": dec_avg_ms,
+            "roofline": {"kernel": "decode call (decode_split_kernel + window + combine)", "bound": "hbm",
+                         "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "peak_kind": peak_kind, "traffic": None,
+                         "algorithmic_bytes_per_launch": decode_bytes,
+                         "frac_of_8tbs_spec": achieved / 8000.0},
+            "quantize": {"workload": f"prefill {B}x{q_tokens} tokens x {H} kv-heads, K 2-bit + V 2-bit, bf16 in",
+                         "tokens_per_s": B * q_tokens / (quant_ms_best * 1e-3),
+                         "token_heads_per_s": qtoken_heads / (quant_ms_best * 1e-3),
+                         "ms": quant_ms_best, "gbs": q_bytes / (quant_ms_best * 1e-3) / 1e9,
+                         "hbm_frac": q_bytes / (quant_ms_best * 1e-3) / 1e9 / hbm,
+                         "roofline": {"kernel": "quantize_prefill_kernel", "bound": "alu", "achieved": q_ach,
+                                      "peak": alu_peak, "unit": "T FMA/s (fp32)", "frac": q_ach / alu_peak,
+                                      "algorithmic_fma_per_token_head": fma_per_th}},
+            "e2e": {"value": world * B * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": K * 4,
+            "clocks": clocks,
+            "cache_status": status,
+            "cpu_baseline": {"value": B / cpu_step, "unit": "tokens/s", "cores": cpu_threads, "kind": "oracle",
+                             "sample": f"oracle decode attention of {cpu_n} sampled (batch, kv-head) sequences "
+                                       f"({nq} quantized + 128 window tokens, {g} q-heads) scaled to "
+                                       f"{B}x{H} sequences per step",
+                             "quantize_token_heads_per_s": 128 / cq_t,
+                             "quantize_sample": f"{cq_n} oracle 128-token 2-bit blocks"},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,109 @@
+// Host-side codebook construction (nsn_build_codebook_host in include/nsn.h).
+//
+// "NSNQuant: A Double Normalization Approach ...", technical summary,
+// Metodologia 3: the single global codebook is initialised by k-means on
+// synthetic standard-normal data; the README's "Codebook tuning" builds the
+// 2-bit codebook over absolute values (--abs).
+//
+// Standard normals: Philox4x64-10 counter-based generator (Salmon, Moraes, Dror,
+// Shaw, SC'11) + Box-Muller transform (Box & Muller, 1958); stream layout in nsn.h.
+
+#include <cmath>
+#include <cstdint>
+#include <vector>
+
+#include <cuda_fp16.h>
+
+#include "nsn.h"
+
+namespace {
+
+constexpr uint64_t kM0 = 0xD2E7470EE14C6C93ull;
+constexpr uint64_t kM1 = 0xCA5A826395121157ull;
+constexpr uint64_t kW0 = 0x9E3779B97F4A7C15ull;
+constexpr uint64_t kW1 = 0xBB67AE8584CAA73Bull;
+constexpr uint64_t kStreamKey1 = 0x4E534E51ull;
+
+struct Block4 {
+  uint64_t w[4];
+};
+
+Block4 philox4x64_10(uint64_t c0, uint64_t c1, uint64_t c2, uint64_t c3, uint64_t k0, uint64_t k1) {
+  for (int r = 0; r < 10; ++r) {
+    const unsigned __int128 p0 = (unsigned __int128)kM0 * c0;
+    const unsigned __int128 p1 = (unsigned __int128)kM1 * c2;
+    const uint64_t hi0 = (uint64_t)(p0 >> 64), lo0 = (uint64_t)p0;
+    const uint64_t hi1 = (uint64_t)(p1 >> 64), lo1 = (uint64_t)p1;
+    const uint64_t n0 = hi1 ^ c1 ^ k0, n1 = lo1, n2 = hi0 ^ c3 ^ k1, n3 = lo0;
+    c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    k0 += kW0;
+    k1 += kW1;
+  }
+  return Block4{{c0, c1, c2, c3}};
+}
+
+double uniform_open(uint64_t w) { return ((double)(w >> 12) + 0.5) * 0x1.0p-52; }
+
+void normal_stream(uint64_t seed, size_t count, double* out) {
+  const double two_pi = 2.0 * M_PI;
+  for (size_t j = 0; 4 * j < count; ++j) {
+    const Block4 b = philox4x64_10(j, 0, 0, 0, seed, kStreamKey1);
+    double z[4];
+    for (int pr = 0; pr < 2; ++pr) {
+      const double ua = uniform_open(b.w[2 * pr]), ub = uniform_open(b.w[2 * pr + 1]);
+      const double r = std::sqrt(-2.0 * std::log(ua));
+      z[2 * pr] = r * std::cos(two_pi * ub);
+      z[2 * pr + 1] = r * std::sin(two_pi * ub);
+    }
+    for (int i = 0; i < 4 && 4 * j + i < count; ++i) out[4 * j + i] = z[i];
+  }
+}
+
+}  // namespace
+
+extern "C" nsn_status nsn_build_codebook_host(uint64_t seed, int n_samples, int n_codes, int dim, int abs_mode,
+                                              int iters, float* out) {
+  if (!out || n_codes <= 0 || dim <= 0 || n_samples < n_codes || iters < 0) return NSN_ERR_INVALID_ARG;
+  const size_t n = (size_t)n_samples, k = (size_t)n_codes, d = (size_t)dim;
+  std::vector<double> x(n * d);
+  normal_stream(seed, n * d, x.data());
+  if (abs_mode)
+    for (double& v : x) v = std::fabs(v);
+
+  std::vector<double> cent(x.begin(), x.begin() + k * d);  // first n_codes samples
+  std::vector<double> sums(k * d);
+  std::vector<int64_t> counts(k);
+  std::vector<int32_t> label(n);
+  for (int it = 0; it < iters; ++it) {
+    for (size_t i = 0; i < n; ++i) {
+      const double* xi = &x[i * d];
+      double best = INFINITY;
+      int32_t bi = 0;
+      for (size_t c = 0; c < k; ++c) {
+        const double* cc = &cent[c * d];
+        double s = 0.0;
+        for (size_t e = 0; e < d; ++e) {
+          const double df = xi[e] - cc[e];
+          s += df * df;
+        }
+        if (s < best) {
+          best = s;
+          bi = (int32_t)c;
+        }
+      }
+      label[i] = bi;
+    }
+    std::fill(sums.begin(), sums.end(), 0.0);
+    std::fill(counts.begin(), counts.end(), 0);
+    for (size_t i = 0; i < n; ++i) {
+      const size_t c = (size_t)label[i];
+      counts[c] += 1;
+      for (size_t e = 0; e < d; ++e) sums[c * d + e] += x[i * d + e];
+    }
+    for (size_t c = 0; c < k; ++c)
+      if (counts[c] > 0)
+        for (size_t e = 0; e < d; ++e) cent[c * d + e] = sums[c * d + e] / (double)counts[c];
+  }
+  for (size_t i = 0; i < k * d; ++i) out[i] = __half2float(__double2half(cent[i]));
+  return NSN_OK;
+}

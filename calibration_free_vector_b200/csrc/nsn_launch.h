@@ -1,0 +1,47 @@
+// Internal interface between the C ABI (nsn_api.cpp) and the kernels.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace nsn {
+
+// Device view of one nsn_cache (same buffers, typed pointers).
+struct CacheView {
+  int batch, n_kv_heads, capacity, window_len, mode, scale_adjust;
+  uint8_t* codes;
+  uint8_t* signs;
+  __half2* norms;
+  __half* means;
+  __half* window;
+  int32_t* n_quant;
+  int32_t* n_window;
+  int32_t* status;
+};
+
+// Decode split geometry: the quantized range of every (b, kv-head) is cut into
+// chunks of `chunk` tokens; one more partial slot holds the residual window.
+struct DecodeGeom {
+  int chunk;         // tokens per split (multiple of 128)
+  int nsplit_q;      // splits over the quantized part
+  int g;             // query heads per kv-head
+};
+
+DecodeGeom decode_geometry(int capacity, int n_q_heads, int n_kv_heads);
+size_t decode_workspace_bytes(int batch, int n_kv_heads, const DecodeGeom& geom);
+
+size_t quant_smem_bytes();
+
+cudaError_t launch_quantize_prefill(const void* x, int dtype, int64_t sb, int64_t st, int64_t sh, int q_tokens,
+                                    int n_tokens, const CacheView& cv, const float* cb, cudaStream_t s);
+
+cudaError_t launch_append(const CacheView& kc, const CacheView& vc, const void* kn, const void* vn, int dtype,
+                          int64_t sb, int64_t sh, const float* cbk, const float* cbv, cudaStream_t s);
+
+cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                          int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
+                          float* out, void* ws, const DecodeGeom& geom, cudaStream_t s);
+
+}  // namespace nsn

@@ -1,0 +1,544 @@
+// NSNQuant KV quantizer kernels (sm_100a).
+//
+// Method: "NSNQuant: A Double Normalization Approach for Calibration-Free Low-Bit
+// Vector Quantization of KV Cache", technical summary, Metodologia 1 (NSN),
+// 2 (Hadamard), 3 (VQ with one global codebook, adaptive scale) and 4 (KIVI-style
+// residual that is flushed into the quantized part when full).
+//
+// One CTA of 128 threads quantizes one block of <= 128 tokens of one (batch,
+// kv-head); thread t owns token t.  Per block:
+//   r      = column mean of the raw tokens (fp64 sum, stored as fp32)
+//   d_t    = FWHT(x_t - r)                 fp32, in registers (exact algebra:
+//   w_t    = d_t + FWHT(r)                 FWHT is linear; FWHT(r) in fp64)
+//   s1     = ||x_t|| / sqrt(128)  (= ||H x_t|| / sqrt(128), H orthonormal)
+//   n1_t   = w_t rr_t, rr_t = 1/||x_t||;  o = FWHT(r) mean(rr) + mean_t(d_t rr_t)
+//   z_t    = d_t rr_t + FWHT(r)(rr_t - mean rr) - mean_t(d_t rr_t)       (fp64 -> fp32)
+//   s2     = ||z_t|| / sqrt(128),  u_t = z_t / s2                          (u: fp32)
+// Subtracting r before the fp32 transform keeps the large token-constant channel
+// offsets (outliers) out of the fp32 rounding, so u carries fp32 precision
+// relative to the token-varying part that survives the shift step.
+//
+// Nearest codeword: exhaustive fp32 search over the 256 codewords held in shared
+// memory (broadcast reads), score_k = u.c_k - ||c_k||^2/2, tracking the best and
+// second-best score.  Whenever the second best lies within the rigorous fp32
+// error bound of the best, the sub-vector is re-decided exactly in fp64 over all
+// codewords inside that bound (ties to the lowest index).  The stored code is
+// therefore the exact nearest codeword of the fp32 u.
+
+#include "nsn_common.cuh"
+#include "nsn_launch.h"
+
+namespace nsn {
+
+// Shared-memory fp64 load that the compiler may not merge with other loads of the
+// same address (keeps 128-entry fp64 tables from being cached in registers).
+__device__ __forceinline__ double lds_f64(const double* p) {
+  double r;
+  asm volatile("ld.shared.f64 %0, [%1];" : "=d"(r) : "r"((unsigned)__cvta_generic_to_shared(p)));
+  return r;
+}
+
+struct QuantSmem {
+  alignas(16) float cb[NCODES][SUB];   // codebook (fp32)
+  alignas(16) float bias[NCODES];      // -||c_k||^2 / 2
+  alignas(16) float cnorm[4];          // [0] = max ||c||, [1] = max ||c||^2 (rounded up)
+  alignas(16) double rr[BLK];          // 1 / ||x_t|| (0 for a zero token)
+  alignas(16) double s1[BLK];          // per-token s1 and s2 (fp64) until the final store
+  alignas(16) double s2[BLK];
+  alignas(16) double big_r[D];         // FWHT(r) in fp64
+  alignas(16) double o[D];             // D_c = mean_t(d_t,c rr_t) (the token-varying part of o)
+  alignas(16) float r[D];              // column mean of raw tokens (fp32)
+  alignas(16) float tile[BLK][D + 4];  // raw tokens, then d_t rows, then u rows; padded by 16 B
+  alignas(16) float thr[BLK][NSUB];    // per (token, sub-vector) threshold of the exact re-decision
+  alignas(16) uint8_t code[BLK][NSUB]; // chosen codes
+};
+
+// Stages the codebook, its biases and norm bounds.  All 128 threads.
+__device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook) {
+  const int t = threadIdx.x;
+  for (int i = t; i < NCODES * SUB / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(&sm.cb[0][0])[i] = __ldg(reinterpret_cast<const float4*>(codebook) + i);
+  __syncthreads();
+  float my_max = 0.f;
+  for (int k = t; k < NCODES; k += blockDim.x) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) s = fmaf(sm.cb[k][i], sm.cb[k][i], s);
+    sm.bias[k] = -0.5f * s;
+    my_max = fmaxf(my_max, s);
+  }
+  my_max = warp_max(my_max);
+  __shared__ float red[4];
+  if ((t & 31) == 0) red[t >> 5] = my_max;
+  __syncthreads();
+  if (t == 0) {
+    float m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    m *= 1.0001f;  // upper bound on max ||c||^2 despite the fp32 rounding above
+    sm.cnorm[1] = m;
+    sm.cnorm[0] = sqrtf(m) * 1.0001f;
+  }
+  __syncthreads();
+}
+
+// Quantizes one block of n (1..128) tokens.  Rows are at
+// src + row0 + t*row_stride (elements).  Output pointers are already offset to
+// the block's first token (codes, signs, norms) and to its mean row (means).
+template <int DT, int MODE>
+__device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, int64_t row0,
+                                   int64_t row_stride, int n, uint8_t* __restrict__ codes,
+                                   uint8_t* __restrict__ signs, __half2* __restrict__ norms,
+                                   __half* __restrict__ means, int scale_adjust) {
+  const int t = threadIdx.x;
+  const bool valid = t < n;
+  constexpr int ESZ = (DT == NSN_DTYPE_F32) ? 4 : 2;
+  constexpr int CHUNKS = D * ESZ / 16;  // 16-byte chunks per row
+
+  // ---- cooperative, coalesced load of the raw tile into shared memory --------
+  {
+    char* tile_bytes = reinterpret_cast<char*>(&sm.tile[0][0]);
+    constexpr int ROWB = (D + 4) * 4;  // padded row stride in bytes (fits both dtypes)
+    for (int q = t; q < BLK * CHUNKS; q += blockDim.x) {
+      const int row = q / CHUNKS, ch = q % CHUNKS;
+      if (row < n) {
+        const char* g = static_cast<const char*>(src) + (row0 + (int64_t)row * row_stride) * ESZ + ch * 16;
+        *reinterpret_cast<uint4*>(tile_bytes + row * ROWB + ch * 16) = __ldg(reinterpret_cast<const uint4*>(g));
+      }
+    }
+  }
+  __syncthreads();
+
+  auto raw_at = [&](int row, int c) -> float {
+    const char* tb = reinterpret_cast<const char*>(&sm.tile[0][0]) + row * (D + 4) * 4;
+    if constexpr (DT == NSN_DTYPE_F32) return reinterpret_cast<const float*>(tb)[c];
+    else if constexpr (DT == NSN_DTYPE_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(tb)[c]);
+    else return __half2float(reinterpret_cast<const __half*>(tb)[c]);
+  };
+
+  // ---- reference r = column mean of the raw tokens ---------------------------
+  {
+    double s = 0.0;
+    for (int row = 0; row < n; ++row) s += (double)raw_at(row, t);
+    sm.r[t] = (float)(s / n);
+  }
+  __syncthreads();
+  // FWHT(r) in fp64 by warp 0 (lane l holds elements 4l..4l+3).
+  if (t < 32) {
+    double v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = (double)sm.r[4 * t + i];
+    double a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
+    v[0] = a0 + a2; v[2] = a0 - a2; v[1] = a1 + a3; v[3] = a1 - a3;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const bool upper = (t & m) != 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        double other = __shfl_xor_sync(0xffffffffu, v[i], m);
+        v[i] = upper ? (other - v[i]) : (v[i] + other);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sm.big_r[4 * t + i] = v[i];
+  }
+
+  // ---- d_t = FWHT(x_t - r) in registers; ||x_t||^2 from the raw values -------
+  float v[D];
+  double ssx0 = 0.0, ssx1 = 0.0;
+  if (valid) {
+    const char* tb = reinterpret_cast<const char*>(&sm.tile[t][0]);
+#pragma unroll
+    for (int ch = 0; ch < CHUNKS; ++ch) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(tb + ch * 16);
+      float xs[8];
+      constexpr int PER = (DT == NSN_DTYPE_F32) ? 4 : 8;
+      if constexpr (DT == NSN_DTYPE_F32) {
+        const float* f = reinterpret_cast<const float*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xs[i] = f[i];
+      } else if constexpr (DT == NSN_DTYPE_BF16) {
+        const __nv_bfloat162* f = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 p = __bfloat1622float2(f[i]);
+          xs[2 * i] = p.x;
+          xs[2 * i + 1] = p.y;
+        }
+      } else {
+        const __half2* f = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 p = __half22float2(f[i]);
+          xs[2 * i] = p.x;
+          xs[2 * i + 1] = p.y;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        v[PER * ch + i] = xs[i] - sm.r[PER * ch + i];
+        if (i & 1) ssx1 = fma((double)xs[i], (double)xs[i], ssx1);
+        else ssx0 = fma((double)xs[i], (double)xs[i], ssx0);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < D; ++c) v[c] = 0.f;
+  }
+  fwht128_regs(v);
+  __syncthreads();  // raw tile fully consumed; big_r ready
+
+  // ---- first normalization: s1 = ||H x|| / sqrt(128) = ||x|| / sqrt(128) -----
+  // (H is orthonormal.)  n1_t = w_t * rr_t with w_t = FWHT(x_t) = d_t + FWHT(r)
+  // and rr_t = 1/||x_t|| (||w_t|| = sqrt(128) ||x_t||); a zero token gets rr = 0.
+  {
+    const double ssx = ssx0 + ssx1;
+    const double norm_x = sqrt(ssx);
+    sm.s1[t] = norm_x / 11.313708498984761;
+    const double rr = (ssx > 0.0) ? 1.0 / norm_x : 0.0;
+    if (valid) {
+#pragma unroll
+      for (int c = 0; c < D; c += 4)
+        *reinterpret_cast<float4*>(&sm.tile[t][c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+      sm.rr[t] = rr;
+    }
+  }
+  __syncthreads();
+
+  // ---- shift: o = mean_t n1_t = FWHT(r) * mean(rr) + mean_t(d_t rr_t) --------
+  // mean(rr) is accumulated as deviations from rr_0 so that equal rr give it
+  // exactly (identical tokens then give z = 0 exactly, as the definition does).
+  double rr_mean;
+  {
+    const double rr0 = sm.rr[0];
+    double dev = 0.0, sd = 0.0;
+    for (int row = 0; row < n; ++row) {
+      const double rrow = sm.rr[row];
+      dev += rrow - rr0;
+      sd = fma((double)sm.tile[row][t], rrow, sd);
+    }
+    rr_mean = rr0 + dev / n;
+    const double dc = sd / n;
+    sm.o[t] = dc;  // holds D_c = mean_t(d_t,c rr_t) until the next barrier
+    means[t] = __double2half(fma(sm.big_r[t], rr_mean, dc));
+  }
+  __syncthreads();
+
+  // ---- second normalization --------------------------------------------------
+  // z_t = n1_t - o = d_t rr_t + FWHT(r) (rr_t - mean rr) - D.  The last two terms
+  // are formed in fp64 and rounded once (they are at the scale of z), then one
+  // fp32 fma per channel.
+  const double rr_t = valid ? sm.rr[t] : 0.0;
+  const double delta = rr_t - rr_mean;
+  const float rrf = (float)rr_t;
+  double zz0 = 0.0, zz1 = 0.0;
+#pragma unroll
+  for (int c = 0; c < D; c += 2) {
+    const float c0 = (float)fma(lds_f64(&sm.big_r[c]), delta, -lds_f64(&sm.o[c]));
+    const float c1 = (float)fma(lds_f64(&sm.big_r[c + 1]), delta, -lds_f64(&sm.o[c + 1]));
+    const float z0 = fmaf(v[c], rrf, c0);
+    const float z1 = fmaf(v[c + 1], rrf, c1);
+    v[c] = z0;
+    v[c + 1] = z1;
+    zz0 = fma((double)z0, (double)z0, zz0);
+    zz1 = fma((double)z1, (double)z1, zz1);
+  }
+  const double zz = zz0 + zz1;
+  sm.s2[t] = sqrt(zz) / 11.313708498984761;
+  const float inv2 = (zz > 0.0) ? (float)(11.313708498984761 / sqrt(zz)) : 0.f;
+#pragma unroll
+  for (int c = 0; c < D; ++c) v[c] *= inv2;
+  // v now holds u (fp32).
+
+  // ---- sign bits (2-bit) and search operand a = |u| or u ---------------------
+  // In 2-bit mode v is replaced by |u| after the sign bits are taken; every later
+  // use only needs |u| (u_c * u_hat_c = |u_c| * A_code,c because the signs match).
+  uint32_t sgn[4] = {0u, 0u, 0u, 0u};
+  if constexpr (MODE == NSN_MODE_2BIT) {
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      sgn[c >> 5] |= (v[c] < 0.f ? 1u : 0u) << (c & 31);
+      v[c] = fabsf(v[c]);
+    }
+  }
+
+  // ---- exhaustive fp32 search with best / second-best tracking ---------------
+  // Two passes over the codebook, 8 sub-vectors each (bounded register use).
+  // After each pass the codes, the exact-path thresholds and the "close second"
+  // flags go to shared memory.
+  const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1];
+  constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
+  uint32_t need = 0u;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float best1[NSUB / 2], best2[NSUB / 2];
+    int idx[NSUB / 2];
+#pragma unroll
+    for (int jj = 0; jj < NSUB / 2; ++jj) {
+      best1[jj] = -INFINITY;
+      best2[jj] = -INFINITY;
+      idx[jj] = 0;
+    }
+#pragma unroll 1
+    for (int k = 0; k < NCODES; ++k) {
+      const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
+      const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
+      const float bk = sm.bias[k];
+#pragma unroll
+      for (int jj = 0; jj < NSUB / 2; ++jj) {
+        const int j = 8 * half + jj;
+        float s = bk;
+        s = fmaf(v[8 * j + 0], c0.x, s);
+        s = fmaf(v[8 * j + 1], c0.y, s);
+        s = fmaf(v[8 * j + 2], c0.z, s);
+        s = fmaf(v[8 * j + 3], c0.w, s);
+        s = fmaf(v[8 * j + 4], c1.x, s);
+        s = fmaf(v[8 * j + 5], c1.y, s);
+        s = fmaf(v[8 * j + 6], c1.z, s);
+        s = fmaf(v[8 * j + 7], c1.w, s);
+        const float lo = fminf(best1[jj], s);
+        idx[jj] = (s > best1[jj]) ? k : idx[jj];
+        best1[jj] = fmaxf(best1[jj], s);
+        best2[jj] = fmaxf(best2[jj], lo);
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < NSUB / 2; ++jj) {
+      const int j = 8 * half + jj;
+      float na = 0.f;
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) na = fmaf(v[8 * j + i], v[8 * j + i], na);
+      na = sqrtf(na) * 1.0001f;
+      // |fp32 score - exact score| <= gamma_9 (max||c||^2 + ||a|| max||c||) for every
+      // codeword, so a rival within twice that bound of the best may be the true best.
+      const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
+      sm.thr[t][j] = best1[jj] - margin;
+      need |= (best2[jj] >= best1[jj] - margin ? 1u : 0u) << j;
+      sm.code[t][j] = (uint8_t)idx[jj];
+    }
+  }
+
+  // ---- hand u to shared memory (the tile rows are free again) ----------------
+  // From here on u is read from shared memory so that no register array stays
+  // live across the rarely taken exact path.
+#pragma unroll
+  for (int c = 0; c < D; c += 4)
+    *reinterpret_cast<float4*>(&sm.tile[t][c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+
+  // ---- exact fp64 re-decision of sub-vectors with a close second -------------
+  // Candidates: codewords whose fp32 score (same operation order as the main
+  // search) reaches the threshold; winner by fp64 squared distance, ties to the
+  // lowest index.
+#pragma unroll 1
+  for (int j = 0; j < NSUB; ++j) {
+    if (!((need >> j) & 1u)) continue;
+    const float* a = &sm.tile[t][8 * j];
+    const float thr = sm.thr[t][j];
+    double bestd = INFINITY;
+    int bi = sm.code[t][j];
+#pragma unroll 1
+    for (int k = 0; k < NCODES; ++k) {
+      float sc = sm.bias[k];
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) sc = fmaf(a[i], sm.cb[k][i], sc);
+      if (sc >= thr) {
+        double dd = 0.0;
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) {
+          const double e = (double)a[i] - (double)sm.cb[k][i];
+          dd = fma(e, e, dd);
+        }
+        if (dd < bestd) { bestd = dd; bi = k; }
+      }
+    }
+    sm.code[t][j] = (uint8_t)bi;
+  }
+
+  // ---- adaptive scale: alpha = ||u||^2 / (u . u_hat) --------------------------
+  double dot = 0.0, uu = 0.0;
+#pragma unroll 4
+  for (int j = 0; j < NSUB; ++j) {
+    const int cj = sm.code[t][j];
+    const float4 q0 = *reinterpret_cast<const float4*>(&sm.cb[cj][0]);
+    const float4 q1 = *reinterpret_cast<const float4*>(&sm.cb[cj][4]);
+    const float4 u0 = *reinterpret_cast<const float4*>(&sm.tile[t][8 * j]);
+    const float4 u1 = *reinterpret_cast<const float4*>(&sm.tile[t][8 * j + 4]);
+    const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    float dj = 0.f, uj = 0.f;
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) {
+      dj = fmaf(uv[i], qv[i], dj);
+      uj = fmaf(uv[i], uv[i], uj);
+    }
+    dot += (double)dj;
+    uu += (double)uj;
+  }
+  double alpha = (dot > 0.0) ? uu / dot : 1.0;
+  if (!scale_adjust) alpha = 1.0;
+
+  // ---- packed stores ---------------------------------------------------------
+  if (valid) {
+    *reinterpret_cast<uint4*>(codes + (int64_t)t * NSUB) = *reinterpret_cast<const uint4*>(&sm.code[t][0]);
+    if constexpr (MODE == NSN_MODE_2BIT)
+      *reinterpret_cast<uint4*>(signs + (int64_t)t * NSUB) = make_uint4(sgn[0], sgn[1], sgn[2], sgn[3]);
+    norms[t] = __halves2half2(__double2half(sm.s1[t]), __double2half(alpha * sm.s2[t]));
+  }
+  __syncthreads();  // shared memory is reused by the caller's next block
+}
+
+// ---------------------------------------------------------------------------
+// Prefill: grid (blocks, kv-heads, batch).
+// ---------------------------------------------------------------------------
+template <int DT, int MODE>
+__global__ void __launch_bounds__(128, 2)
+quantize_prefill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int64_t sh, int q_tokens,
+                        CacheView cv, const float* __restrict__ codebook) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw);
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int n = min(BLK, q_tokens - blk * BLK);
+  if (n <= 0) return;
+  stage_codebook(sm, codebook);
+  const int64_t seq = (int64_t)b * cv.n_kv_heads + h;
+  const int64_t tok0 = seq * cv.capacity + (int64_t)blk * BLK;
+  quantize_block_dev<DT, MODE>(sm, x, (int64_t)b * sb + (int64_t)blk * BLK * st + (int64_t)h * sh, st, n,
+                               cv.codes + tok0 * NSUB, MODE == NSN_MODE_2BIT ? cv.signs + tok0 * NSUB : nullptr,
+                               cv.norms + tok0, cv.means + (seq * (cv.capacity / BLK) + blk) * D,
+                               cv.scale_adjust);
+}
+
+// Prefill tail: copies tokens [q, L) to the residual window (fp16) and sets the
+// counters.  grid (kv-heads, batch), 128 threads.
+template <int DT>
+__global__ void window_fill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int64_t sh, int q_tokens,
+                                   int n_tokens, CacheView cv) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int64_t seq = (int64_t)b * cv.n_kv_heads + h;
+  const int nw = n_tokens - q_tokens;
+  for (int q = threadIdx.x; q < nw * (D / 8); q += blockDim.x) {
+    const int row = q / (D / 8), ch = q % (D / 8);
+    float vals[8];
+    load8<DT>(x, (int64_t)b * sb + (int64_t)(q_tokens + row) * st + (int64_t)h * sh + ch * 8, vals);
+    *reinterpret_cast<uint4*>(cv.window + (seq * cv.window_len + row) * D + ch * 8) = pack8_f16(vals);
+  }
+  if (threadIdx.x == 0) {
+    cv.n_quant[seq] = q_tokens;
+    cv.n_window[seq] = nw;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Append one token per (b, h) to K (blockIdx.z == 0) and V (blockIdx.z == 1),
+// flushing a full window into the quantized part first.  grid (kv-heads, batch, 2).
+// ---------------------------------------------------------------------------
+template <int DTN>
+__global__ void __launch_bounds__(128, 2)
+append_kernel(CacheView kc, CacheView vc, const void* __restrict__ k_new, const void* __restrict__ v_new,
+              int64_t sb, int64_t sh, const float* __restrict__ cbk, const float* __restrict__ cbv) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw);
+  __shared__ int state[2];
+  const bool is_v = blockIdx.z == 1;
+  const CacheView c = is_v ? vc : kc;
+  const void* src_new = is_v ? v_new : k_new;
+  const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  const int64_t seq = (int64_t)b * c.n_kv_heads + h;
+  if (t == 0) { state[0] = c.n_quant[seq]; state[1] = c.n_window[seq]; }
+  __syncthreads();
+  int nq = state[0], nw = state[1];
+  bool ok = true;
+  if (nw >= c.window_len) {
+    if (nq + BLK > c.capacity || (nq % BLK) != 0) {
+      ok = false;
+      if (t == 0 && c.status) atomicOr(c.status, 1);
+    } else {
+      stage_codebook(sm, is_v ? cbv : cbk);
+      const int64_t tok0 = seq * c.capacity + nq;
+      const int blk = nq / BLK;
+      uint8_t* sg = c.mode == NSN_MODE_2BIT ? c.signs + tok0 * NSUB : nullptr;
+      __half* mn = c.means + (seq * (c.capacity / BLK) + blk) * D;
+      if (c.mode == NSN_MODE_2BIT)
+        quantize_block_dev<NSN_DTYPE_F16, NSN_MODE_2BIT>(sm, c.window, seq * c.window_len * D, D, BLK,
+                                                         c.codes + tok0 * NSUB, sg, c.norms + tok0, mn,
+                                                         c.scale_adjust);
+      else
+        quantize_block_dev<NSN_DTYPE_F16, NSN_MODE_1BIT>(sm, c.window, seq * c.window_len * D, D, BLK,
+                                                         c.codes + tok0 * NSUB, sg, c.norms + tok0, mn,
+                                                         c.scale_adjust);
+      nq += BLK;
+      nw = 0;
+    }
+  }
+  __syncthreads();  // the flushed window rows are consumed before row 0 is overwritten
+  if (!ok) return;
+  if (t < D / 8) {
+    float vals[8];
+    load8<DTN>(src_new, (int64_t)b * sb + (int64_t)h * sh + t * 8, vals);
+    *reinterpret_cast<uint4*>(c.window + (seq * c.window_len + nw) * D + t * 8) = pack8_f16(vals);
+  }
+  if (t == 0) {
+    c.n_quant[seq] = nq;
+    c.n_window[seq] = nw + 1;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+size_t quant_smem_bytes() { return sizeof(QuantSmem); }
+
+template <int DT, int MODE>
+static cudaError_t launch_prefill_t(const void* x, int64_t sb, int64_t st, int64_t sh, int q_tokens,
+                                    const CacheView& cv, const float* cb, cudaStream_t s) {
+  const size_t smem = sizeof(QuantSmem);
+  cudaError_t e = cudaFuncSetAttribute(quantize_prefill_kernel<DT, MODE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int nblk = (q_tokens + BLK - 1) / BLK;
+  if (nblk > 0) {
+    dim3 grid(nblk, cv.n_kv_heads, cv.batch);
+    quantize_prefill_kernel<DT, MODE><<<grid, 128, smem, s>>>(x, sb, st, sh, q_tokens, cv, cb);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_prefill(const void* x, int dtype, int64_t sb, int64_t st, int64_t sh, int q_tokens,
+                                    int n_tokens, const CacheView& cv, const float* cb, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  if (q_tokens > 0) {
+    if (cv.mode == NSN_MODE_1BIT) {
+      if (dtype == NSN_DTYPE_F32) e = launch_prefill_t<NSN_DTYPE_F32, NSN_MODE_1BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
+      else if (dtype == NSN_DTYPE_BF16) e = launch_prefill_t<NSN_DTYPE_BF16, NSN_MODE_1BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
+      else e = launch_prefill_t<NSN_DTYPE_F16, NSN_MODE_1BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
+    } else {
+      if (dtype == NSN_DTYPE_F32) e = launch_prefill_t<NSN_DTYPE_F32, NSN_MODE_2BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
+      else if (dtype == NSN_DTYPE_BF16) e = launch_prefill_t<NSN_DTYPE_BF16, NSN_MODE_2BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
+      else e = launch_prefill_t<NSN_DTYPE_F16, NSN_MODE_2BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
+    }
+    if (e != cudaSuccess) return e;
+  }
+  dim3 g2(cv.n_kv_heads, cv.batch);
+  if (dtype == NSN_DTYPE_F32) window_fill_kernel<NSN_DTYPE_F32><<<g2, 128, 0, s>>>(x, sb, st, sh, q_tokens, n_tokens, cv);
+  else if (dtype == NSN_DTYPE_BF16) window_fill_kernel<NSN_DTYPE_BF16><<<g2, 128, 0, s>>>(x, sb, st, sh, q_tokens, n_tokens, cv);
+  else window_fill_kernel<NSN_DTYPE_F16><<<g2, 128, 0, s>>>(x, sb, st, sh, q_tokens, n_tokens, cv);
+  return cudaGetLastError();
+}
+
+template <int DTN>
+static cudaError_t launch_append_t(const CacheView& kc, const CacheView& vc, const void* kn, const void* vn,
+                                   int64_t sb, int64_t sh, const float* cbk, const float* cbv, cudaStream_t s) {
+  const size_t smem = sizeof(QuantSmem);
+  cudaError_t e = cudaFuncSetAttribute(append_kernel<DTN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(kc.n_kv_heads, kc.batch, 2);
+  append_kernel<DTN><<<grid, 128, smem, s>>>(kc, vc, kn, vn, sb, sh, cbk, cbv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const CacheView& kc, const CacheView& vc, const void* kn, const void* vn, int dtype,
+                          int64_t sb, int64_t sh, const float* cbk, const float* cbv, cudaStream_t s) {
+  if (dtype == NSN_DTYPE_F32) return launch_append_t<NSN_DTYPE_F32>(kc, vc, kn, vn, sb, sh, cbk, cbv, s);
+  if (dtype == NSN_DTYPE_BF16) return launch_append_t<NSN_DTYPE_BF16>(kc, vc, kn, vn, sb, sh, cbk, cbv, s);
+  return launch_append_t<NSN_DTYPE_F16>(kc, vc, kn, vn, sb, sh, cbk, cbv, s);
+}
+
+}  // namespace nsn

@@ -255,6 +255,7 @@ def quantize_sequence(x: np.ndarray, codebook: np.ndarray, mode: int,
         "s2": cat("s2", (0,)),
         "o": np.stack([p["o"] for p in parts]) if parts else np.zeros((0, d)),
         "gap": cat("gap", (0, nsub)),
+        "u": cat("u", (0, d)),
         "window": to_f16(x[q:]),
     }
 

@@ -1,0 +1,97 @@
+"""CPU checks of the C ABI: the library builds/loads, exports every symbol that
+include/nsn.h declares, validates arguments without a GPU, and its host-side
+codebook builder matches the oracle's k-means bit for bit."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from calibration_free_vector_b200 import nsn
+from calibration_free_vector_b200.build import build
+from oracle import codebook_oracle as cbo
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "nsn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return nsn.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nsn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.nsn_version() >= 100
+    assert lib.nsn_status_string(0) == b"ok"
+    assert lib.nsn_status_string(3) == b"workspace too small"
+
+
+def test_buffer_sizes(lib):
+    s = nsn.nsn_cache_buffer_sizes(16, 8, 32896, 128, 2)
+    assert s["codes"] == 16 * 8 * 32896 * 16 == s["signs"]
+    assert s["norms"] == 16 * 8 * 32896 * 4
+    assert s["means"] == 16 * 8 * (32896 // 128) * 128 * 2
+    assert s["window_buf"] == 16 * 8 * 128 * 128 * 2
+    s1 = nsn.nsn_cache_buffer_sizes(1, 1, 256, 0, 1)
+    assert s1["signs"] == 0 and s1["window_buf"] == 0
+    with pytest.raises(nsn.NsnError):
+        nsn.nsn_cache_buffer_sizes(1, 1, 100, 128, 2)   # capacity not a multiple of 128
+    with pytest.raises(nsn.NsnError):
+        nsn.nsn_cache_buffer_sizes(1, 1, 128, 64, 2)    # window must be 0 or 128
+
+
+def test_host_validation_without_gpu(lib):
+    # Every device entry point rejects bad arguments before touching the GPU.
+    c = nsn.nsn_cache(1, 1, 128, 128, 2, 1, 16, 16, 16, 16, 16, 16, 16, None)
+    assert lib.nsn_quantize_kv(ctypes.byref(c), None, 1, 0, 0, 0, 10, 16, None) == 1
+    bad = nsn.nsn_cache(1, 1, 100, 128, 2, 1, 16, 16, 16, 16, 16, 16, 16, None)
+    assert lib.nsn_quantize_kv(ctypes.byref(bad), 16, 1, 0, 0, 0, 10, 16, None) == 1
+    odd = nsn.nsn_cache(1, 1, 128, 64, 2, 1, 16, 16, 16, 16, 16, 16, 16, None)
+    assert lib.nsn_quantize_kv(ctypes.byref(odd), 16, 1, 0, 0, 0, 10, 16, None) == 2
+    # misaligned x, unaligned token stride, too many tokens
+    assert lib.nsn_quantize_kv(ctypes.byref(c), 18, 1, 0, 1024, 128, 10, 16, None) == 1
+    assert lib.nsn_quantize_kv(ctypes.byref(c), 16, 1, 0, 1020, 128, 10, 16, None) == 1
+    assert lib.nsn_quantize_kv(ctypes.byref(c), 16, 1, 0, 1024, 128, 300, 16, None) == 1
+    # decode: head count not a multiple, GQA group > 8, workspace too small
+    c2 = nsn.nsn_cache(1, 2, 128, 128, 2, 1, 16, 16, 16, 16, 16, 16, 16, None)
+    assert lib.nsn_decode_attention(ctypes.byref(c2), ctypes.byref(c2), 16, 1, 3, 0, 128, 0.1, 16, 16, 16, 16,
+                                    1 << 20, None) == 1
+    assert lib.nsn_decode_attention(ctypes.byref(c2), ctypes.byref(c2), 16, 1, 32, 0, 128, 0.1, 16, 16, 16, 16,
+                                    1 << 20, None) == 2
+    assert lib.nsn_decode_attention(ctypes.byref(c2), ctypes.byref(c2), 16, 1, 8, 0, 128, 0.1, 16, 16, 16, 16,
+                                    16, None) == 3
+    need = lib.nsn_decode_workspace_bytes(ctypes.byref(c2), 8)
+    assert need > 0
+    # append: window 0 caches cannot append; shapes must agree
+    c0 = nsn.nsn_cache(1, 2, 128, 0, 2, 1, 16, 16, 16, 16, None, 16, 16, None)
+    assert lib.nsn_append_residual(ctypes.byref(c0), ctypes.byref(c0), 16, 16, 1, 0, 128, 16, 16, None) == 2
+    assert lib.nsn_append_residual(ctypes.byref(c), ctypes.byref(c2), 16, 16, 1, 0, 128, 16, 16, None) == 1
+
+
+def test_host_codebook_matches_oracle(lib):
+    for abs_mode in (False, True):
+        ours = nsn.nsn_build_codebook_host(0x1234, 8192, 64, 8, abs_mode, 12)
+        ref = cbo.build_codebook(0x1234, 8192, 64, 8, abs_mode, 12)
+        assert np.array_equal(ours.astype(np.float64), ref)
+
+
+def test_host_codebook_full_size_properties(lib):
+    cb = nsn.nsn_build_codebook_host(7, 65536, 256, 8, True, 3)
+    assert cb.shape == (256, 8) and np.all(cb >= 0)
+    assert np.array_equal(cb, cb.astype(np.float16).astype(np.float32))
+    with pytest.raises(nsn.NsnError):
+        nsn.nsn_build_codebook_host(7, 100, 256, 8, False, 3)
