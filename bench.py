@@ -67,7 +67,7 @@ class ClockSampler:
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
@@ -253,8 +253,9 @@ def run_ours(args):
         torch.cuda.synchronize()
         quant_ms.append(e0.elapsed_time(e1))
     quant_ms_best = min(quant_ms[1:])
-    new_k = rk.tokens(B, total_steps, torch.bfloat16, dev, stream_id=1)
-    new_v = rv.tokens(B, total_steps, torch.bfloat16, dev, stream_id=1)
+    # per-step new tokens, [steps, B, H_kv, 128]
+    new_k = rk.tokens(B, total_steps, torch.bfloat16, dev, stream_id=1).transpose(0, 1).contiguous()
+    new_v = rv.tokens(B, total_steps, torch.bfloat16, dev, stream_id=1).transpose(0, 1).contiguous()
     qs = torch.stack([synthetic.queries(synthetic.config_seed(3, "q") + s, B, HQ, torch.bfloat16, dev)
                       for s in range(total_steps)])
     del xk, xv
@@ -276,7 +277,11 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     # ---- timed region ----
-    gpu_id = getattr(torch.cuda.get_device_properties(dev), "pci_bus_id", None) or str(local_rank)
+    props = torch.cuda.get_device_properties(dev)
+    try:
+        gpu_id = f"{int(props.pci_domain_id):08X}:{int(props.pci_bus_id):02X}:{int(props.pci_device_id):02X}.0"
+    except (AttributeError, TypeError, ValueError):
+        gpu_id = str(local_rank)
     sampler = ClockSampler(gpu_id)
     sampler.start()
     time.sleep(0.3)

@@ -108,7 +108,8 @@ nsn_status nsn_quantize_kv(nsn_cache* cache, const void* x, int dtype, int64_t s
                            int64_t stride_h, int n_tokens, const float* codebook, void* stream) {
   nsn_status st = check_cache(cache);
   if (st != NSN_OK) return st;
-  if (!x || !codebook || !valid_dtype(dtype) || n_tokens < 0) return NSN_ERR_INVALID_ARG;
+  if (!codebook || !valid_dtype(dtype) || n_tokens < 0) return NSN_ERR_INVALID_ARG;
+  if (n_tokens > 0 && !x) return NSN_ERR_INVALID_ARG;   // x is not read when n_tokens == 0
   if (!aligned16(x) || !aligned16(codebook)) return NSN_ERR_INVALID_ARG;
   const int64_t e16 = elems16(dtype);
   if (stride_b < 0 || stride_t < 0 || stride_h < 0) return NSN_ERR_INVALID_ARG;

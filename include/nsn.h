@@ -145,6 +145,7 @@ nsn_status nsn_build_codebook_host(uint64_t seed, int n_samples, int n_codes, in
  * (counters are overwritten).  [TS] Metodologia 1-3 (+ 4 for the residual split).
  *   x          device, dtype element type, token (b, t, h) row at
  *              x + b*stride_b + t*stride_t + h*stride_h (elements), 128 contiguous values.
+ *              May be NULL when n_tokens == 0 (only the counters are reset then).
  *   n_tokens   L >= 0, same for every batch row.  With window 128 the first
  *              Q = 128*floor((L-1)/128) tokens are quantized in blocks of 128 and the
  *              remaining L-Q (1..128) are copied (as fp16) to the window; with
