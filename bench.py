@@ -219,17 +219,18 @@ def run_ours(args):
     nsn.load()
 
     W = WORKLOAD
-    B, H, HQ, T = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["seq"]
+    B, H, HQ, T = args.batch or W["batch"], W["n_kv_heads"], W["n_q_heads"], W["seq"]
     g = HQ // H
     K, WU = args.steps, args.warmup
-    e2e_steps = max(4, K // 2)
+    e2e_steps = 0 if args.lite else max(4, K // 2)
     total_steps = WU + K + e2e_steps
     cap = ((T + K + e2e_steps + 255) // 128) * 128
 
     # codebooks from the host builder (k-means on seeded randn)
-    cbk_np = nsn.nsn_build_codebook_host(0x4E534E02, 65536, 256, 8, W["mode_k"] == 2, 20)
+    iters = 3 if args.lite else 20
+    cbk_np = nsn.nsn_build_codebook_host(0x4E534E02, 65536, 256, 8, W["mode_k"] == 2, iters)
     cbv_np = nsn.nsn_build_codebook_host(0x4E534E02 if W["mode_v"] == 2 else 0x4E534E01, 65536, 256, 8,
-                                         W["mode_v"] == 2, 20)
+                                         W["mode_v"] == 2, iters)
     cbk, cbv = torch.from_numpy(cbk_np).to(dev), torch.from_numpy(cbv_np).to(dev)
 
     rk = synthetic.KVRecipe(synthetic.config_seed(3, "k") + 7 * rank, H)
@@ -243,7 +244,7 @@ def run_ours(args):
     xv = rv.tokens(B, T, torch.bfloat16, dev, stream_id=0)
     q_tokens = 128 * ((T - 1) // 128)
     quant_ms = []
-    for rep in range(3):
+    for rep in range(2 if args.lite else 3):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         e0.record(stream)
@@ -302,7 +303,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     # keep the same load for ~1 s more so that the clock sampler sees it
-    soak_end = time.perf_counter() + 1.0
+    soak_end = time.perf_counter() + (0.0 if args.lite else 1.0)
     while time.perf_counter() < soak_end:
         for _ in range(20):
             nsn.nsn_decode_attention(kc, vc, qs[WU + K - 1], scale, cbk, cbv, out, ws)
@@ -333,33 +334,35 @@ def run_ours(args):
     achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers ----
-    pin_k = new_k.cpu().pin_memory()
-    pin_v = new_v.cpu().pin_memory()
-    pin_q = qs.cpu().pin_memory()
-    host_out = torch.empty((B, HQ, 128), dtype=torch.float32).pin_memory()
-    dk = torch.empty_like(new_k[0])
-    dv = torch.empty_like(new_v[0])
-    dq = torch.empty_like(qs[0])
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        s = WU + K + i
-        dk.copy_(pin_k[s], non_blocking=True)
-        dv.copy_(pin_v[s], non_blocking=True)
-        dq.copy_(pin_q[s], non_blocking=True)
-        nsn.nsn_append_residual(kc, vc, dk, dv, cbk, cbv)
-        nsn.nsn_decode_attention(kc, vc, dq, scale, cbk, cbv, out, ws)
-        host_out.copy_(out, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    h2d = (dk.numel() + dv.numel() + dq.numel()) * 2
-    d2h = host_out.numel() * 4
+    e2e_ms, h2d, d2h = 0.0, 0, 0
+    if not args.lite:
+        pin_k = new_k.cpu().pin_memory()
+        pin_v = new_v.cpu().pin_memory()
+        pin_q = qs.cpu().pin_memory()
+        host_out = torch.empty((B, HQ, 128), dtype=torch.float32).pin_memory()
+        dk = torch.empty_like(new_k[0])
+        dv = torch.empty_like(new_v[0])
+        dq = torch.empty_like(qs[0])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            s = WU + K + i
+            dk.copy_(pin_k[s], non_blocking=True)
+            dv.copy_(pin_v[s], non_blocking=True)
+            dq.copy_(pin_q[s], non_blocking=True)
+            nsn.nsn_append_residual(kc, vc, dk, dv, cbk, cbv)
+            nsn.nsn_decode_attention(kc, vc, dq, scale, cbk, cbv, out, ws)
+            host_out.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        h2d = (dk.numel() + dv.numel() + dq.numel()) * 2
+        d2h = host_out.numel() * 4
 
     status = int(kc.status.item()) | int(vc.status.item())
 
@@ -371,7 +374,11 @@ def run_ours(args):
     alu_peak = 148 * 128 * 1.965e9 / 1e12   # FP32 FMA lanes x max SM clock, in T FMA/s
     q_ach = qtoken_heads * fma_per_th / (quant_ms_best * 1e-3) / 1e12
 
-    if rank == 0:
+    if rank == 0 and args.lite:
+        print(json.dumps({"lite": True, "batch": B, "steps": K, "ms_per_step": ms_per_step,
+                          "decode_call_ms": dec_avg_ms, "decode_gbs": achieved, "quantize_ms": quant_ms_best,
+                          "cache_status": int(kc.status.item()) | int(vc.status.item())}), flush=True)
+    elif rank == 0:
         cpu_t, cpu_n, cpu_threads = oracle_decode_sample(float(os.environ.get("NSN_CPU_BUDGET_S", "15")))
         cpu_step = cpu_t * B * H
         cq_t, cq_n = oracle_quantize_sample(8.0)
@@ -425,6 +432,9 @@ def main():
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling runs)")
+    ap.add_argument("--lite", action="store_true",
+                    help="profiling run: no e2e leg, no clock soak, no CPU baseline; short summary line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
