@@ -94,219 +94,403 @@ __device__ __host__ __forceinline__ int64_t acc_offset(int64_t P, int G) { retur
 __device__ __forceinline__ float* partial_ml(float* ws, int64_t p, int G, int h) { return ws + (p * G + h) * 2; }
 
 // ---------------------------------------------------------------------------
-// Quantized part: grid (nsplit_q, kv-heads, batch), 128 threads.
+// Tensor-core building blocks (mma.sync m16n8k16, fp16 in / fp32 accumulate;
+// ldmatrix gathers of whole 8-dim codewords).
 // ---------------------------------------------------------------------------
-// Every member is 16-byte aligned (vector loads); unused tables shrink to 4 floats.
-template <int G, int MK, int MV>
-struct SplitSmem {
-  alignas(16) float qt[G][D];
-  alignas(16) float lut[MK == NSN_MODE_1BIT ? NSUB * NCODES * G : 4];  // [s][k][h]
-  alignas(16) float cbk[MK == NSN_MODE_2BIT ? NCODES * SUB : 4];
-  alignas(16) float cbv[NCODES * SUB];
-  alignas(16) float w[BLK][G];
-  alignas(16) uint4 vcode[BLK];
-  alignas(16) uint4 vsign[BLK];
-  alignas(16) float red[4][16];
-  alignas(16) float racc[8][G][D];  // final reduction over the 8 token groups
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+// d += A(16x16, rows a0/a1/a2/a3) * B(16x8, b0/b1); rows 8-15 of A are zero here.
+__device__ __forceinline__ void mma_rows0_7(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_full(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// 2^x with the hardware approximation (ex2.approx.ftz: ~2 ulp); 2^(-1e30) = 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Applies stored sign bits to a half2 fragment: `w` holds the two signs at bits
+// 15 - s and 31 - s; after the shift by s they sit on the fp16 sign bits.
+__device__ __forceinline__ uint32_t apply_signs(uint32_t x, uint32_t w, int s) {
+  return x ^ ((w << s) & 0x80008000u);
+}
+
+__device__ __forceinline__ uint32_t u4_word(const uint4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// ---------------------------------------------------------------------------
+// Quantized part.  One CTA of 16 warps per SM; every warp owns one split: a
+// contiguous range of 128-token blocks of one (batch, kv-head) sequence, and
+// writes its own partial (m, l, O).  The CTA shares only the two replicated
+// fp16 codebooks (staged once).  Compressed tokens stream through a per-warp
+// double-buffered ring of 64-token stages filled by cp.async, so one stage is
+// always in flight while the previous one is consumed.
+//
+// Per 16-token tile a warp computes, on the tensor cores,
+//   S^T[h][t]  = sum_k q~[h][k] u_hat[t][k]   (M = heads, N = 8 tokens, K = 16 dims)
+//   O^T[d][h] += sum_t u_hat_v[t][d] w[t][h]   (M = 16 dims, N = heads, K = 16 tokens)
+// with u_hat fragments gathered by ldmatrix from an 8-fold replicated fp16
+// codebook (replica r of code c at byte 128c + 16r: the 8 rows of each 8x8
+// matrix always hit 8 different bank groups), stored sign bits XOR-ed onto the
+// fp16 sign bits (2-bit mode), and w = p * s1 * s2 of the value tokens.  The S^T
+// accumulator fragment (head g, tokens 2p, 2p+1) is exactly the B fragment of
+// the value product, so no transpose is needed.  A rows g + 8 carry the fp16
+// rounding residual of q~ (the score adds both accumulator rows).
+// ---------------------------------------------------------------------------
+constexpr int DEC_WARPS = 16;
+constexpr int STAGE_TOK = 64;
+// stage layout (bytes): K codes | K signs | K norms | V codes | V signs | V norms | K mean | V mean
+constexpr int ST_KC = 0, ST_KS = 1024, ST_KN = 2048, ST_VC = 2304, ST_VS = 3328, ST_VN = 4352, ST_KM = 4608,
+              ST_VM = 4864, STAGE_BYTES = 5120;
+
+struct DecSmem {
+  alignas(128) uint4 cbk[NCODES][8];  // replicated fp16 codebooks (32 KB each)
+  alignas(128) uint4 cbv[NCODES][8];
+  alignas(128) unsigned char stage[DEC_WARPS][2][STAGE_BYTES];
 };
 
+__device__ __forceinline__ uint4 cb_row_f16(const float* __restrict__ cb, int c) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(cb + c * SUB));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(cb + c * SUB) + 1);
+  return make_uint4(pack_half2(a.x, a.y), pack_half2(a.z, a.w), pack_half2(b.x, b.y), pack_half2(b.z, b.w));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+// Copies `bytes` (multiple of 16) from global src to shared dst, lanes striding 16 B.
+__device__ __forceinline__ void warp_copy(uint32_t dst, const unsigned char* src, int bytes, int lane) {
+  for (int o = lane * 16; o < bytes; o += 32 * 16) cp_async16(dst + o, src + o);
+}
+
+template <int MK, int MV>
+__device__ __forceinline__ void issue_stage(uint32_t dst, const CacheView& kc, const CacheView& vc, int64_t seq,
+                                           int t0, int lane) {
+  const int64_t cap = kc.capacity;
+  const int64_t tok = seq * cap + t0;
+  const int64_t mrow = (seq * (cap / BLK) + t0 / BLK) * D;
+  warp_copy(dst + ST_KC, kc.codes + tok * NSUB, STAGE_TOK * 16, lane);
+  if constexpr (MK == NSN_MODE_2BIT) warp_copy(dst + ST_KS, kc.signs + tok * NSUB, STAGE_TOK * 16, lane);
+  warp_copy(dst + ST_KN, reinterpret_cast<const unsigned char*>(kc.norms + tok), STAGE_TOK * 4, lane);
+  warp_copy(dst + ST_VC, vc.codes + tok * NSUB, STAGE_TOK * 16, lane);
+  if constexpr (MV == NSN_MODE_2BIT) warp_copy(dst + ST_VS, vc.signs + tok * NSUB, STAGE_TOK * 16, lane);
+  warp_copy(dst + ST_VN, reinterpret_cast<const unsigned char*>(vc.norms + tok), STAGE_TOK * 4, lane);
+  warp_copy(dst + ST_KM, reinterpret_cast<const unsigned char*>(kc.means + mrow), D * 2, lane);
+  warp_copy(dst + ST_VM, reinterpret_cast<const unsigned char*>(vc.means + mrow), D * 2, lane);
+  cp_async_commit();
+}
+
 template <int G, int MK, int MV>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(32 * DEC_WARPS, 1)
 decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb, int64_t qsh,
-                    float qscale, const float* __restrict__ cbk, const float* __restrict__ cbv,
+                    float qscale, const float* __restrict__ cbk_g, const float* __restrict__ cbv_g,
                     float* __restrict__ ws, DecodeGeom geom) {
-  static_assert(2 * G <= 16, "reduction scratch holds 16 values");
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  using Smem = SplitSmem<G, MK, MV>;
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
-  const int64_t seq = (int64_t)b * kc.n_kv_heads + hk;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, p = lane & 3;
+
+  // ---- stage the replicated fp16 codebooks (whole CTA, once) ----
+  for (int e = tid; e < NCODES * 8; e += blockDim.x) {
+    const int c = e >> 3, r = e & 7;
+    sm.cbk[c][r] = cb_row_f16(cbk_g, c);
+    sm.cbv[c][r] = cb_row_f16(cbv_g, c);
+  }
+  __syncthreads();
+
+  const int nseq = kc.batch * kc.n_kv_heads;
+  const int gw = blockIdx.x * DEC_WARPS + warp;  // global split id
+  if (gw >= nseq * geom.nsplit_q) return;
+  const int64_t seq = gw / geom.nsplit_q;
+  const int split = gw % geom.nsplit_q;
+  const int b = (int)(seq / kc.n_kv_heads), hk = (int)(seq % kc.n_kv_heads);
   const int64_t pidx = seq * (geom.nsplit_q + 1) + split;
-  const int64_t P = (int64_t)kc.batch * kc.n_kv_heads * (geom.nsplit_q + 1);
+  const int64_t P = (int64_t)nseq * (geom.nsplit_q + 1);
   float* ws_acc = ws + acc_offset(P, G);
 
   const int nq = min(min(kc.n_quant[seq], vc.n_quant[seq]), kc.capacity);
-  const int start = split * geom.chunk;
-  const int end = min(start + geom.chunk, nq);
-  if (start >= end) {
-    for (int i = t; i < G * D; i += blockDim.x) ws_acc[pidx * G * D + i] = 0.f;
-    if (t < G) {
-      partial_ml(ws, pidx, G, t)[0] = NEG_BIG;
-      partial_ml(ws, pidx, G, t)[1] = 0.f;
+  const int nblk = (nq + BLK - 1) / BLK;
+  const int bps = (nblk + geom.nsplit_q - 1) / geom.nsplit_q;  // blocks per split
+  const int tok_begin = split * bps * BLK;
+  const int tok_end = min(nq, (split + 1) * bps * BLK);
+  if (tok_begin >= tok_end) {
+    for (int i = lane; i < G * D; i += 32) ws_acc[pidx * G * D + i] = 0.f;
+    if (lane < G) {
+      partial_ml(ws, pidx, G, lane)[0] = NEG_BIG;
+      partial_ml(ws, pidx, G, lane)[1] = 0.f;
     }
     return;
   }
+  const int nstages = (tok_end - tok_begin + STAGE_TOK - 1) / STAGE_TOK;
+  const uint32_t st_base = smem_addr(&sm.stage[warp][0][0]);
 
-  load_queries<G>(&sm.qt[0][0], q, dtype, qsb, qsh, b, hk, qscale, true);
-  for (int i = t; i < NCODES * SUB; i += blockDim.x) {
-    sm.cbv[i] = f16r(__ldg(cbv + i));
-    if constexpr (MK == NSN_MODE_2BIT) sm.cbk[i] = f16r(__ldg(cbk + i));
-  }
-  __syncthreads();
-  if constexpr (MK == NSN_MODE_1BIT) {
-    for (int e = t; e < NSUB * NCODES; e += blockDim.x) {
-      const int s = e / NCODES, k = e % NCODES;
-      float c[SUB];
-#pragma unroll
-      for (int i = 0; i < SUB; ++i) c[i] = f16r(__ldg(cbk + k * SUB + i));
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < SUB; ++i) acc = fmaf(sm.qt[h][SUB * s + i], c[i], acc);
-        sm.lut[e * G + h] = acc;
-      }
-    }
-    __syncthreads();
-  }
+  // prologue: two stages in flight
+  issue_stage<MK, MV>(st_base, kc, vc, seq, tok_begin, lane);
+  if (nstages > 1) issue_stage<MK, MV>(st_base + STAGE_BYTES, kc, vc, seq, tok_begin + STAGE_TOK, lane);
+  else cp_async_commit();
 
-  const int64_t cap = kc.capacity;
-  const int64_t nblk_cap = cap / BLK;
-  const uint4* kcodes = reinterpret_cast<const uint4*>(kc.codes) + seq * cap;
-  const uint4* ksigns = MK == NSN_MODE_2BIT ? reinterpret_cast<const uint4*>(kc.signs) + seq * cap : nullptr;
-  const __half2* knorm = kc.norms + seq * cap;
-  const __half* kmean = kc.means + seq * nblk_cap * D;
-  const uint4* vcodes = reinterpret_cast<const uint4*>(vc.codes) + seq * cap;
-  const uint4* vsigns = MV == NSN_MODE_2BIT ? reinterpret_cast<const uint4*>(vc.signs) + seq * cap : nullptr;
-  const __half2* vnorm = vc.norms + seq * cap;
-  const __half* vmean = vc.means + seq * nblk_cap * D;
-
-  float m_run[G], l_run[G], accm[G], acc[G][SUB];
+  // ---- rotated query fragments (built in registers while the copies fly) ----
+  // A row g = fp16(q~_g), row g + 8 = fp16(q~_g - fp16(q~_g)).
+  uint32_t qa[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) qa[j][0] = qa[j][1] = qa[j][2] = qa[j][3] = 0u;
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    m_run[h] = NEG_BIG;
-    l_run[h] = 0.f;
-    accm[h] = 0.f;
-#pragma unroll
-    for (int i = 0; i < SUB; ++i) acc[h][i] = 0.f;
-  }
-  const int my_s = t % NSUB, my_tg = t / NSUB;
-
-  for (int tile0 = start; tile0 < end; tile0 += BLK) {
-    const int tok = tile0 + t;
-    const bool valid = tok < end;
-    const int blk = tile0 / BLK;
-    const float oK = __half2float(kmean[(int64_t)blk * D + t]);
-    const float oV = __half2float(vmean[(int64_t)blk * D + t]);
-
-    uint4 kcw = make_uint4(0, 0, 0, 0), ksw = make_uint4(0, 0, 0, 0), vcw = make_uint4(0, 0, 0, 0),
-          vsw = make_uint4(0, 0, 0, 0);
-    float2 kn = make_float2(0.f, 0.f), vn = make_float2(0.f, 0.f);
-    if (valid) {
-      kcw = kcodes[tok];
-      if constexpr (MK == NSN_MODE_2BIT) ksw = ksigns[tok];
-      kn = __half22float2(knorm[tok]);
-      vcw = vcodes[tok];
-      if constexpr (MV == NSN_MODE_2BIT) vsw = vsigns[tok];
-      vn = __half22float2(vnorm[tok]);
-    }
-    sm.vcode[t] = vcw;
-    sm.vsign[t] = vsw;
-
-    // (Hq) . o_b for the K block of this tile
-    float qo[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) qo[h] = sm.qt[h][t] * oK;
-    block_reduce<G, false>(qo, sm.red);
-
-    // q~ . u_hat from the codes
-    float dot[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) dot[h] = 0.f;
-    const uint32_t kcs[4] = {kcw.x, kcw.y, kcw.z, kcw.w};
-    const uint32_t kss[4] = {ksw.x, ksw.y, ksw.z, ksw.w};
-#pragma unroll
-    for (int s = 0; s < NSUB; ++s) {
-      const int code = (kcs[s >> 2] >> (8 * (s & 3))) & 0xff;
-      if constexpr (MK == NSN_MODE_1BIT) {
-        const float* e = &sm.lut[(s * NCODES + code) * G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) dot[h] += e[h];
+    const int64_t off = (int64_t)b * qsb + (int64_t)(hk * G + h) * qsh + 4 * lane;
+    float v[4];
+    if (dtype == NSN_DTYPE_F32) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(q) + off));
+      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    } else {
+      const uint2 r = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(q) + off));
+      float2 a, c;
+      if (dtype == NSN_DTYPE_BF16) {
+        a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+        c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
       } else {
-        const uint32_t sb = (kss[s >> 2] >> (8 * (s & 3))) & 0xff;
-        const float4 c0 = *reinterpret_cast<const float4*>(&sm.cbk[code * SUB]);
-        const float4 c1 = *reinterpret_cast<const float4*>(&sm.cbk[code * SUB + 4]);
-        float cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        a = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
+        c = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
+      }
+      v[0] = a.x; v[1] = a.y; v[2] = c.x; v[3] = c.y;
+    }
+    fwht128_warp(v, lane);
 #pragma unroll
-        for (int i = 0; i < SUB; ++i) cw[i] = ((sb >> i) & 1) ? -cw[i] : cw[i];
+    for (int i = 0; i < 4; ++i) v[i] *= qscale * INV_SQRT_D;
+    // element c lives in lane c/4, slot c%4; lane (g, p) needs c = 16j + 8hf + 2p, +1
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+    for (int j = 0; j < 8; ++j) {
 #pragma unroll
-          for (int i = 0; i < SUB; ++i) dot[h] = fmaf(sm.qt[h][SUB * s + i], cw[i], dot[h]);
+      for (int hf = 0; hf < 2; ++hf) {
+        const int src = 4 * j + 2 * hf + (p >> 1);
+        const float e0 = __shfl_sync(0xffffffffu, v[0], src), e2 = __shfl_sync(0xffffffffu, v[2], src);
+        const float e1 = __shfl_sync(0xffffffffu, v[1], src), e3 = __shfl_sync(0xffffffffu, v[3], src);
+        const float x0 = (p & 1) ? e2 : e0, x1 = (p & 1) ? e3 : e1;
+        if (g == h) {
+          const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+          qa[j][2 * hf] = pack_half2(__half2float(h0), __half2float(h1));
+          qa[j][2 * hf + 1] = pack_half2(x0 - __half2float(h0), x1 - __half2float(h1));
         }
       }
     }
-    float sc[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) sc[h] = valid ? kn.x * fmaf(kn.y, dot[h], qo[h]) : NEG_BIG;
+  }
 
-    // online softmax
-    float tmax[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) tmax[h] = sc[h];
-    block_reduce<G, true>(tmax, sm.red);
-    float corr[G], sums[2 * G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float mn = fmaxf(m_run[h], tmax[h]);
-      corr[h] = exp2f(m_run[h] - mn);
-      m_run[h] = mn;
-      const float p = valid ? exp2f(sc[h] - mn) : 0.f;
-      sm.w[t][h] = p * vn.x * vn.y;
-      sums[h] = p;
-      sums[G + h] = p * vn.x;
-    }
-    block_reduce<2 * G, false>(sums, sm.red);  // also publishes sm.w / vcode / vsign
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      l_run[h] = fmaf(l_run[h], corr[h], sums[h]);
-      accm[h] = fmaf(accm[h], corr[h], sums[G + h] * oV);
-#pragma unroll
-      for (int i = 0; i < SUB; ++i) acc[h][i] *= corr[h];
-    }
+  const uint32_t lane_row = (uint32_t)(lane & 7) * 16u;
+  const uint32_t cbk_base = smem_addr(&sm.cbk[0][0]) + lane_row;
+  const uint32_t cbv_base = smem_addr(&sm.cbv[0][0]) + lane_row;
+  const uint32_t sel_k = 0x4440u | (uint32_t)(lane >> 3);
+  const uint32_t sel_v0 = 0x4440u | (uint32_t)((lane >> 3) & 1);
+  const uint32_t sel_v1 = 0x4440u | (uint32_t)(2 + ((lane >> 3) & 1));
 
-    // value accumulation in the rotated domain: thread (s, tg) takes tokens tg, tg+8, ...
-    const int nvalid = min(BLK, end - tile0);
-    for (int tt = my_tg; tt < nvalid; tt += 8) {
-      const uint4 cw4 = sm.vcode[tt];
-      const uint32_t cws[4] = {cw4.x, cw4.y, cw4.z, cw4.w};
-      const int code = (cws[my_s >> 2] >> (8 * (my_s & 3))) & 0xff;
-      const float4 c0 = *reinterpret_cast<const float4*>(&sm.cbv[code * SUB]);
-      const float4 c1 = *reinterpret_cast<const float4*>(&sm.cbv[code * SUB + 4]);
-      float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  float m = NEG_BIG, l = 0.f;
+  float O[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
+
+  for (int st = 0; st < nstages; ++st) {
+    cp_async_wait<1>();
+    __syncwarp();
+    const int t_stage = tok_begin + st * STAGE_TOK;
+    const unsigned char* sb = &sm.stage[warp][st & 1][0];
+    const uint32_t sba = st_base + (uint32_t)((st & 1) * STAGE_BYTES);
+
+    // (H q) . o_K of this stage's block, for head g (the mean row as all 8 "tokens")
+    float qo;
+    {
+      float d4[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t mrow = sba + ST_KM + (uint32_t)(lane >> 3) * 16u;
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        uint32_t bb[4];
+        ldsm_x4(mrow + 64u * qq, bb);
+        mma_full(d4, qa[2 * qq], bb[0], bb[1]);
+        mma_full(d4, qa[2 * qq + 1], bb[2], bb[3]);
+      }
+      qo = d4[0] + d4[2];
+    }
+    float cmean = 0.f;
+    const int ntile = min(STAGE_TOK, tok_end - t_stage + 15) >> 4;
+    const bool full = t_stage + STAGE_TOK <= tok_end;  // every token of the stage is valid
+    for (int tile = 0; tile < ntile; ++tile) {
+      const int tt = 16 * tile;  // token offset inside the stage
+      const uint4 kc0 = *reinterpret_cast<const uint4*>(sb + ST_KC + (tt + (lane & 7)) * 16);
+      const uint4 kc1 = *reinterpret_cast<const uint4*>(sb + ST_KC + (tt + 8 + (lane & 7)) * 16);
+      uint32_t ks0 = 0u, ks1 = 0u;
+      if constexpr (MK == NSN_MODE_2BIT) {
+        ks0 = *reinterpret_cast<const uint32_t*>(sb + ST_KS + (tt + g) * 16 + 4 * p);
+        ks1 = *reinterpret_cast<const uint32_t*>(sb + ST_KS + (tt + 8 + g) * 16 + 4 * p);
+      }
+      const uint2 kn0 = *reinterpret_cast<const uint2*>(sb + ST_KN + (tt + 2 * p) * 4);
+      const uint2 kn1 = *reinterpret_cast<const uint2*>(sb + ST_KN + (tt + 8 + 2 * p) * 4);
+      const uint4 vcw = *reinterpret_cast<const uint4*>(sb + ST_VC + (tt + (lane & 7) + 8 * (lane >> 4)) * 16);
+      uint32_t W0 = 0u, W1 = 0u;
       if constexpr (MV == NSN_MODE_2BIT) {
-        const uint4 sw4 = sm.vsign[tt];
-        const uint32_t sws[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
-        const uint32_t sb = (sws[my_s >> 2] >> (8 * (my_s & 3))) & 0xff;
-#pragma unroll
-        for (int i = 0; i < SUB; ++i) cv[i] = ((sb >> i) & 1) ? -cv[i] : cv[i];
+        const uint16_t* vs = reinterpret_cast<const uint16_t*>(sb + ST_VS);
+        W0 = (uint32_t)vs[(tt + 2 * p) * 8 + g] | ((uint32_t)vs[(tt + 2 * p + 1) * 8 + g] << 16);
+        W1 = (uint32_t)vs[(tt + 8 + 2 * p) * 8 + g] | ((uint32_t)vs[(tt + 9 + 2 * p) * 8 + g] << 16);
       }
+      const uint2 vn0 = *reinterpret_cast<const uint2*>(sb + ST_VN + (tt + 2 * p) * 4);
+      const uint2 vn1 = *reinterpret_cast<const uint2*>(sb + ST_VN + (tt + 8 + 2 * p) * 4);
+
+      // ---- scores S^T = q~ u_hat^T for the two 8-token groups ----
+      float S[2][2];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float wt = sm.w[tt][h];
+      for (int grp = 0; grp < 2; ++grp) {
+        const uint4 kcw = grp ? kc1 : kc0;
+        const uint32_t ksw = grp ? ks1 : ks0;
+        float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < SUB; ++i) acc[h][i] = fmaf(wt, cv[i], acc[h][i]);
+        for (int qq = 0; qq < 4; ++qq) {
+          const uint32_t code = __byte_perm(u4_word(kcw, qq), 0u, sel_k);
+          uint32_t bb[4];
+          ldsm_x4(cbk_base + code * 128u, bb);
+          if constexpr (MK == NSN_MODE_2BIT) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) bb[i] = apply_signs(bb[i], ksw, 4 * qq + i);
+          }
+          mma_full(Sa, qa[2 * qq], bb[0], bb[1]);
+          mma_full(Sb, qa[2 * qq + 1], bb[2], bb[3]);
+        }
+        S[grp][0] = (Sa[0] + Sa[2]) + (Sb[0] + Sb[2]);  // rows g and g + 8
+        S[grp][1] = (Sa[1] + Sa[3]) + (Sb[1] + Sb[3]);
+      }
+
+      // ---- scores with the NSN byproducts, online softmax (head g) ----
+      const __half2* kh0 = reinterpret_cast<const __half2*>(&kn0);
+      const __half2* kh1 = reinterpret_cast<const __half2*>(&kn1);
+      const __half2* vh0 = reinterpret_cast<const __half2*>(&vn0);
+      const __half2* vh1 = reinterpret_cast<const __half2*>(&vn1);
+      const float2 kn[4] = {__half22float2(kh0[0]), __half22float2(kh0[1]), __half22float2(kh1[0]),
+                            __half22float2(kh1[1])};
+      const float2 vn[4] = {__half22float2(vh0[0]), __half22float2(vh0[1]), __half22float2(vh1[0]),
+                            __half22float2(vh1[1])};
+      const float dk[4] = {S[0][0], S[0][1], S[1][0], S[1][1]};  // tokens 2p, 2p+1, 8+2p, 9+2p
+      const int tk[4] = {tt + 2 * p, tt + 2 * p + 1, tt + 8 + 2 * p, tt + 9 + 2 * p};
+      float sc[4];
+      float tmax = NEG_BIG;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool ok = (g < G) && (full || t_stage + tk[i] < tok_end);
+        sc[i] = ok ? kn[i].x * fmaf(kn[i].y, dk[i], qo) : NEG_BIG;
+        tmax = fmaxf(tmax, sc[i]);
+      }
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+      const float mnew = fmaxf(m, tmax);
+      if (__any_sync(0xffffffffu, mnew > m)) {
+        const float corr = fast_exp2(m - mnew);
+        const float ca = __shfl_sync(0xffffffffu, corr, 8 * p);
+        const float cb = __shfl_sync(0xffffffffu, corr, 8 * p + 4);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          O[i][0] *= ca; O[i][1] *= cb; O[i][2] *= ca; O[i][3] *= cb;
+        }
+        l *= corr;
+        cmean *= corr;
+        m = mnew;
+      }
+      float w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float pr = (g < G) ? fast_exp2(sc[i] - m) : 0.f;
+        l += pr;
+        cmean = fmaf(pr, vn[i].x, cmean);
+        w[i] = pr * vn[i].x * vn[i].y;
+      }
+      const uint32_t pb0 = pack_half2(w[0], w[1]);
+      const uint32_t pb1 = pack_half2(w[2], w[3]);
+
+      // ---- values: O^T += u_hat_v^T w ----
+#pragma unroll
+      for (int mm = 0; mm < 8; ++mm) {
+        const uint32_t code = __byte_perm(u4_word(vcw, mm >> 1), 0u, (mm & 1) ? sel_v1 : sel_v0);
+        uint32_t aa[4];
+        ldsm_x4_t(cbv_base + code * 128u, aa);
+        if constexpr (MV == NSN_MODE_2BIT) {
+          aa[0] = apply_signs(aa[0], W0, 2 * mm);
+          aa[1] = apply_signs(aa[1], W0, 2 * mm + 1);
+          aa[2] = apply_signs(aa[2], W1, 2 * mm);
+          aa[3] = apply_signs(aa[3], W1, 2 * mm + 1);
+        }
+        mma_full(O[mm], aa, pb0, pb1);
       }
     }
-    __syncthreads();  // w / vcode / vsign are rewritten by the next tile
-  }
 
-  // reduce the 8 token groups; thread t owns rotated dim t
+    // ---- block mean of V for this stage's tokens: O^T[d][h] += o_V[d] * sum_t p_t s1_t ----
+    cmean += __shfl_xor_sync(0xffffffffu, cmean, 1);
+    cmean += __shfl_xor_sync(0xffffffffu, cmean, 2);
+    {
+      const float ca = __shfl_sync(0xffffffffu, cmean, 8 * p);
+      const float cb = __shfl_sync(0xffffffffu, cmean, 8 * p + 4);
+      const __half* ov = reinterpret_cast<const __half*>(sb + ST_VM);
 #pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int i = 0; i < SUB; ++i) sm.racc[my_tg][h][my_s * SUB + i] = acc[h][i];
-  __syncthreads();
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float s = accm[h];
-#pragma unroll
-    for (int g2 = 0; g2 < 8; ++g2) s += sm.racc[g2][h][t];
-    ws_acc[(pidx * G + h) * D + t] = s;
+      for (int mm = 0; mm < 8; ++mm) {
+        const float oa = __half2float(ov[16 * mm + g]);
+        const float ob = __half2float(ov[16 * mm + 8 + g]);
+        O[mm][0] = fmaf(oa, ca, O[mm][0]);
+        O[mm][1] = fmaf(oa, cb, O[mm][1]);
+        O[mm][2] = fmaf(ob, ca, O[mm][2]);
+        O[mm][3] = fmaf(ob, cb, O[mm][3]);
+      }
+    }
+    __syncwarp();  // every lane is done with this stage buffer
+    if (st + 2 < nstages) issue_stage<MK, MV>(sba, kc, vc, seq, t_stage + 2 * STAGE_TOK, lane);
+    else cp_async_commit();  // keep the group count uniform for wait_group
   }
-  if (t < G) {
-    partial_ml(ws, pidx, G, t)[0] = m_run[t];
-    partial_ml(ws, pidx, G, t)[1] = l_run[t];
+  cp_async_wait<0>();
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
+
+  // ---- this warp's partial ----
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = 2 * p + hh;
+    if (h < G) {
+      float* dst = ws_acc + (pidx * G + h) * D;
+#pragma unroll
+      for (int mm = 0; mm < 8; ++mm) {
+        dst[16 * mm + g] = O[mm][hh];
+        dst[16 * mm + 8 + g] = O[mm][2 + hh];
+      }
+    }
+  }
+  if (p == 0 && g < G) {
+    partial_ml(ws, pidx, G, g)[0] = m;
+    partial_ml(ws, pidx, G, g)[1] = l;
   }
 }
 
@@ -431,11 +615,30 @@ decode_combine_kernel(const float* __restrict__ ws, float* __restrict__ out, int
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-DecodeGeom decode_geometry(int capacity, int n_q_heads, int n_kv_heads) {
+static int sm_count() {
+  static int cached = 0;
+  if (cached == 0) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+      cached = n;
+    else
+      cached = 148;
+  }
+  return cached;
+}
+
+DecodeGeom decode_geometry(int batch, int capacity, int n_q_heads, int n_kv_heads) {
   DecodeGeom g;
   g.g = n_q_heads / n_kv_heads;
-  g.chunk = capacity < 1024 ? capacity : 1024;
-  g.nsplit_q = (capacity + g.chunk - 1) / g.chunk;
+  g.chunk = 0;
+  // splits per sequence: fill one 16-warp CTA per SM, at most one split per block
+  const int nseq = batch * n_kv_heads;
+  const int warps = sm_count() * DEC_WARPS;
+  int sp = warps / (nseq > 0 ? nseq : 1);
+  const int maxsp = capacity / BLK;
+  if (sp > maxsp) sp = maxsp;
+  if (sp < 1) sp = 1;
+  g.nsplit_q = sp;
   return g;
 }
 
@@ -448,12 +651,13 @@ template <int G, int MK, int MV>
 static cudaError_t launch_split_t(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int64_t qsb,
                                   int64_t qsh, float qscale, const float* cbk, const float* cbv, float* ws,
                                   const DecodeGeom& geom, cudaStream_t s) {
-  const size_t smem = sizeof(SplitSmem<G, MK, MV>);
+  const size_t smem = sizeof(DecSmem);
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<G, MK, MV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(geom.nsplit_q, kc.n_kv_heads, kc.batch);
-  decode_split_kernel<G, MK, MV><<<grid, 128, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, ws, geom);
+  const int nwarps = kc.batch * kc.n_kv_heads * geom.nsplit_q;
+  dim3 grid((nwarps + DEC_WARPS - 1) / DEC_WARPS);
+  decode_split_kernel<G, MK, MV><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, ws, geom);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2(kc.n_kv_heads, kc.batch);

@@ -143,7 +143,7 @@ nsn_status nsn_append_residual(nsn_cache* k_cache, nsn_cache* v_cache, const voi
 
 size_t nsn_decode_workspace_bytes(const nsn_cache* k_cache, int n_q_heads) {
   if (check_cache(k_cache) != NSN_OK || n_q_heads <= 0 || n_q_heads % k_cache->n_kv_heads) return 0;
-  const nsn::DecodeGeom g = nsn::decode_geometry(k_cache->capacity, n_q_heads, k_cache->n_kv_heads);
+  const nsn::DecodeGeom g = nsn::decode_geometry(k_cache->batch, k_cache->capacity, n_q_heads, k_cache->n_kv_heads);
   return nsn::decode_workspace_bytes(k_cache->batch, k_cache->n_kv_heads, g);
 }
 
@@ -165,7 +165,7 @@ nsn_status nsn_decode_attention(const nsn_cache* k_cache, const nsn_cache* v_cac
   const int64_t e16 = elems16(dtype);
   if (q_stride_b < 0 || q_stride_h < 0 || q_stride_b % e16 || q_stride_h % e16) return NSN_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return NSN_ERR_INVALID_ARG;
-  const nsn::DecodeGeom geom = nsn::decode_geometry(k_cache->capacity, n_q_heads, k_cache->n_kv_heads);
+  const nsn::DecodeGeom geom = nsn::decode_geometry(k_cache->batch, k_cache->capacity, n_q_heads, k_cache->n_kv_heads);
   if (ws_bytes < nsn::decode_workspace_bytes(k_cache->batch, k_cache->n_kv_heads, geom)) return NSN_ERR_WORKSPACE;
   return cuda_status(nsn::launch_decode(view(k_cache), view(v_cache), q, dtype, n_q_heads, q_stride_b, q_stride_h,
                                         softmax_scale, cb_k, cb_v, out, workspace, geom,

@@ -21,15 +21,16 @@ struct CacheView {
   int32_t* status;
 };
 
-// Decode split geometry: the quantized range of every (b, kv-head) is cut into
-// chunks of `chunk` tokens; one more partial slot holds the residual window.
+// Decode split geometry: the quantized blocks of every (b, kv-head) are dealt
+// out to nsplit_q warps in contiguous ranges; one more partial slot holds the
+// residual window.
 struct DecodeGeom {
-  int chunk;         // tokens per split (multiple of 128)
-  int nsplit_q;      // splits over the quantized part
+  int chunk;         // unused (kept 0)
+  int nsplit_q;      // splits per sequence over the quantized part (blocks are dealt out evenly)
   int g;             // query heads per kv-head
 };
 
-DecodeGeom decode_geometry(int capacity, int n_q_heads, int n_kv_heads);
+DecodeGeom decode_geometry(int batch, int capacity, int n_q_heads, int n_kv_heads);
 size_t decode_workspace_bytes(int batch, int n_kv_heads, const DecodeGeom& geom);
 
 size_t quant_smem_bytes();

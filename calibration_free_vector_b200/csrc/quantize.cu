@@ -251,11 +251,15 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   // ---- sign bits (2-bit) and search operand a = |u| or u ---------------------
   // In 2-bit mode v is replaced by |u| after the sign bits are taken; every later
   // use only needs |u| (u_c * u_hat_c = |u_c| * A_code,c because the signs match).
+  // Sign-bit layout (see include/nsn.h): 16-bit field i (i = dim within the
+  // sub-vector) holds the sign of u[8s + i] at bit 15 - s; fields 2j, 2j+1 form
+  // 32-bit word j (bit 15 - s and bit 31 - s).
   uint32_t sgn[4] = {0u, 0u, 0u, 0u};
   if constexpr (MODE == NSN_MODE_2BIT) {
 #pragma unroll
     for (int c = 0; c < D; ++c) {
-      sgn[c >> 5] |= (v[c] < 0.f ? 1u : 0u) << (c & 31);
+      const int s = c >> 3, i = c & 7;
+      sgn[i >> 1] |= (v[c] < 0.f ? 1u : 0u) << (16 * (i & 1) + 15 - s);
       v[c] = fabsf(v[c]);
     }
   }

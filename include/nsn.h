@@ -70,8 +70,11 @@ typedef enum { NSN_DTYPE_F32 = 0, NSN_DTYPE_BF16 = 1, NSN_DTYPE_F16 = 2 } nsn_dt
  * Compressed cache of one tensor (K or V) of one layer.  All pointers are
  * device pointers owned by the caller.  Layout (row-major, per (b, h) contiguous):
  *   codes    uint8  [batch][n_kv_heads][capacity][16]   code of sub-vector s at byte s
- *   signs    uint8  [batch][n_kv_heads][capacity][16]   2-bit mode only (NULL in 1-bit):
- *                                                       byte s, bit i = sign of u[8s+i]
+ *   signs    uint8  [batch][n_kv_heads][capacity][16]   2-bit mode only (NULL in 1-bit): the
+ *                                                       128 sign bits of a token as eight
+ *                                                       little-endian 16-bit fields; field i
+ *                                                       (bytes 2i, 2i+1) bit 15-s is set iff
+ *                                                       u[8s+i] < 0 (s = sub-vector 0..15)
  *   norms    fp16   [batch][n_kv_heads][capacity][2]    (s1, alpha*s2) per token
  *   means    fp16   [batch][n_kv_heads][capacity/128][128]   o of each block (rotated domain)
  *   window   fp16   [batch][n_kv_heads][window][128]    residual tokens, original domain

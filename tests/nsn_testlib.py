@@ -30,6 +30,34 @@ def codebook(mode: int) -> np.ndarray:
     return np.loadtxt(os.path.join(GOLDEN, name)).astype(np.float32)
 
 
+def signs_to_natural(stored: np.ndarray) -> np.ndarray:
+    """Stored sign bytes [..., 16] (eight 16-bit fields; field i bit 15-s = sign of
+    dim 8s+i) -> the oracle's layout [..., 16] (byte s bit i = sign of dim 8s+i)."""
+    stored = np.asarray(stored, dtype=np.uint8)
+    fields = stored.reshape(stored.shape[:-1] + (8, 2)).astype(np.uint32)
+    fields = fields[..., 0] | (fields[..., 1] << 8)                     # [..., 8] field i
+    out = np.zeros(stored.shape, dtype=np.uint8)
+    for s in range(16):
+        for i in range(8):
+            bit = (fields[..., i] >> (15 - s)) & 1
+            out[..., s] |= (bit << i).astype(np.uint8)
+    return out
+
+
+def natural_to_signs(natural: np.ndarray) -> np.ndarray:
+    """Inverse of signs_to_natural."""
+    natural = np.asarray(natural, dtype=np.uint8)
+    fields = np.zeros(natural.shape[:-1] + (8,), dtype=np.uint32)
+    for s in range(16):
+        for i in range(8):
+            bit = (natural[..., s].astype(np.uint32) >> i) & 1
+            fields[..., i] |= bit << (15 - s)
+    out = np.zeros(natural.shape, dtype=np.uint8)
+    out[..., 0::2] = (fields & 0xFF).astype(np.uint8)
+    out[..., 1::2] = (fields >> 8).astype(np.uint8)
+    return out
+
+
 def read_cache(cache, b: int, h: int) -> dict:
     """Stored contents of one (b, h) sequence of an nsn.Cache as numpy (oracle layout)."""
     nq = int(cache.n_quant[b, h].item())
@@ -38,7 +66,7 @@ def read_cache(cache, b: int, h: int) -> dict:
         "n_quant": nq,
         "n_window": nw,
         "codes": cache.codes[b, h, :nq].cpu().numpy().astype(np.int64),
-        "signs": None if cache.signs is None else cache.signs[b, h, :nq].cpu().numpy(),
+        "signs": None if cache.signs is None else signs_to_natural(cache.signs[b, h, :nq].cpu().numpy()),
         "s1": cache.norms[b, h, :nq, 0].float().cpu().numpy().astype(np.float64),
         "s2": cache.norms[b, h, :nq, 1].float().cpu().numpy().astype(np.float64),
         "o": cache.means[b, h, :(nq + 127) // 128].float().cpu().numpy().astype(np.float64),

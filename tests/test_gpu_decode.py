@@ -33,8 +33,10 @@ def fill_cache(cache, contents):
 
 
 def oracle_seq(c):
+    """The same random contents in the oracle's layout (sign bits reordered)."""
     f = lambda a: None if a is None else np.asarray(a, dtype=np.float64)  # noqa: E731
-    return {"codes": c["codes"].astype(np.int64), "signs": c["signs"], "s1": f(c["s1"]), "s2": f(c["s2"]),
+    signs = None if c["signs"] is None else tl.signs_to_natural(c["signs"])
+    return {"codes": c["codes"].astype(np.int64), "signs": signs, "s1": f(c["s1"]), "s2": f(c["s2"]),
             "o": f(c["o"])}
 
 

@@ -101,3 +101,16 @@ def test_f16_rounding_is_round_to_nearest_even():
     assert orc.to_f16(1.0 + 3 * 2.0 ** -11)[()] == 1.0 + 2.0 ** -9
     with np.errstate(over="ignore"):
         assert orc.to_f16(65520.0)[()] == np.inf
+
+
+def test_sign_layout_conversion_roundtrip():
+    import nsn_testlib as tl
+    rng = np.random.default_rng(15)
+    nat = rng.integers(0, 256, size=(50, 16)).astype(np.uint8)
+    stored = tl.natural_to_signs(nat)
+    assert np.array_equal(tl.signs_to_natural(stored), nat)
+    # single bit: dim 8*3 + 5 (sub 3, i 5) -> field 5 (bytes 10, 11), bit 15 - 3 = 12 -> byte 11 bit 4
+    one = np.zeros((1, 16), np.uint8)
+    one[0, 3] = 1 << 5
+    st = tl.natural_to_signs(one)
+    assert st[0, 11] == 1 << 4 and st.sum() == 16
