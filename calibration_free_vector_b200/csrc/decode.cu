@@ -12,12 +12,13 @@
 // Residual-window tokens are attended in the original domain.
 //
 // Kernels:
-//   decode_split_kernel     one CTA per (split of the quantized range, kv-head, batch):
-//                           rotated query, scores from the codes, online softmax,
-//                           value accumulation from the codewords -> partial (m, l, acc)
-//   decode_window_kernel    one CTA per (kv-head, batch): the residual window -> partial
-//   decode_combine_kernel   one warp per (q-head, batch): log-sum-exp merge of the
-//                           partials, H applied to the rotated sum, normalisation.
+//   decode_split_kernel           one warp per split (a contiguous range of 128-token
+//                                 blocks of one (batch, kv-head)): rotated query, scores
+//                                 from the codes, online softmax, value accumulation
+//                                 from the codewords -> partial (m, l, acc)
+//   decode_window_combine_kernel  one warp per query head: residual window attention
+//                                 (original domain), log-sum-exp merge with the split
+//                                 partials, H applied to their rotated value sum.
 // Scores are carried in log2 units (the query is pre-scaled by softmax_scale*log2 e).
 
 #include "nsn_common.cuh"
@@ -27,66 +28,6 @@ namespace nsn {
 
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float INV_SQRT_D = 0.08838834764831845f;  // 1/sqrt(128)
-
-__device__ __forceinline__ void load8_rt(const void* base, int64_t off, int dtype, float* out) {
-  if (dtype == NSN_DTYPE_F32) load8<NSN_DTYPE_F32>(base, off, out);
-  else if (dtype == NSN_DTYPE_BF16) load8<NSN_DTYPE_BF16>(base, off, out);
-  else load8<NSN_DTYPE_F16>(base, off, out);
-}
-
-__device__ __forceinline__ float f16r(float x) { return __half2float(__float2half_rn(x)); }
-
-// Block-wide reduction of N values per thread (128 threads): op = sum or max.
-template <int N, bool IS_MAX>
-__device__ __forceinline__ void block_reduce(float* vals, float (*red)[16]) {
-  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    float x = vals[i];
-    x = IS_MAX ? warp_max(x) : warp_sum(x);
-    if (lane == 0) red[w][i] = x;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    float a = red[0][i], b = red[1][i], c = red[2][i], d = red[3][i];
-    vals[i] = IS_MAX ? fmaxf(fmaxf(a, b), fmaxf(c, d)) : (a + b) + (c + d);
-  }
-  __syncthreads();
-}
-
-// Loads the g query rows of kv-head hk, rotates them (H q = FWHT(q)/sqrt(128))
-// when `rotate`, scales by `scale` and stores [g][128] fp32 to qt.
-template <int G>
-__device__ void load_queries(float* qt, const void* q, int dtype, int64_t qsb, int64_t qsh, int b, int hk,
-                             float scale, bool rotate) {
-  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-  for (int h = w; h < G; h += 4) {
-    const int64_t off = (int64_t)b * qsb + (int64_t)(hk * G + h) * qsh + 4 * lane;
-    float v[4];
-    if (dtype == NSN_DTYPE_F32) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(q) + off));
-      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-    } else if (dtype == NSN_DTYPE_BF16) {
-      const uint2 r = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(q) + off));
-      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-      const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-      v[0] = a.x; v[1] = a.y; v[2] = c.x; v[3] = c.y;
-    } else {
-      const uint2 r = __ldg(reinterpret_cast<const uint2*>(static_cast<const __half*>(q) + off));
-      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
-      const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
-      v[0] = a.x; v[1] = a.y; v[2] = c.x; v[3] = c.y;
-    }
-    float sc = scale;
-    if (rotate) {
-      fwht128_warp(v, lane);
-      sc *= INV_SQRT_D;
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) qt[h * D + 4 * lane + i] = v[i] * sc;
-  }
-}
 
 // Workspace layout: [P][G][2] (m, l) floats, then -- from a 16-byte aligned
 // offset -- [P][G][128] accumulators; P = batch * kv-heads * (nsplit_q + 1).
@@ -171,14 +112,22 @@ __device__ __forceinline__ uint32_t u4_word(const uint4& v, int i) {
 // ---------------------------------------------------------------------------
 constexpr int DEC_WARPS = 16;
 constexpr int STAGE_TOK = 64;
-// stage layout (bytes): K codes | K signs | K norms | V codes | V signs | V norms | K mean | V mean
-constexpr int ST_KC = 0, ST_KS = 1024, ST_KN = 2048, ST_VC = 2304, ST_VS = 3328, ST_VN = 4352, ST_KM = 4608,
-              ST_VM = 4864, STAGE_BYTES = 5120;
+// stage layout (bytes): K codes | K signs | K norms | V codes | V signs | V norms
+constexpr int ST_KC = 0, ST_KS = 1024, ST_KN = 2048, ST_VC = 2304, ST_VS = 3328, ST_VN = 4352, STAGE_BYTES = 4608;
+constexpr int MEAN_BYTES = 512;  // K mean row | V mean row of one block (fp16)
+// The running max is re-based only when a score exceeds it by more than this
+// (log2 units): weights stay below 2^8 and exact in fp32, and most tiles skip the
+// max reduction.
+constexpr float LAZY_MAX_SLACK = 8.0f;
+// Upper bound on mbarrier polls before a wait gives up (error flag, no hang).
+constexpr uint32_t WAIT_LIMIT = 1u << 26;
 
 struct DecSmem {
   alignas(128) uint4 cbk[NCODES][8];  // replicated fp16 codebooks (32 KB each)
   alignas(128) uint4 cbv[NCODES][8];
   alignas(128) unsigned char stage[DEC_WARPS][2][STAGE_BYTES];
+  alignas(128) unsigned char means[DEC_WARPS][2][MEAN_BYTES];
+  alignas(8) uint64_t bar[DEC_WARPS][2];
 };
 
 __device__ __forceinline__ uint4 cb_row_f16(const float* __restrict__ cb, int c) {
@@ -187,33 +136,56 @@ __device__ __forceinline__ uint4 cb_row_f16(const float* __restrict__ cb, int c)
   return make_uint4(pack_half2(a.x, a.y), pack_half2(a.z, a.w), pack_half2(b.x, b.y), pack_half2(b.z, b.w));
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+// ---- mbarrier + 1-D bulk copy (TMA) helpers ----
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
-
-// Copies `bytes` (multiple of 16) from global src to shared dst, lanes striding 16 B.
-__device__ __forceinline__ void warp_copy(uint32_t dst, const unsigned char* src, int bytes, int lane) {
-  for (int o = lane * 16; o < bytes; o += 32 * 16) cp_async16(dst + o, src + o);
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// Bounded wait; false if the limit was reached.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (uint32_t i = 0; i < WAIT_LIMIT; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
 }
 
+// Lane 0 issues the bulk copies of one 64-token stage (+ the block's mean rows
+// when `with_means`) and arms the stage's barrier with the byte count.
 template <int MK, int MV>
-__device__ __forceinline__ void issue_stage(uint32_t dst, const CacheView& kc, const CacheView& vc, int64_t seq,
-                                           int t0, int lane) {
+__device__ __forceinline__ void issue_stage(uint32_t dst, uint32_t mdst, uint32_t bar, const CacheView& kc,
+                                           const CacheView& vc, int64_t seq, int t0, bool with_means) {
   const int64_t cap = kc.capacity;
   const int64_t tok = seq * cap + t0;
-  const int64_t mrow = (seq * (cap / BLK) + t0 / BLK) * D;
-  warp_copy(dst + ST_KC, kc.codes + tok * NSUB, STAGE_TOK * 16, lane);
-  if constexpr (MK == NSN_MODE_2BIT) warp_copy(dst + ST_KS, kc.signs + tok * NSUB, STAGE_TOK * 16, lane);
-  warp_copy(dst + ST_KN, reinterpret_cast<const unsigned char*>(kc.norms + tok), STAGE_TOK * 4, lane);
-  warp_copy(dst + ST_VC, vc.codes + tok * NSUB, STAGE_TOK * 16, lane);
-  if constexpr (MV == NSN_MODE_2BIT) warp_copy(dst + ST_VS, vc.signs + tok * NSUB, STAGE_TOK * 16, lane);
-  warp_copy(dst + ST_VN, reinterpret_cast<const unsigned char*>(vc.norms + tok), STAGE_TOK * 4, lane);
-  warp_copy(dst + ST_KM, reinterpret_cast<const unsigned char*>(kc.means + mrow), D * 2, lane);
-  warp_copy(dst + ST_VM, reinterpret_cast<const unsigned char*>(vc.means + mrow), D * 2, lane);
-  cp_async_commit();
+  constexpr uint32_t CB = STAGE_TOK * 16, NB = STAGE_TOK * 4;
+  const uint32_t bytes = CB * 2 + NB * 2 + (MK == NSN_MODE_2BIT ? CB : 0) + (MV == NSN_MODE_2BIT ? CB : 0) +
+                         (with_means ? MEAN_BYTES : 0);
+  mbar_expect_tx(bar, bytes);
+  bulk_g2s(dst + ST_KC, kc.codes + tok * NSUB, CB, bar);
+  if constexpr (MK == NSN_MODE_2BIT) bulk_g2s(dst + ST_KS, kc.signs + tok * NSUB, CB, bar);
+  bulk_g2s(dst + ST_KN, kc.norms + tok, NB, bar);
+  bulk_g2s(dst + ST_VC, vc.codes + tok * NSUB, CB, bar);
+  if constexpr (MV == NSN_MODE_2BIT) bulk_g2s(dst + ST_VS, vc.signs + tok * NSUB, CB, bar);
+  bulk_g2s(dst + ST_VN, vc.norms + tok, NB, bar);
+  if (with_means) {
+    const int64_t mrow = (seq * (cap / BLK) + t0 / BLK) * D;
+    bulk_g2s(mdst, kc.means + mrow, D * 2, bar);
+    bulk_g2s(mdst + D * 2, vc.means + mrow, D * 2, bar);
+  }
 }
 
 template <int G, int MK, int MV>
@@ -230,6 +202,11 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
     const int c = e >> 3, r = e & 7;
     sm.cbk[c][r] = cb_row_f16(cbk_g, c);
     sm.cbv[c][r] = cb_row_f16(cbv_g, c);
+  }
+  if (lane == 0) {
+    mbar_init(smem_addr(&sm.bar[warp][0]), 1);
+    mbar_init(smem_addr(&sm.bar[warp][1]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   __syncthreads();
 
@@ -258,11 +235,16 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
   }
   const int nstages = (tok_end - tok_begin + STAGE_TOK - 1) / STAGE_TOK;
   const uint32_t st_base = smem_addr(&sm.stage[warp][0][0]);
+  const uint32_t mb_base = smem_addr(&sm.means[warp][0][0]);
+  const uint32_t bar0 = smem_addr(&sm.bar[warp][0]);
 
-  // prologue: two stages in flight
-  issue_stage<MK, MV>(st_base, kc, vc, seq, tok_begin, lane);
-  if (nstages > 1) issue_stage<MK, MV>(st_base + STAGE_BYTES, kc, vc, seq, tok_begin + STAGE_TOK, lane);
-  else cp_async_commit();
+  // prologue: two stages in flight (stage s -> buffer s & 1; means buffer = block & 1)
+  if (lane == 0) {
+    issue_stage<MK, MV>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc, seq,
+                        tok_begin, true);
+    if (nstages > 1)
+      issue_stage<MK, MV>(st_base + STAGE_BYTES, mb_base, bar0 + 8, kc, vc, seq, tok_begin + STAGE_TOK, false);
+  }
 
   // ---- rotated query fragments (built in registers while the copies fly) ----
   // A row g = fp16(q~_g), row g + 8 = fp16(q~_g - fp16(q~_g)).
@@ -316,23 +298,32 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
   const uint32_t sel_v0 = 0x4440u | (uint32_t)((lane >> 3) & 1);
   const uint32_t sel_v1 = 0x4440u | (uint32_t)(2 + ((lane >> 3) & 1));
 
-  float m = NEG_BIG, l = 0.f;
+  float m = NEG_BIG, l = 0.f, cmean = 0.f, qo = 0.f;
   float O[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
+  uint32_t phase = 0u;  // bit k = parity of the next wait on buffer k
+  bool failed = false;
 
   for (int st = 0; st < nstages; ++st) {
-    cp_async_wait<1>();
-    __syncwarp();
+    const int buf = st & 1;
+    const bool arrived = mbar_wait(bar0 + 8u * buf, (phase >> buf) & 1u);
+    if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform decision
+      failed = true;
+      break;
+    }
+    phase ^= 1u << buf;
     const int t_stage = tok_begin + st * STAGE_TOK;
-    const unsigned char* sb = &sm.stage[warp][st & 1][0];
-    const uint32_t sba = st_base + (uint32_t)((st & 1) * STAGE_BYTES);
+    const bool block_start = (t_stage % BLK) == 0;
+    const bool block_end = ((t_stage + STAGE_TOK) % BLK) == 0 || st == nstages - 1;
+    const int mbuf = (t_stage / BLK) & 1;
+    const unsigned char* sb = &sm.stage[warp][buf][0];
+    const unsigned char* mb = &sm.means[warp][mbuf][0];
 
-    // (H q) . o_K of this stage's block, for head g (the mean row as all 8 "tokens")
-    float qo;
-    {
+    if (block_start) {
+      // (H q) . o_K of this block, for head g (the mean row as all 8 "tokens")
       float d4[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t mrow = sba + ST_KM + (uint32_t)(lane >> 3) * 16u;
+      const uint32_t mrow = mb_base + (uint32_t)(mbuf * MEAN_BYTES) + (uint32_t)(lane >> 3) * 16u;
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) {
         uint32_t bb[4];
@@ -342,7 +333,6 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
       }
       qo = d4[0] + d4[2];
     }
-    float cmean = 0.f;
     const int ntile = min(STAGE_TOK, tok_end - t_stage + 15) >> 4;
     const bool full = t_stage + STAGE_TOK <= tok_end;  // every token of the stage is valid
     for (int tile = 0; tile < ntile; ++tile) {
@@ -401,17 +391,18 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
       const float dk[4] = {S[0][0], S[0][1], S[1][0], S[1][1]};  // tokens 2p, 2p+1, 8+2p, 9+2p
       const int tk[4] = {tt + 2 * p, tt + 2 * p + 1, tt + 8 + 2 * p, tt + 9 + 2 * p};
       float sc[4];
-      float tmax = NEG_BIG;
+      float lmax = NEG_BIG;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const bool ok = (g < G) && (full || t_stage + tk[i] < tok_end);
         sc[i] = ok ? kn[i].x * fmaf(kn[i].y, dk[i], qo) : NEG_BIG;
-        tmax = fmaxf(tmax, sc[i]);
+        lmax = fmaxf(lmax, sc[i]);
       }
-      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
-      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-      const float mnew = fmaxf(m, tmax);
-      if (__any_sync(0xffffffffu, mnew > m)) {
+      // lazy re-basing of the running max (rare after the first tile)
+      if (__any_sync(0xffffffffu, lmax > m + LAZY_MAX_SLACK)) {
+        float tmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, 1));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+        const float mnew = fmaxf(m, tmax);
         const float corr = fast_exp2(m - mnew);
         const float ca = __shfl_sync(0xffffffffu, corr, 8 * p);
         const float cb = __shfl_sync(0xffffffffu, corr, 8 * p + 4);
@@ -450,13 +441,13 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
       }
     }
 
-    // ---- block mean of V for this stage's tokens: O^T[d][h] += o_V[d] * sum_t p_t s1_t ----
-    cmean += __shfl_xor_sync(0xffffffffu, cmean, 1);
-    cmean += __shfl_xor_sync(0xffffffffu, cmean, 2);
-    {
+    if (block_end) {
+      // ---- block mean of V: O^T[d][h] += o_V[d] * sum_{t in block} p_t s1_t ----
+      cmean += __shfl_xor_sync(0xffffffffu, cmean, 1);
+      cmean += __shfl_xor_sync(0xffffffffu, cmean, 2);
       const float ca = __shfl_sync(0xffffffffu, cmean, 8 * p);
       const float cb = __shfl_sync(0xffffffffu, cmean, 8 * p + 4);
-      const __half* ov = reinterpret_cast<const __half*>(sb + ST_VM);
+      const __half* ov = reinterpret_cast<const __half*>(mb + D * 2);
 #pragma unroll
       for (int mm = 0; mm < 8; ++mm) {
         const float oa = __half2float(ov[16 * mm + g]);
@@ -466,12 +457,20 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
         O[mm][2] = fmaf(ob, ca, O[mm][2]);
         O[mm][3] = fmaf(ob, cb, O[mm][3]);
       }
+      cmean = 0.f;
     }
-    __syncwarp();  // every lane is done with this stage buffer
-    if (st + 2 < nstages) issue_stage<MK, MV>(sba, kc, vc, seq, t_stage + 2 * STAGE_TOK, lane);
-    else cp_async_commit();  // keep the group count uniform for wait_group
+    __syncwarp();  // every lane is done with this stage buffer (and, at a block end, its means)
+    if (lane == 0 && st + 2 < nstages) {
+      const int tn = t_stage + 2 * STAGE_TOK;
+      issue_stage<MK, MV>(st_base + (uint32_t)(buf * STAGE_BYTES), mb_base + (uint32_t)(((tn / BLK) & 1) * MEAN_BYTES),
+                          bar0 + 8u * buf, kc, vc, seq, tn, (tn % BLK) == 0);
+    }
   }
-  cp_async_wait<0>();
+  if (failed) {
+    // A copy never completed: report it; wait (bounded) for the other buffer's copy.
+    if (lane == 0 && kc.status) atomicOr(kc.status, 2);
+    mbar_wait(bar0 + 8u, (phase >> 1) & 1u);
+  }
   l += __shfl_xor_sync(0xffffffffu, l, 1);
   l += __shfl_xor_sync(0xffffffffu, l, 2);
 
@@ -495,121 +494,139 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
 }
 
 // ---------------------------------------------------------------------------
-// Residual window: grid (kv-heads, batch), 128 threads; thread t owns window
-// token t for the scores and dim t for the value sum.  Original domain.
+// Residual window + combine: grid (kv-heads, batch), one warp per query head of
+// the group.  The window's K and V rows (fp16, original domain) are staged in
+// shared memory with coalesced loads; each warp scores them against its head,
+// merges the split partials of the quantized part (log-sum-exp), applies H to
+// their rotated value sum (H^T = H) and normalises both parts together.
+// Lane l owns dims 4l..4l+3.
 // ---------------------------------------------------------------------------
+constexpr int WROW = D + 8;  // padded fp16 row of the staged window (272 B: conflict-free row reads)
+
 template <int G>
-__global__ void __launch_bounds__(128)
-decode_window_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb, int64_t qsh,
-                     float qscale, float* __restrict__ ws, DecodeGeom geom) {
-  __shared__ float qp[G][D];
-  __shared__ float pw[BLK][G];
-  __shared__ float red[4][16];
-  const int hk = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+__global__ void __launch_bounds__(32 * G)
+decode_window_combine_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb,
+                             int64_t qsh, float qscale, const float* __restrict__ ws, float* __restrict__ out,
+                             int n_q_heads, DecodeGeom geom) {
+  extern __shared__ __align__(16) unsigned char wsm_raw[];
+  __half* kwin = reinterpret_cast<__half*>(wsm_raw);             // [BLK][WROW]
+  __half* vwin = kwin + BLK * WROW;                               // [BLK][D]
+  float* qp = reinterpret_cast<float*>(vwin + BLK * D);           // [G][D]
+  float* pw = qp + G * D;                                         // [G][BLK]
+  const int hk = blockIdx.x, b = blockIdx.y, h = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t seq = (int64_t)b * kc.n_kv_heads + hk;
-  const int64_t pidx = seq * (geom.nsplit_q + 1) + geom.nsplit_q;
-  const int64_t P = (int64_t)kc.batch * kc.n_kv_heads * (geom.nsplit_q + 1);
-  float* ws_acc = ws + acc_offset(P, G);
-  const int nw = (kc.window_len > 0) ? min(min(kc.n_window[seq], vc.n_window[seq]), kc.window_len) : 0;
-  if (nw <= 0) {
-    for (int i = t; i < G * D; i += blockDim.x) ws_acc[pidx * G * D + i] = 0.f;
-    if (t < G) {
-      partial_ml(ws, pidx, G, t)[0] = NEG_BIG;
-      partial_ml(ws, pidx, G, t)[1] = 0.f;
-    }
-    return;
-  }
-  load_queries<G>(&qp[0][0], q, dtype, qsb, qsh, b, hk, qscale, false);
-  __syncthreads();
-  const bool valid = t < nw;
-  float sc[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) sc[h] = 0.f;
-  if (valid) {
-    const __half* krow = kc.window + (seq * kc.window_len + t) * D;
-#pragma unroll 4
-    for (int c = 0; c < D; c += 8) {
-      float kv[8];
-      load8<NSN_DTYPE_F16>(krow, c, kv);
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sc[h] = fmaf(qp[h][c + i], kv[i], sc[h]);
-    }
-  }
-  float tmax[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    sc[h] = valid ? sc[h] : NEG_BIG;
-    tmax[h] = sc[h];
-  }
-  block_reduce<G, true>(tmax, red);
-  float sums[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const float p = valid ? exp2f(sc[h] - tmax[h]) : 0.f;
-    pw[t][h] = p;
-    sums[h] = p;
-  }
-  block_reduce<G, false>(sums, red);
-  float acc[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) acc[h] = 0.f;
-  const __half* vbase = vc.window + seq * vc.window_len * D;
-  for (int j = 0; j < nw; ++j) {
-    const float vv = __half2float(vbase[(int64_t)j * D + t]);
-#pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] = fmaf(pw[j][h], vv, acc[h]);
-  }
-#pragma unroll
-  for (int h = 0; h < G; ++h) ws_acc[(pidx * G + h) * D + t] = acc[h];
-  if (t < G) {
-    partial_ml(ws, pidx, G, t)[0] = tmax[t];
-    partial_ml(ws, pidx, G, t)[1] = sums[t];
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Combine: grid (q-heads, batch), 32 threads.  Lane l owns dims 4l..4l+3.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(32)
-decode_combine_kernel(const float* __restrict__ ws, float* __restrict__ out, int n_q_heads, int n_kv_heads,
-                      int batch, DecodeGeom geom) {
-  const int hq = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
-  const int G = geom.g;
-  const int hk = hq / G, h = hq % G;
+  const int hq = hk * G + h;
   const int nslots = geom.nsplit_q + 1;
-  const int64_t P = (int64_t)batch * n_kv_heads * nslots;
+  const int64_t P = (int64_t)kc.batch * kc.n_kv_heads * nslots;
   const float* ws_acc = ws + acc_offset(P, G);
-  const int64_t p0 = ((int64_t)b * n_kv_heads + hk) * nslots;
+  const int64_t p0 = seq * nslots;
+  const int nw = (kc.window_len > 0) ? min(min(kc.n_window[seq], vc.n_window[seq]), kc.window_len) : 0;
 
+  // ---- stage the window rows (coalesced 16-byte loads) and this head's query ----
+  if (nw > 0) {
+    const uint4* ksrc = reinterpret_cast<const uint4*>(kc.window + seq * kc.window_len * D);
+    const uint4* vsrc = reinterpret_cast<const uint4*>(vc.window + seq * vc.window_len * D);
+    for (int e = threadIdx.x; e < nw * (D / 8); e += blockDim.x) {
+      const int row = e >> 4, ch = e & 15;
+      *reinterpret_cast<uint4*>(kwin + row * WROW + ch * 8) = __ldg(ksrc + e);
+      *reinterpret_cast<uint4*>(vwin + row * D + ch * 8) = __ldg(vsrc + e);
+    }
+    const int64_t off = (int64_t)b * qsb + (int64_t)hq * qsh + 4 * lane;
+    float v[4];
+    if (dtype == NSN_DTYPE_F32) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(q) + off));
+      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    } else {
+      const uint2 r = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(q) + off));
+      float2 a2, c2;
+      if (dtype == NSN_DTYPE_BF16) {
+        a2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+        c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+      } else {
+        a2 = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
+        c2 = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
+      }
+      v[0] = a2.x; v[1] = a2.y; v[2] = c2.x; v[3] = c2.y;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qp[h * D + 4 * lane + i] = v[i] * qscale;
+  }
+  __syncthreads();
+
+  // ---- window scores of this head (original domain, log2 units) ----
+  float mw = NEG_BIG, lw = 0.f, aw[4] = {0.f, 0.f, 0.f, 0.f};
+  if (nw > 0) {
+    float sc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = lane + 32 * i;
+      float acc0 = 0.f, acc1 = 0.f;
+      if (t < nw) {
+        const __half* row = kwin + t * WROW;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 r = *reinterpret_cast<const uint4*>(row + 8 * c);
+          const __half2* hv = reinterpret_cast<const __half2*>(&r);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __half22float2(hv[k]);
+            acc0 = fmaf(qp[h * D + 8 * c + 2 * k], f.x, acc0);
+            acc1 = fmaf(qp[h * D + 8 * c + 2 * k + 1], f.y, acc1);
+          }
+        }
+      }
+      sc[i] = t < nw ? acc0 + acc1 : NEG_BIG;
+      mw = fmaxf(mw, sc[i]);
+    }
+    mw = warp_max(mw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float pr = (lane + 32 * i < nw) ? fast_exp2(sc[i] - mw) : 0.f;
+      pw[h * BLK + lane + 32 * i] = pr;
+      lw += pr;
+    }
+    lw = warp_sum(lw);
+    __syncwarp();
+#pragma unroll 8
+    for (int t = 0; t < nw; ++t) {
+      const float pr = pw[h * BLK + t];
+      const uint2 r = *reinterpret_cast<const uint2*>(vwin + t * D + 4 * lane);
+      const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
+      const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
+      aw[0] = fmaf(pr, x0.x, aw[0]); aw[1] = fmaf(pr, x0.y, aw[1]);
+      aw[2] = fmaf(pr, x1.x, aw[2]); aw[3] = fmaf(pr, x1.y, aw[3]);
+    }
+  }
+
+  // ---- quantized part: merge the split partials, rotate back ----
   float mrot = NEG_BIG;
   for (int s = 0; s < geom.nsplit_q; ++s) mrot = fmaxf(mrot, ws[((p0 + s) * G + h) * 2]);
   float lrot = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
   for (int s = 0; s < geom.nsplit_q; ++s) {
-    const float* ml = ws + ((p0 + s) * G + h) * 2;
-    const float l = ml[1];
-    if (l == 0.f) continue;
-    const float f = exp2f(ml[0] - mrot);
-    lrot = fmaf(l, f, lrot);
+    const float2 ml = *reinterpret_cast<const float2*>(ws + ((p0 + s) * G + h) * 2);
+    const float f = ml.y > 0.f ? fast_exp2(ml.x - mrot) : 0.f;
+    lrot = fmaf(ml.y, f, lrot);
     const float4 v = *reinterpret_cast<const float4*>(ws_acc + ((p0 + s) * G + h) * D + 4 * lane);
     a[0] = fmaf(v.x, f, a[0]); a[1] = fmaf(v.y, f, a[1]); a[2] = fmaf(v.z, f, a[2]); a[3] = fmaf(v.w, f, a[3]);
   }
   fwht128_warp(a, lane);
-  const int64_t pr = p0 + geom.nsplit_q;
-  const float mres = ws[(pr * G + h) * 2], lres = ws[(pr * G + h) * 2 + 1];
-  const float4 r = *reinterpret_cast<const float4*>(ws_acc + (pr * G + h) * D + 4 * lane);
-  const float mt = fmaxf(mrot, mres);
-  const float fa = lrot > 0.f ? exp2f(mrot - mt) : 0.f;
-  const float fr = lres > 0.f ? exp2f(mres - mt) : 0.f;
-  const float den = lrot * fa + lres * fr;
+  const float mt = fmaxf(mrot, mw);
+  const float fa = lrot > 0.f ? fast_exp2(mrot - mt) : 0.f;
+  const float fr = lw > 0.f ? fast_exp2(mw - mt) : 0.f;
+  const float den = lrot * fa + lw * fr;
   const float inv = den > 0.f ? 1.f / den : 0.f;
   float4 o;
-  o.x = (a[0] * INV_SQRT_D * fa + r.x * fr) * inv;
-  o.y = (a[1] * INV_SQRT_D * fa + r.y * fr) * inv;
-  o.z = (a[2] * INV_SQRT_D * fa + r.z * fr) * inv;
-  o.w = (a[3] * INV_SQRT_D * fa + r.w * fr) * inv;
+  o.x = (a[0] * INV_SQRT_D * fa + aw[0] * fr) * inv;
+  o.y = (a[1] * INV_SQRT_D * fa + aw[1] * fr) * inv;
+  o.z = (a[2] * INV_SQRT_D * fa + aw[2] * fr) * inv;
+  o.w = (a[3] * INV_SQRT_D * fa + aw[3] * fr) * inv;
   *reinterpret_cast<float4*>(out + ((int64_t)b * n_q_heads + hq) * D + 4 * lane) = o;
+}
+
+template <int G>
+constexpr size_t window_smem_bytes() {
+  return (size_t)BLK * WROW * 2 + (size_t)BLK * D * 2 + (size_t)G * D * 4 + (size_t)G * BLK * 4;
 }
 
 // ---------------------------------------------------------------------------
@@ -648,8 +665,8 @@ size_t decode_workspace_bytes(int batch, int n_kv_heads, const DecodeGeom& geom)
 }
 
 template <int G, int MK, int MV>
-static cudaError_t launch_split_t(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int64_t qsb,
-                                  int64_t qsh, float qscale, const float* cbk, const float* cbv, float* ws,
+static cudaError_t launch_split_t(const CacheView& kc, const CacheView& vc, const float* cbk, const float* cbv,
+                                  const void* q, int dtype, int64_t qsb, int64_t qsh, float qscale, float* ws,
                                   const DecodeGeom& geom, cudaStream_t s) {
   const size_t smem = sizeof(DecSmem);
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<G, MK, MV>,
@@ -657,25 +674,32 @@ static cudaError_t launch_split_t(const CacheView& kc, const CacheView& vc, cons
   if (e != cudaSuccess) return e;
   const int nwarps = kc.batch * kc.n_kv_heads * geom.nsplit_q;
   dim3 grid((nwarps + DEC_WARPS - 1) / DEC_WARPS);
-  decode_split_kernel<G, MK, MV><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, ws, geom);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  dim3 g2(kc.n_kv_heads, kc.batch);
-  decode_window_kernel<G><<<g2, 128, 0, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, ws, geom);
+  decode_split_kernel<G, MK, MV><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv,
+                                                                   ws, geom);
   return cudaGetLastError();
 }
 
 template <int G>
-static cudaError_t launch_modes(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int64_t qsb,
-                                int64_t qsh, float qscale, const float* cbk, const float* cbv, float* ws,
-                                const DecodeGeom& geom, cudaStream_t s) {
+static cudaError_t launch_g(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                            int64_t qsb, int64_t qsh, float qscale, const float* cbk, const float* cbv, float* out,
+                            float* ws, const DecodeGeom& geom, cudaStream_t s) {
+  cudaError_t e;
   if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_1BIT)
-    return launch_split_t<G, 1, 1>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, ws, geom, s);
-  if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_2BIT)
-    return launch_split_t<G, 1, 2>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, ws, geom, s);
-  if (kc.mode == NSN_MODE_2BIT && vc.mode == NSN_MODE_1BIT)
-    return launch_split_t<G, 2, 1>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, ws, geom, s);
-  return launch_split_t<G, 2, 2>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, ws, geom, s);
+    e = launch_split_t<G, 1, 1>(kc, vc, cbk, cbv, q, dtype, qsb, qsh, qscale, ws, geom, s);
+  else if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_2BIT)
+    e = launch_split_t<G, 1, 2>(kc, vc, cbk, cbv, q, dtype, qsb, qsh, qscale, ws, geom, s);
+  else if (kc.mode == NSN_MODE_2BIT && vc.mode == NSN_MODE_1BIT)
+    e = launch_split_t<G, 2, 1>(kc, vc, cbk, cbv, q, dtype, qsb, qsh, qscale, ws, geom, s);
+  else
+    e = launch_split_t<G, 2, 2>(kc, vc, cbk, cbv, q, dtype, qsb, qsh, qscale, ws, geom, s);
+  if (e != cudaSuccess) return e;
+  dim3 g2(kc.n_kv_heads, kc.batch);
+  const size_t wsmem = window_smem_bytes<G>();
+  e = cudaFuncSetAttribute(decode_window_combine_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem);
+  if (e != cudaSuccess) return e;
+  decode_window_combine_kernel<G><<<g2, 32 * G, wsmem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, ws, out, n_q_heads,
+                                                            geom);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
@@ -683,17 +707,12 @@ cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* 
                           float* out, void* ws, const DecodeGeom& geom, cudaStream_t s) {
   const float qscale = softmax_scale * LOG2E;
   float* w = static_cast<float*>(ws);
-  cudaError_t e;
   switch (geom.g) {
-    case 1: e = launch_modes<1>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, w, geom, s); break;
-    case 2: e = launch_modes<2>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, w, geom, s); break;
-    case 4: e = launch_modes<4>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, w, geom, s); break;
-    default: e = launch_modes<8>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, w, geom, s); break;
+    case 1: return launch_g<1>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
+    case 2: return launch_g<2>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
+    case 4: return launch_g<4>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
+    default: return launch_g<8>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
   }
-  if (e != cudaSuccess) return e;
-  dim3 g3(n_q_heads, kc.batch);
-  decode_combine_kernel<<<g3, 32, 0, s>>>(w, out, n_q_heads, kc.n_kv_heads, kc.batch, geom);
-  return cudaGetLastError();
 }
 
 }  // namespace nsn
