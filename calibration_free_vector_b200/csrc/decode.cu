@@ -119,8 +119,9 @@ constexpr int MEAN_BYTES = 512;  // K mean row | V mean row of one block (fp16)
 // (log2 units): weights stay below 2^8 and exact in fp32, and most tiles skip the
 // max reduction.
 constexpr float LAZY_MAX_SLACK = 8.0f;
-// Upper bound on mbarrier polls before a wait gives up (error flag, no hang).
-constexpr uint32_t WAIT_LIMIT = 1u << 26;
+// Upper bound on suspended mbarrier wait attempts before a wait gives up (error
+// flag, no hang): a few seconds in total.
+constexpr uint32_t WAIT_LIMIT = 4096u;
 
 struct DecSmem {
   alignas(128) uint4 cbk[NCODES][8];  // replicated fp16 codebooks (32 KB each)
@@ -148,16 +149,19 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
 }
+// One wait attempt: the thread may sleep in hardware for up to SUSPEND_NS while the
+// phase is incomplete (no polling instructions are issued meanwhile).
+constexpr uint32_t SUSPEND_NS = 1000000u;
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(done)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(SUSPEND_NS)
       : "memory");
   return done != 0;
 }
-// Bounded wait; false if the limit was reached.
+// Bounded wait (at most WAIT_LIMIT suspended attempts); false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   for (uint32_t i = 0; i < WAIT_LIMIT; ++i)
     if (mbar_try_wait(bar, parity)) return true;
@@ -188,14 +192,32 @@ __device__ __forceinline__ void issue_stage(uint32_t dst, uint32_t mdst, uint32_
   }
 }
 
-template <int G, int MK, int MV>
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// One warp = one split of one (sequence, head group).  GH <= 4 query heads per
+// warp (a group of 8 runs as two head groups).
+//
+// Scores:  S[t][c] = sum_k u_hat[t][k] Qc[k][c]   M = 16 tokens, N = 8 columns, K = 16
+//          (columns 0-3: fp16(q~) of the GH heads, 4-7: their fp16 rounding residual).
+//          A lane swap (xor 2) adds the two halves so that lane (g, p) holds the
+//          scores of token g + 8 (p >> 1) for heads 2 (p & 1), 2 (p & 1) + 1.
+// Values:  O^T[d][h] += sum_t u_hat_v[t][d] w[t][h]  M = 16 dims, N = 8 heads, K = 16 tokens;
+//          the B operand is the weight matrix moved into place with movmatrix.trans.
+template <int GH, int MK, int MV>
 __global__ void __launch_bounds__(32 * DEC_WARPS, 1)
 decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb, int64_t qsh,
                     float qscale, const float* __restrict__ cbk_g, const float* __restrict__ cbv_g,
                     float* __restrict__ ws, DecodeGeom geom) {
+  static_assert(GH == 1 || GH == 2 || GH == 4, "1, 2 or 4 heads per warp");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, p = lane & 3;
+  const int G = geom.g;           // query heads per kv-head
+  const int ngroups = G / GH;     // head groups per kv-head
 
   // ---- stage the replicated fp16 codebooks (whole CTA, once) ----
   for (int e = tid; e < NCODES * 8; e += blockDim.x) {
@@ -211,11 +233,13 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
   __syncthreads();
 
   const int nseq = kc.batch * kc.n_kv_heads;
-  const int gw = blockIdx.x * DEC_WARPS + warp;  // global split id
-  if (gw >= nseq * geom.nsplit_q) return;
-  const int64_t seq = gw / geom.nsplit_q;
-  const int split = gw % geom.nsplit_q;
+  const int gw = blockIdx.x * DEC_WARPS + warp;  // global warp job id
+  if (gw >= nseq * geom.nsplit_q * ngroups) return;
+  const int hg = gw % ngroups;
+  const int64_t seq = (gw / ngroups) / geom.nsplit_q;
+  const int split = (gw / ngroups) % geom.nsplit_q;
   const int b = (int)(seq / kc.n_kv_heads), hk = (int)(seq % kc.n_kv_heads);
+  const int hbase = hg * GH;                      // first head of the group within the kv-head
   const int64_t pidx = seq * (geom.nsplit_q + 1) + split;
   const int64_t P = (int64_t)nseq * (geom.nsplit_q + 1);
   float* ws_acc = ws + acc_offset(P, G);
@@ -226,10 +250,10 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
   const int tok_begin = split * bps * BLK;
   const int tok_end = min(nq, (split + 1) * bps * BLK);
   if (tok_begin >= tok_end) {
-    for (int i = lane; i < G * D; i += 32) ws_acc[pidx * G * D + i] = 0.f;
-    if (lane < G) {
-      partial_ml(ws, pidx, G, lane)[0] = NEG_BIG;
-      partial_ml(ws, pidx, G, lane)[1] = 0.f;
+    for (int i = lane; i < GH * D; i += 32) ws_acc[(pidx * G + hbase) * D + i] = 0.f;
+    if (lane < GH) {
+      partial_ml(ws, pidx, G, hbase + lane)[0] = NEG_BIG;
+      partial_ml(ws, pidx, G, hbase + lane)[1] = 0.f;
     }
     return;
   }
@@ -238,7 +262,6 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
   const uint32_t mb_base = smem_addr(&sm.means[warp][0][0]);
   const uint32_t bar0 = smem_addr(&sm.bar[warp][0]);
 
-  // prologue: two stages in flight (stage s -> buffer s & 1; means buffer = block & 1)
   if (lane == 0) {
     issue_stage<MK, MV>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc, seq,
                         tok_begin, true);
@@ -246,14 +269,14 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
       issue_stage<MK, MV>(st_base + STAGE_BYTES, mb_base, bar0 + 8, kc, vc, seq, tok_begin + STAGE_TOK, false);
   }
 
-  // ---- rotated query fragments (built in registers while the copies fly) ----
-  // A row g = fp16(q~_g), row g + 8 = fp16(q~_g - fp16(q~_g)).
-  uint32_t qa[8][4];
+  // ---- query operand (B of the score product), built while the copies fly ----
+  // lane (g, p): column g, k rows 2p, 2p+1 (qb[j][0]) and 8 + 2p, 9 + 2p (qb[j][1]) of step j.
+  uint32_t qb[8][2];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) qa[j][0] = qa[j][1] = qa[j][2] = qa[j][3] = 0u;
+  for (int j = 0; j < 8; ++j) qb[j][0] = qb[j][1] = 0u;
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const int64_t off = (int64_t)b * qsb + (int64_t)(hk * G + h) * qsh + 4 * lane;
+  for (int h = 0; h < GH; ++h) {
+    const int64_t off = (int64_t)b * qsb + (int64_t)(hk * G + hbase + h) * qsh + 4 * lane;
     float v[4];
     if (dtype == NSN_DTYPE_F32) {
       const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(q) + off));
@@ -273,20 +296,17 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
     fwht128_warp(v, lane);
 #pragma unroll
     for (int i = 0; i < 4; ++i) v[i] *= qscale * INV_SQRT_D;
-    // element c lives in lane c/4, slot c%4; lane (g, p) needs c = 16j + 8hf + 2p, +1
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
-        const int src = 4 * j + 2 * hf + (p >> 1);
+        const int src = 4 * j + 2 * hf + (p >> 1);  // element 16j + 8hf + 2p lives in lane 4j + 2hf + p/2
         const float e0 = __shfl_sync(0xffffffffu, v[0], src), e2 = __shfl_sync(0xffffffffu, v[2], src);
         const float e1 = __shfl_sync(0xffffffffu, v[1], src), e3 = __shfl_sync(0xffffffffu, v[3], src);
         const float x0 = (p & 1) ? e2 : e0, x1 = (p & 1) ? e3 : e1;
-        if (g == h) {
-          const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-          qa[j][2 * hf] = pack_half2(__half2float(h0), __half2float(h1));
-          qa[j][2 * hf + 1] = pack_half2(x0 - __half2float(h0), x1 - __half2float(h1));
-        }
+        const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+        if (g == h) qb[j][hf] = pack_half2(__half2float(h0), __half2float(h1));
+        if (g == h + 4) qb[j][hf] = pack_half2(x0 - __half2float(h0), x1 - __half2float(h1));
       }
     }
   }
@@ -294,21 +314,29 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
   const uint32_t lane_row = (uint32_t)(lane & 7) * 16u;
   const uint32_t cbk_base = smem_addr(&sm.cbk[0][0]) + lane_row;
   const uint32_t cbv_base = smem_addr(&sm.cbv[0][0]) + lane_row;
-  const uint32_t sel_k = 0x4440u | (uint32_t)(lane >> 3);
+  const int tok_a = (lane & 7) + 8 * ((lane >> 3) & 1);   // token of this lane's K ldmatrix row
+  const int tok_v = (lane & 7) + 8 * (lane >> 4);         // token of this lane's V ldmatrix row
+  const uint32_t sel_k0 = 0x4440u | (uint32_t)(lane >> 4);
+  const uint32_t sel_k1 = 0x4440u | (uint32_t)(2 + (lane >> 4));
   const uint32_t sel_v0 = 0x4440u | (uint32_t)((lane >> 3) & 1);
   const uint32_t sel_v1 = 0x4440u | (uint32_t)(2 + ((lane >> 3) & 1));
-
-  float m = NEG_BIG, l = 0.f, cmean = 0.f, qo = 0.f;
+  const bool lo_lane = p < 2;                      // keeps token g (else g + 8) after the swap
+  const int t_l = g + (lo_lane ? 0 : 8);           // token of this lane's two scores
+  const int h0 = 2 * (p & 1);                      // its two heads: h0, h0 + 1 (within the group)
+  // Padding heads get a running max of +1e30: their weights are exactly 0 and they
+  // never trigger a re-base.
+  float m0 = h0 < GH ? NEG_BIG : -NEG_BIG, m1 = h0 + 1 < GH ? NEG_BIG : -NEG_BIG;
+  float l0 = 0.f, l1 = 0.f, cm0 = 0.f, cm1 = 0.f, qo0 = 0.f, qo1 = 0.f;
   float O[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
-  uint32_t phase = 0u;  // bit k = parity of the next wait on buffer k
+  uint32_t phase = 0u;
   bool failed = false;
 
   for (int st = 0; st < nstages; ++st) {
     const int buf = st & 1;
     const bool arrived = mbar_wait(bar0 + 8u * buf, (phase >> buf) & 1u);
-    if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform decision
+    if (!__all_sync(0xffffffffu, arrived)) {
       failed = true;
       break;
     }
@@ -321,109 +349,93 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
     const unsigned char* mb = &sm.means[warp][mbuf][0];
 
     if (block_start) {
-      // (H q) . o_K of this block, for head g (the mean row as all 8 "tokens")
+      // (H q) . o_K of this block: the mean row as all 16 "tokens" of one score tile
       float d4[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t mrow = mb_base + (uint32_t)(mbuf * MEAN_BYTES) + (uint32_t)(lane >> 3) * 16u;
+      const uint32_t mrow = mb_base + (uint32_t)(mbuf * MEAN_BYTES) + (uint32_t)(lane >> 4) * 16u;
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        uint32_t bb[4];
-        ldsm_x4(mrow + 64u * qq, bb);
-        mma_full(d4, qa[2 * qq], bb[0], bb[1]);
-        mma_full(d4, qa[2 * qq + 1], bb[2], bb[3]);
+      for (int j = 0; j < 8; ++j) {
+        uint32_t aa[4];
+        ldsm_x4(mrow + 32u * j, aa);
+        mma_full(d4, aa, qb[j][0], qb[j][1]);
       }
-      qo = d4[0] + d4[2];
+      const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? d4[2] : d4[0], 2);
+      const float r1 = __shfl_xor_sync(0xffffffffu, lo_lane ? d4[3] : d4[1], 2);
+      qo0 = (lo_lane ? d4[0] : d4[2]) + r0;
+      qo1 = (lo_lane ? d4[1] : d4[3]) + r1;
     }
     const int ntile = min(STAGE_TOK, tok_end - t_stage + 15) >> 4;
     const bool full = t_stage + STAGE_TOK <= tok_end;  // every token of the stage is valid
     for (int tile = 0; tile < ntile; ++tile) {
       const int tt = 16 * tile;  // token offset inside the stage
-      const uint4 kc0 = *reinterpret_cast<const uint4*>(sb + ST_KC + (tt + (lane & 7)) * 16);
-      const uint4 kc1 = *reinterpret_cast<const uint4*>(sb + ST_KC + (tt + 8 + (lane & 7)) * 16);
+      const uint4 kcw = *reinterpret_cast<const uint4*>(sb + ST_KC + (tt + tok_a) * 16);
       uint32_t ks0 = 0u, ks1 = 0u;
       if constexpr (MK == NSN_MODE_2BIT) {
         ks0 = *reinterpret_cast<const uint32_t*>(sb + ST_KS + (tt + g) * 16 + 4 * p);
         ks1 = *reinterpret_cast<const uint32_t*>(sb + ST_KS + (tt + 8 + g) * 16 + 4 * p);
       }
-      const uint2 kn0 = *reinterpret_cast<const uint2*>(sb + ST_KN + (tt + 2 * p) * 4);
-      const uint2 kn1 = *reinterpret_cast<const uint2*>(sb + ST_KN + (tt + 8 + 2 * p) * 4);
-      const uint4 vcw = *reinterpret_cast<const uint4*>(sb + ST_VC + (tt + (lane & 7) + 8 * (lane >> 4)) * 16);
+      const uint32_t knw = *reinterpret_cast<const uint32_t*>(sb + ST_KN + (tt + t_l) * 4);
+      const uint4 vcw = *reinterpret_cast<const uint4*>(sb + ST_VC + (tt + tok_v) * 16);
       uint32_t W0 = 0u, W1 = 0u;
       if constexpr (MV == NSN_MODE_2BIT) {
         const uint16_t* vs = reinterpret_cast<const uint16_t*>(sb + ST_VS);
-        W0 = (uint32_t)vs[(tt + 2 * p) * 8 + g] | ((uint32_t)vs[(tt + 2 * p + 1) * 8 + g] << 16);
-        W1 = (uint32_t)vs[(tt + 8 + 2 * p) * 8 + g] | ((uint32_t)vs[(tt + 9 + 2 * p) * 8 + g] << 16);
+        W0 = __byte_perm((uint32_t)vs[(tt + 2 * p) * 8 + g], (uint32_t)vs[(tt + 2 * p + 1) * 8 + g], 0x5410u);
+        W1 = __byte_perm((uint32_t)vs[(tt + 8 + 2 * p) * 8 + g], (uint32_t)vs[(tt + 9 + 2 * p) * 8 + g], 0x5410u);
       }
-      const uint2 vn0 = *reinterpret_cast<const uint2*>(sb + ST_VN + (tt + 2 * p) * 4);
-      const uint2 vn1 = *reinterpret_cast<const uint2*>(sb + ST_VN + (tt + 8 + 2 * p) * 4);
+      const uint32_t vnw = *reinterpret_cast<const uint32_t*>(sb + ST_VN + (tt + t_l) * 4);
 
-      // ---- scores S^T = q~ u_hat^T for the two 8-token groups ----
-      float S[2][2];
+      // ---- scores: 8 k-steps of 16 dims ----
+      float S[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int grp = 0; grp < 2; ++grp) {
-        const uint4 kcw = grp ? kc1 : kc0;
-        const uint32_t ksw = grp ? ks1 : ks0;
-        float Sa[4] = {0.f, 0.f, 0.f, 0.f}, Sb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const uint32_t code = __byte_perm(u4_word(kcw, qq), 0u, sel_k);
-          uint32_t bb[4];
-          ldsm_x4(cbk_base + code * 128u, bb);
-          if constexpr (MK == NSN_MODE_2BIT) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) bb[i] = apply_signs(bb[i], ksw, 4 * qq + i);
-          }
-          mma_full(Sa, qa[2 * qq], bb[0], bb[1]);
-          mma_full(Sb, qa[2 * qq + 1], bb[2], bb[3]);
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t code = __byte_perm(u4_word(kcw, j >> 1), 0u, (j & 1) ? sel_k1 : sel_k0);
+        uint32_t aa[4];
+        ldsm_x4(cbk_base + code * 128u, aa);
+        if constexpr (MK == NSN_MODE_2BIT) {
+          aa[0] = apply_signs(aa[0], ks0, 2 * j);
+          aa[1] = apply_signs(aa[1], ks1, 2 * j);
+          aa[2] = apply_signs(aa[2], ks0, 2 * j + 1);
+          aa[3] = apply_signs(aa[3], ks1, 2 * j + 1);
         }
-        S[grp][0] = (Sa[0] + Sa[2]) + (Sb[0] + Sb[2]);  // rows g and g + 8
-        S[grp][1] = (Sa[1] + Sa[3]) + (Sb[1] + Sb[3]);
+        mma_full(S, aa, qb[j][0], qb[j][1]);
       }
+      // hi + lo columns -> (token t_l, heads h0, h0 + 1)
+      const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[2] : S[0], 2);
+      const float r1 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[3] : S[1], 2);
+      const float d0 = (lo_lane ? S[0] : S[2]) + r0;
+      const float d1 = (lo_lane ? S[1] : S[3]) + r1;
 
-      // ---- scores with the NSN byproducts, online softmax (head g) ----
-      const __half2* kh0 = reinterpret_cast<const __half2*>(&kn0);
-      const __half2* kh1 = reinterpret_cast<const __half2*>(&kn1);
-      const __half2* vh0 = reinterpret_cast<const __half2*>(&vn0);
-      const __half2* vh1 = reinterpret_cast<const __half2*>(&vn1);
-      const float2 kn[4] = {__half22float2(kh0[0]), __half22float2(kh0[1]), __half22float2(kh1[0]),
-                            __half22float2(kh1[1])};
-      const float2 vn[4] = {__half22float2(vh0[0]), __half22float2(vh0[1]), __half22float2(vh1[0]),
-                            __half22float2(vh1[1])};
-      const float dk[4] = {S[0][0], S[0][1], S[1][0], S[1][1]};  // tokens 2p, 2p+1, 8+2p, 9+2p
-      const int tk[4] = {tt + 2 * p, tt + 2 * p + 1, tt + 8 + 2 * p, tt + 9 + 2 * p};
-      float sc[4];
-      float lmax = NEG_BIG;
+      // ---- scores with the NSN byproducts; online softmax (lazy re-basing) ----
+      const float2 kn = __half22float2(*reinterpret_cast<const __half2*>(&knw));
+      const float2 vn = __half22float2(*reinterpret_cast<const __half2*>(&vnw));
+      float sc0 = kn.x * fmaf(kn.y, d0, qo0);
+      float sc1 = kn.x * fmaf(kn.y, d1, qo1);
+      if (!full && t_stage + tt + t_l >= tok_end) sc0 = sc1 = NEG_BIG;
+      if (__any_sync(0xffffffffu, fmaxf(sc0 - m0, sc1 - m1) > LAZY_MAX_SLACK)) {
+        float t0 = sc0, t1 = sc1;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const bool ok = (g < G) && (full || t_stage + tk[i] < tok_end);
-        sc[i] = ok ? kn[i].x * fmaf(kn[i].y, dk[i], qo) : NEG_BIG;
-        lmax = fmaxf(lmax, sc[i]);
-      }
-      // lazy re-basing of the running max (rare after the first tile)
-      if (__any_sync(0xffffffffu, lmax > m + LAZY_MAX_SLACK)) {
-        float tmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, 1));
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-        const float mnew = fmaxf(m, tmax);
-        const float corr = fast_exp2(m - mnew);
-        const float ca = __shfl_sync(0xffffffffu, corr, 8 * p);
-        const float cb = __shfl_sync(0xffffffffu, corr, 8 * p + 4);
+        for (int x = 2; x < 32; x <<= 1) {  // lanes sharing the head pair: xor 2, 4, 8, 16
+          t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, x));
+          t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, x));
+        }
+        const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
+        const float c0 = fast_exp2(m0 - n0), c1 = fast_exp2(m1 - n1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          O[i][0] *= ca; O[i][1] *= cb; O[i][2] *= ca; O[i][3] *= cb;
+          O[i][0] *= c0; O[i][1] *= c1; O[i][2] *= c0; O[i][3] *= c1;
         }
-        l *= corr;
-        cmean *= corr;
-        m = mnew;
+        l0 *= c0; l1 *= c1; cm0 *= c0; cm1 *= c1;
+        m0 = n0; m1 = n1;
       }
-      float w[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float pr = (g < G) ? fast_exp2(sc[i] - m) : 0.f;
-        l += pr;
-        cmean = fmaf(pr, vn[i].x, cmean);
-        w[i] = pr * vn[i].x * vn[i].y;
-      }
-      const uint32_t pb0 = pack_half2(w[0], w[1]);
-      const uint32_t pb1 = pack_half2(w[2], w[3]);
+      const float pr0 = fast_exp2(sc0 - m0), pr1 = fast_exp2(sc1 - m1);
+      l0 += pr0;
+      l1 += pr1;
+      cm0 = fmaf(pr0, vn.x, cm0);
+      cm1 = fmaf(pr1, vn.x, cm1);
+      const float s12 = vn.x * vn.y;
+      const uint32_t wpk = pack_half2(pr0 * s12, pr1 * s12);
+      const uint32_t wother = __shfl_xor_sync(0xffffffffu, wpk, 2);
+      const uint32_t pb0 = movmatrix_t(lo_lane ? wpk : 0u);     // tokens 0-7
+      const uint32_t pb1 = movmatrix_t(lo_lane ? wother : 0u);  // tokens 8-15
 
       // ---- values: O^T += u_hat_v^T w ----
 #pragma unroll
@@ -443,21 +455,23 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
 
     if (block_end) {
       // ---- block mean of V: O^T[d][h] += o_V[d] * sum_{t in block} p_t s1_t ----
-      cmean += __shfl_xor_sync(0xffffffffu, cmean, 1);
-      cmean += __shfl_xor_sync(0xffffffffu, cmean, 2);
-      const float ca = __shfl_sync(0xffffffffu, cmean, 8 * p);
-      const float cb = __shfl_sync(0xffffffffu, cmean, 8 * p + 4);
+      float c0 = cm0, c1 = cm1;
+#pragma unroll
+      for (int x = 2; x < 32; x <<= 1) {
+        c0 += __shfl_xor_sync(0xffffffffu, c0, x);
+        c1 += __shfl_xor_sync(0xffffffffu, c1, x);
+      }
       const __half* ov = reinterpret_cast<const __half*>(mb + D * 2);
 #pragma unroll
       for (int mm = 0; mm < 8; ++mm) {
         const float oa = __half2float(ov[16 * mm + g]);
         const float ob = __half2float(ov[16 * mm + 8 + g]);
-        O[mm][0] = fmaf(oa, ca, O[mm][0]);
-        O[mm][1] = fmaf(oa, cb, O[mm][1]);
-        O[mm][2] = fmaf(ob, ca, O[mm][2]);
-        O[mm][3] = fmaf(ob, cb, O[mm][3]);
+        O[mm][0] = fmaf(oa, c0, O[mm][0]);
+        O[mm][1] = fmaf(oa, c1, O[mm][1]);
+        O[mm][2] = fmaf(ob, c0, O[mm][2]);
+        O[mm][3] = fmaf(ob, c1, O[mm][3]);
       }
-      cmean = 0.f;
+      cm0 = cm1 = 0.f;
     }
     __syncwarp();  // every lane is done with this stage buffer (and, at a block end, its means)
     if (lane == 0 && st + 2 < nstages) {
@@ -467,29 +481,39 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
     }
   }
   if (failed) {
-    // A copy never completed: report it; wait (bounded) for the other buffer's copy.
     if (lane == 0 && kc.status) atomicOr(kc.status, 2);
     mbar_wait(bar0 + 8u, (phase >> 1) & 1u);
   }
-  l += __shfl_xor_sync(0xffffffffu, l, 1);
-  l += __shfl_xor_sync(0xffffffffu, l, 2);
+#pragma unroll
+  for (int x = 2; x < 32; x <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, x);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, x);
+  }
 
-  // ---- this warp's partial ----
+  // ---- this warp's partial: lanes p < 2 own heads 2p, 2p + 1 of the group ----
+  if (lo_lane) {
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int h = 2 * p + hh;
-    if (h < G) {
-      float* dst = ws_acc + (pidx * G + h) * D;
+    for (int hh = 0; hh < 2; ++hh) {
+      const int h = 2 * p + hh;
+      if (h < GH) {
+        float* dst = ws_acc + (pidx * G + hbase + h) * D;
 #pragma unroll
-      for (int mm = 0; mm < 8; ++mm) {
-        dst[16 * mm + g] = O[mm][hh];
-        dst[16 * mm + 8 + g] = O[mm][2 + hh];
+        for (int mm = 0; mm < 8; ++mm) {
+          dst[16 * mm + g] = O[mm][hh];
+          dst[16 * mm + 8 + g] = O[mm][2 + hh];
+        }
       }
     }
-  }
-  if (p == 0 && g < G) {
-    partial_ml(ws, pidx, G, g)[0] = m;
-    partial_ml(ws, pidx, G, g)[1] = l;
+    if (g == 0) {
+      if (h0 < GH) {
+        partial_ml(ws, pidx, G, hbase + h0)[0] = m0;
+        partial_ml(ws, pidx, G, hbase + h0)[1] = l0;
+      }
+      if (h0 + 1 < GH) {
+        partial_ml(ws, pidx, G, hbase + h0 + 1)[0] = m1;
+        partial_ml(ws, pidx, G, hbase + h0 + 1)[1] = l1;
+      }
+    }
   }
 }
 
@@ -650,8 +674,9 @@ DecodeGeom decode_geometry(int batch, int capacity, int n_q_heads, int n_kv_head
   g.chunk = 0;
   // splits per sequence: fill one 16-warp CTA per SM, at most one split per block
   const int nseq = batch * n_kv_heads;
+  const int groups = g.g > 4 ? g.g / 4 : 1;
   const int warps = sm_count() * DEC_WARPS;
-  int sp = warps / (nseq > 0 ? nseq : 1);
+  int sp = warps / (nseq * groups > 0 ? nseq * groups : 1);
   const int maxsp = capacity / BLK;
   if (sp > maxsp) sp = maxsp;
   if (sp < 1) sp = 1;
@@ -668,14 +693,15 @@ template <int G, int MK, int MV>
 static cudaError_t launch_split_t(const CacheView& kc, const CacheView& vc, const float* cbk, const float* cbv,
                                   const void* q, int dtype, int64_t qsb, int64_t qsh, float qscale, float* ws,
                                   const DecodeGeom& geom, cudaStream_t s) {
+  constexpr int GH = G < 4 ? G : 4;  // heads per warp job
   const size_t smem = sizeof(DecSmem);
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<G, MK, MV>,
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<GH, MK, MV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int nwarps = kc.batch * kc.n_kv_heads * geom.nsplit_q;
+  const int nwarps = kc.batch * kc.n_kv_heads * geom.nsplit_q * (G / GH);
   dim3 grid((nwarps + DEC_WARPS - 1) / DEC_WARPS);
-  decode_split_kernel<G, MK, MV><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv,
-                                                                   ws, geom);
+  decode_split_kernel<GH, MK, MV><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv,
+                                                                    ws, geom);
   return cudaGetLastError();
 }
 
