@@ -20,10 +20,11 @@
 //
 // Nearest codeword: exhaustive fp32 search over the 256 codewords held in shared
 // memory (broadcast reads), score_k = u.c_k - ||c_k||^2/2, tracking the best and
-// second-best score.  Whenever the second best lies within the rigorous fp32
-// error bound of the best, the sub-vector is re-decided exactly in fp64 over all
-// codewords inside that bound (ties to the lowest index).  The stored code is
-// therefore the exact nearest codeword of the fp32 u.
+// second-best score (per group of 8 codewords, then inside the winning group).
+// Whenever the second best lies within the rigorous fp32 error bound of the best,
+// the sub-vector is re-decided exactly in fp64 over all codewords inside that
+// bound (ties to the lowest index).  The stored code is therefore the exact
+// nearest codeword of the fp32 u.
 
 #include "nsn_common.cuh"
 #include "nsn_launch.h"
@@ -264,32 +265,72 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     }
   }
 
-  // ---- exhaustive fp32 search with best / second-best tracking ---------------
-  // Two passes over the codebook, 8 sub-vectors each (bounded register use).
-  // After each pass the codes, the exact-path thresholds and the "close second"
-  // flags go to shared memory.
+  // ---- exhaustive fp32 search ------------------------------------------------
+  // score_k = u.c_k - ||c_k||^2 / 2 (maximised).  Two passes over the codebook,
+  // 8 sub-vectors each.  Codewords are scanned in groups of 8: a running max
+  // per group (one FMNMX per codeword), then the best and second-best group
+  // maxima with the best group's index.  The winning group is rescanned to find
+  // the code (lowest index on ties) and its runner-up inside the group; the
+  // overall runner-up is the larger of that and the second-best group max.
   const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1];
   constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
   uint32_t need = 0u;
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
-    float best1[NSUB / 2], best2[NSUB / 2];
-    int idx[NSUB / 2];
+    float b1[NSUB / 2], b2[NSUB / 2];
+    int bg[NSUB / 2];
 #pragma unroll
     for (int jj = 0; jj < NSUB / 2; ++jj) {
-      best1[jj] = -INFINITY;
-      best2[jj] = -INFINITY;
-      idx[jj] = 0;
+      b1[jj] = -INFINITY;
+      b2[jj] = -INFINITY;
+      bg[jj] = 0;
     }
 #pragma unroll 1
-    for (int k = 0; k < NCODES; ++k) {
-      const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
-      const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
-      const float bk = sm.bias[k];
+    for (int grp = 0; grp < NCODES / 8; ++grp) {
+      float gm[NSUB / 2];
+#pragma unroll
+      for (int jj = 0; jj < NSUB / 2; ++jj) gm[jj] = -INFINITY;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int k = 8 * grp + kk;
+        const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
+        const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
+        const float bk = sm.bias[k];
+#pragma unroll
+        for (int jj = 0; jj < NSUB / 2; ++jj) {
+          const int j = 8 * half + jj;
+          float s = bk;
+          s = fmaf(v[8 * j + 0], c0.x, s);
+          s = fmaf(v[8 * j + 1], c0.y, s);
+          s = fmaf(v[8 * j + 2], c0.z, s);
+          s = fmaf(v[8 * j + 3], c0.w, s);
+          s = fmaf(v[8 * j + 4], c1.x, s);
+          s = fmaf(v[8 * j + 5], c1.y, s);
+          s = fmaf(v[8 * j + 6], c1.z, s);
+          s = fmaf(v[8 * j + 7], c1.w, s);
+          gm[jj] = fmaxf(gm[jj], s);
+        }
+      }
 #pragma unroll
       for (int jj = 0; jj < NSUB / 2; ++jj) {
-        const int j = 8 * half + jj;
-        float s = bk;
+        const float lo = fminf(b1[jj], gm[jj]);
+        bg[jj] = (gm[jj] > b1[jj]) ? grp : bg[jj];
+        b1[jj] = fmaxf(b1[jj], gm[jj]);
+        b2[jj] = fmaxf(b2[jj], lo);
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < NSUB / 2; ++jj) {
+      const int j = 8 * half + jj;
+      // rescan the winning group with the same arithmetic as above
+      float best = -INFINITY, second = -INFINITY;
+      int idx = 8 * bg[jj];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int k = 8 * bg[jj] + kk;
+        const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
+        const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
+        float s = sm.bias[k];
         s = fmaf(v[8 * j + 0], c0.x, s);
         s = fmaf(v[8 * j + 1], c0.y, s);
         s = fmaf(v[8 * j + 2], c0.z, s);
@@ -298,15 +339,12 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
         s = fmaf(v[8 * j + 5], c1.y, s);
         s = fmaf(v[8 * j + 6], c1.z, s);
         s = fmaf(v[8 * j + 7], c1.w, s);
-        const float lo = fminf(best1[jj], s);
-        idx[jj] = (s > best1[jj]) ? k : idx[jj];
-        best1[jj] = fmaxf(best1[jj], s);
-        best2[jj] = fmaxf(best2[jj], lo);
+        const float lo = fminf(best, s);
+        idx = (s > best) ? k : idx;
+        best = fmaxf(best, s);
+        second = fmaxf(second, lo);
       }
-    }
-#pragma unroll
-    for (int jj = 0; jj < NSUB / 2; ++jj) {
-      const int j = 8 * half + jj;
+      const float runner = fmaxf(b2[jj], second);
       float na = 0.f;
 #pragma unroll
       for (int i = 0; i < SUB; ++i) na = fmaf(v[8 * j + i], v[8 * j + i], na);
@@ -314,9 +352,9 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
       // |fp32 score - exact score| <= gamma_9 (max||c||^2 + ||a|| max||c||) for every
       // codeword, so a rival within twice that bound of the best may be the true best.
       const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
-      sm.thr[t][j] = best1[jj] - margin;
-      need |= (best2[jj] >= best1[jj] - margin ? 1u : 0u) << j;
-      sm.code[t][j] = (uint8_t)idx[jj];
+      sm.thr[t][j] = best - margin;
+      need |= (runner >= best - margin ? 1u : 0u) << j;
+      sm.code[t][j] = (uint8_t)idx;
     }
   }
 
