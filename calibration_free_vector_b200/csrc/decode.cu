@@ -21,6 +21,8 @@
 //                                 partials, H applied to their rotated value sum.
 // Scores are carried in log2 units (the query is pre-scaled by softmax_scale*log2 e).
 
+#include <mutex>
+
 #include "nsn_common.cuh"
 #include "nsn_launch.h"
 
@@ -739,6 +741,49 @@ cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* 
     case 4: return launch_g<4>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
     default: return launch_g<8>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode.  Some callers cannot allocate device memory at the
+// moment they need to attend: code running inside a custom allocator or a
+// memory-pool callback, processes whose device memory is fully reserved up
+// front by a framework, or embedded hosts that forbid cudaMalloc after start-up.
+// For them the decode partials live in this fixed file-scope device array
+// instead of a caller-provided workspace.  Every GPU that loads the library
+// holds the array until the process exits.  All calls share it, so two such
+// calls that overlap on the GPU (different streams, no ordering) race on it.
+// The kernels write every partial they later read, so nothing needs clearing
+// between calls.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_decode_scratch[NSN_DECODE_SCRATCH_BYTES];
+
+// Device address of the scratch array for the current device.  Resolved once per
+// device (cudaGetSymbolAddress with that device current) and cached.
+static cudaError_t decode_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static void* ptrs[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode_static(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                                 int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
+                                 float* out, const DecodeGeom& geom, cudaStream_t s) {
+  void* ws = nullptr;
+  const cudaError_t e = decode_scratch_ptr(&ws);
+  if (e != cudaSuccess) return e;
+  return launch_decode(kc, vc, q, dtype, n_q_heads, qsb, qsh, softmax_scale, cbk, cbv, out, ws, geom, s);
 }
 
 }  // namespace nsn

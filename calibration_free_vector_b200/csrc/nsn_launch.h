@@ -45,4 +45,9 @@ cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* 
                           int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
                           float* out, void* ws, const DecodeGeom& geom, cudaStream_t s);
 
+// Same as launch_decode with the file-scope scratch array as the workspace.
+cudaError_t launch_decode_static(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                                 int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
+                                 float* out, const DecodeGeom& geom, cudaStream_t s);
+
 }  // namespace nsn

@@ -81,6 +81,9 @@ def load():
     lib.nsn_decode_attention.argtypes = [POINTER(nsn_cache), POINTER(nsn_cache), c_void_p, c_int, c_int, c_int64,
                                          c_int64, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                          c_void_p]
+    lib.nsn_decode_attention_static.restype = c_int
+    lib.nsn_decode_attention_static.argtypes = [POINTER(nsn_cache), POINTER(nsn_cache), c_void_p, c_int, c_int,
+                                                c_int64, c_int64, c_float, c_void_p, c_void_p, c_void_p, c_void_p]
     _lib = lib
     return lib
 
@@ -212,3 +215,25 @@ def nsn_decode_attention(k_cache: Cache, v_cache: Cache, q, softmax_scale: float
                                      cb_k.data_ptr(), cb_v.data_ptr(), out.data_ptr(), workspace.data_ptr(),
                                      workspace.numel(), _stream_ptr(stream))
     _check(st, "nsn_decode_attention")
+
+
+def nsn_decode_attention_static(k_cache: Cache, v_cache: Cache, q, softmax_scale: float, cb_k, cb_v, out,
+                                stream=None) -> None:
+    """Decode attention without a workspace argument.
+
+    For callers that cannot allocate device memory when they decode (for example
+    code running inside an allocator callback, or a framework that reserved all
+    device memory up front).  The partial results go to a fixed device array
+    inside the library instead (include/nsn.h: NSN_DECODE_SCRATCH_BYTES); calls
+    that overlap on the GPU race on it.  Same result as nsn_decode_attention.
+    """
+    if q.dim() != 3 or q.shape[-1] != HEAD_DIM or q.stride(-1) != 1:
+        raise ValueError("q must be [B, H_q, 128] with a contiguous last dimension")
+    import torch
+    if out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must be a contiguous float32 tensor shaped like q")
+    st = load().nsn_decode_attention_static(ctypes.byref(k_cache.c), ctypes.byref(v_cache.c), q.data_ptr(),
+                                            _dtype_code(q), q.shape[1], q.stride(0), q.stride(1),
+                                            float(softmax_scale), cb_k.data_ptr(), cb_v.data_ptr(),
+                                            out.data_ptr(), _stream_ptr(stream))
+    _check(st, "nsn_decode_attention_static")

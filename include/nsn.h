@@ -200,6 +200,31 @@ nsn_status nsn_decode_attention(const nsn_cache* k_cache, const nsn_cache* v_cac
                                 const float* cb_v, float* out, void* workspace, size_t ws_bytes,
                                 void* stream);
 
+/*
+ * Allocation-free variant of nsn_decode_attention.  The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory when they
+ * decode -- code running inside an allocator or memory-pool callback, frameworks
+ * that reserve all device memory up front, hosts that forbid cudaMalloc after
+ * start-up.  It takes the same arguments as nsn_decode_attention minus the
+ * workspace and computes the same result; its decode partials go to a fixed
+ * file-scope device array of NSN_DECODE_SCRATCH_BYTES bytes instead, which every
+ * GPU that loads the library holds until the process exits.
+ *   - Nothing is allocated or freed (no cudaMalloc / cudaFree / allocating library).
+ *   - Returns NSN_ERR_WORKSPACE if this shape needs more than NSN_DECODE_SCRATCH_BYTES
+ *     (nsn_decode_workspace_bytes() tells how much it needs).
+ *   - The first call on a device resolves the array's device address (with that
+ *     device current) and caches it; make that first call before any stream capture.
+ *   - All calls share the one array: two calls whose work overlaps on the GPU (e.g. on
+ *     different streams without ordering between them) race on it and must not be
+ *     issued.  Every value the kernels read from it is written earlier in the same
+ *     call, so nothing needs clearing between calls.
+ */
+#define NSN_DECODE_SCRATCH_BYTES (8u << 20)
+nsn_status nsn_decode_attention_static(const nsn_cache* k_cache, const nsn_cache* v_cache, const void* q,
+                                       int dtype, int n_q_heads, int64_t q_stride_b, int64_t q_stride_h,
+                                       float softmax_scale, const float* cb_k, const float* cb_v, float* out,
+                                       void* stream);
+
 #ifdef __cplusplus
 }
 #endif
