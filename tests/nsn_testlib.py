@@ -127,3 +127,33 @@ def attn_error(out: np.ndarray, ref: np.ndarray) -> float:
     num = np.abs(out - ref).max(axis=1)
     den = np.maximum(np.abs(ref).max(axis=1), 1e-30)
     return float((num / den).max())
+
+
+# ---------------------------------------------------------------------------
+# Oracle pipeline of one (batch, kv-head) sequence, block quantization spread over
+# a process pool (the oracle itself is unchanged; blocks are independent).
+# ---------------------------------------------------------------------------
+def _oracle_block(args):
+    from oracle import nsn_oracle as orc
+    x, cb, mode = args
+    r = orc.quantize_block(x, cb, mode)
+    return {k: r[k] for k in ("codes", "signs", "s1", "s2", "o", "gap", "u")}
+
+
+def oracle_cache_sequence(pool, x, n_prefill, n_total, cb, mode, window=128):
+    """Oracle cache of one sequence x [T, 128] (fp64) after a prefill of n_prefill
+    tokens and appends up to n_total: (quantized dict, fp16 window rows)."""
+    from oracle import nsn_oracle as orc
+    q = orc.prefill_split(n_prefill, 128, window)
+    blocks = [(x[a:min(a + 128, q)], cb, mode) for a in range(0, q, 128)]
+    parts = list(pool.map(_oracle_block, blocks, chunksize=4)) if blocks else []
+    win = list(orc.to_f16(x[q:n_prefill]))
+    for t in range(n_prefill, n_total):
+        if len(win) == window:
+            parts.append(_oracle_block((np.array(win), cb, mode)))
+            win = []
+        win.append(orc.to_f16(x[t]))
+    cat = lambda k: np.concatenate([p[k] for p in parts])  # noqa: E731
+    seq = {"codes": cat("codes"), "signs": None if mode == 1 else cat("signs"), "s1": cat("s1"),
+           "s2": cat("s2"), "o": np.stack([p["o"] for p in parts]), "gap": cat("gap"), "u": cat("u")}
+    return seq, np.array(win).reshape(-1, 128)
