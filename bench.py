@@ -54,6 +54,27 @@ def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The largest of the ranks' times (every rank gets it); ms itself when alone."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job units/s: what all ranks processed over the slowest rank's time."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each replica draws its own synthetic batch."""
+    return 7 * rank
+
+
 # ---------------------------------------------------------------------------
 # clocks sampler (nvidia-smi during the timed region)
 # ---------------------------------------------------------------------------
@@ -233,8 +254,8 @@ def run_ours(args):
                                          W["mode_v"] == 2, iters)
     cbk, cbv = torch.from_numpy(cbk_np).to(dev), torch.from_numpy(cbv_np).to(dev)
 
-    rk = synthetic.KVRecipe(synthetic.config_seed(3, "k") + 7 * rank, H)
-    rv = synthetic.KVRecipe(synthetic.config_seed(3, "v") + 7 * rank, H)
+    rk = synthetic.KVRecipe(synthetic.config_seed(3, "k") + rank_seed_offset(rank), H)
+    rv = synthetic.KVRecipe(synthetic.config_seed(3, "v") + rank_seed_offset(rank), H)
     kc = nsn.Cache(B, H, cap, W["window"], W["mode_k"], device=dev)
     vc = nsn.Cache(B, H, cap, W["window"], W["mode_v"], device=dev)
     stream = torch.cuda.current_stream()
@@ -311,12 +332,8 @@ def run_ours(args):
     clocks = sampler.stop()
     clocks["window"] = "timed region + 1 s of the same decode call right after it"
 
-    ms = t0.elapsed_time(t1)
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     decode_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
     ms_per_step = ms / K
 
     # ---- algorithmic bytes of one decode call ----
@@ -356,11 +373,7 @@ def run_ours(args):
             host_out.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         h2d = (dk.numel() + dv.numel() + dq.numel()) * 2
         d2h = host_out.numel() * 4
 
@@ -384,7 +397,7 @@ def run_ours(args):
         cq_t, cq_n = oracle_quantize_sample(8.0)
         line = {
             "metric": METRIC,
-            "value": world * B * K / (ms * 1e-3),
+            "value": job_throughput(B * K, world, ms),
             "unit": "tokens/s",
             "n_gpus": world, "steps": K, "warmup": WU, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -407,7 +420,7 @@ def run_ours(args):
                          "roofline": {"kernel": "quantize_prefill_kernel", "bound": "alu", "achieved": q_ach,
                                       "peak": alu_peak, "unit": "T FMA/s (fp32)", "frac": q_ach / alu_peak,
                                       "algorithmic_fma_per_token_head": fma_per_th}},
-            "e2e": {"value": world * B * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": job_throughput(B * e2e_steps, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": K * 4,
             "clocks": clocks,
