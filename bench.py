@@ -38,6 +38,9 @@ WORKLOAD = dict(config=3, name="decode-b16-32k-2bit", batch=16, n_kv_heads=8, n_
                 mode_k=2, mode_v=2, window=128)
 BYTES_PER_TOKEN = {1: 16 + 4, 2: 16 + 16 + 4}   # codes (+ signs) + (s1, s2) per token-head
 MEAN_BYTES_PER_BLOCK = 128 * 2
+# Kernels one decode step launches: append_kernel (K and V, flush included),
+# decode_split_kernel, decode_window_combine_kernel.
+LAUNCHES_PER_STEP = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
@@ -422,7 +425,7 @@ def run_ours(args):
                                       "algorithmic_fma_per_token_head": fma_per_th}},
             "e2e": {"value": job_throughput(B * e2e_steps, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": K * 4,
+            "gpu_launches": K * LAUNCHES_PER_STEP,
             "clocks": clocks,
             "cache_status": status,
             "cpu_baseline": {"value": B / cpu_step, "unit": "tokens/s", "cores": cpu_threads, "kind": "oracle",
