@@ -11,14 +11,16 @@
 //   sum_t p_t v_hat_t = H [ sum_t (p_t s1 s2) u_hat_t + sum_b (sum_{t in b} p_t s1) o_b ].
 // Residual-window tokens are attended in the original domain.
 //
-// Kernels:
-//   decode_split_kernel           one warp per split (a contiguous range of 128-token
-//                                 blocks of one (batch, kv-head)): rotated query, scores
-//                                 from the codes, online softmax, value accumulation
-//                                 from the codewords -> partial (m, l, acc)
-//   decode_window_combine_kernel  one warp per query head: residual window attention
-//                                 (original domain), log-sum-exp merge with the split
-//                                 partials, H applied to their rotated value sum.
+// One kernel (decode_kernel) does the whole call:
+//   - one warp per split (a contiguous range of 128-token blocks of one (batch,
+//     kv-head) and a group of up to 4 query heads): rotated query, scores from the
+//     codes, online softmax, value accumulation from the codewords -> partial
+//     (m, l, acc) in the rotated domain;
+//   - the last split of a sequence also attends the residual window (original
+//     domain) -> a second partial;
+//   - the warp that finishes a (sequence, head group) last (a self-resetting
+//     counter decides) merges the partials by log-sum-exp, applies H to the
+//     rotated value sum and writes the output rows.
 // Scores are carried in log2 units (the query is pre-scaled by softmax_scale*log2 e).
 
 #include <mutex>
@@ -31,8 +33,9 @@ namespace nsn {
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float INV_SQRT_D = 0.08838834764831845f;  // 1/sqrt(128)
 
-// Workspace layout: [P][G][2] (m, l) floats, then -- from a 16-byte aligned
-// offset -- [P][G][128] accumulators; P = batch * kv-heads * (nsplit_q + 1).
+// Partials layout: [P][G][2] (m, l) floats, then -- from a 16-byte aligned
+// offset -- [P][G][128] accumulators; P = batch * kv-heads * (nsplit_q + 1)
+// (slot nsplit_q of each sequence is its residual window).
 __device__ __host__ __forceinline__ int64_t acc_offset(int64_t P, int G) { return ((P * G * 2 + 3) / 4) * 4; }
 __device__ __forceinline__ float* partial_ml(float* ws, int64_t p, int G, int h) { return ws + (p * G + h) * 2; }
 
@@ -200,85 +203,41 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
   return y;
 }
 
-// One warp = one split of one (sequence, head group).  GH <= 4 query heads per
-// warp (a group of 8 runs as two head groups).
-//
-// Scores:  S[t][c] = sum_k u_hat[t][k] Qc[k][c]   M = 16 tokens, N = 8 columns, K = 16
-//          (columns 0-3: fp16(q~) of the GH heads, 4-7: their fp16 rounding residual).
-//          A lane swap (xor 2) adds the two halves so that lane (g, p) holds the
-//          scores of token g + 8 (p >> 1) for heads 2 (p & 1), 2 (p & 1) + 1.
-// Values:  O^T[d][h] += sum_t u_hat_v[t][d] w[t][h]  M = 16 dims, N = 8 heads, K = 16 tokens;
-//          the B operand is the weight matrix moved into place with movmatrix.trans.
-template <int GH, int MK, int MV>
-__global__ void __launch_bounds__(32 * DEC_WARPS, 1)
-decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb, int64_t qsh,
-                    float qscale, const float* __restrict__ cbk_g, const float* __restrict__ cbv_g,
-                    float* __restrict__ ws, DecodeGeom geom) {
-  static_assert(GH == 1 || GH == 2 || GH == 4, "1, 2 or 4 heads per warp");
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, p = lane & 3;
-  const int G = geom.g;           // query heads per kv-head
-  const int ngroups = G / GH;     // head groups per kv-head
+// ---- residual-window chunks: 8 fp16 rows of K and of V per stage buffer ----
+// Rows are copied one by one (one lane per row) into 272-byte slots so that the
+// 8 rows of an ldmatrix fetch start in 8 different bank groups.
+constexpr int WCHUNK = 8;
+constexpr int WROWB = (D + 8) * 2;    // 272
+constexpr int WC_V = WCHUNK * WROWB;  // V rows follow the K rows
+static_assert(2 * WC_V <= STAGE_BYTES, "a window chunk fits one stage buffer");
+// The residual window counts as this many 128-token blocks when the quantized
+// blocks of a sequence are dealt out to its splits (the last split takes it).
+constexpr int WINDOW_COST_BLOCKS = 2;
 
-  // ---- stage the replicated fp16 codebooks (whole CTA, once) ----
-  for (int e = tid; e < NCODES * 8; e += blockDim.x) {
-    const int c = e >> 3, r = e & 7;
-    sm.cbk[c][r] = cb_row_f16(cbk_g, c);
-    sm.cbv[c][r] = cb_row_f16(cbv_g, c);
+__device__ __forceinline__ void issue_window_chunk(uint32_t dst, uint32_t bar, const __half* krow, const __half* vrow,
+                                                   int rows, int lane) {
+  if (lane == 0) mbar_expect_tx(bar, (uint32_t)rows * 2u * (uint32_t)(D * 2));
+  __syncwarp();
+  if (lane < 2 * rows) {
+    const int r = lane >> 1;
+    const bool isv = (lane & 1) != 0;
+    bulk_g2s(dst + (isv ? WC_V : 0) + (uint32_t)(r * WROWB), (isv ? vrow : krow) + r * D, D * 2, bar);
   }
-  if (lane == 0) {
-    mbar_init(smem_addr(&sm.bar[warp][0]), 1);
-    mbar_init(smem_addr(&sm.bar[warp][1]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  }
-  __syncthreads();
+}
 
-  const int nseq = kc.batch * kc.n_kv_heads;
-  const int gw = blockIdx.x * DEC_WARPS + warp;  // global warp job id
-  if (gw >= nseq * geom.nsplit_q * ngroups) return;
-  const int hg = gw % ngroups;
-  const int64_t seq = (gw / ngroups) / geom.nsplit_q;
-  const int split = (gw / ngroups) % geom.nsplit_q;
-  const int b = (int)(seq / kc.n_kv_heads), hk = (int)(seq % kc.n_kv_heads);
-  const int hbase = hg * GH;                      // first head of the group within the kv-head
-  const int64_t pidx = seq * (geom.nsplit_q + 1) + split;
-  const int64_t P = (int64_t)nseq * (geom.nsplit_q + 1);
-  float* ws_acc = ws + acc_offset(P, G);
-
-  const int nq = min(min(kc.n_quant[seq], vc.n_quant[seq]), kc.capacity);
-  const int nblk = (nq + BLK - 1) / BLK;
-  const int bps = (nblk + geom.nsplit_q - 1) / geom.nsplit_q;  // blocks per split
-  const int tok_begin = split * bps * BLK;
-  const int tok_end = min(nq, (split + 1) * bps * BLK);
-  if (tok_begin >= tok_end) {
-    for (int i = lane; i < GH * D; i += 32) ws_acc[(pidx * G + hbase) * D + i] = 0.f;
-    if (lane < GH) {
-      partial_ml(ws, pidx, G, hbase + lane)[0] = NEG_BIG;
-      partial_ml(ws, pidx, G, hbase + lane)[1] = 0.f;
-    }
-    return;
-  }
-  const int nstages = (tok_end - tok_begin + STAGE_TOK - 1) / STAGE_TOK;
-  const uint32_t st_base = smem_addr(&sm.stage[warp][0][0]);
-  const uint32_t mb_base = smem_addr(&sm.means[warp][0][0]);
-  const uint32_t bar0 = smem_addr(&sm.bar[warp][0]);
-
-  if (lane == 0) {
-    issue_stage<MK, MV>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc, seq,
-                        tok_begin, true);
-    if (nstages > 1)
-      issue_stage<MK, MV>(st_base + STAGE_BYTES, mb_base, bar0 + 8, kc, vc, seq, tok_begin + STAGE_TOK, false);
-  }
-
-  // ---- query operand (B of the score product), built while the copies fly ----
-  // lane (g, p): column g, k rows 2p, 2p+1 (qb[j][0]) and 8 + 2p, 9 + 2p (qb[j][1]) of step j.
-  uint32_t qb[8][2];
+// B operand of the score product for GH query heads: lane (g, p) holds column g
+// (head g for g < 4, the fp16 rounding residual of head g - 4 for g >= 4), k rows
+// 2p, 2p+1 (qb[j][0]) and 8+2p, 9+2p (qb[j][1]) of k-step j.  With `rotate` the
+// query is taken to the Hadamard domain first (orthonormal H).
+template <int GH>
+__device__ __forceinline__ void build_q_operand(uint32_t (&qb)[8][2], const void* __restrict__ q, int dtype,
+                                                int64_t off0, int64_t qsh, float scale, bool rotate, int lane) {
+  const int g = lane >> 2, p = lane & 3;
 #pragma unroll
   for (int j = 0; j < 8; ++j) qb[j][0] = qb[j][1] = 0u;
 #pragma unroll
   for (int h = 0; h < GH; ++h) {
-    const int64_t off = (int64_t)b * qsb + (int64_t)(hk * G + hbase + h) * qsh + 4 * lane;
+    const int64_t off = off0 + (int64_t)h * qsh + 4 * lane;
     float v[4];
     if (dtype == NSN_DTYPE_F32) {
       const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(q) + off));
@@ -295,9 +254,9 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
       }
       v[0] = a.x; v[1] = a.y; v[2] = c.x; v[3] = c.y;
     }
-    fwht128_warp(v, lane);
+    if (rotate) fwht128_warp(v, lane);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] *= qscale * INV_SQRT_D;
+    for (int i = 0; i < 4; ++i) v[i] *= scale;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
 #pragma unroll
@@ -312,6 +271,218 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
       }
     }
   }
+}
+
+// Online-softmax state of one warp for its head pair (h0, h0 + 1): running max in
+// log2 units, denominator and the O^T accumulator fragment (rows = dims, columns =
+// heads).  `lazy_update` re-bases the running max only when a score exceeds it by
+// more than LAZY_MAX_SLACK, so most tiles skip the max reduction.
+struct SoftmaxState {
+  float m0, m1, l0, l1;
+  float O[8][4];
+};
+
+__device__ __forceinline__ void lazy_update(SoftmaxState& st, float sc0, float sc1, float& cm0, float& cm1) {
+  if (__any_sync(0xffffffffu, fmaxf(sc0 - st.m0, sc1 - st.m1) > LAZY_MAX_SLACK)) {
+    float t0 = sc0, t1 = sc1;
+#pragma unroll
+    for (int x = 2; x < 32; x <<= 1) {  // lanes sharing the head pair: xor 2, 4, 8, 16
+      t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, x));
+      t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, x));
+    }
+    const float n0 = fmaxf(st.m0, t0), n1 = fmaxf(st.m1, t1);
+    const float c0 = fast_exp2(st.m0 - n0), c1 = fast_exp2(st.m1 - n1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      st.O[i][0] *= c0; st.O[i][1] *= c1; st.O[i][2] *= c0; st.O[i][3] *= c1;
+    }
+    st.l0 *= c0; st.l1 *= c1; cm0 *= c0; cm1 *= c1;
+    st.m0 = n0; st.m1 = n1;
+  }
+}
+
+// Writes a warp's partial (m, l, O^T) for the GH heads of its group: lanes p < 2
+// own heads 2p, 2p + 1.  Reduces l across the lanes first.
+template <int GH>
+__device__ __forceinline__ void store_partial(SoftmaxState& st, float* __restrict__ ws, float* __restrict__ ws_acc,
+                                              int64_t slot, int G, int hbase, int lane) {
+  const int g = lane >> 2, p = lane & 3, h0 = 2 * (p & 1);
+#pragma unroll
+  for (int x = 2; x < 32; x <<= 1) {
+    st.l0 += __shfl_xor_sync(0xffffffffu, st.l0, x);
+    st.l1 += __shfl_xor_sync(0xffffffffu, st.l1, x);
+  }
+  if (p < 2) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int h = 2 * p + hh;
+      if (h < GH) {
+        float* dst = ws_acc + (slot * G + hbase + h) * D;
+#pragma unroll
+        for (int mm = 0; mm < 8; ++mm) {
+          dst[16 * mm + g] = st.O[mm][hh];
+          dst[16 * mm + 8 + g] = st.O[mm][2 + hh];
+        }
+      }
+    }
+    if (g == 0) {
+      if (h0 < GH) {
+        partial_ml(ws, slot, G, hbase + h0)[0] = st.m0;
+        partial_ml(ws, slot, G, hbase + h0)[1] = st.l0;
+      }
+      if (h0 + 1 < GH) {
+        partial_ml(ws, slot, G, hbase + h0 + 1)[0] = st.m1;
+        partial_ml(ws, slot, G, hbase + h0 + 1)[1] = st.l1;
+      }
+    }
+  }
+}
+
+// Log-sum-exp merge of the partials of one (sequence, head group), done by the
+// warp that finished last.  Slots 0 .. nsplit-1 hold the quantized part (rotated
+// domain), slot nsplit the residual window (original domain).  The rotated value
+// sum is taken back with H (H^T = H) before both parts are normalised together.
+// Lane l owns dims 4l .. 4l+3.  Partials written by other SMs are read through L2.
+template <int GH>
+__device__ __noinline__ void merge_partials(const float* ws, const float* ws_acc, int64_t p0, int nsplit, int G, int hbase,
+                               float* __restrict__ out_rows, int lane) {
+  float mrot[GH], lrot[GH], a[GH][4];
+#pragma unroll
+  for (int h = 0; h < GH; ++h) {
+    mrot[h] = NEG_BIG;
+    lrot[h] = 0.f;
+    a[h][0] = a[h][1] = a[h][2] = a[h][3] = 0.f;
+  }
+  for (int s = lane; s < nsplit; s += 32) {
+#pragma unroll
+    for (int h = 0; h < GH; ++h) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(ws + ((p0 + s) * G + hbase + h) * 2));
+      if (ml.y > 0.f) mrot[h] = fmaxf(mrot[h], ml.x);
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < GH; ++h) mrot[h] = warp_max(mrot[h]);
+  for (int s0 = 0; s0 < nsplit; s0 += 32) {
+    float f[GH];
+#pragma unroll
+    for (int h = 0; h < GH; ++h) {
+      f[h] = 0.f;
+      if (s0 + lane < nsplit) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(ws + ((p0 + s0 + lane) * G + hbase + h) * 2));
+        f[h] = ml.y > 0.f ? fast_exp2(ml.x - mrot[h]) : 0.f;
+        lrot[h] = fmaf(ml.y, f[h], lrot[h]);
+      }
+    }
+    const int cnt = min(32, nsplit - s0);
+#pragma unroll 4
+    for (int k = 0; k < cnt; ++k) {
+#pragma unroll
+      for (int h = 0; h < GH; ++h) {
+        const float fk = __shfl_sync(0xffffffffu, f[h], k);
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(ws_acc + ((p0 + s0 + k) * G + hbase + h) * D) + lane);
+        a[h][0] = fmaf(v.x, fk, a[h][0]);
+        a[h][1] = fmaf(v.y, fk, a[h][1]);
+        a[h][2] = fmaf(v.z, fk, a[h][2]);
+        a[h][3] = fmaf(v.w, fk, a[h][3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < GH; ++h) {
+    const float lr = warp_sum(lrot[h]);
+    fwht128_warp(a[h], lane);
+    const float2 mlw = __ldcg(reinterpret_cast<const float2*>(ws + ((p0 + nsplit) * G + hbase + h) * 2));
+    const float4 aw = __ldcg(reinterpret_cast<const float4*>(ws_acc + ((p0 + nsplit) * G + hbase + h) * D) + lane);
+    const float mw = mlw.y > 0.f ? mlw.x : NEG_BIG, lw = mlw.y;
+    const float mt = fmaxf(mrot[h], mw);
+    const float fa = lr > 0.f ? fast_exp2(mrot[h] - mt) : 0.f;
+    const float fr = lw > 0.f ? fast_exp2(mw - mt) : 0.f;
+    const float den = lr * fa + lw * fr;
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    float4 o;
+    o.x = (a[h][0] * INV_SQRT_D * fa + aw.x * fr) * inv;
+    o.y = (a[h][1] * INV_SQRT_D * fa + aw.y * fr) * inv;
+    o.z = (a[h][2] * INV_SQRT_D * fa + aw.z * fr) * inv;
+    o.w = (a[h][3] * INV_SQRT_D * fa + aw.w * fr) * inv;
+    *reinterpret_cast<float4*>(out_rows + (int64_t)h * D + 4 * lane) = o;
+  }
+}
+
+// One warp = one split of one (sequence, head group); GH <= 4 query heads per
+// warp (a group of 8 runs as two head groups).  A split is a contiguous range of
+// 128-token blocks; the last split of a sequence also attends the residual window.
+// The warp that completes a (sequence, head group) last merges its partials into
+// the output, so one launch does the whole decode.
+//
+// Scores:  S[t][c] = sum_k u_hat[t][k] Qc[k][c]   M = 16 tokens, N = 8 columns, K = 16
+//          (columns 0-3: fp16(q~) of the GH heads, 4-7: their fp16 rounding residual),
+//          accumulated in two independent chains (even and odd k-steps).
+//          A lane swap (xor 2) adds the two halves so that lane (g, p) holds the
+//          scores of token g + 8 (p >> 1) for heads 2 (p & 1), 2 (p & 1) + 1.
+// Values:  O^T[d][h] += sum_t u_hat_v[t][d] w[t][h]  M = 16 dims, N = 8 heads, K = 16 tokens;
+//          the B operand is the weight matrix moved into place with movmatrix.trans.
+template <int GH, int MK, int MV>
+__global__ void __launch_bounds__(32 * DEC_WARPS, 1)
+decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb, int64_t qsh,
+              float qscale, const float* __restrict__ cbk_g, const float* __restrict__ cbv_g,
+              unsigned int* __restrict__ counters, float* __restrict__ ws, float* __restrict__ out, int n_q_heads,
+              DecodeGeom geom) {
+  static_assert(GH == 1 || GH == 2 || GH == 4, "1, 2 or 4 heads per warp");
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, p = lane & 3;
+  const int G = geom.g;           // query heads per kv-head
+  const int ngroups = G / GH;     // head groups per kv-head
+  const int nsplit = geom.nsplit_q;
+
+  // ---- stage the replicated fp16 codebooks (whole CTA, once) ----
+  for (int e = tid; e < NCODES * 8; e += blockDim.x) {
+    const int c = e >> 3, r = e & 7;
+    sm.cbk[c][r] = cb_row_f16(cbk_g, c);
+    sm.cbv[c][r] = cb_row_f16(cbv_g, c);
+  }
+  if (lane == 0) {
+    mbar_init(smem_addr(&sm.bar[warp][0]), 1);
+    mbar_init(smem_addr(&sm.bar[warp][1]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+
+  const int nseq = kc.batch * kc.n_kv_heads;
+  const int gw = blockIdx.x * DEC_WARPS + warp;  // global warp job id
+  if (gw >= nseq * nsplit * ngroups) return;
+  const int hg = gw % ngroups;
+  const int64_t seq = (gw / ngroups) / nsplit;
+  const int split = (gw / ngroups) % nsplit;
+  const int b = (int)(seq / kc.n_kv_heads), hk = (int)(seq % kc.n_kv_heads);
+  const int hbase = hg * GH;                      // first head of the group within the kv-head
+  const int64_t p0 = seq * (nsplit + 1);          // first partial slot of the sequence
+  const int64_t P = (int64_t)nseq * (nsplit + 1);
+  float* ws_acc = ws + acc_offset(P, G);
+  const int64_t q_off = (int64_t)b * qsb + (int64_t)(hk * G + hbase) * qsh;
+
+  const int nq = min(min(kc.n_quant[seq], vc.n_quant[seq]), kc.capacity);
+  const int nw = (kc.window_len > 0) ? max(0, min(min(kc.n_window[seq], vc.n_window[seq]), kc.window_len)) : 0;
+  const int nblk = (nq + BLK - 1) / BLK;
+  const int bps = max(1, (nblk + (nw > 0 ? WINDOW_COST_BLOCKS : 0) + nsplit - 1) / nsplit);  // blocks per split
+  const int tok_begin = min(nq, split * bps * BLK);
+  const int tok_end = min(nq, (split + 1) * bps * BLK);
+  const bool has_window = split == nsplit - 1;
+  const uint32_t st_base = smem_addr(&sm.stage[warp][0][0]);
+  const uint32_t mb_base = smem_addr(&sm.means[warp][0][0]);
+  const uint32_t bar0 = smem_addr(&sm.bar[warp][0]);
+  const int nstages = (tok_end - tok_begin + STAGE_TOK - 1) / STAGE_TOK;
+
+  if (lane == 0 && nstages > 0) {
+    issue_stage<MK, MV>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc, seq,
+                        tok_begin, true);
+    if (nstages > 1)
+      issue_stage<MK, MV>(st_base + STAGE_BYTES, mb_base, bar0 + 8, kc, vc, seq, tok_begin + STAGE_TOK, false);
+  }
+
+  // ---- query operand (B of the score product), built while the copies fly ----
+  uint32_t qb[8][2];
+  build_q_operand<GH>(qb, q, dtype, q_off, qsh, qscale * INV_SQRT_D, true, lane);
 
   const uint32_t lane_row = (uint32_t)(lane & 7) * 16u;
   const uint32_t cbk_base = smem_addr(&sm.cbk[0][0]) + lane_row;
@@ -327,19 +498,22 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
   const int h0 = 2 * (p & 1);                      // its two heads: h0, h0 + 1 (within the group)
   // Padding heads get a running max of +1e30: their weights are exactly 0 and they
   // never trigger a re-base.
-  float m0 = h0 < GH ? NEG_BIG : -NEG_BIG, m1 = h0 + 1 < GH ? NEG_BIG : -NEG_BIG;
-  float l0 = 0.f, l1 = 0.f, cm0 = 0.f, cm1 = 0.f, qo0 = 0.f, qo1 = 0.f;
-  float O[8][4];
+  const float m_init0 = h0 < GH ? NEG_BIG : -NEG_BIG, m_init1 = h0 + 1 < GH ? NEG_BIG : -NEG_BIG;
+  SoftmaxState sx;
+  sx.m0 = m_init0; sx.m1 = m_init1; sx.l0 = sx.l1 = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
+  for (int i = 0; i < 8; ++i) sx.O[i][0] = sx.O[i][1] = sx.O[i][2] = sx.O[i][3] = 0.f;
+  float cm0 = 0.f, cm1 = 0.f, qo0 = 0.f, qo1 = 0.f;
   uint32_t phase = 0u;
   bool failed = false;
+  int pending = 0;  // buffers whose copy may still be in flight when a wait gives up (bit per buffer)
 
   for (int st = 0; st < nstages; ++st) {
     const int buf = st & 1;
     const bool arrived = mbar_wait(bar0 + 8u * buf, (phase >> buf) & 1u);
     if (!__all_sync(0xffffffffu, arrived)) {
       failed = true;
+      pending = (1 << buf) | (st + 1 < nstages ? (1 << (buf ^ 1)) : 0);
       break;
     }
     phase ^= 1u << buf;
@@ -385,8 +559,8 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
       }
       const uint32_t vnw = *reinterpret_cast<const uint32_t*>(sb + ST_VN + (tt + t_l) * 4);
 
-      // ---- scores: 8 k-steps of 16 dims ----
-      float S[4] = {0.f, 0.f, 0.f, 0.f};
+      // ---- scores: 8 k-steps of 16 dims in two independent accumulation chains ----
+      float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const uint32_t code = __byte_perm(u4_word(kcw, j >> 1), 0u, (j & 1) ? sel_k1 : sel_k0);
@@ -398,8 +572,11 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
           aa[2] = apply_signs(aa[2], ks0, 2 * j + 1);
           aa[3] = apply_signs(aa[3], ks1, 2 * j + 1);
         }
-        mma_full(S, aa, qb[j][0], qb[j][1]);
+        if (j & 1) mma_full(S2, aa, qb[j][0], qb[j][1]);
+        else mma_full(S, aa, qb[j][0], qb[j][1]);
       }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) S[i] += S2[i];
       // hi + lo columns -> (token t_l, heads h0, h0 + 1)
       const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[2] : S[0], 2);
       const float r1 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[3] : S[1], 2);
@@ -408,29 +585,17 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
 
       // ---- scores with the NSN byproducts; online softmax (lazy re-basing) ----
       const float2 kn = __half22float2(*reinterpret_cast<const __half2*>(&knw));
-      const float2 vn = __half22float2(*reinterpret_cast<const __half2*>(&vnw));
+      float2 vn = __half22float2(*reinterpret_cast<const __half2*>(&vnw));
       float sc0 = kn.x * fmaf(kn.y, d0, qo0);
       float sc1 = kn.x * fmaf(kn.y, d1, qo1);
-      if (!full && t_stage + tt + t_l >= tok_end) sc0 = sc1 = NEG_BIG;
-      if (__any_sync(0xffffffffu, fmaxf(sc0 - m0, sc1 - m1) > LAZY_MAX_SLACK)) {
-        float t0 = sc0, t1 = sc1;
-#pragma unroll
-        for (int x = 2; x < 32; x <<= 1) {  // lanes sharing the head pair: xor 2, 4, 8, 16
-          t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, x));
-          t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, x));
-        }
-        const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
-        const float c0 = fast_exp2(m0 - n0), c1 = fast_exp2(m1 - n1);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          O[i][0] *= c0; O[i][1] *= c1; O[i][2] *= c0; O[i][3] *= c1;
-        }
-        l0 *= c0; l1 *= c1; cm0 *= c0; cm1 *= c1;
-        m0 = n0; m1 = n1;
+      if (!full && t_stage + tt + t_l >= tok_end) {  // past the end: no weight, and no stale norms
+        sc0 = sc1 = NEG_BIG;
+        vn = make_float2(0.f, 0.f);
       }
-      const float pr0 = fast_exp2(sc0 - m0), pr1 = fast_exp2(sc1 - m1);
-      l0 += pr0;
-      l1 += pr1;
+      lazy_update(sx, sc0, sc1, cm0, cm1);
+      const float pr0 = fast_exp2(sc0 - sx.m0), pr1 = fast_exp2(sc1 - sx.m1);
+      sx.l0 += pr0;
+      sx.l1 += pr1;
       cm0 = fmaf(pr0, vn.x, cm0);
       cm1 = fmaf(pr1, vn.x, cm1);
       const float s12 = vn.x * vn.y;
@@ -451,7 +616,7 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
           aa[2] = apply_signs(aa[2], W1, 2 * mm);
           aa[3] = apply_signs(aa[3], W1, 2 * mm + 1);
         }
-        mma_full(O[mm], aa, pb0, pb1);
+        mma_full(sx.O[mm], aa, pb0, pb1);
       }
     }
 
@@ -468,10 +633,10 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
       for (int mm = 0; mm < 8; ++mm) {
         const float oa = __half2float(ov[16 * mm + g]);
         const float ob = __half2float(ov[16 * mm + 8 + g]);
-        O[mm][0] = fmaf(oa, c0, O[mm][0]);
-        O[mm][1] = fmaf(oa, c1, O[mm][1]);
-        O[mm][2] = fmaf(ob, c0, O[mm][2]);
-        O[mm][3] = fmaf(ob, c1, O[mm][3]);
+        sx.O[mm][0] = fmaf(oa, c0, sx.O[mm][0]);
+        sx.O[mm][1] = fmaf(oa, c1, sx.O[mm][1]);
+        sx.O[mm][2] = fmaf(ob, c0, sx.O[mm][2]);
+        sx.O[mm][3] = fmaf(ob, c1, sx.O[mm][3]);
       }
       cm0 = cm1 = 0.f;
     }
@@ -482,177 +647,90 @@ decode_split_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int 
                           bar0 + 8u * buf, kc, vc, seq, tn, (tn % BLK) == 0);
     }
   }
-  if (failed) {
-    if (lane == 0 && kc.status) atomicOr(kc.status, 2);
-    mbar_wait(bar0 + 8u, (phase >> 1) & 1u);
-  }
-#pragma unroll
-  for (int x = 2; x < 32; x <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, x);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, x);
-  }
+  store_partial<GH>(sx, ws, ws_acc, p0 + split, G, hbase, lane);
 
-  // ---- this warp's partial: lanes p < 2 own heads 2p, 2p + 1 of the group ----
-  if (lo_lane) {
+  // ---- residual window (original domain), last split only ----
+  if (has_window) {
+    sx.m0 = m_init0; sx.m1 = m_init1; sx.l0 = sx.l1 = 0.f;
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int h = 2 * p + hh;
-      if (h < GH) {
-        float* dst = ws_acc + (pidx * G + hbase + h) * D;
+    for (int i = 0; i < 8; ++i) sx.O[i][0] = sx.O[i][1] = sx.O[i][2] = sx.O[i][3] = 0.f;
+    const int nch = failed ? 0 : (nw + WCHUNK - 1) / WCHUNK;
+    if (nch > 0) {
+      const __half* kw0 = kc.window + seq * kc.window_len * D;
+      const __half* vw0 = vc.window + seq * vc.window_len * D;
+      issue_window_chunk(st_base, bar0, kw0, vw0, min(WCHUNK, nw), lane);
+      if (nch > 1) issue_window_chunk(st_base + STAGE_BYTES, bar0 + 8u, kw0 + WCHUNK * D, vw0 + WCHUNK * D,
+                                      min(WCHUNK, nw - WCHUNK), lane);
+      build_q_operand<GH>(qb, q, dtype, q_off, qsh, qscale, false, lane);
+      const int wr = lane & 7;  // ldmatrix row (token) of this lane; rows 8-15 repeat rows 0-7
+      for (int c = 0; c < nch; ++c) {
+        const int buf = c & 1;
+        const bool arrived = mbar_wait(bar0 + 8u * buf, (phase >> buf) & 1u);
+        if (!__all_sync(0xffffffffu, arrived)) {
+          failed = true;
+          pending = (1 << buf) | (c + 1 < nch ? (1 << (buf ^ 1)) : 0);
+          break;
+        }
+        phase ^= 1u << buf;
+        const int rows = min(WCHUNK, nw - c * WCHUNK);
+        const uint32_t kbuf = st_base + (uint32_t)(buf * STAGE_BYTES);
+        const uint32_t vbuf = kbuf + (uint32_t)WC_V;
+        const uint32_t rowoff = (uint32_t)(min(wr, rows - 1) * WROWB);
+        float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint32_t aa[4];
+          ldsm_x4(kbuf + rowoff + (uint32_t)(32 * j + 16 * (lane >> 4)), aa);
+          if (j & 1) mma_full(S2, aa, qb[j][0], qb[j][1]);
+          else mma_full(S, aa, qb[j][0], qb[j][1]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) S[i] += S2[i];
+        const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[2] : S[0], 2);
+        const float r1 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[3] : S[1], 2);
+        float sc0 = (lo_lane ? S[0] : S[2]) + r0;
+        float sc1 = (lo_lane ? S[1] : S[3]) + r1;
+        if (t_l >= rows) sc0 = sc1 = NEG_BIG;  // tokens 8-15 of the tile and rows past the window
+        float unused0 = 0.f, unused1 = 0.f;
+        lazy_update(sx, sc0, sc1, unused0, unused1);
+        const float pr0 = fast_exp2(sc0 - sx.m0), pr1 = fast_exp2(sc1 - sx.m1);
+        sx.l0 += pr0;
+        sx.l1 += pr1;
+        const uint32_t wpk = pack_half2(pr0, pr1);
+        const uint32_t pb0 = movmatrix_t(lo_lane ? wpk : 0u);  // tokens 0-7; tokens 8-15 weigh 0
 #pragma unroll
         for (int mm = 0; mm < 8; ++mm) {
-          dst[16 * mm + g] = O[mm][hh];
-          dst[16 * mm + 8 + g] = O[mm][2 + hh];
+          uint32_t aa[4];
+          ldsm_x4_t(vbuf + rowoff + (uint32_t)(32 * mm + 16 * ((lane >> 3) & 1)), aa);
+          mma_full(sx.O[mm], aa, pb0, 0u);
+        }
+        __syncwarp();
+        if (c + 2 < nch) {
+          const int t2 = (c + 2) * WCHUNK;
+          issue_window_chunk(kbuf, bar0 + 8u * buf, kw0 + t2 * D, vw0 + t2 * D, min(WCHUNK, nw - t2), lane);
         }
       }
     }
-    if (g == 0) {
-      if (h0 < GH) {
-        partial_ml(ws, pidx, G, hbase + h0)[0] = m0;
-        partial_ml(ws, pidx, G, hbase + h0)[1] = l0;
-      }
-      if (h0 + 1 < GH) {
-        partial_ml(ws, pidx, G, hbase + h0 + 1)[0] = m1;
-        partial_ml(ws, pidx, G, hbase + h0 + 1)[1] = l1;
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Residual window + combine: grid (kv-heads, batch), one warp per query head of
-// the group.  The window's K and V rows (fp16, original domain) are staged in
-// shared memory with coalesced loads; each warp scores them against its head,
-// merges the split partials of the quantized part (log-sum-exp), applies H to
-// their rotated value sum (H^T = H) and normalises both parts together.
-// Lane l owns dims 4l..4l+3.
-// ---------------------------------------------------------------------------
-constexpr int WROW = D + 8;  // padded fp16 row of the staged window (272 B: conflict-free row reads)
-
-template <int G>
-__global__ void __launch_bounds__(32 * G)
-decode_window_combine_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb,
-                             int64_t qsh, float qscale, const float* __restrict__ ws, float* __restrict__ out,
-                             int n_q_heads, DecodeGeom geom) {
-  extern __shared__ __align__(16) unsigned char wsm_raw[];
-  __half* kwin = reinterpret_cast<__half*>(wsm_raw);             // [BLK][WROW]
-  __half* vwin = kwin + BLK * WROW;                               // [BLK][D]
-  float* qp = reinterpret_cast<float*>(vwin + BLK * D);           // [G][D]
-  float* pw = qp + G * D;                                         // [G][BLK]
-  const int hk = blockIdx.x, b = blockIdx.y, h = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t seq = (int64_t)b * kc.n_kv_heads + hk;
-  const int hq = hk * G + h;
-  const int nslots = geom.nsplit_q + 1;
-  const int64_t P = (int64_t)kc.batch * kc.n_kv_heads * nslots;
-  const float* ws_acc = ws + acc_offset(P, G);
-  const int64_t p0 = seq * nslots;
-  const int nw = (kc.window_len > 0) ? min(min(kc.n_window[seq], vc.n_window[seq]), kc.window_len) : 0;
-
-  // ---- stage the window rows (coalesced 16-byte loads) and this head's query ----
-  if (nw > 0) {
-    const uint4* ksrc = reinterpret_cast<const uint4*>(kc.window + seq * kc.window_len * D);
-    const uint4* vsrc = reinterpret_cast<const uint4*>(vc.window + seq * vc.window_len * D);
-    for (int e = threadIdx.x; e < nw * (D / 8); e += blockDim.x) {
-      const int row = e >> 4, ch = e & 15;
-      *reinterpret_cast<uint4*>(kwin + row * WROW + ch * 8) = __ldg(ksrc + e);
-      *reinterpret_cast<uint4*>(vwin + row * D + ch * 8) = __ldg(vsrc + e);
-    }
-    const int64_t off = (int64_t)b * qsb + (int64_t)hq * qsh + 4 * lane;
-    float v[4];
-    if (dtype == NSN_DTYPE_F32) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(q) + off));
-      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-    } else {
-      const uint2 r = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(q) + off));
-      float2 a2, c2;
-      if (dtype == NSN_DTYPE_BF16) {
-        a2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-        c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-      } else {
-        a2 = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
-        c2 = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
-      }
-      v[0] = a2.x; v[1] = a2.y; v[2] = c2.x; v[3] = c2.y;
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) qp[h * D + 4 * lane + i] = v[i] * qscale;
-  }
-  __syncthreads();
-
-  // ---- window scores of this head (original domain, log2 units) ----
-  float mw = NEG_BIG, lw = 0.f, aw[4] = {0.f, 0.f, 0.f, 0.f};
-  if (nw > 0) {
-    float sc[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = lane + 32 * i;
-      float acc0 = 0.f, acc1 = 0.f;
-      if (t < nw) {
-        const __half* row = kwin + t * WROW;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 r = *reinterpret_cast<const uint4*>(row + 8 * c);
-          const __half2* hv = reinterpret_cast<const __half2*>(&r);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f = __half22float2(hv[k]);
-            acc0 = fmaf(qp[h * D + 8 * c + 2 * k], f.x, acc0);
-            acc1 = fmaf(qp[h * D + 8 * c + 2 * k + 1], f.y, acc1);
-          }
-        }
-      }
-      sc[i] = t < nw ? acc0 + acc1 : NEG_BIG;
-      mw = fmaxf(mw, sc[i]);
-    }
-    mw = warp_max(mw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float pr = (lane + 32 * i < nw) ? fast_exp2(sc[i] - mw) : 0.f;
-      pw[h * BLK + lane + 32 * i] = pr;
-      lw += pr;
-    }
-    lw = warp_sum(lw);
-    __syncwarp();
-#pragma unroll 8
-    for (int t = 0; t < nw; ++t) {
-      const float pr = pw[h * BLK + t];
-      const uint2 r = *reinterpret_cast<const uint2*>(vwin + t * D + 4 * lane);
-      const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
-      const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
-      aw[0] = fmaf(pr, x0.x, aw[0]); aw[1] = fmaf(pr, x0.y, aw[1]);
-      aw[2] = fmaf(pr, x1.x, aw[2]); aw[3] = fmaf(pr, x1.y, aw[3]);
-    }
+    store_partial<GH>(sx, ws, ws_acc, p0 + nsplit, G, hbase, lane);
   }
 
-  // ---- quantized part: merge the split partials, rotate back ----
-  float mrot = NEG_BIG;
-  for (int s = 0; s < geom.nsplit_q; ++s) mrot = fmaxf(mrot, ws[((p0 + s) * G + h) * 2]);
-  float lrot = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-  for (int s = 0; s < geom.nsplit_q; ++s) {
-    const float2 ml = *reinterpret_cast<const float2*>(ws + ((p0 + s) * G + h) * 2);
-    const float f = ml.y > 0.f ? fast_exp2(ml.x - mrot) : 0.f;
-    lrot = fmaf(ml.y, f, lrot);
-    const float4 v = *reinterpret_cast<const float4*>(ws_acc + ((p0 + s) * G + h) * D + 4 * lane);
-    a[0] = fmaf(v.x, f, a[0]); a[1] = fmaf(v.y, f, a[1]); a[2] = fmaf(v.z, f, a[2]); a[3] = fmaf(v.w, f, a[3]);
+  if (failed) {
+    if (lane == 0 && kc.status) atomicOr(kc.status, 2);
+    // let copies that may still be in flight land before the CTA can exit
+    if (pending & 1) mbar_wait(bar0, phase & 1u);
+    if (pending & 2) mbar_wait(bar0 + 8u, (phase >> 1) & 1u);
   }
-  fwht128_warp(a, lane);
-  const float mt = fmaxf(mrot, mw);
-  const float fa = lrot > 0.f ? fast_exp2(mrot - mt) : 0.f;
-  const float fr = lw > 0.f ? fast_exp2(mw - mt) : 0.f;
-  const float den = lrot * fa + lw * fr;
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-  float4 o;
-  o.x = (a[0] * INV_SQRT_D * fa + aw[0] * fr) * inv;
-  o.y = (a[1] * INV_SQRT_D * fa + aw[1] * fr) * inv;
-  o.z = (a[2] * INV_SQRT_D * fa + aw[2] * fr) * inv;
-  o.w = (a[3] * INV_SQRT_D * fa + aw[3] * fr) * inv;
-  *reinterpret_cast<float4*>(out + ((int64_t)b * n_q_heads + hq) * D + 4 * lane) = o;
-}
 
-template <int G>
-constexpr size_t window_smem_bytes() {
-  return (size_t)BLK * WROW * 2 + (size_t)BLK * D * 2 + (size_t)G * D * 4 + (size_t)G * BLK * 4;
+  // ---- the last warp of this (sequence, head group) merges the partials ----
+  __threadfence();  // this warp's partial stores are visible device-wide ...
+  __syncwarp();      // ... for every lane before lane 0 takes the ticket
+  unsigned int ticket = 0u;
+  if (lane == 0) ticket = atomicInc(&counters[seq * ngroups + hg], (unsigned int)(nsplit - 1));
+  ticket = __shfl_sync(0xffffffffu, ticket, 0);
+  if (ticket != (unsigned int)(nsplit - 1)) return;
+  __threadfence();
+  merge_partials<GH>(ws, ws_acc, p0, nsplit, G, hbase,
+                     out + ((int64_t)b * n_q_heads + hk * G + hbase) * D, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -686,61 +764,67 @@ DecodeGeom decode_geometry(int batch, int capacity, int n_q_heads, int n_kv_head
   return g;
 }
 
-size_t decode_workspace_bytes(int batch, int n_kv_heads, const DecodeGeom& geom) {
+// Merge counters: two 32-bit words per (batch, kv-head) (one per head group),
+// padded to 256 bytes.
+static int64_t counter_words(int64_t nseq) { return ((2 * nseq + 63) / 64) * 64; }
+
+size_t decode_partial_bytes(int batch, int n_kv_heads, const DecodeGeom& geom) {
   const int64_t P = (int64_t)batch * n_kv_heads * (geom.nsplit_q + 1);
   return (size_t)(acc_offset(P, geom.g) + P * geom.g * D) * sizeof(float);
 }
 
+size_t decode_workspace_bytes(int batch, int n_kv_heads, const DecodeGeom& geom) {
+  return (size_t)counter_words((int64_t)batch * n_kv_heads) * 4u + decode_partial_bytes(batch, n_kv_heads, geom);
+}
+
 template <int G, int MK, int MV>
-static cudaError_t launch_split_t(const CacheView& kc, const CacheView& vc, const float* cbk, const float* cbv,
-                                  const void* q, int dtype, int64_t qsb, int64_t qsh, float qscale, float* ws,
-                                  const DecodeGeom& geom, cudaStream_t s) {
+static cudaError_t launch_t(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                            int64_t qsb, int64_t qsh, float qscale, const float* cbk, const float* cbv, float* out,
+                            unsigned int* counters, float* partials, const DecodeGeom& geom, cudaStream_t s) {
   constexpr int GH = G < 4 ? G : 4;  // heads per warp job
   const size_t smem = sizeof(DecSmem);
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<GH, MK, MV>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<GH, MK, MV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   const int nwarps = kc.batch * kc.n_kv_heads * geom.nsplit_q * (G / GH);
   dim3 grid((nwarps + DEC_WARPS - 1) / DEC_WARPS);
-  decode_split_kernel<GH, MK, MV><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv,
-                                                                    ws, geom);
+  decode_kernel<GH, MK, MV><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv,
+                                                               counters, partials, out, n_q_heads, geom);
   return cudaGetLastError();
 }
 
 template <int G>
 static cudaError_t launch_g(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
                             int64_t qsb, int64_t qsh, float qscale, const float* cbk, const float* cbv, float* out,
-                            float* ws, const DecodeGeom& geom, cudaStream_t s) {
-  cudaError_t e;
+                            unsigned int* counters, float* partials, const DecodeGeom& geom, cudaStream_t s) {
   if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_1BIT)
-    e = launch_split_t<G, 1, 1>(kc, vc, cbk, cbv, q, dtype, qsb, qsh, qscale, ws, geom, s);
-  else if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_2BIT)
-    e = launch_split_t<G, 1, 2>(kc, vc, cbk, cbv, q, dtype, qsb, qsh, qscale, ws, geom, s);
-  else if (kc.mode == NSN_MODE_2BIT && vc.mode == NSN_MODE_1BIT)
-    e = launch_split_t<G, 2, 1>(kc, vc, cbk, cbv, q, dtype, qsb, qsh, qscale, ws, geom, s);
-  else
-    e = launch_split_t<G, 2, 2>(kc, vc, cbk, cbv, q, dtype, qsb, qsh, qscale, ws, geom, s);
-  if (e != cudaSuccess) return e;
-  dim3 g2(kc.n_kv_heads, kc.batch);
-  const size_t wsmem = window_smem_bytes<G>();
-  e = cudaFuncSetAttribute(decode_window_combine_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem);
-  if (e != cudaSuccess) return e;
-  decode_window_combine_kernel<G><<<g2, 32 * G, wsmem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, ws, out, n_q_heads,
-                                                            geom);
-  return cudaGetLastError();
+    return launch_t<G, 1, 1>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+  if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_2BIT)
+    return launch_t<G, 1, 2>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+  if (kc.mode == NSN_MODE_2BIT && vc.mode == NSN_MODE_1BIT)
+    return launch_t<G, 2, 1>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+  return launch_t<G, 2, 2>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+}
+
+static cudaError_t launch_any(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                              int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
+                              float* out, unsigned int* counters, float* partials, const DecodeGeom& geom,
+                              cudaStream_t s) {
+  const float qscale = softmax_scale * LOG2E;
+  switch (geom.g) {
+    case 1: return launch_g<1>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+    case 2: return launch_g<2>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+    case 4: return launch_g<4>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+    default: return launch_g<8>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+  }
 }
 
 cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
                           int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
                           float* out, void* ws, const DecodeGeom& geom, cudaStream_t s) {
-  const float qscale = softmax_scale * LOG2E;
-  float* w = static_cast<float*>(ws);
-  switch (geom.g) {
-    case 1: return launch_g<1>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
-    case 2: return launch_g<2>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
-    case 4: return launch_g<4>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
-    default: return launch_g<8>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, w, geom, s);
-  }
+  unsigned int* counters = static_cast<unsigned int*>(ws);
+  float* partials = static_cast<float*>(ws) + counter_words((int64_t)kc.batch * kc.n_kv_heads);
+  return launch_any(kc, vc, q, dtype, n_q_heads, qsb, qsh, softmax_scale, cbk, cbv, out, counters, partials, geom, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -749,41 +833,55 @@ cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* 
 // memory-pool callback, processes whose device memory is fully reserved up
 // front by a framework, or embedded hosts that forbid cudaMalloc after start-up.
 // For them the decode partials live in this fixed file-scope device array
-// instead of a caller-provided workspace.  Every GPU that loads the library
-// holds the array until the process exits.  All calls share it, so two such
-// calls that overlap on the GPU (different streams, no ordering) race on it.
-// The kernels write every partial they later read, so nothing needs clearing
-// between calls.
+// instead of a caller-provided workspace, and the merge counters in a second
+// one.  Every GPU that loads the library holds both until the process exits.
+// All calls share them, so two such calls that overlap on the GPU (different
+// streams, no ordering) race on them.  The kernel writes every partial it later
+// reads, and each completed call leaves every counter it used at zero (both
+// arrays start zero-filled), so nothing needs clearing between calls.
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_decode_scratch[NSN_DECODE_SCRATCH_BYTES];
+static __device__ __align__(256) unsigned int g_decode_counters[NSN_DECODE_STATIC_COUNTERS];
 
-// Device address of the scratch array for the current device.  Resolved once per
+bool decode_static_fits(int batch, int n_kv_heads, const DecodeGeom& geom) {
+  return decode_partial_bytes(batch, n_kv_heads, geom) <= (size_t)NSN_DECODE_SCRATCH_BYTES &&
+         2 * (int64_t)batch * n_kv_heads <= (int64_t)NSN_DECODE_STATIC_COUNTERS;
+}
+
+// Device addresses of the two arrays for the current device.  Resolved once per
 // device (cudaGetSymbolAddress with that device current) and cached.
-static cudaError_t decode_scratch_ptr(void** out) {
+static cudaError_t decode_static_ptrs(void** scratch, void** counters) {
   static std::mutex mu;
-  static void* ptrs[64] = {};
+  static void* ptrs[64][2] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
+  if (!ptrs[dev][0]) {
     void* p = nullptr;
+    void* c = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    ptrs[dev] = p;
+    e = cudaGetSymbolAddress(&c, g_decode_counters);
+    if (e != cudaSuccess) return e;
+    ptrs[dev][0] = p;
+    ptrs[dev][1] = c;
   }
-  *out = ptrs[dev];
+  *scratch = ptrs[dev][0];
+  *counters = ptrs[dev][1];
   return cudaSuccess;
 }
 
 cudaError_t launch_decode_static(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
                                  int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
                                  float* out, const DecodeGeom& geom, cudaStream_t s) {
-  void* ws = nullptr;
-  const cudaError_t e = decode_scratch_ptr(&ws);
+  void* scratch = nullptr;
+  void* counters = nullptr;
+  const cudaError_t e = decode_static_ptrs(&scratch, &counters);
   if (e != cudaSuccess) return e;
-  return launch_decode(kc, vc, q, dtype, n_q_heads, qsb, qsh, softmax_scale, cbk, cbv, out, ws, geom, s);
+  return launch_any(kc, vc, q, dtype, n_q_heads, qsb, qsh, softmax_scale, cbk, cbv, out,
+                    static_cast<unsigned int*>(counters), static_cast<float*>(scratch), geom, s);
 }
 
 }  // namespace nsn

@@ -189,9 +189,8 @@ nsn_status nsn_decode_attention_static(const nsn_cache* k_cache, const nsn_cache
   if (q_stride_b < 0 || q_stride_h < 0 || q_stride_b % e16 || q_stride_h % e16) return NSN_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return NSN_ERR_INVALID_ARG;
   const nsn::DecodeGeom geom = nsn::decode_geometry(k_cache->batch, k_cache->capacity, n_q_heads, k_cache->n_kv_heads);
-  // the partials of this shape must fit in the fixed scratch array
-  if (nsn::decode_workspace_bytes(k_cache->batch, k_cache->n_kv_heads, geom) > (size_t)NSN_DECODE_SCRATCH_BYTES)
-    return NSN_ERR_WORKSPACE;
+  // the partials and counters of this shape must fit in the fixed arrays
+  if (!nsn::decode_static_fits(k_cache->batch, k_cache->n_kv_heads, geom)) return NSN_ERR_WORKSPACE;
   return cuda_status(nsn::launch_decode_static(view(k_cache), view(v_cache), q, dtype, n_q_heads, q_stride_b,
                                                q_stride_h, softmax_scale, cb_k, cb_v, out, geom,
                                                static_cast<cudaStream_t>(stream)));

@@ -68,15 +68,16 @@ __device__ __forceinline__ uint4 pack8_f16(const float* v) {
 }
 
 // ---------------------------------------------------------------------------
-// Unnormalized Walsh-Hadamard transform of 128 values held in registers by one
-// thread: w_i = sum_j (-1)^popcount(i & j) v_j (Sylvester / natural order).
-// Seven butterfly stages with compile-time strides, so every index is a
-// constant and the array stays in registers.
+// Unnormalized Walsh-Hadamard transform, w_i = sum_j (-1)^popcount(i & j) v_j
+// (Sylvester / natural order), of 128 values held by a pair of adjacent lanes:
+// lane 2k + h holds elements 64h .. 64h+63 in v[0..63].  Six butterfly stages in
+// registers (compile-time strides, so the array stays in registers), then the
+// stride-64 stage across the pair with one shuffle per element.
 // ---------------------------------------------------------------------------
 template <int H>
-__device__ __forceinline__ void fwht_stage(float* v) {
+__device__ __forceinline__ void fwht64_stage(float* v) {
 #pragma unroll
-  for (int i = 0; i < D; i += 2 * H) {
+  for (int i = 0; i < D / 2; i += 2 * H) {
 #pragma unroll
     for (int j = 0; j < H; ++j) {
       const float a = v[i + j], b = v[i + j + H];
@@ -86,14 +87,18 @@ __device__ __forceinline__ void fwht_stage(float* v) {
   }
 }
 
-__device__ __forceinline__ void fwht128_regs(float* v) {
-  fwht_stage<1>(v);
-  fwht_stage<2>(v);
-  fwht_stage<4>(v);
-  fwht_stage<8>(v);
-  fwht_stage<16>(v);
-  fwht_stage<32>(v);
-  fwht_stage<64>(v);
+__device__ __forceinline__ void fwht128_pair(float* v, int h) {
+  fwht64_stage<1>(v);
+  fwht64_stage<2>(v);
+  fwht64_stage<4>(v);
+  fwht64_stage<8>(v);
+  fwht64_stage<16>(v);
+  fwht64_stage<32>(v);
+#pragma unroll
+  for (int i = 0; i < D / 2; ++i) {
+    const float o = __shfl_xor_sync(0xffffffffu, v[i], 1);
+    v[i] = h ? (o - v[i]) : (v[i] + o);  // (a + b, a - b) with a in the low half
+  }
 }
 
 // Unnormalized WHT of 128 values spread over a warp, lane l holding elements

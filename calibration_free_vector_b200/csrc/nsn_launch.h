@@ -31,7 +31,11 @@ struct DecodeGeom {
 };
 
 DecodeGeom decode_geometry(int batch, int capacity, int n_q_heads, int n_kv_heads);
+// Workspace = merge counters (zero at rest) followed by the partials.
 size_t decode_workspace_bytes(int batch, int n_kv_heads, const DecodeGeom& geom);
+size_t decode_partial_bytes(int batch, int n_kv_heads, const DecodeGeom& geom);
+// Whether a shape fits the allocation-free decode's fixed arrays.
+bool decode_static_fits(int batch, int n_kv_heads, const DecodeGeom& geom);
 
 size_t quant_smem_bytes();
 
@@ -45,7 +49,7 @@ cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* 
                           int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
                           float* out, void* ws, const DecodeGeom& geom, cudaStream_t s);
 
-// Same as launch_decode with the file-scope scratch array as the workspace.
+// Same as launch_decode with the file-scope arrays as the workspace.
 cudaError_t launch_decode_static(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
                                  int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
                                  float* out, const DecodeGeom& geom, cudaStream_t s);

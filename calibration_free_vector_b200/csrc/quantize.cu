@@ -5,8 +5,9 @@
 // 2 (Hadamard), 3 (VQ with one global codebook, adaptive scale) and 4 (KIVI-style
 // residual that is flushed into the quantized part when full).
 //
-// One CTA of 128 threads quantizes one block of <= 128 tokens of one (batch,
-// kv-head); thread t owns token t.  Per block:
+// One CTA of 256 threads quantizes one block of <= 128 tokens of one (batch,
+// kv-head); the adjacent lanes 2t, 2t+1 own token t (64 dims, 8 sub-vectors
+// each).  Per block:
 //   r      = column mean of the raw tokens (fp64 sum, stored as fp32)
 //   d_t    = FWHT(x_t - r)                 fp32, in registers (exact algebra:
 //   w_t    = d_t + FWHT(r)                 FWHT is linear; FWHT(r) in fp64)
@@ -39,6 +40,10 @@ __device__ __forceinline__ double lds_f64(const double* p) {
   return r;
 }
 
+constexpr int QTHREADS = 2 * BLK;  // two threads per token
+constexpr int HD = D / 2;           // dims per thread
+constexpr int HSUB = NSUB / 2;      // sub-vectors per thread
+
 struct QuantSmem {
   alignas(16) float cb[NCODES][SUB];   // codebook (fp32)
   alignas(16) float bias[NCODES];      // -||c_k||^2 / 2
@@ -48,13 +53,16 @@ struct QuantSmem {
   alignas(16) double s2[BLK];
   alignas(16) double big_r[D];         // FWHT(r) in fp64
   alignas(16) double o[D];             // D_c = mean_t(d_t,c rr_t) (the token-varying part of o)
+  alignas(16) double part[2][D];       // per-half column partial sums
+  alignas(16) double dev_part[2];      // per-half sums of rr_t - rr_0
   alignas(16) float r[D];              // column mean of raw tokens (fp32)
   alignas(16) float tile[BLK][D + 4];  // raw tokens, then d_t rows, then u rows; padded by 16 B
-  alignas(16) float thr[BLK][NSUB];    // per (token, sub-vector) threshold of the exact re-decision
+  alignas(16) float thr[BLK][NSUB + 1];  // per (token, sub-vector) threshold of the exact re-decision
   alignas(16) uint8_t code[BLK][NSUB]; // chosen codes
+  alignas(16) uint32_t sgn[BLK][4];    // packed sign bits (2-bit mode)
 };
 
-// Stages the codebook, its biases and norm bounds.  All 128 threads.
+// Stages the codebook, its biases and norm bounds.  All QTHREADS threads.
 __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook) {
   const int t = threadIdx.x;
   for (int i = t; i < NCODES * SUB / 4; i += blockDim.x)
@@ -69,11 +77,12 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
     my_max = fmaxf(my_max, s);
   }
   my_max = warp_max(my_max);
-  __shared__ float red[4];
+  __shared__ float red[QTHREADS / 32];
   if ((t & 31) == 0) red[t >> 5] = my_max;
   __syncthreads();
   if (t == 0) {
-    float m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    float m = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
     m *= 1.0001f;  // upper bound on max ||c||^2 despite the fp32 rounding above
     sm.cnorm[1] = m;
     sm.cnorm[0] = sqrtf(m) * 1.0001f;
@@ -81,16 +90,21 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
   __syncthreads();
 }
 
-// Quantizes one block of n (1..128) tokens.  Rows are at
-// src + row0 + t*row_stride (elements).  Output pointers are already offset to
-// the block's first token (codes, signs, norms) and to its mean row (means).
+__device__ __forceinline__ double shfl_pair_sum(double x) { return x + __shfl_xor_sync(0xffffffffu, x, 1); }
+
+// Quantizes one block of n (1..128) tokens with QTHREADS threads: thread
+// t = 2 tk + h works on token tk, dims 64h .. 64h+63 (sub-vectors 8h .. 8h+7).
+// Rows are at src + row0 + tk*row_stride (elements).  Output pointers are
+// already offset to the block's first token (codes, signs, norms) and to its
+// mean row (means).
 template <int DT, int MODE>
 __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, int64_t row0,
                                    int64_t row_stride, int n, uint8_t* __restrict__ codes,
                                    uint8_t* __restrict__ signs, __half2* __restrict__ norms,
                                    __half* __restrict__ means, int scale_adjust) {
-  const int t = threadIdx.x;
-  const bool valid = t < n;
+  const int t = threadIdx.x, tk = t >> 1, h = t & 1;
+  const int col = t & (D - 1), rhalf = t >> 7;  // column-sum roles: column, half of the rows
+  const bool valid = tk < n;
   constexpr int ESZ = (DT == NSN_DTYPE_F32) ? 4 : 2;
   constexpr int CHUNKS = D * ESZ / 16;  // 16-byte chunks per row
 
@@ -98,7 +112,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   {
     char* tile_bytes = reinterpret_cast<char*>(&sm.tile[0][0]);
     constexpr int ROWB = (D + 4) * 4;  // padded row stride in bytes (fits both dtypes)
-    for (int q = t; q < BLK * CHUNKS; q += blockDim.x) {
+    for (int q = t; q < BLK * CHUNKS; q += QTHREADS) {
       const int row = q / CHUNKS, ch = q % CHUNKS;
       if (row < n) {
         const char* g = static_cast<const char*>(src) + (row0 + (int64_t)row * row_stride) * ESZ + ch * 16;
@@ -116,11 +130,21 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   };
 
   // ---- reference r = column mean of the raw tokens ---------------------------
+  // Column `col`, rows split in two halves (two accumulators each), combined in
+  // a fixed order.
   {
-    double s = 0.0;
-    for (int row = 0; row < n; ++row) s += (double)raw_at(row, t);
-    sm.r[t] = (float)(s / n);
+    const int lo = rhalf * (BLK / 2), hi = min(n, lo + BLK / 2);
+    double s0 = 0.0, s1 = 0.0;
+    int row = lo;
+    for (; row + 1 < hi; row += 2) {
+      s0 += (double)raw_at(row, col);
+      s1 += (double)raw_at(row + 1, col);
+    }
+    if (row < hi) s0 += (double)raw_at(row, col);
+    sm.part[rhalf][col] = s0 + s1;
   }
+  __syncthreads();
+  if (t < D) sm.r[t] = (float)((sm.part[0][t] + sm.part[1][t]) / n);
   __syncthreads();
   // FWHT(r) in fp64 by warp 0 (lane l holds elements 4l..4l+3).
   if (t < 32) {
@@ -142,16 +166,17 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     for (int i = 0; i < 4; ++i) sm.big_r[4 * t + i] = v[i];
   }
 
-  // ---- d_t = FWHT(x_t - r) in registers; ||x_t||^2 from the raw values -------
-  float v[D];
+  // ---- d_t = FWHT(x_t - r) over the lane pair; ||x_t||^2 from the raw values --
+  float v[HD];
   double ssx0 = 0.0, ssx1 = 0.0;
   if (valid) {
-    const char* tb = reinterpret_cast<const char*>(&sm.tile[t][0]);
+    const char* tb = reinterpret_cast<const char*>(&sm.tile[tk][0]) + HD * ESZ * h;
+    constexpr int HCHUNKS = CHUNKS / 2;
+    constexpr int PER = (DT == NSN_DTYPE_F32) ? 4 : 8;
 #pragma unroll
-    for (int ch = 0; ch < CHUNKS; ++ch) {
+    for (int ch = 0; ch < HCHUNKS; ++ch) {
       const uint4 raw = *reinterpret_cast<const uint4*>(tb + ch * 16);
       float xs[8];
-      constexpr int PER = (DT == NSN_DTYPE_F32) ? 4 : 8;
       if constexpr (DT == NSN_DTYPE_F32) {
         const float* f = reinterpret_cast<const float*>(&raw);
 #pragma unroll
@@ -175,31 +200,33 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
       }
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
-        v[PER * ch + i] = xs[i] - sm.r[PER * ch + i];
+        v[PER * ch + i] = xs[i] - sm.r[HD * h + PER * ch + i];
         if (i & 1) ssx1 = fma((double)xs[i], (double)xs[i], ssx1);
         else ssx0 = fma((double)xs[i], (double)xs[i], ssx0);
       }
     }
   } else {
 #pragma unroll
-    for (int c = 0; c < D; ++c) v[c] = 0.f;
+    for (int c = 0; c < HD; ++c) v[c] = 0.f;
   }
-  fwht128_regs(v);
+  fwht128_pair(v, h);
+  const double ssx = shfl_pair_sum(ssx0 + ssx1);
   __syncthreads();  // raw tile fully consumed; big_r ready
 
   // ---- first normalization: s1 = ||H x|| / sqrt(128) = ||x|| / sqrt(128) -----
   // (H is orthonormal.)  n1_t = w_t * rr_t with w_t = FWHT(x_t) = d_t + FWHT(r)
   // and rr_t = 1/||x_t|| (||w_t|| = sqrt(128) ||x_t||); a zero token gets rr = 0.
   {
-    const double ssx = ssx0 + ssx1;
     const double norm_x = sqrt(ssx);
-    sm.s1[t] = norm_x / 11.313708498984761;
     const double rr = (ssx > 0.0) ? 1.0 / norm_x : 0.0;
     if (valid) {
 #pragma unroll
-      for (int c = 0; c < D; c += 4)
-        *reinterpret_cast<float4*>(&sm.tile[t][c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-      sm.rr[t] = rr;
+      for (int c = 0; c < HD; c += 4)
+        *reinterpret_cast<float4*>(&sm.tile[tk][HD * h + c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+      if (h == 0) {
+        sm.rr[tk] = rr;
+        sm.s1[tk] = norm_x / 11.313708498984761;
+      }
     }
   }
   __syncthreads();
@@ -207,18 +234,31 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   // ---- shift: o = mean_t n1_t = FWHT(r) * mean(rr) + mean_t(d_t rr_t) --------
   // mean(rr) is accumulated as deviations from rr_0 so that equal rr give it
   // exactly (identical tokens then give z = 0 exactly, as the definition does).
-  double rr_mean;
+  // Column `col`, rows split in two halves, combined in a fixed order.
   {
     const double rr0 = sm.rr[0];
-    double dev = 0.0, sd = 0.0;
-    for (int row = 0; row < n; ++row) {
-      const double rrow = sm.rr[row];
-      dev += rrow - rr0;
-      sd = fma((double)sm.tile[row][t], rrow, sd);
+    const int lo = rhalf * (BLK / 2), hi = min(n, lo + BLK / 2);
+    double dev = 0.0, sd0 = 0.0, sd1 = 0.0;
+    int row = lo;
+    for (; row + 1 < hi; row += 2) {
+      const double ra = sm.rr[row], rb = sm.rr[row + 1];
+      dev += (ra - rr0) + (rb - rr0);
+      sd0 = fma((double)sm.tile[row][col], ra, sd0);
+      sd1 = fma((double)sm.tile[row + 1][col], rb, sd1);
     }
-    rr_mean = rr0 + dev / n;
-    const double dc = sd / n;
-    sm.o[t] = dc;  // holds D_c = mean_t(d_t,c rr_t) until the next barrier
+    if (row < hi) {
+      const double ra = sm.rr[row];
+      dev += ra - rr0;
+      sd0 = fma((double)sm.tile[row][col], ra, sd0);
+    }
+    sm.part[rhalf][col] = sd0 + sd1;
+    if (col == 0) sm.dev_part[rhalf] = dev;
+  }
+  __syncthreads();
+  const double rr_mean = sm.rr[0] + (sm.dev_part[0] + sm.dev_part[1]) / n;
+  if (t < D) {
+    const double dc = (sm.part[0][t] + sm.part[1][t]) / n;
+    sm.o[t] = dc;  // D_c = mean_t(d_t,c rr_t)
     means[t] = __double2half(fma(sm.big_r[t], rr_mean, dc));
   }
   __syncthreads();
@@ -227,14 +267,15 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   // z_t = n1_t - o = d_t rr_t + FWHT(r) (rr_t - mean rr) - D.  The last two terms
   // are formed in fp64 and rounded once (they are at the scale of z), then one
   // fp32 fma per channel.
-  const double rr_t = valid ? sm.rr[t] : 0.0;
+  const double rr_t = valid ? sm.rr[tk] : 0.0;
   const double delta = rr_t - rr_mean;
   const float rrf = (float)rr_t;
   double zz0 = 0.0, zz1 = 0.0;
 #pragma unroll
-  for (int c = 0; c < D; c += 2) {
-    const float c0 = (float)fma(lds_f64(&sm.big_r[c]), delta, -lds_f64(&sm.o[c]));
-    const float c1 = (float)fma(lds_f64(&sm.big_r[c + 1]), delta, -lds_f64(&sm.o[c + 1]));
+  for (int c = 0; c < HD; c += 2) {
+    const int cg = HD * h + c;
+    const float c0 = (float)fma(lds_f64(&sm.big_r[cg]), delta, -lds_f64(&sm.o[cg]));
+    const float c1 = (float)fma(lds_f64(&sm.big_r[cg + 1]), delta, -lds_f64(&sm.o[cg + 1]));
     const float z0 = fmaf(v[c], rrf, c0);
     const float z1 = fmaf(v[c + 1], rrf, c1);
     v[c] = z0;
@@ -242,12 +283,12 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     zz0 = fma((double)z0, (double)z0, zz0);
     zz1 = fma((double)z1, (double)z1, zz1);
   }
-  const double zz = zz0 + zz1;
-  sm.s2[t] = sqrt(zz) / 11.313708498984761;
+  const double zz = shfl_pair_sum(zz0 + zz1);
+  if (valid && h == 0) sm.s2[tk] = sqrt(zz) / 11.313708498984761;
   const float inv2 = (zz > 0.0) ? (float)(11.313708498984761 / sqrt(zz)) : 0.f;
 #pragma unroll
-  for (int c = 0; c < D; ++c) v[c] *= inv2;
-  // v now holds u (fp32).
+  for (int c = 0; c < HD; ++c) v[c] *= inv2;
+  // v now holds u (fp32) for dims 64h .. 64h+63.
 
   // ---- sign bits (2-bit) and search operand a = |u| or u ---------------------
   // In 2-bit mode v is replaced by |u| after the sign bits are taken; every later
@@ -258,38 +299,40 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   uint32_t sgn[4] = {0u, 0u, 0u, 0u};
   if constexpr (MODE == NSN_MODE_2BIT) {
 #pragma unroll
-    for (int c = 0; c < D; ++c) {
-      const int s = c >> 3, i = c & 7;
+    for (int c = 0; c < HD; ++c) {
+      const int s = HSUB * h + (c >> 3), i = c & 7;
       sgn[i >> 1] |= (v[c] < 0.f ? 1u : 0u) << (16 * (i & 1) + 15 - s);
       v[c] = fabsf(v[c]);
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sgn[k] |= __shfl_xor_sync(0xffffffffu, sgn[k], 1);
+    if (h == 0) *reinterpret_cast<uint4*>(&sm.sgn[tk][0]) = make_uint4(sgn[0], sgn[1], sgn[2], sgn[3]);
   }
 
   // ---- exhaustive fp32 search ------------------------------------------------
-  // score_k = u.c_k - ||c_k||^2 / 2 (maximised).  Two passes over the codebook,
-  // 8 sub-vectors each.  Codewords are scanned in groups of 8: a running max
-  // per group (one FMNMX per codeword), then the best and second-best group
+  // score_k = u.c_k - ||c_k||^2 / 2 (maximised), one pass over the codebook for
+  // the thread's 8 sub-vectors.  Codewords are scanned in groups of 8: a running
+  // max per group (one FMNMX per codeword), then the best and second-best group
   // maxima with the best group's index.  The winning group is rescanned to find
   // the code (lowest index on ties) and its runner-up inside the group; the
   // overall runner-up is the larger of that and the second-best group max.
   const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1];
   constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
   uint32_t need = 0u;
+  {
+    float b1[HSUB], b2[HSUB];
+    int bg[HSUB];
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    float b1[NSUB / 2], b2[NSUB / 2];
-    int bg[NSUB / 2];
-#pragma unroll
-    for (int jj = 0; jj < NSUB / 2; ++jj) {
+    for (int jj = 0; jj < HSUB; ++jj) {
       b1[jj] = -INFINITY;
       b2[jj] = -INFINITY;
       bg[jj] = 0;
     }
 #pragma unroll 1
     for (int grp = 0; grp < NCODES / 8; ++grp) {
-      float gm[NSUB / 2];
+      float gm[HSUB];
 #pragma unroll
-      for (int jj = 0; jj < NSUB / 2; ++jj) gm[jj] = -INFINITY;
+      for (int jj = 0; jj < HSUB; ++jj) gm[jj] = -INFINITY;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const int k = 8 * grp + kk;
@@ -297,22 +340,21 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
         const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
         const float bk = sm.bias[k];
 #pragma unroll
-        for (int jj = 0; jj < NSUB / 2; ++jj) {
-          const int j = 8 * half + jj;
+        for (int jj = 0; jj < HSUB; ++jj) {
           float s = bk;
-          s = fmaf(v[8 * j + 0], c0.x, s);
-          s = fmaf(v[8 * j + 1], c0.y, s);
-          s = fmaf(v[8 * j + 2], c0.z, s);
-          s = fmaf(v[8 * j + 3], c0.w, s);
-          s = fmaf(v[8 * j + 4], c1.x, s);
-          s = fmaf(v[8 * j + 5], c1.y, s);
-          s = fmaf(v[8 * j + 6], c1.z, s);
-          s = fmaf(v[8 * j + 7], c1.w, s);
+          s = fmaf(v[8 * jj + 0], c0.x, s);
+          s = fmaf(v[8 * jj + 1], c0.y, s);
+          s = fmaf(v[8 * jj + 2], c0.z, s);
+          s = fmaf(v[8 * jj + 3], c0.w, s);
+          s = fmaf(v[8 * jj + 4], c1.x, s);
+          s = fmaf(v[8 * jj + 5], c1.y, s);
+          s = fmaf(v[8 * jj + 6], c1.z, s);
+          s = fmaf(v[8 * jj + 7], c1.w, s);
           gm[jj] = fmaxf(gm[jj], s);
         }
       }
 #pragma unroll
-      for (int jj = 0; jj < NSUB / 2; ++jj) {
+      for (int jj = 0; jj < HSUB; ++jj) {
         const float lo = fminf(b1[jj], gm[jj]);
         bg[jj] = (gm[jj] > b1[jj]) ? grp : bg[jj];
         b1[jj] = fmaxf(b1[jj], gm[jj]);
@@ -320,8 +362,8 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
       }
     }
 #pragma unroll
-    for (int jj = 0; jj < NSUB / 2; ++jj) {
-      const int j = 8 * half + jj;
+    for (int jj = 0; jj < HSUB; ++jj) {
+      const int j = HSUB * h + jj;
       // rescan the winning group with the same arithmetic as above
       float best = -INFINITY, second = -INFINITY;
       int idx = 8 * bg[jj];
@@ -331,14 +373,14 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
         const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
         const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
         float s = sm.bias[k];
-        s = fmaf(v[8 * j + 0], c0.x, s);
-        s = fmaf(v[8 * j + 1], c0.y, s);
-        s = fmaf(v[8 * j + 2], c0.z, s);
-        s = fmaf(v[8 * j + 3], c0.w, s);
-        s = fmaf(v[8 * j + 4], c1.x, s);
-        s = fmaf(v[8 * j + 5], c1.y, s);
-        s = fmaf(v[8 * j + 6], c1.z, s);
-        s = fmaf(v[8 * j + 7], c1.w, s);
+        s = fmaf(v[8 * jj + 0], c0.x, s);
+        s = fmaf(v[8 * jj + 1], c0.y, s);
+        s = fmaf(v[8 * jj + 2], c0.z, s);
+        s = fmaf(v[8 * jj + 3], c0.w, s);
+        s = fmaf(v[8 * jj + 4], c1.x, s);
+        s = fmaf(v[8 * jj + 5], c1.y, s);
+        s = fmaf(v[8 * jj + 6], c1.z, s);
+        s = fmaf(v[8 * jj + 7], c1.w, s);
         const float lo = fminf(best, s);
         idx = (s > best) ? k : idx;
         best = fmaxf(best, s);
@@ -347,14 +389,14 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
       const float runner = fmaxf(b2[jj], second);
       float na = 0.f;
 #pragma unroll
-      for (int i = 0; i < SUB; ++i) na = fmaf(v[8 * j + i], v[8 * j + i], na);
+      for (int i = 0; i < SUB; ++i) na = fmaf(v[8 * jj + i], v[8 * jj + i], na);
       na = sqrtf(na) * 1.0001f;
       // |fp32 score - exact score| <= gamma_9 (max||c||^2 + ||a|| max||c||) for every
       // codeword, so a rival within twice that bound of the best may be the true best.
       const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
-      sm.thr[t][j] = best - margin;
-      need |= (runner >= best - margin ? 1u : 0u) << j;
-      sm.code[t][j] = (uint8_t)idx;
+      sm.thr[tk][j] = best - margin;
+      need |= (runner >= best - margin ? 1u : 0u) << jj;
+      sm.code[tk][j] = (uint8_t)idx;
     }
   }
 
@@ -362,20 +404,21 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   // From here on u is read from shared memory so that no register array stays
   // live across the rarely taken exact path.
 #pragma unroll
-  for (int c = 0; c < D; c += 4)
-    *reinterpret_cast<float4*>(&sm.tile[t][c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+  for (int c = 0; c < HD; c += 4)
+    *reinterpret_cast<float4*>(&sm.tile[tk][HD * h + c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
 
   // ---- exact fp64 re-decision of sub-vectors with a close second -------------
   // Candidates: codewords whose fp32 score (same operation order as the main
   // search) reaches the threshold; winner by fp64 squared distance, ties to the
   // lowest index.
 #pragma unroll 1
-  for (int j = 0; j < NSUB; ++j) {
-    if (!((need >> j) & 1u)) continue;
-    const float* a = &sm.tile[t][8 * j];
-    const float thr = sm.thr[t][j];
+  for (int jj = 0; jj < HSUB; ++jj) {
+    if (!((need >> jj) & 1u)) continue;
+    const int j = HSUB * h + jj;
+    const float* a = &sm.tile[tk][8 * j];
+    const float thr = sm.thr[tk][j];
     double bestd = INFINITY;
-    int bi = sm.code[t][j];
+    int bi = sm.code[tk][j];
 #pragma unroll 1
     for (int k = 0; k < NCODES; ++k) {
       float sc = sm.bias[k];
@@ -391,18 +434,19 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
         if (dd < bestd) { bestd = dd; bi = k; }
       }
     }
-    sm.code[t][j] = (uint8_t)bi;
+    sm.code[tk][j] = (uint8_t)bi;
   }
 
   // ---- adaptive scale: alpha = ||u||^2 / (u . u_hat) --------------------------
   double dot = 0.0, uu = 0.0;
 #pragma unroll 4
-  for (int j = 0; j < NSUB; ++j) {
-    const int cj = sm.code[t][j];
+  for (int jj = 0; jj < HSUB; ++jj) {
+    const int j = HSUB * h + jj;
+    const int cj = sm.code[tk][j];
     const float4 q0 = *reinterpret_cast<const float4*>(&sm.cb[cj][0]);
     const float4 q1 = *reinterpret_cast<const float4*>(&sm.cb[cj][4]);
-    const float4 u0 = *reinterpret_cast<const float4*>(&sm.tile[t][8 * j]);
-    const float4 u1 = *reinterpret_cast<const float4*>(&sm.tile[t][8 * j + 4]);
+    const float4 u0 = *reinterpret_cast<const float4*>(&sm.tile[tk][8 * j]);
+    const float4 u1 = *reinterpret_cast<const float4*>(&sm.tile[tk][8 * j + 4]);
     const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
     const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
     float dj = 0.f, uj = 0.f;
@@ -414,15 +458,22 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     dot += (double)dj;
     uu += (double)uj;
   }
+  // halves combined in a fixed order (low half first) so both lanes agree bit for bit
+  const double dot_o = __shfl_xor_sync(0xffffffffu, dot, 1), uu_o = __shfl_xor_sync(0xffffffffu, uu, 1);
+  dot = h ? dot_o + dot : dot + dot_o;
+  uu = h ? uu_o + uu : uu + uu_o;
   double alpha = (dot > 0.0) ? uu / dot : 1.0;
   if (!scale_adjust) alpha = 1.0;
 
   // ---- packed stores ---------------------------------------------------------
   if (valid) {
-    *reinterpret_cast<uint4*>(codes + (int64_t)t * NSUB) = *reinterpret_cast<const uint4*>(&sm.code[t][0]);
-    if constexpr (MODE == NSN_MODE_2BIT)
-      *reinterpret_cast<uint4*>(signs + (int64_t)t * NSUB) = make_uint4(sgn[0], sgn[1], sgn[2], sgn[3]);
-    norms[t] = __halves2half2(__double2half(sm.s1[t]), __double2half(alpha * sm.s2[t]));
+    *reinterpret_cast<uint2*>(codes + (int64_t)tk * NSUB + HSUB * h) =
+        *reinterpret_cast<const uint2*>(&sm.code[tk][HSUB * h]);
+    if (h == 0) {
+      if constexpr (MODE == NSN_MODE_2BIT)
+        *reinterpret_cast<uint4*>(signs + (int64_t)tk * NSUB) = *reinterpret_cast<const uint4*>(&sm.sgn[tk][0]);
+      norms[tk] = __halves2half2(__double2half(sm.s1[tk]), __double2half(alpha * sm.s2[tk]));
+    }
   }
   __syncthreads();  // shared memory is reused by the caller's next block
 }
@@ -431,7 +482,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
 // Prefill: grid (blocks, kv-heads, batch).
 // ---------------------------------------------------------------------------
 template <int DT, int MODE>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(QTHREADS, 2)
 quantize_prefill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int64_t sh, int q_tokens,
                         CacheView cv, const float* __restrict__ codebook) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -473,7 +524,7 @@ __global__ void window_fill_kernel(const void* __restrict__ x, int64_t sb, int64
 // flushing a full window into the quantized part first.  grid (kv-heads, batch, 2).
 // ---------------------------------------------------------------------------
 template <int DTN>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(QTHREADS, 2)
 append_kernel(CacheView kc, CacheView vc, const void* __restrict__ k_new, const void* __restrict__ v_new,
               int64_t sb, int64_t sh, const float* __restrict__ cbk, const float* __restrict__ cbv) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -538,7 +589,7 @@ static cudaError_t launch_prefill_t(const void* x, int64_t sb, int64_t st, int64
   const int nblk = (q_tokens + BLK - 1) / BLK;
   if (nblk > 0) {
     dim3 grid(nblk, cv.n_kv_heads, cv.batch);
-    quantize_prefill_kernel<DT, MODE><<<grid, 128, smem, s>>>(x, sb, st, sh, q_tokens, cv, cb);
+    quantize_prefill_kernel<DT, MODE><<<grid, QTHREADS, smem, s>>>(x, sb, st, sh, q_tokens, cv, cb);
   }
   return cudaGetLastError();
 }
@@ -572,7 +623,7 @@ static cudaError_t launch_append_t(const CacheView& kc, const CacheView& vc, con
   cudaError_t e = cudaFuncSetAttribute(append_kernel<DTN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(kc.n_kv_heads, kc.batch, 2);
-  append_kernel<DTN><<<grid, 128, smem, s>>>(kc, vc, kn, vn, sb, sh, cbk, cbv);
+  append_kernel<DTN><<<grid, QTHREADS, smem, s>>>(kc, vc, kn, vn, sb, sh, cbk, cbv);
   return cudaGetLastError();
 }
 

@@ -199,7 +199,8 @@ def decode_workspace(k_cache: Cache, n_q_heads: int, device="cuda"):
     n = nsn_decode_workspace_bytes(k_cache, n_q_heads)
     if n == 0:
         raise ValueError("invalid cache or head count for decode")
-    return torch.empty((n,), dtype=torch.uint8, device=device)
+    # zero-filled: the leading merge counters must start at zero
+    return torch.zeros((n,), dtype=torch.uint8, device=device)
 
 
 def nsn_decode_attention(k_cache: Cache, v_cache: Cache, q, softmax_scale: float, cb_k, cb_v, out, workspace,

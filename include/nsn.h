@@ -179,6 +179,8 @@ nsn_status nsn_append_residual(nsn_cache* k_cache, nsn_cache* v_cache, const voi
 
 /*
  * Workspace bytes that nsn_decode_attention needs for these caches and n_q_heads.
+ * The workspace starts with 2 * batch * n_kv_heads 32-bit merge counters (padded
+ * to 256 bytes); the decode partials follow.
  */
 size_t nsn_decode_workspace_bytes(const nsn_cache* k_cache, int n_q_heads);
 
@@ -192,7 +194,17 @@ size_t nsn_decode_workspace_bytes(const nsn_cache* k_cache, int n_q_heads);
  *   cb_k, cb_v     device float[256*8] codebooks; decode reads them rounded to fp16.
  *   out            device float [b][n_q_heads][128].  A (b, h) with no tokens at all
  *                  yields zeros.
- *   workspace      device, >= nsn_decode_workspace_bytes() bytes, 256-byte aligned.
+ *   workspace      device, >= nsn_decode_workspace_bytes() bytes, 256-byte aligned,
+ *                  caller-owned.  It must be zero-filled before its first use with
+ *                  caches of a given batch x n_kv_heads (its leading counters must be
+ *                  zero); every completed call leaves those counters zero again, so
+ *                  later calls need no clearing.  Calls sharing one workspace must not
+ *                  overlap on the GPU.
+ * One kernel launch: the quantized blocks of each (b, kv-head) are dealt out to
+ * splits, the last split also attends the window, and the split that completes a
+ * (b, kv-head, head group) last merges the partials into `out`.  Status bit 2 of
+ * k_cache->status is set if a copy into shared memory did not complete in time
+ * (the affected outputs are then not meaningful).
  */
 nsn_status nsn_decode_attention(const nsn_cache* k_cache, const nsn_cache* v_cache,
                                 const void* q, int dtype, int n_q_heads, int64_t q_stride_b,
@@ -207,19 +219,23 @@ nsn_status nsn_decode_attention(const nsn_cache* k_cache, const nsn_cache* v_cac
  * that reserve all device memory up front, hosts that forbid cudaMalloc after
  * start-up.  It takes the same arguments as nsn_decode_attention minus the
  * workspace and computes the same result; its decode partials go to a fixed
- * file-scope device array of NSN_DECODE_SCRATCH_BYTES bytes instead, which every
- * GPU that loads the library holds until the process exits.
+ * file-scope device array of NSN_DECODE_SCRATCH_BYTES bytes instead, and its merge
+ * counters to a second one of NSN_DECODE_STATIC_COUNTERS 32-bit words (both
+ * zero-filled at load); every GPU that loads the library holds them until the
+ * process exits.
  *   - Nothing is allocated or freed (no cudaMalloc / cudaFree / allocating library).
- *   - Returns NSN_ERR_WORKSPACE if this shape needs more than NSN_DECODE_SCRATCH_BYTES
- *     (nsn_decode_workspace_bytes() tells how much it needs).
+ *   - Returns NSN_ERR_WORKSPACE if this shape's partials need more than
+ *     NSN_DECODE_SCRATCH_BYTES or 2 * batch * n_kv_heads > NSN_DECODE_STATIC_COUNTERS.
  *   - The first call on a device resolves the array's device address (with that
  *     device current) and caches it; make that first call before any stream capture.
  *   - All calls share the one array: two calls whose work overlaps on the GPU (e.g. on
  *     different streams without ordering between them) race on it and must not be
- *     issued.  Every value the kernels read from it is written earlier in the same
- *     call, so nothing needs clearing between calls.
+ *     issued.  Every partial the kernel reads is written earlier in the same call and
+ *     each completed call leaves the counters it used at zero, so nothing needs
+ *     clearing between calls.
  */
 #define NSN_DECODE_SCRATCH_BYTES (8u << 20)
+#define NSN_DECODE_STATIC_COUNTERS 16384u
 nsn_status nsn_decode_attention_static(const nsn_cache* k_cache, const nsn_cache* v_cache, const void* q,
                                        int dtype, int n_q_heads, int64_t q_stride_b, int64_t q_stride_h,
                                        float softmax_scale, const float* cb_k, const float* cb_v, float* out,

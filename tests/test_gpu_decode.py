@@ -148,3 +148,39 @@ def test_e2e_config2_llama_layer():
 def test_e2e_mixed_modes_across_flushes():
     # 2-bit K / 1-bit V (the long-context mix), 130 appends crossing a flush.
     run_e2e(2, 2, 4, 1000, 130, 2, 1, torch.bfloat16, "llama", (31, 32, 33))
+
+
+def test_workspace_counters_return_to_zero_and_calls_repeat():
+    # The decode merges its split partials through one counter per (sequence,
+    # head group) at the start of the workspace; every completed call leaves the
+    # counters at zero, so back-to-back calls on one workspace agree exactly.
+    B, H, g, mk, mv = 2, 2, 8, 2, 1
+    shape = {(0, 0): (2304, 128), (0, 1): (640, 7), (1, 0): (128, 0), (1, 1): (0, 33)}
+    kc, vc = nsn.Cache(B, H, 2304, 128, mk), nsn.Cache(B, H, 2304, 128, mv)
+    kcont, vcont = {}, {}
+    for (b, h), (nq, nw) in shape.items():
+        kcont[(b, h)] = synthetic.random_cache_contents(50 + 10 * b + h, nq, nw, mk)
+        vcont[(b, h)] = synthetic.random_cache_contents(70 + 10 * b + h, nq, nw, mv)
+    fill_cache(kc, kcont)
+    fill_cache(vc, vcont)
+    cbk = torch.from_numpy(tl.codebook(mk)).cuda()
+    cbv = torch.from_numpy(tl.codebook(mv)).cuda()
+    q = synthetic.queries(9, B, H * g, torch.bfloat16, "cuda")
+    ws = nsn.decode_workspace(kc, H * g)
+    outs = []
+    for _ in range(3):
+        out = torch.full((B, H * g, 128), float("nan"), dtype=torch.float32, device="cuda")
+        nsn.nsn_decode_attention(kc, vc, q, SCALE, cbk, cbv, out, ws)
+        torch.cuda.synchronize()
+        outs.append(out.cpu())
+        counters = ws[: 4 * 2 * B * H].view(torch.int32).cpu()
+        assert int(counters.abs().sum()) == 0, "merge counters not back to zero"
+    assert torch.isfinite(outs[0]).all()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    qf = q.float().cpu().numpy().astype(np.float64)
+    cbk64, cbv64 = tl.codebook(mk).astype(np.float64), tl.codebook(mv).astype(np.float64)
+    for (b, h) in shape:
+        ref = orc.decode_attention(qf[b, h * g:(h + 1) * g], oracle_seq(kcont[(b, h)]), oracle_seq(vcont[(b, h)]),
+                                   kcont[(b, h)]["window"].astype(np.float64),
+                                   vcont[(b, h)]["window"].astype(np.float64), cbk64, cbv64, mk, mv, SCALE)
+        assert tl.attn_error(outs[0][b, h * g:(h + 1) * g].numpy(), ref) <= tl.ATTN_TOL
