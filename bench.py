@@ -44,6 +44,28 @@ LAUNCHES_PER_STEP = 2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
+# DRAM bytes (read + write) per decode_kernel launch on this workload, from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum; command and numbers
+# in profiles/launches-decode_b16_32k_2bit.md), valid only for the decode sources
+# with this SHA-256 (decode.cu, nsn_common.cuh, nsn_launch.h).  Any later change
+# to those files makes the figure stale, and the bench then reports null.
+DECODE_TRAFFIC = {"sha256": "150c974ccef32724836b1cb33dbb02515b03be4a614812d3a96723e5633616e2",
+                  "bytes_per_launch": 320636544 + 2836480}
+
+
+def decode_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("decode.cu", "nsn_common.cuh", "nsn_launch.h"):
+        with open(os.path.join(ROOT, "calibration_free_vector_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def decode_traffic():
+    return DECODE_TRAFFIC["bytes_per_launch"] if decode_sources_sha256() == DECODE_TRAFFIC["sha256"] else None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -424,7 +446,7 @@ def run_ours(args):
             "decode_call_ms": dec_avg_ms,
             "roofline": {"kernel": "decode_kernel (one launch per decode call)", "bound": "hbm",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                         "peak_kind": peak_kind, "traffic": None,
+                         "peak_kind": peak_kind, "traffic": decode_traffic(),
                          "algorithmic_bytes_per_launch": decode_bytes,
                          "frac_of_8tbs_spec": achieved / 8000.0},
             "quantize": {"workload": f"prefill {B}x{q_tokens} tokens x {H} kv-heads, K 2-bit + V 2-bit, bf16 in",

@@ -62,3 +62,10 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
         steps, warmup = 1, 3
     assert bench.run_reference(A()) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_decode_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
+    import bench
+    assert bench.decode_traffic() in (None, bench.DECODE_TRAFFIC["bytes_per_launch"])
+    monkeypatch.setitem(bench.DECODE_TRAFFIC, "sha256", "0" * 64)
+    assert bench.decode_traffic() is None
