@@ -5,6 +5,10 @@
 // synthetic standard-normal data; the README's "Codebook tuning" builds the
 // 2-bit codebook over absolute values (--abs).
 //
+// The same passage: the k-means codebook is then fine-tuned to minimise the
+// cosine distance between vectors and their quantized versions
+// (nsn_build_codebook_cosine_host; the README's "--method learned").
+//
 // Standard normals: Philox4x64-10 counter-based generator (Salmon, Moraes, Dror,
 // Shaw, SC'11) + Box-Muller transform (Box & Muller, 1958); stream layout in nsn.h.
 
@@ -59,40 +63,36 @@ void normal_stream(uint64_t seed, size_t count, double* out) {
   }
 }
 
-}  // namespace
+// Lloyd k-means from the first k samples (ties to the lowest centroid, empty
+// clusters keep their centroid); `label` receives the last assignment.
+void assign(const std::vector<double>& x, const std::vector<double>& cent, size_t n, size_t k, size_t d,
+            std::vector<int32_t>& label) {
+  for (size_t i = 0; i < n; ++i) {
+    const double* xi = &x[i * d];
+    double best = INFINITY;
+    int32_t bi = 0;
+    for (size_t c = 0; c < k; ++c) {
+      const double* cc = &cent[c * d];
+      double s = 0.0;
+      for (size_t e = 0; e < d; ++e) {
+        const double df = xi[e] - cc[e];
+        s += df * df;
+      }
+      if (s < best) {
+        best = s;
+        bi = (int32_t)c;
+      }
+    }
+    label[i] = bi;
+  }
+}
 
-extern "C" nsn_status nsn_build_codebook_host(uint64_t seed, int n_samples, int n_codes, int dim, int abs_mode,
-                                              int iters, float* out) {
-  if (!out || n_codes <= 0 || dim <= 0 || n_samples < n_codes || iters < 0) return NSN_ERR_INVALID_ARG;
-  const size_t n = (size_t)n_samples, k = (size_t)n_codes, d = (size_t)dim;
-  std::vector<double> x(n * d);
-  normal_stream(seed, n * d, x.data());
-  if (abs_mode)
-    for (double& v : x) v = std::fabs(v);
-
-  std::vector<double> cent(x.begin(), x.begin() + k * d);  // first n_codes samples
+void kmeans(const std::vector<double>& x, std::vector<double>& cent, size_t n, size_t k, size_t d, int iters) {
   std::vector<double> sums(k * d);
   std::vector<int64_t> counts(k);
   std::vector<int32_t> label(n);
   for (int it = 0; it < iters; ++it) {
-    for (size_t i = 0; i < n; ++i) {
-      const double* xi = &x[i * d];
-      double best = INFINITY;
-      int32_t bi = 0;
-      for (size_t c = 0; c < k; ++c) {
-        const double* cc = &cent[c * d];
-        double s = 0.0;
-        for (size_t e = 0; e < d; ++e) {
-          const double df = xi[e] - cc[e];
-          s += df * df;
-        }
-        if (s < best) {
-          best = s;
-          bi = (int32_t)c;
-        }
-      }
-      label[i] = bi;
-    }
+    assign(x, cent, n, k, d, label);
     std::fill(sums.begin(), sums.end(), 0.0);
     std::fill(counts.begin(), counts.end(), 0);
     for (size_t i = 0; i < n; ++i) {
@@ -104,6 +104,91 @@ extern "C" nsn_status nsn_build_codebook_host(uint64_t seed, int n_samples, int 
       if (counts[c] > 0)
         for (size_t e = 0; e < d; ++e) cent[c * d + e] = sums[c * d + e] / (double)counts[c];
   }
-  for (size_t i = 0; i < k * d; ++i) out[i] = __half2float(__double2half(cent[i]));
+}
+
+// Cosine fine-tuning.  With the samples assigned to their nearest codeword (as
+// the quantizer assigns), codeword c is turned to the direction that maximises
+// the summed cosine with its members -- the normalised sum of their unit
+// vectors -- and given the least-squares length along it, the mean projection
+// of its members.  Codewords without members, with a zero direction sum or a
+// non-positive mean projection are kept.
+void cosine_finetune(const std::vector<double>& x, std::vector<double>& cent, size_t n, size_t k, size_t d,
+                     int iters) {
+  std::vector<double> unit(n * d);
+  for (size_t i = 0; i < n; ++i) {
+    double ss = 0.0;
+    for (size_t e = 0; e < d; ++e) ss += x[i * d + e] * x[i * d + e];
+    const double nr = std::sqrt(ss);
+    for (size_t e = 0; e < d; ++e) unit[i * d + e] = nr > 0.0 ? x[i * d + e] / nr : 0.0;
+  }
+  std::vector<double> dir(k * d), proj(k);
+  std::vector<int64_t> counts(k);
+  std::vector<int32_t> label(n);
+  for (int it = 0; it < iters; ++it) {
+    assign(x, cent, n, k, d, label);
+    std::fill(dir.begin(), dir.end(), 0.0);
+    std::fill(counts.begin(), counts.end(), 0);
+    for (size_t i = 0; i < n; ++i) {
+      const size_t c = (size_t)label[i];
+      counts[c] += 1;
+      for (size_t e = 0; e < d; ++e) dir[c * d + e] += unit[i * d + e];
+    }
+    for (size_t c = 0; c < k; ++c) {
+      double ss = 0.0;
+      for (size_t e = 0; e < d; ++e) ss += dir[c * d + e] * dir[c * d + e];
+      const double nr = std::sqrt(ss);
+      for (size_t e = 0; e < d; ++e) dir[c * d + e] = nr > 0.0 ? dir[c * d + e] / nr : 0.0;
+    }
+    std::fill(proj.begin(), proj.end(), 0.0);
+    for (size_t i = 0; i < n; ++i) {
+      const size_t c = (size_t)label[i];
+      double p = 0.0;
+      for (size_t e = 0; e < d; ++e) p += x[i * d + e] * dir[c * d + e];
+      proj[c] += p;
+    }
+    for (size_t c = 0; c < k; ++c) {
+      if (counts[c] == 0) continue;
+      const double len = proj[c] / (double)counts[c];
+      if (!(len > 0.0)) continue;
+      for (size_t e = 0; e < d; ++e) cent[c * d + e] = dir[c * d + e] * len;
+    }
+  }
+}
+
+std::vector<double> samples(uint64_t seed, size_t n, size_t d, int abs_mode) {
+  std::vector<double> x(n * d);
+  normal_stream(seed, n * d, x.data());
+  if (abs_mode)
+    for (double& v : x) v = std::fabs(v);
+  return x;
+}
+
+void store_f16(const std::vector<double>& cent, size_t count, float* out) {
+  for (size_t i = 0; i < count; ++i) out[i] = __half2float(__double2half(cent[i]));
+}
+
+}  // namespace
+
+extern "C" nsn_status nsn_build_codebook_host(uint64_t seed, int n_samples, int n_codes, int dim, int abs_mode,
+                                              int iters, float* out) {
+  if (!out || n_codes <= 0 || dim <= 0 || n_samples < n_codes || iters < 0) return NSN_ERR_INVALID_ARG;
+  const size_t n = (size_t)n_samples, k = (size_t)n_codes, d = (size_t)dim;
+  const std::vector<double> x = samples(seed, n, d, abs_mode);
+  std::vector<double> cent(x.begin(), x.begin() + k * d);  // first n_codes samples
+  kmeans(x, cent, n, k, d, iters);
+  store_f16(cent, k * d, out);
+  return NSN_OK;
+}
+
+extern "C" nsn_status nsn_build_codebook_cosine_host(uint64_t seed, int n_samples, int n_codes, int dim,
+                                                     int abs_mode, int kmeans_iters, int cosine_iters, float* out) {
+  if (!out || n_codes <= 0 || dim <= 0 || n_samples < n_codes || kmeans_iters < 0 || cosine_iters < 0)
+    return NSN_ERR_INVALID_ARG;
+  const size_t n = (size_t)n_samples, k = (size_t)n_codes, d = (size_t)dim;
+  const std::vector<double> x = samples(seed, n, d, abs_mode);
+  std::vector<double> cent(x.begin(), x.begin() + k * d);
+  kmeans(x, cent, n, k, d, kmeans_iters);
+  cosine_finetune(x, cent, n, k, d, cosine_iters);
+  store_f16(cent, k * d, out);
   return NSN_OK;
 }

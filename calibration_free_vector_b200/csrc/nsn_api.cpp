@@ -104,8 +104,10 @@ nsn_status nsn_cache_buffer_sizes(int batch, int n_kv_heads, int capacity, int w
   return NSN_OK;
 }
 
-nsn_status nsn_quantize_kv(nsn_cache* cache, const void* x, int dtype, int64_t stride_b, int64_t stride_t,
-                           int64_t stride_h, int n_tokens, const float* codebook, void* stream) {
+// Validation shared by the common-length and ragged prefills; sets q, the
+// quantized prefix of n_tokens.
+static nsn_status check_prefill(const nsn_cache* cache, const void* x, int dtype, int64_t stride_b, int64_t stride_t,
+                                int64_t stride_h, int n_tokens, const float* codebook, int* q_out) {
   nsn_status st = check_cache(cache);
   if (st != NSN_OK) return st;
   if (!codebook || !valid_dtype(dtype) || n_tokens < 0) return NSN_ERR_INVALID_ARG;
@@ -120,8 +122,28 @@ nsn_status nsn_quantize_kv(nsn_cache* cache, const void* x, int dtype, int64_t s
   else q = NSN_BLOCK * ((n_tokens - 1) / NSN_BLOCK);
   if (q > cache->capacity) return NSN_ERR_INVALID_ARG;
   if (n_tokens - q > cache->window) return NSN_ERR_INVALID_ARG;
-  return cuda_status(nsn::launch_quantize_prefill(x, dtype, stride_b, stride_t, stride_h, q, n_tokens, view(cache),
-                                                  codebook, static_cast<cudaStream_t>(stream)));
+  *q_out = q;
+  return NSN_OK;
+}
+
+nsn_status nsn_quantize_kv_ragged(nsn_cache* cache, const void* x, int dtype, int64_t stride_b, int64_t stride_t,
+                                  int64_t stride_h, const int32_t* lengths, int max_tokens, const float* codebook,
+                                  void* stream) {
+  if (!lengths || (reinterpret_cast<uintptr_t>(lengths) & 3u)) return NSN_ERR_INVALID_ARG;
+  int q = 0;
+  const nsn_status st = check_prefill(cache, x, dtype, stride_b, stride_t, stride_h, max_tokens, codebook, &q);
+  if (st != NSN_OK) return st;
+  return cuda_status(nsn::launch_quantize_prefill(x, dtype, stride_b, stride_t, stride_h, q, max_tokens, lengths,
+                                                  view(cache), codebook, static_cast<cudaStream_t>(stream)));
+}
+
+nsn_status nsn_quantize_kv(nsn_cache* cache, const void* x, int dtype, int64_t stride_b, int64_t stride_t,
+                           int64_t stride_h, int n_tokens, const float* codebook, void* stream) {
+  int q = 0;
+  const nsn_status st = check_prefill(cache, x, dtype, stride_b, stride_t, stride_h, n_tokens, codebook, &q);
+  if (st != NSN_OK) return st;
+  return cuda_status(nsn::launch_quantize_prefill(x, dtype, stride_b, stride_t, stride_h, q, n_tokens, nullptr,
+                                                  view(cache), codebook, static_cast<cudaStream_t>(stream)));
 }
 
 nsn_status nsn_append_residual(nsn_cache* k_cache, nsn_cache* v_cache, const void* k_new, const void* v_new,

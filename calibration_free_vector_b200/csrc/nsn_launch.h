@@ -39,8 +39,11 @@ bool decode_static_fits(int batch, int n_kv_heads, const DecodeGeom& geom);
 
 size_t quant_smem_bytes();
 
+// `lengths` (device int32[batch]) is NULL for a common length; otherwise n_tokens is
+// the bound of the lengths and q_tokens the quantized prefix of that bound.
 cudaError_t launch_quantize_prefill(const void* x, int dtype, int64_t sb, int64_t st, int64_t sh, int q_tokens,
-                                    int n_tokens, const CacheView& cv, const float* cb, cudaStream_t s);
+                                    int n_tokens, const int32_t* lengths, const CacheView& cv, const float* cb,
+                                    cudaStream_t s);
 
 cudaError_t launch_append(const CacheView& kc, const CacheView& vc, const void* kn, const void* vn, int dtype,
                           int64_t sb, int64_t sh, const float* cbk, const float* cbv, cudaStream_t s);

@@ -481,14 +481,35 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
 // ---------------------------------------------------------------------------
 // Prefill: grid (blocks, kv-heads, batch).
 // ---------------------------------------------------------------------------
+// Tokens of sequence b and its quantized prefix.  Without `lengths` every
+// sequence has the common n_tokens / q_tokens; with it, sequence b has
+// lengths[b] tokens (an entry outside [0, max_tokens] counts as 0 and is
+// flagged) and the same split rule: window 0 quantizes all of them, window 128
+// quantizes 128 floor((L - 1) / 128) and keeps the rest (1..128) in the window.
+struct PrefillSplit {
+  int n, q;
+  bool bad;
+};
+
+__device__ __forceinline__ PrefillSplit prefill_split(const int32_t* __restrict__ lengths, int b, int n_tokens,
+                                                      int q_tokens, int window_len) {
+  if (!lengths) return {n_tokens, q_tokens, false};
+  int L = lengths[b];
+  const bool bad = L < 0 || L > n_tokens;
+  if (bad) L = 0;
+  const int q = L == 0 ? 0 : (window_len == 0 ? L : BLK * ((L - 1) / BLK));
+  return {L, q, bad};
+}
+
 template <int DT, int MODE>
 __global__ void __launch_bounds__(QTHREADS, 2)
-quantize_prefill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int64_t sh, int q_tokens,
-                        CacheView cv, const float* __restrict__ codebook) {
+quantize_prefill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int64_t sh, int q_tokens, int n_tokens,
+                        const int32_t* __restrict__ lengths, CacheView cv, const float* __restrict__ codebook) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw);
   const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int n = min(BLK, q_tokens - blk * BLK);
+  const PrefillSplit ps = prefill_split(lengths, b, n_tokens, q_tokens, cv.window_len);
+  const int n = min(BLK, ps.q - blk * BLK);
   if (n <= 0) return;
   stage_codebook(sm, codebook);
   const int64_t seq = (int64_t)b * cv.n_kv_heads + h;
@@ -499,23 +520,26 @@ quantize_prefill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int6
                                cv.scale_adjust);
 }
 
-// Prefill tail: copies tokens [q, L) to the residual window (fp16) and sets the
-// counters.  grid (kv-heads, batch), 128 threads.
+// Prefill tail: copies tokens [q, L) of each sequence to the residual window
+// (fp16) and sets the counters; a rejected ragged length sets status bit 4.
+// grid (kv-heads, batch), 128 threads.
 template <int DT>
 __global__ void window_fill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int64_t sh, int q_tokens,
-                                   int n_tokens, CacheView cv) {
+                                   int n_tokens, const int32_t* __restrict__ lengths, CacheView cv) {
   const int h = blockIdx.x, b = blockIdx.y;
   const int64_t seq = (int64_t)b * cv.n_kv_heads + h;
-  const int nw = n_tokens - q_tokens;
+  const PrefillSplit ps = prefill_split(lengths, b, n_tokens, q_tokens, cv.window_len);
+  const int nw = ps.n - ps.q;
   for (int q = threadIdx.x; q < nw * (D / 8); q += blockDim.x) {
     const int row = q / (D / 8), ch = q % (D / 8);
     float vals[8];
-    load8<DT>(x, (int64_t)b * sb + (int64_t)(q_tokens + row) * st + (int64_t)h * sh + ch * 8, vals);
+    load8<DT>(x, (int64_t)b * sb + (int64_t)(ps.q + row) * st + (int64_t)h * sh + ch * 8, vals);
     *reinterpret_cast<uint4*>(cv.window + (seq * cv.window_len + row) * D + ch * 8) = pack8_f16(vals);
   }
   if (threadIdx.x == 0) {
-    cv.n_quant[seq] = q_tokens;
+    cv.n_quant[seq] = ps.q;
     cv.n_window[seq] = nw;
+    if (ps.bad && h == 0 && cv.status) atomicOr(cv.status, 4);
   }
 }
 
@@ -580,8 +604,8 @@ append_kernel(CacheView kc, CacheView vc, const void* __restrict__ k_new, const 
 size_t quant_smem_bytes() { return sizeof(QuantSmem); }
 
 template <int DT, int MODE>
-static cudaError_t launch_prefill_t(const void* x, int64_t sb, int64_t st, int64_t sh, int q_tokens,
-                                    const CacheView& cv, const float* cb, cudaStream_t s) {
+static cudaError_t launch_prefill_t(const void* x, int64_t sb, int64_t st, int64_t sh, int q_tokens, int n_tokens,
+                                    const int32_t* lengths, const CacheView& cv, const float* cb, cudaStream_t s) {
   const size_t smem = sizeof(QuantSmem);
   cudaError_t e = cudaFuncSetAttribute(quantize_prefill_kernel<DT, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -589,30 +613,39 @@ static cudaError_t launch_prefill_t(const void* x, int64_t sb, int64_t st, int64
   const int nblk = (q_tokens + BLK - 1) / BLK;
   if (nblk > 0) {
     dim3 grid(nblk, cv.n_kv_heads, cv.batch);
-    quantize_prefill_kernel<DT, MODE><<<grid, QTHREADS, smem, s>>>(x, sb, st, sh, q_tokens, cv, cb);
+    quantize_prefill_kernel<DT, MODE><<<grid, QTHREADS, smem, s>>>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv, cb);
   }
   return cudaGetLastError();
 }
 
+template <int MODE>
+static cudaError_t launch_prefill_m(const void* x, int dtype, int64_t sb, int64_t st, int64_t sh, int q_tokens,
+                                    int n_tokens, const int32_t* lengths, const CacheView& cv, const float* cb,
+                                    cudaStream_t s) {
+  if (dtype == NSN_DTYPE_F32)
+    return launch_prefill_t<NSN_DTYPE_F32, MODE>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv, cb, s);
+  if (dtype == NSN_DTYPE_BF16)
+    return launch_prefill_t<NSN_DTYPE_BF16, MODE>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv, cb, s);
+  return launch_prefill_t<NSN_DTYPE_F16, MODE>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv, cb, s);
+}
+
 cudaError_t launch_quantize_prefill(const void* x, int dtype, int64_t sb, int64_t st, int64_t sh, int q_tokens,
-                                    int n_tokens, const CacheView& cv, const float* cb, cudaStream_t s) {
-  cudaError_t e = cudaSuccess;
+                                    int n_tokens, const int32_t* lengths, const CacheView& cv, const float* cb,
+                                    cudaStream_t s) {
   if (q_tokens > 0) {
-    if (cv.mode == NSN_MODE_1BIT) {
-      if (dtype == NSN_DTYPE_F32) e = launch_prefill_t<NSN_DTYPE_F32, NSN_MODE_1BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
-      else if (dtype == NSN_DTYPE_BF16) e = launch_prefill_t<NSN_DTYPE_BF16, NSN_MODE_1BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
-      else e = launch_prefill_t<NSN_DTYPE_F16, NSN_MODE_1BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
-    } else {
-      if (dtype == NSN_DTYPE_F32) e = launch_prefill_t<NSN_DTYPE_F32, NSN_MODE_2BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
-      else if (dtype == NSN_DTYPE_BF16) e = launch_prefill_t<NSN_DTYPE_BF16, NSN_MODE_2BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
-      else e = launch_prefill_t<NSN_DTYPE_F16, NSN_MODE_2BIT>(x, sb, st, sh, q_tokens, cv, cb, s);
-    }
+    const cudaError_t e =
+        cv.mode == NSN_MODE_1BIT
+            ? launch_prefill_m<NSN_MODE_1BIT>(x, dtype, sb, st, sh, q_tokens, n_tokens, lengths, cv, cb, s)
+            : launch_prefill_m<NSN_MODE_2BIT>(x, dtype, sb, st, sh, q_tokens, n_tokens, lengths, cv, cb, s);
     if (e != cudaSuccess) return e;
   }
   dim3 g2(cv.n_kv_heads, cv.batch);
-  if (dtype == NSN_DTYPE_F32) window_fill_kernel<NSN_DTYPE_F32><<<g2, 128, 0, s>>>(x, sb, st, sh, q_tokens, n_tokens, cv);
-  else if (dtype == NSN_DTYPE_BF16) window_fill_kernel<NSN_DTYPE_BF16><<<g2, 128, 0, s>>>(x, sb, st, sh, q_tokens, n_tokens, cv);
-  else window_fill_kernel<NSN_DTYPE_F16><<<g2, 128, 0, s>>>(x, sb, st, sh, q_tokens, n_tokens, cv);
+  if (dtype == NSN_DTYPE_F32)
+    window_fill_kernel<NSN_DTYPE_F32><<<g2, 128, 0, s>>>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv);
+  else if (dtype == NSN_DTYPE_BF16)
+    window_fill_kernel<NSN_DTYPE_BF16><<<g2, 128, 0, s>>>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv);
+  else
+    window_fill_kernel<NSN_DTYPE_F16><<<g2, 128, 0, s>>>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv);
   return cudaGetLastError();
 }
 

@@ -69,9 +69,15 @@ def load():
     lib.nsn_cache_buffer_sizes.argtypes = [c_int, c_int, c_int, c_int, c_int, POINTER(nsn_cache_sizes)]
     lib.nsn_build_codebook_host.restype = c_int
     lib.nsn_build_codebook_host.argtypes = [c_uint64, c_int, c_int, c_int, c_int, c_int, POINTER(c_float)]
+    lib.nsn_build_codebook_cosine_host.restype = c_int
+    lib.nsn_build_codebook_cosine_host.argtypes = [c_uint64, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                   POINTER(c_float)]
     lib.nsn_quantize_kv.restype = c_int
     lib.nsn_quantize_kv.argtypes = [POINTER(nsn_cache), c_void_p, c_int, c_int64, c_int64, c_int64, c_int,
                                     c_void_p, c_void_p]
+    lib.nsn_quantize_kv_ragged.restype = c_int
+    lib.nsn_quantize_kv_ragged.argtypes = [POINTER(nsn_cache), c_void_p, c_int, c_int64, c_int64, c_int64, c_void_p,
+                                           c_int, c_void_p, c_void_p]
     lib.nsn_append_residual.restype = c_int
     lib.nsn_append_residual.argtypes = [POINTER(nsn_cache), POINTER(nsn_cache), c_void_p, c_void_p, c_int,
                                         c_int64, c_int64, c_void_p, c_void_p, c_void_p]
@@ -119,6 +125,18 @@ def nsn_build_codebook_host(seed: int, n_samples: int = 65536, n_codes: int = N_
                                         1 if abs_mode else 0, iters,
                                         out.ctypes.data_as(POINTER(c_float)))
     _check(st, "nsn_build_codebook_host")
+    return out
+
+
+def nsn_build_codebook_cosine_host(seed: int, n_samples: int = 65536, n_codes: int = N_CODES, dim: int = SUB_DIM,
+                                   abs_mode: bool = False, kmeans_iters: int = 50,
+                                   cosine_iters: int = 10) -> np.ndarray:
+    """k-means codebook fine-tuned for cosine distance [n_codes, dim] float32 (see include/nsn.h)."""
+    out = np.empty((n_codes, dim), dtype=np.float32)
+    st = load().nsn_build_codebook_cosine_host(c_uint64(seed & (2**64 - 1)), n_samples, n_codes, dim,
+                                               1 if abs_mode else 0, kmeans_iters, cosine_iters,
+                                               out.ctypes.data_as(POINTER(c_float)))
+    _check(st, "nsn_build_codebook_cosine_host")
     return out
 
 
@@ -176,6 +194,27 @@ def nsn_quantize_kv(cache: Cache, x, codebook, stream=None) -> None:
     st = load().nsn_quantize_kv(ctypes.byref(cache.c), x.data_ptr(), _dtype_code(x), x.stride(0), x.stride(1),
                                 x.stride(2), x.shape[1], codebook.data_ptr(), _stream_ptr(stream))
     _check(st, "nsn_quantize_kv")
+
+
+def nsn_quantize_kv_ragged(cache: Cache, x, lengths, codebook, max_tokens=None, stream=None) -> None:
+    """Ragged prefill of x [B, T, H_kv, 128]: sequence b takes lengths[b] tokens
+    (lengths: device int32 [B]); max_tokens defaults to T."""
+    if x.dim() != 4 or x.shape[-1] != HEAD_DIM or x.stride(-1) != 1:
+        raise ValueError("x must be [B, T, H_kv, 128] with a contiguous last dimension")
+    if x.shape[0] != cache.batch or x.shape[2] != cache.n_kv_heads:
+        raise ValueError("x batch / kv-head count does not match the cache")
+    import torch
+    if lengths.dtype != torch.int32 or lengths.dim() != 1 or lengths.shape[0] != cache.batch:
+        raise ValueError("lengths must be int32 [B]")
+    if lengths.stride(0) != 1 or lengths.device != x.device:
+        raise ValueError("lengths must be contiguous and on the device of x")
+    mt = x.shape[1] if max_tokens is None else int(max_tokens)
+    if mt > x.shape[1]:
+        raise ValueError("max_tokens exceeds the rows of x")
+    st = load().nsn_quantize_kv_ragged(ctypes.byref(cache.c), x.data_ptr(), _dtype_code(x), x.stride(0),
+                                       x.stride(1), x.stride(2), lengths.data_ptr(), mt, codebook.data_ptr(),
+                                       _stream_ptr(stream))
+    _check(st, "nsn_quantize_kv_ragged")
 
 
 def nsn_append_residual(k_cache: Cache, v_cache: Cache, k_new, v_new, cb_k, cb_v, stream=None) -> None:

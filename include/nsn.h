@@ -82,7 +82,9 @@ typedef enum { NSN_DTYPE_F32 = 0, NSN_DTYPE_BF16 = 1, NSN_DTYPE_F16 = 2 } nsn_dt
  *                                                       when window > 0)
  *   n_window int32  [batch][n_kv_heads]                 tokens in the residual window
  *   status   int32  [1] or NULL                         device error bits, OR-ed by kernels:
- *                                                       1 = capacity overflow on flush
+ *                                                       1 = capacity overflow on flush,
+ *                                                       2 = decode copy timeout,
+ *                                                       4 = ragged prefill length out of range
  * capacity must be a positive multiple of 128.  window must be 0 (quantize every
  * token, no append) or 128 (KIVI-style residual of one block).
  */
@@ -144,6 +146,24 @@ nsn_status nsn_build_codebook_host(uint64_t seed, int n_samples, int n_codes, in
                                    int abs_mode, int iters, float* out);
 
 /*
+ * Cosine-tuned codebook ([TS] Metodologia 3: the k-means codebook is fine-tuned to
+ * minimise the cosine distance between vectors and their quantized versions; [GH]
+ * Codebook tuning, "--method learned").  The pages give no procedure; this one
+ * alternates, cosine_iters times:
+ *   1. assign every sample to its nearest codeword (squared Euclidean, lowest index
+ *      on ties), as the quantizer assigns;
+ *   2. turn codeword c to the normalised sum of its members' unit vectors (the
+ *      direction that maximises their summed cosine) and give it the mean projection
+ *      of its members on that direction (the least-squares length).  A codeword with
+ *      no members, a zero direction sum or a non-positive mean projection is kept.
+ * Samples, k-means start (kmeans_iters Lloyd iterations) and the fp16 rounding of
+ * the result are those of nsn_build_codebook_host; cosine_iters = 0 gives its result.
+ */
+nsn_status nsn_build_codebook_cosine_host(uint64_t seed, int n_samples, int n_codes, int dim,
+                                          int abs_mode, int kmeans_iters, int cosine_iters,
+                                          float* out);
+
+/*
  * Prefill: quantizes n_tokens tokens of every (b, h) of x into a FRESH cache
  * (counters are overwritten).  [TS] Metodologia 1-3 (+ 4 for the residual split).
  *   x          device, dtype element type, token (b, t, h) row at
@@ -161,6 +181,23 @@ nsn_status nsn_build_codebook_host(uint64_t seed, int n_samples, int n_codes, in
 nsn_status nsn_quantize_kv(nsn_cache* cache, const void* x, int dtype, int64_t stride_b,
                            int64_t stride_t, int64_t stride_h, int n_tokens,
                            const float* codebook, void* stream);
+
+/*
+ * Ragged prefill: nsn_quantize_kv with one prompt length per batch row.  Sequence
+ * b takes lengths[b] tokens and is split by the same rule as a common length L
+ * ([TS] Metodologia 1-4 per sequence; the pages' runs use one sequence at a time).
+ *   lengths     device int32[batch], read by the kernels (no host synchronisation).
+ *               An entry outside [0, max_tokens] is treated as 0 and sets status
+ *               bit 4 (that sequence is left empty).
+ *   max_tokens  host bound on the lengths; it must satisfy the capacity rule that
+ *               n_tokens satisfies in nsn_quantize_kv.  Rows t >= lengths[b] of
+ *               sequence b are never read, so x may be padded or shorter per row.
+ * Everything else (x layout, codebook, stored values) is as in nsn_quantize_kv; with
+ * every length equal to L the cache bytes equal those of nsn_quantize_kv(..., L, ...).
+ */
+nsn_status nsn_quantize_kv_ragged(nsn_cache* cache, const void* x, int dtype, int64_t stride_b,
+                                  int64_t stride_t, int64_t stride_h, const int32_t* lengths,
+                                  int max_tokens, const float* codebook, void* stream);
 
 /*
  * Decode-time append of one new token per (b, h) to K and V ([TS] Metodologia 4,

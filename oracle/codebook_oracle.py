@@ -3,8 +3,10 @@
 The pages build the single global codebook by k-means on synthetic standard
 normal samples (torch.randn) -- "NSNQuant ... technical summary", Metodologia 3
 "Codebook: construccion" -- and the 2-bit variant on absolute values
-("NSNQuant" README, "Codebook tuning": ``--abs``).  The fine-tuning for cosine
-distance that the pages mention afterwards is not part of this path.
+("NSNQuant" README, "Codebook tuning": ``--abs``).  The same passage then
+fine-tunes the codebook to minimise the cosine distance between vectors and
+their quantized versions (README: ``--method learned``); `cosine_finetune`
+restates the reading of that step given below.
 
 The seeded standard-normal samples come from a counter-based generator that
 each side implements from its published definition:
@@ -24,6 +26,13 @@ the first K samples, nearest centroid by squared Euclidean distance with ties to
 the lowest index, empty clusters keep their centroid, a fixed iteration count;
 the result is rounded to fp16-representable values so that the fp32 quantizer
 and the fp16 decode read identical codewords.
+
+Cosine fine-tuning (a reading; the pages give no procedure): alternate
+(1) nearest-codeword assignment as above and (2) for every codeword with
+members, the direction maximising the summed cosine with its members (the
+normalised sum of their unit vectors) with the least-squares length along it
+(the members' mean projection); a codeword with no members, a zero direction
+sum or a non-positive mean projection is kept.
 
 Pinned by tests/test_oracle_codebook.py against numpy's own Philox bit
 generator, the moments and a Kolmogorov-Smirnov test of the normal stream, scipy's
@@ -110,6 +119,63 @@ def kmeans(samples: np.ndarray, n_codes: int, iters: int) -> np.ndarray:
             if members.shape[0] > 0:
                 cent[k] = members.sum(axis=0) / members.shape[0]
     return cent
+
+
+def nearest(x: np.ndarray, cent: np.ndarray) -> np.ndarray:
+    """Index of the nearest centroid (squared Euclidean, lowest index on ties)."""
+    diff_sq = np.empty((x.shape[0], cent.shape[0]))
+    for a in range(0, x.shape[0], 4096):
+        diff = x[a:a + 4096, None, :] - cent[None, :, :]
+        diff_sq[a:a + 4096] = np.sum(diff * diff, axis=2)
+    return np.argmin(diff_sq, axis=1)
+
+
+def cosine_step(x: np.ndarray, cent: np.ndarray, label: np.ndarray) -> np.ndarray:
+    """One cosine update of the centroids for fixed assignments `label`."""
+    x = np.asarray(x, dtype=np.float64)
+    new = np.array(cent, dtype=np.float64, copy=True)
+    norms = np.sqrt(np.sum(x * x, axis=1))
+    unit = np.divide(x, norms[:, None], out=np.zeros_like(x), where=norms[:, None] > 0)
+    for k in range(cent.shape[0]):
+        members = label == k
+        if not members.any():
+            continue
+        direction = unit[members].sum(axis=0)
+        length = math.sqrt(float(np.sum(direction * direction)))
+        if length == 0.0:
+            continue
+        direction = direction / length
+        proj = float(np.mean(x[members] @ direction))
+        if proj > 0.0:
+            new[k] = direction * proj
+    return new
+
+
+def cosine_finetune(samples: np.ndarray, cent: np.ndarray, iters: int) -> np.ndarray:
+    """Alternating nearest assignment and cosine update, `iters` times."""
+    x = np.asarray(samples, dtype=np.float64)
+    c = np.array(cent, dtype=np.float64, copy=True)
+    for _ in range(iters):
+        c = cosine_step(x, c, nearest(x, c))
+    return c
+
+
+def cosine_distance(x: np.ndarray, cent: np.ndarray) -> float:
+    """Mean 1 - cos(x, nearest codeword) over the samples (zero rows count 1)."""
+    x = np.asarray(x, dtype=np.float64)
+    q = cent[nearest(x, cent)]
+    num = np.sum(x * q, axis=1)
+    den = np.sqrt(np.sum(x * x, axis=1) * np.sum(q * q, axis=1))
+    cos = np.divide(num, den, out=np.zeros_like(num), where=den > 0)
+    return float(np.mean(1.0 - cos))
+
+
+def build_codebook_cosine(seed: int, n_samples: int, n_codes: int, dim: int, abs_mode: bool,
+                          kmeans_iters: int, cosine_iters: int) -> np.ndarray:
+    """k-means codebook fine-tuned for cosine distance, as fp16-representable values (fp64)."""
+    x = normal_samples(seed, n_samples, dim, abs_mode)
+    cent = cosine_finetune(x, kmeans(x, n_codes, kmeans_iters), cosine_iters)
+    return cent.astype(np.float16).astype(np.float64)
 
 
 def build_codebook(seed: int, n_samples: int, n_codes: int, dim: int,

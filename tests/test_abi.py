@@ -66,6 +66,12 @@ def test_host_validation_without_gpu(lib):
     assert lib.nsn_quantize_kv(ctypes.byref(c), 18, 1, 0, 1024, 128, 10, 16, None) == 1
     assert lib.nsn_quantize_kv(ctypes.byref(c), 16, 1, 0, 1020, 128, 10, 16, None) == 1
     assert lib.nsn_quantize_kv(ctypes.byref(c), 16, 1, 0, 1024, 128, 300, 16, None) == 1
+    # ragged prefill: lengths missing or misaligned, bound over capacity, negative bound
+    assert lib.nsn_quantize_kv_ragged(ctypes.byref(c), 16, 1, 0, 1024, 128, None, 10, 16, None) == 1
+    assert lib.nsn_quantize_kv_ragged(ctypes.byref(c), 16, 1, 0, 1024, 128, 18, 10, 16, None) == 1
+    assert lib.nsn_quantize_kv_ragged(ctypes.byref(c), 16, 1, 0, 1024, 128, 16, 300, 16, None) == 1
+    assert lib.nsn_quantize_kv_ragged(ctypes.byref(c), 16, 1, 0, 1024, 128, 16, -1, 16, None) == 1
+    assert lib.nsn_quantize_kv_ragged(ctypes.byref(odd), 16, 1, 0, 1024, 128, 16, 10, 16, None) == 2
     # decode: head count not a multiple, GQA group > 8, workspace too small
     c2 = nsn.nsn_cache(1, 2, 128, 128, 2, 1, 16, 16, 16, 16, 16, 16, 16, None)
     assert lib.nsn_decode_attention(ctypes.byref(c2), ctypes.byref(c2), 16, 1, 3, 0, 128, 0.1, 16, 16, 16, 16,
@@ -87,6 +93,15 @@ def test_host_codebook_matches_oracle(lib):
         ours = nsn.nsn_build_codebook_host(0x1234, 8192, 64, 8, abs_mode, 12)
         ref = cbo.build_codebook(0x1234, 8192, 64, 8, abs_mode, 12)
         assert np.array_equal(ours.astype(np.float64), ref)
+
+
+def test_host_cosine_codebook_matches_oracle(lib):
+    for abs_mode in (False, True):
+        ours = nsn.nsn_build_codebook_cosine_host(0x77, 8192, 64, 8, abs_mode, 8, 4)
+        ref = cbo.build_codebook_cosine(0x77, 8192, 64, 8, abs_mode, 8, 4)
+        assert np.array_equal(ours.astype(np.float64), ref)
+    with pytest.raises(nsn.NsnError):
+        nsn.nsn_build_codebook_cosine_host(1, 100, 256, 8, False, 3, -1)
 
 
 def test_host_codebook_full_size_properties(lib):

@@ -2,6 +2,8 @@
 own Philox bit generator, Box-Muller output statistics, and k-means against
 scipy's Lloyd iteration from the same initial centroids plus the fixed-point
 property."""
+import math
+
 import numpy as np
 import pytest
 from scipy import stats
@@ -67,3 +69,58 @@ def test_build_codebook_is_fp16_representable():
     cb = cbo.build_codebook(3, 1024, 16, 8, abs_mode=True, iters=3)
     assert np.array_equal(cb, cb.astype(np.float16).astype(np.float64))
     assert np.all(cb >= 0)
+
+
+# ---- cosine fine-tuning -------------------------------------------------------
+
+def test_cosine_step_2d_closed_form():
+    # One codeword, members on the plane: the summed cosine is maximised by the
+    # direction of the summed unit vectors, atan2(sum sin, sum cos), and the
+    # least-squares length is the mean projection on it.
+    rng = np.random.default_rng(3)
+    theta = rng.uniform(-0.7, 0.9, 50)
+    r = rng.uniform(0.5, 2.0, 50)
+    x = np.stack([r * np.cos(theta), r * np.sin(theta)], axis=1)
+    new = cbo.cosine_step(x, np.array([[1.0, 0.0]]), np.zeros(50, dtype=np.int64))
+    phi = math.atan2(np.sin(theta).sum(), np.cos(theta).sum())
+    length = np.mean(r * np.cos(theta - phi))
+    assert np.allclose(new[0], length * np.array([math.cos(phi), math.sin(phi)]), rtol=0, atol=1e-12)
+
+
+def test_cosine_step_is_locally_optimal_and_least_squares():
+    x = cbo.normal_samples(11, 2000, 8, False)
+    cent = cbo.kmeans(x, 16, 4)
+    label = cbo.nearest(x, cent)
+    new = cbo.cosine_step(x, cent, label)
+    rng = np.random.default_rng(0)
+    for k in range(16):
+        m = x[label == k]
+        u = new[k] / np.linalg.norm(new[k])
+        base = np.sum(m @ u / np.linalg.norm(m, axis=1))
+        for _ in range(20):   # no small turn of the direction raises the summed cosine
+            v = u + 1e-3 * rng.standard_normal(8)
+            v /= np.linalg.norm(v)
+            assert np.sum(m @ v / np.linalg.norm(m, axis=1)) <= base + 1e-12
+        s = np.linalg.norm(new[k])   # d/ds sum ||x - s u||^2 = 2 sum (s - x.u) = 0
+        assert abs(np.sum(s - m @ u)) <= 1e-9 * len(m)
+
+
+def test_cosine_step_keeps_codewords_without_members():
+    x = np.array([[1.0, 0.0], [0.9, 0.1]])
+    cent = np.array([[1.0, 0.0], [-5.0, 3.0]])
+    new = cbo.cosine_step(x, cent, np.array([0, 0]))
+    assert np.array_equal(new[1], cent[1])
+
+
+@pytest.mark.parametrize("abs_mode", [False, True])
+def test_cosine_finetune_lowers_the_cosine_distance(abs_mode):
+    x = cbo.normal_samples(21, 8192, 8, abs_mode)
+    km = cbo.kmeans(x, 32, 6)
+    ft = cbo.cosine_finetune(x, km, 5)
+    assert cbo.cosine_distance(x, ft) < cbo.cosine_distance(x, km)
+
+
+def test_cosine_zero_iterations_is_the_kmeans_codebook():
+    a = cbo.build_codebook_cosine(9, 4096, 32, 8, True, 5, 0)
+    b = cbo.build_codebook(9, 4096, 32, 8, True, 5)
+    assert np.array_equal(a, b)
