@@ -46,17 +46,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 # DRAM bytes (read + write) per decode_kernel launch on this workload, from one
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum; command and numbers
-# in profiles/launches-decode_b16_32k_2bit.md), valid only for the decode sources
-# with this SHA-256 (decode.cu, nsn_common.cuh, nsn_launch.h).  Any later change
-# to those files makes the figure stale, and the bench then reports null.
-DECODE_TRAFFIC = {"sha256": "150c974ccef32724836b1cb33dbb02515b03be4a614812d3a96723e5633616e2",
+# in profiles/launches-decode_b16_32k_2bit.md), valid only for the sources the
+# decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh).
+# Any later change to those files makes the figure stale; the bench then reports null.
+DECODE_TRAFFIC = {"sha256": "5a08e739df43722fa00263f71cb0330226fba0d7c1adb09305a58d8e73220af8",
                   "bytes_per_launch": 320636544 + 2836480}
 
 
 def decode_sources_sha256() -> str:
     import hashlib
     h = hashlib.sha256()
-    for name in ("decode.cu", "nsn_common.cuh", "nsn_launch.h"):
+    for name in ("decode.cu", "nsn_common.cuh"):
         with open(os.path.join(ROOT, "calibration_free_vector_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -393,26 +393,47 @@ def run_ours(args):
         pin_k = new_k.cpu().pin_memory()
         pin_v = new_v.cpu().pin_memory()
         pin_q = qs.cpu().pin_memory()
-        host_out = torch.empty((B, HQ, 128), dtype=torch.float32).pin_memory()
-        dk = torch.empty_like(new_k[0])
-        dv = torch.empty_like(new_v[0])
-        dq = torch.empty_like(qs[0])
+        # Pipelined like a serving loop: step s+1's inputs go up on one copy
+        # stream and step s-1's output comes down on another while step s runs;
+        # device inputs and outputs are double-buffered and ordered by events.
+        host_out = [torch.empty((B, HQ, 128), dtype=torch.float32).pin_memory() for _ in range(2)]
+        d_in = [(torch.empty_like(new_k[0]), torch.empty_like(new_v[0]), torch.empty_like(qs[0])) for _ in range(2)]
+        d_out = [torch.empty((B, HQ, 128), dtype=torch.float32, device=dev) for _ in range(2)]
+        up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of a buffer are on the device
+        ev_done = [torch.cuda.Event() for _ in range(2)]   # the step using a buffer has finished
+        ev_out = [torch.cuda.Event() for _ in range(2)]    # the output of a buffer is on the host
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        up.wait_event(e0)
+        down.wait_event(e0)
         for i in range(e2e_steps):
-            s = WU + K + i
-            dk.copy_(pin_k[s], non_blocking=True)
-            dv.copy_(pin_v[s], non_blocking=True)
-            dq.copy_(pin_q[s], non_blocking=True)
+            s, j = WU + K + i, i % 2
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(ev_done[j])
+                for dst, src in zip(d_in[j], (pin_k[s], pin_v[s], pin_q[s])):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[j].record(up)
+            stream.wait_event(ev_in[j])
+            if i >= 2:
+                stream.wait_event(ev_out[j])
+            dk, dv, dq = d_in[j]
             nsn.nsn_append_residual(kc, vc, dk, dv, cbk, cbv)
-            nsn.nsn_decode_attention(kc, vc, dq, scale, cbk, cbv, out, ws)
-            host_out.copy_(out, non_blocking=True)
+            nsn.nsn_decode_attention(kc, vc, dq, scale, cbk, cbv, d_out[j], ws)
+            ev_done[j].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_done[j])
+                host_out[j].copy_(d_out[j], non_blocking=True)
+                ev_out[j].record(down)
+        for j in range(2):
+            stream.wait_event(ev_out[j])
         e1.record(stream)
         torch.cuda.synchronize()
+        h2d = int(sum(t.numel() * t.element_size() for t in d_in[0]))
+        d2h = int(d_out[0].numel() * d_out[0].element_size())
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        h2d = (dk.numel() + dv.numel() + dq.numel()) * 2
-        d2h = host_out.numel() * 4
 
     status = int(kc.status.item()) | int(vc.status.item())
 
@@ -458,7 +479,9 @@ def run_ours(args):
                                       "peak": alu_peak, "unit": "T FMA/s (fp32)", "frac": q_ach / alu_peak,
                                       "algorithmic_fma_per_token_head": fma_per_th}},
             "e2e": {"value": job_throughput(B * e2e_steps, world, e2e_ms), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "copies": "every step: its new K/V token and q from pinned host memory, its output back; "
+                              "uploads of step s+1 and the download of step s-1 overlap step s"},
             "gpu_launches": K * LAUNCHES_PER_STEP,
             "clocks": clocks,
             "cache_status": status,

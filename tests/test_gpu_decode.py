@@ -40,7 +40,7 @@ def oracle_seq(c):
             "o": f(c["o"])}
 
 
-@pytest.mark.parametrize("g", [1, 4, 8])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
 @pytest.mark.parametrize("mk,mv", [(1, 1), (1, 2), (2, 1), (2, 2)])
 def test_decode_random_cache(mk, mv, g):
     B, H, cap = 3, 2, 2304
