@@ -49,8 +49,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # in profiles/launches-decode_b16_32k_2bit.md), valid only for the sources the
 # decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh).
 # Any later change to those files makes the figure stale; the bench then reports null.
-DECODE_TRAFFIC = {"sha256": "5a08e739df43722fa00263f71cb0330226fba0d7c1adb09305a58d8e73220af8",
-                  "bytes_per_launch": 320636544 + 2836480}
+DECODE_TRAFFIC = {"sha256": "c5a492144be6804a0b977c1b73172ac05ee1432866c35d8a68d7c6e4ea3b772f",
+                  "bytes_per_launch": 320970880 + 2323456}
 
 
 def decode_sources_sha256() -> str:

@@ -134,6 +134,9 @@ struct DecSmem {
   alignas(128) unsigned char stage[DEC_WARPS][2][STAGE_BYTES];
   alignas(128) unsigned char means[DEC_WARPS][2][MEAN_BYTES];
   alignas(8) uint64_t bar[DEC_WARPS][2];
+  int merge_n;                    // (sequence, head group)s whose last ticket a warp of this CTA took
+  int merge_seq[DEC_WARPS];
+  int merge_hg[DEC_WARPS];
 };
 
 __device__ __forceinline__ uint4 cb_row_f16(const float* __restrict__ cb, int c) {
@@ -166,9 +169,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
-// Bounded wait (at most WAIT_LIMIT suspended attempts); false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (uint32_t i = 0; i < WAIT_LIMIT; ++i)
+// Bounded wait (at most `limit` suspended attempts); false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit = WAIT_LIMIT) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }
@@ -210,9 +213,9 @@ constexpr int WCHUNK = 8;
 constexpr int WROWB = (D + 8) * 2;    // 272
 constexpr int WC_V = WCHUNK * WROWB;  // V rows follow the K rows
 static_assert(2 * WC_V <= STAGE_BYTES, "a window chunk fits one stage buffer");
-// The residual window counts as this many 128-token blocks when the quantized
-// blocks of a sequence are dealt out to its splits (the last split takes it).
-constexpr int WINDOW_COST_BLOCKS = 2;
+// The residual window counts as this many 64-token stages when the quantized
+// stages of a sequence are dealt out to its splits (the last split takes it).
+constexpr int WINDOW_COST_STAGES = 4;
 
 __device__ __forceinline__ void issue_window_chunk(uint32_t dst, uint32_t bar, const __half* krow, const __half* vrow,
                                                    int rows, int lane) {
@@ -225,23 +228,16 @@ __device__ __forceinline__ void issue_window_chunk(uint32_t dst, uint32_t bar, c
   }
 }
 
-// B operand of the score product for GH query heads: lane (g, p) holds column g
-// (head g for g < 4, the fp16 rounding residual of head g - 4 for g >= 4), k rows
-// 2p, 2p+1 (qb[j][0]) and 8+2p, 9+2p (qb[j][1]) of k-step j.  With `rotate` the
-// query is taken to the Hadamard domain first (orthonormal H).
+// Query rows of the GH heads of a group: lane l receives elements 4l..4l+3.
 template <int GH>
-__device__ __forceinline__ void build_q_operand(uint32_t (&qb)[8][2], const void* __restrict__ q, int dtype,
-                                                int64_t off0, int64_t qsh, float scale, bool rotate, int lane) {
-  const int g = lane >> 2, p = lane & 3;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) qb[j][0] = qb[j][1] = 0u;
+__device__ __forceinline__ void load_q_rows(float (&v)[GH][4], const void* __restrict__ q, int dtype, int64_t off0,
+                                            int64_t qsh, int lane) {
 #pragma unroll
   for (int h = 0; h < GH; ++h) {
     const int64_t off = off0 + (int64_t)h * qsh + 4 * lane;
-    float v[4];
     if (dtype == NSN_DTYPE_F32) {
       const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(q) + off));
-      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+      v[h][0] = f.x; v[h][1] = f.y; v[h][2] = f.z; v[h][3] = f.w;
     } else {
       const uint2 r = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(q) + off));
       float2 a, c;
@@ -252,25 +248,55 @@ __device__ __forceinline__ void build_q_operand(uint32_t (&qb)[8][2], const void
         a = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
         c = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
       }
-      v[0] = a.x; v[1] = a.y; v[2] = c.x; v[3] = c.y;
-    }
-    if (rotate) fwht128_warp(v, lane);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] *= scale;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int src = 4 * j + 2 * hf + (p >> 1);  // element 16j + 8hf + 2p lives in lane 4j + 2hf + p/2
-        const float e0 = __shfl_sync(0xffffffffu, v[0], src), e2 = __shfl_sync(0xffffffffu, v[2], src);
-        const float e1 = __shfl_sync(0xffffffffu, v[1], src), e3 = __shfl_sync(0xffffffffu, v[3], src);
-        const float x0 = (p & 1) ? e2 : e0, x1 = (p & 1) ? e3 : e1;
-        const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-        if (g == h) qb[j][hf] = pack_half2(__half2float(h0), __half2float(h1));
-        if (g == h + 4) qb[j][hf] = pack_half2(x0 - __half2float(h0), x1 - __half2float(h1));
-      }
+      v[h][0] = a.x; v[h][1] = a.y; v[h][2] = c.x; v[h][3] = c.y;
     }
   }
+}
+
+// B operand of the score product for GH query heads: lane (g, p) holds column g
+// (head g for g < 4, the fp16 rounding residual of head g - 4 for g >= 4), k rows
+// 2p, 2p+1 (qb[j][0]) and 8+2p, 9+2p (qb[j][1]) of k-step j.  With `rotate` the
+// query is taken to the Hadamard domain first (orthonormal H).  Each lane
+// converts its own 4 values per head once and stores them as rows of an 8 x 128
+// fp16 matrix (rows 0-3: fp16 of the heads, 4-7: rounding residuals; 272-byte
+// rows) in `qs`, a free 2176-byte stretch of this warp's shared memory; four
+// ldmatrix.x4 then deliver the fragments.
+constexpr int QS_ROW = (D + 8) * 2;
+template <int GH>
+__device__ __forceinline__ void build_q_operand(uint32_t (&qb)[8][2], const float (&rows)[GH][4], float scale,
+                                                bool rotate, int lane, unsigned char* qs) {
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    uint2 hi = make_uint2(0u, 0u), lo = make_uint2(0u, 0u);
+    if (h < GH) {
+      float v[4] = {rows[h < GH ? h : 0][0], rows[h < GH ? h : 0][1], rows[h < GH ? h : 0][2],
+                    rows[h < GH ? h : 0][3]};
+      if (rotate) fwht128_warp(v, lane);
+      float r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[i] *= scale;
+        r[i] = v[i] - __half2float(__float2half_rn(v[i]));
+      }
+      hi = make_uint2(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]));
+      lo = make_uint2(pack_half2(r[0], r[1]), pack_half2(r[2], r[3]));
+    }
+    *reinterpret_cast<uint2*>(qs + h * QS_ROW + 8 * lane) = hi;
+    *reinterpret_cast<uint2*>(qs + (h + 4) * QS_ROW + 8 * lane) = lo;
+  }
+  __syncwarp();
+  const uint32_t base = smem_addr(qs) + (uint32_t)((lane & 7) * QS_ROW + 16 * (lane >> 3));
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    uint32_t r4[4];
+    ldsm_x4(base + 64u * jj, r4);
+    qb[2 * jj][0] = r4[0];
+    qb[2 * jj][1] = r4[1];
+    qb[2 * jj + 1][0] = r4[2];
+    qb[2 * jj + 1][1] = r4[3];
+  }
+  __syncwarp();  // every lane has read the stretch ...
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // ... before a bulk copy may overwrite it
 }
 
 // Online-softmax state of one warp for its head pair (h0, h0 + 1): running max in
@@ -338,74 +364,92 @@ __device__ __forceinline__ void store_partial(SoftmaxState& st, float* __restric
   }
 }
 
-// Log-sum-exp merge of the partials of one (sequence, head group), done by the
-// warp that finished last.  Slots 0 .. nsplit-1 hold the quantized part (rotated
-// domain), slot nsplit the residual window (original domain).  The rotated value
-// sum is taken back with H (H^T = H) before both parts are normalised together.
-// Lane l owns dims 4l .. 4l+3.  Partials written by other SMs are read through L2.
+// Log-sum-exp merge of the partials of one (sequence, head group), done by all
+// threads of the CTA whose warp finished the group last.  Slots 0 .. nsplit-1
+// hold the quantized part (rotated domain), slot nsplit the residual window
+// (original domain).  The rotated value sum is taken back with H (H^T = H)
+// before both parts are normalised together.  Partials written by other SMs are
+// read through L2.  `scratch` is shared memory no longer in use (the stage
+// buffers): (nsplit + 1) * GH float2 weights, then GH * 128 floats.
 template <int GH>
-__device__ __noinline__ void merge_partials(const float* ws, const float* ws_acc, int64_t p0, int nsplit, int G, int hbase,
-                               float* __restrict__ out_rows, int lane) {
-  float mrot[GH], lrot[GH], a[GH][4];
+__device__ __noinline__ void cta_merge(const float* ws, const float* ws_acc, int64_t p0, int nsplit, int G, int hbase,
+                                       float* __restrict__ out_rows, float* scratch) {
+  constexpr int CH = 32;  // slots whose accumulators a thread holds in registers at once
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nslot = nsplit + 1;
+  float2* wt = reinterpret_cast<float2*>(scratch);          // [slot][h]: (m, l), then (weight, l)
+  float* rot = scratch + 2 * ((nslot * GH + 1) & ~1);       // [h][128] rotated sums, [h][128] window sums, [h] max
+  float* win = rot + GH * D;
+  const bool own = tid < GH * D;                            // thread (h, d) owns one output element
+  const int h = own ? tid / D : 0, d = tid % D;
+  const float* acc_hd = ws_acc + (p0 * G + hbase + h) * D + d;   // slot s at + s * G * D
+  // The accumulators of the first CH slots and the window element are requested
+  // together with the (m, l) pairs, so all of them share one L2 round trip.
+  float vals[CH];
 #pragma unroll
-  for (int h = 0; h < GH; ++h) {
-    mrot[h] = NEG_BIG;
-    lrot[h] = 0.f;
-    a[h][0] = a[h][1] = a[h][2] = a[h][3] = 0.f;
+  for (int k = 0; k < CH; ++k) vals[k] = (own && k < nsplit) ? __ldcg(acc_hd + (int64_t)k * G * D) : 0.f;
+  const float wv = own ? __ldcg(acc_hd + (int64_t)nsplit * G * D) : 0.f;
+  for (int i = tid; i < nslot * GH; i += blockDim.x) {
+    const int slot = i / GH, hh = i % GH;
+    wt[i] = __ldcg(reinterpret_cast<const float2*>(ws + ((p0 + slot) * G + hbase + hh) * 2));
   }
-  for (int s = lane; s < nsplit; s += 32) {
-#pragma unroll
-    for (int h = 0; h < GH; ++h) {
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(ws + ((p0 + s) * G + hbase + h) * 2));
-      if (ml.y > 0.f) mrot[h] = fmaxf(mrot[h], ml.x);
+  __syncthreads();
+  if (warp < GH) {  // warp hh: running max of the quantized slots, then their weights
+    const int hh = warp;
+    float mx = NEG_BIG;
+    for (int s = lane; s < nsplit; s += 32) {
+      const float2 ml = wt[s * GH + hh];
+      if (ml.y > 0.f) mx = fmaxf(mx, ml.x);
     }
+    mx = warp_max(mx);
+    for (int s = lane; s < nsplit; s += 32) {
+      const float2 ml = wt[s * GH + hh];
+      wt[s * GH + hh] = make_float2(ml.y > 0.f ? fast_exp2(ml.x - mx) : 0.f, ml.y);
+    }
+    if (lane == 0) win[GH * D + hh] = mx;
   }
+  __syncthreads();
+  if (own) {  // thread (h, d): weighted sum over the quantized slots
+    float acc = 0.f;
 #pragma unroll
-  for (int h = 0; h < GH; ++h) mrot[h] = warp_max(mrot[h]);
-  for (int s0 = 0; s0 < nsplit; s0 += 32) {
-    float f[GH];
-#pragma unroll
-    for (int h = 0; h < GH; ++h) {
-      f[h] = 0.f;
-      if (s0 + lane < nsplit) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(ws + ((p0 + s0 + lane) * G + hbase + h) * 2));
-        f[h] = ml.y > 0.f ? fast_exp2(ml.x - mrot[h]) : 0.f;
-        lrot[h] = fmaf(ml.y, f[h], lrot[h]);
-      }
-    }
-    const int cnt = min(32, nsplit - s0);
-#pragma unroll 4
-    for (int k = 0; k < cnt; ++k) {
-#pragma unroll
-      for (int h = 0; h < GH; ++h) {
-        const float fk = __shfl_sync(0xffffffffu, f[h], k);
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(ws_acc + ((p0 + s0 + k) * G + hbase + h) * D) + lane);
-        a[h][0] = fmaf(v.x, fk, a[h][0]);
-        a[h][1] = fmaf(v.y, fk, a[h][1]);
-        a[h][2] = fmaf(v.z, fk, a[h][2]);
-        a[h][3] = fmaf(v.w, fk, a[h][3]);
-      }
-    }
+    for (int k = 0; k < CH; ++k)
+      if (k < nsplit) acc = fmaf(vals[k], wt[k * GH + h].x, acc);
+    for (int s = CH; s < nsplit; ++s) acc = fmaf(__ldcg(acc_hd + (int64_t)s * G * D), wt[s * GH + h].x, acc);
+    rot[h * D + d] = acc;
+    win[h * D + d] = wv;
   }
+  __syncthreads();
+  if (warp < GH) {  // warp hh: H applied to the rotated sum, window part, normalisation
+    const int hh = warp;
+    float lr = 0.f;
+    for (int s = lane; s < nsplit; s += 32) {
+      const float2 wl = wt[s * GH + hh];
+      lr = fmaf(wl.y, wl.x, lr);
+    }
+    lr = warp_sum(lr);
+    const float mrot = win[GH * D + hh];
+    float a[4], aw[4];
 #pragma unroll
-  for (int h = 0; h < GH; ++h) {
-    const float lr = warp_sum(lrot[h]);
-    fwht128_warp(a[h], lane);
-    const float2 mlw = __ldcg(reinterpret_cast<const float2*>(ws + ((p0 + nsplit) * G + hbase + h) * 2));
-    const float4 aw = __ldcg(reinterpret_cast<const float4*>(ws_acc + ((p0 + nsplit) * G + hbase + h) * D) + lane);
+    for (int i = 0; i < 4; ++i) {
+      a[i] = rot[hh * D + 4 * lane + i];
+      aw[i] = win[hh * D + 4 * lane + i];
+    }
+    fwht128_warp(a, lane);
+    const float2 mlw = wt[nsplit * GH + hh];
     const float mw = mlw.y > 0.f ? mlw.x : NEG_BIG, lw = mlw.y;
-    const float mt = fmaxf(mrot[h], mw);
-    const float fa = lr > 0.f ? fast_exp2(mrot[h] - mt) : 0.f;
+    const float mt = fmaxf(mrot, mw);
+    const float fa = lr > 0.f ? fast_exp2(mrot - mt) : 0.f;
     const float fr = lw > 0.f ? fast_exp2(mw - mt) : 0.f;
     const float den = lr * fa + lw * fr;
     const float inv = den > 0.f ? 1.f / den : 0.f;
     float4 o;
-    o.x = (a[h][0] * INV_SQRT_D * fa + aw.x * fr) * inv;
-    o.y = (a[h][1] * INV_SQRT_D * fa + aw.y * fr) * inv;
-    o.z = (a[h][2] * INV_SQRT_D * fa + aw.z * fr) * inv;
-    o.w = (a[h][3] * INV_SQRT_D * fa + aw.w * fr) * inv;
-    *reinterpret_cast<float4*>(out_rows + (int64_t)h * D + 4 * lane) = o;
+    o.x = (a[0] * INV_SQRT_D * fa + aw[0] * fr) * inv;
+    o.y = (a[1] * INV_SQRT_D * fa + aw[1] * fr) * inv;
+    o.z = (a[2] * INV_SQRT_D * fa + aw[2] * fr) * inv;
+    o.w = (a[3] * INV_SQRT_D * fa + aw[3] * fr) * inv;
+    *reinterpret_cast<float4*>(out_rows + (int64_t)hh * D + 4 * lane) = o;
   }
+  __syncthreads();  // the scratch may be reused by the next merge of this CTA
 }
 
 // One warp = one split of one (sequence, head group); GH <= 4 query heads per
@@ -434,25 +478,11 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
   const int G = geom.g;           // query heads per kv-head
   const int ngroups = G / GH;     // head groups per kv-head
   const int nsplit = geom.nsplit_q;
-
-  // ---- stage the replicated fp16 codebooks (whole CTA, once) ----
-  for (int e = tid; e < NCODES * 8; e += blockDim.x) {
-    const int c = e >> 3, r = e & 7;
-    sm.cbk[c][r] = cb_row_f16(cbk_g, c);
-    sm.cbv[c][r] = cb_row_f16(cbv_g, c);
-  }
-  if (lane == 0) {
-    mbar_init(smem_addr(&sm.bar[warp][0]), 1);
-    mbar_init(smem_addr(&sm.bar[warp][1]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  }
-  __syncthreads();
-
   const int nseq = kc.batch * kc.n_kv_heads;
   const int gw = blockIdx.x * DEC_WARPS + warp;  // global warp job id
-  if (gw >= nseq * nsplit * ngroups) return;
+  const bool active = gw < nseq * nsplit * ngroups;
   const int hg = gw % ngroups;
-  const int64_t seq = (gw / ngroups) / nsplit;
+  const int64_t seq = active ? (gw / ngroups) / nsplit : 0;
   const int split = (gw / ngroups) % nsplit;
   const int b = (int)(seq / kc.n_kv_heads), hk = (int)(seq % kc.n_kv_heads);
   const int hbase = hg * GH;                      // first head of the group within the kv-head
@@ -461,28 +491,64 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
   float* ws_acc = ws + acc_offset(P, G);
   const int64_t q_off = (int64_t)b * qsb + (int64_t)(hk * G + hbase) * qsh;
 
-  const int nq = min(min(kc.n_quant[seq], vc.n_quant[seq]), kc.capacity);
+  // The query rows are requested first, before the codebook staging and the bulk
+  // copies, so that they do not queue behind the copies of every warp.
+  // Prologue order: the query rows, the cache counters and this thread's codeword
+  // are requested first; each warp then arms its own barriers and issues its
+  // first bulk copy (no CTA barrier needed), builds its query operand while that
+  // copy flies, issues its second copy, and only then does the CTA store the
+  // codebooks and meet at the one barrier.
+  float qrows[GH][4];
+  if (active) load_q_rows<GH>(qrows, q, dtype, q_off, qsh, lane);
+  static_assert(32 * DEC_WARPS == 2 * NCODES, "one codeword per thread");
+  const int cb_c = tid & (NCODES - 1);
+  const bool cb_isv = tid >= NCODES;
+  const uint4 cb_row = cb_row_f16(cb_isv ? cbv_g : cbk_g, cb_c);
+
+  const int nq = active ? min(min(kc.n_quant[seq], vc.n_quant[seq]), kc.capacity) : 0;
   const int nw = (kc.window_len > 0) ? max(0, min(min(kc.n_window[seq], vc.n_window[seq]), kc.window_len)) : 0;
-  const int nblk = (nq + BLK - 1) / BLK;
-  const int bps = max(1, (nblk + (nw > 0 ? WINDOW_COST_BLOCKS : 0) + nsplit - 1) / nsplit);  // blocks per split
-  const int tok_begin = min(nq, split * bps * BLK);
-  const int tok_end = min(nq, (split + 1) * bps * BLK);
-  const bool has_window = split == nsplit - 1;
+  // Splits are dealt whole 64-token stages, so a split may start or end inside
+  // a 128-token block (the block's mean terms are then split between them too).
+  const int nst_all = (nq + STAGE_TOK - 1) / STAGE_TOK;
+  const int sps = max(1, (nst_all + (nw > 0 ? WINDOW_COST_STAGES : 0) + nsplit - 1) / nsplit);  // stages per split
+  const int tok_begin = min(nq, split * sps * STAGE_TOK);
+  const int tok_end = min(nq, (split + 1) * sps * STAGE_TOK);
+  const bool has_window = active && split == nsplit - 1;
   const uint32_t st_base = smem_addr(&sm.stage[warp][0][0]);
   const uint32_t mb_base = smem_addr(&sm.means[warp][0][0]);
   const uint32_t bar0 = smem_addr(&sm.bar[warp][0]);
   const int nstages = (tok_end - tok_begin + STAGE_TOK - 1) / STAGE_TOK;
 
-  if (lane == 0 && nstages > 0) {
-    issue_stage<MK, MV>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc, seq,
-                        tok_begin, true);
-    if (nstages > 1)
-      issue_stage<MK, MV>(st_base + STAGE_BYTES, mb_base, bar0 + 8, kc, vc, seq, tok_begin + STAGE_TOK, false);
+  if (lane == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8u, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    if (nstages > 0)
+      issue_stage<MK, MV>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc, seq,
+                          tok_begin, true);
+  }
+  __syncwarp();
+
+  // ---- query operand (B of the score product), built while stage 0 flies, in
+  // the second stage buffer, which is filled only afterwards ----
+  uint32_t qb[8][2];
+  if (active) build_q_operand<GH>(qb, qrows, qscale * INV_SQRT_D, true, lane, &sm.stage[warp][1][0]);
+  if (lane == 0 && nstages > 1) {
+    const int t1 = tok_begin + STAGE_TOK;
+    issue_stage<MK, MV>(st_base + STAGE_BYTES, mb_base + (uint32_t)(((t1 / BLK) & 1) * MEAN_BYTES), bar0 + 8, kc, vc,
+                        seq, t1, (t1 % BLK) == 0);
   }
 
-  // ---- query operand (B of the score product), built while the copies fly ----
-  uint32_t qb[8][2];
-  build_q_operand<GH>(qb, q, dtype, q_off, qsh, qscale * INV_SQRT_D, true, lane);
+  // ---- stage the replicated fp16 codebooks (whole CTA, once) ----
+  // One codeword per thread, stored as 8 replicas in a rotated order so that the
+  // 8 lanes of a quarter-warp hit 8 bank groups.
+  {
+    uint4* dst = cb_isv ? &sm.cbv[cb_c][0] : &sm.cbk[cb_c][0];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) dst[(r + cb_c) & 7] = cb_row;
+  }
+  if (tid == 0) sm.merge_n = 0;
+  __syncthreads();
 
   const uint32_t lane_row = (uint32_t)(lane & 7) * 16u;
   const uint32_t cbk_base = smem_addr(&sm.cbk[0][0]) + lane_row;
@@ -518,7 +584,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     }
     phase ^= 1u << buf;
     const int t_stage = tok_begin + st * STAGE_TOK;
-    const bool block_start = (t_stage % BLK) == 0;
+    const bool block_start = (t_stage % BLK) == 0 || st == 0;  // (q~ . o_b needed from the split's first stage)
     const bool block_end = ((t_stage + STAGE_TOK) % BLK) == 0 || st == nstages - 1;
     const int mbuf = (t_stage / BLK) & 1;
     const unsigned char* sb = &sm.stage[warp][buf][0];
@@ -647,7 +713,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
                           bar0 + 8u * buf, kc, vc, seq, tn, (tn % BLK) == 0);
     }
   }
-  store_partial<GH>(sx, ws, ws_acc, p0 + split, G, hbase, lane);
+  if (active) store_partial<GH>(sx, ws, ws_acc, p0 + split, G, hbase, lane);
 
   // ---- residual window (original domain), last split only ----
   if (has_window) {
@@ -659,9 +725,11 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       const __half* kw0 = kc.window + seq * kc.window_len * D;
       const __half* vw0 = vc.window + seq * vc.window_len * D;
       issue_window_chunk(st_base, bar0, kw0, vw0, min(WCHUNK, nw), lane);
+      float wrows[GH][4];  // reloaded: keeping the first rows alive would cost registers in the main loop
+      load_q_rows<GH>(wrows, q, dtype, q_off, qsh, lane);
+      build_q_operand<GH>(qb, wrows, qscale, false, lane, &sm.stage[warp][1][0]);
       if (nch > 1) issue_window_chunk(st_base + STAGE_BYTES, bar0 + 8u, kw0 + WCHUNK * D, vw0 + WCHUNK * D,
                                       min(WCHUNK, nw - WCHUNK), lane);
-      build_q_operand<GH>(qb, q, dtype, q_off, qsh, qscale, false, lane);
       const int wr = lane & 7;  // ldmatrix row (token) of this lane; rows 8-15 repeat rows 0-7
       for (int c = 0; c < nch; ++c) {
         const int buf = c & 1;
@@ -721,16 +789,31 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     if (pending & 2) mbar_wait(bar0 + 8u, (phase >> 1) & 1u);
   }
 
-  // ---- the last warp of this (sequence, head group) merges the partials ----
+  // ---- the last warp of this (sequence, head group) hands it to its CTA ----
   __threadfence();  // this warp's partial stores are visible device-wide ...
-  __syncwarp();      // ... for every lane before lane 0 takes the ticket
-  unsigned int ticket = 0u;
-  if (lane == 0) ticket = atomicInc(&counters[seq * ngroups + hg], (unsigned int)(nsplit - 1));
-  ticket = __shfl_sync(0xffffffffu, ticket, 0);
-  if (ticket != (unsigned int)(nsplit - 1)) return;
+  __syncwarp();     // ... for every lane before lane 0 takes the ticket
+  if (active && lane == 0) {
+    const unsigned int ticket = atomicInc(&counters[seq * ngroups + hg], (unsigned int)(nsplit - 1));
+    if (ticket == (unsigned int)(nsplit - 1)) {
+      __threadfence();
+      const int k = atomicAdd(&sm.merge_n, 1);
+      sm.merge_seq[k] = (int)seq;
+      sm.merge_hg[k] = hg;
+    }
+  }
+
+  // ---- the whole CTA merges the groups whose last ticket it took ----
+  __syncthreads();  // every warp is done with its stage buffers, the merge list is complete
+  const int n_merge = sm.merge_n;
+  if (n_merge == 0) return;
   __threadfence();
-  merge_partials<GH>(ws, ws_acc, p0, nsplit, G, hbase,
-                     out + ((int64_t)b * n_q_heads + hk * G + hbase) * D, lane);
+  float* scratch = reinterpret_cast<float*>(&sm.stage[0][0][0]);
+  for (int m = 0; m < n_merge; ++m) {
+    const int mseq = sm.merge_seq[m], mhg = sm.merge_hg[m];
+    const int mb = mseq / kc.n_kv_heads, mhk = mseq % kc.n_kv_heads;
+    cta_merge<GH>(ws, ws + acc_offset(P, G), (int64_t)mseq * (nsplit + 1), nsplit, G, mhg * GH,
+                  out + ((int64_t)mb * n_q_heads + mhk * G + mhg * GH) * D, scratch);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -825,6 +908,30 @@ cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* 
   unsigned int* counters = static_cast<unsigned int*>(ws);
   float* partials = static_cast<float*>(ws) + counter_words((int64_t)kc.batch * kc.n_kv_heads);
   return launch_any(kc, vc, q, dtype, n_q_heads, qsb, qsh, softmax_scale, cbk, cbv, out, counters, partials, geom, s);
+}
+
+// ---------------------------------------------------------------------------
+// Diagnostic of the bounded wait: one warp arms an mbarrier for a copy that is
+// never issued and waits on it with the decode's wait helper, capped at `limit`
+// attempts.  The wait must give up, set status bit 2 and return, so the error
+// path of a copy that never lands can be tested without a fault or a hang.
+// ---------------------------------------------------------------------------
+__global__ void bounded_wait_selftest_kernel(int32_t* status, uint32_t limit) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    mbar_expect_tx(b, 16u);  // 16 bytes are announced; none will arrive
+  }
+  __syncwarp();
+  const bool arrived = mbar_wait(b, 0u, limit);
+  if (!__all_sync(0xffffffffu, arrived) && threadIdx.x == 0 && status) atomicOr(status, 2);
+}
+
+cudaError_t launch_bounded_wait_selftest(int32_t* status, uint32_t limit, cudaStream_t s) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(status, limit);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------

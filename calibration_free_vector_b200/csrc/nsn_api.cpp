@@ -218,4 +218,11 @@ nsn_status nsn_decode_attention_static(const nsn_cache* k_cache, const nsn_cache
                                                static_cast<cudaStream_t>(stream)));
 }
 
+nsn_status nsn_selftest_bounded_wait(int32_t* status, int max_attempts, void* stream) {
+  if (!status || (reinterpret_cast<uintptr_t>(status) & 3u) || max_attempts <= 0 || max_attempts > 4096)
+    return NSN_ERR_INVALID_ARG;
+  return cuda_status(nsn::launch_bounded_wait_selftest(status, (uint32_t)max_attempts,
+                                                       static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

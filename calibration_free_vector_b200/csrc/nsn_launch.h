@@ -57,4 +57,7 @@ cudaError_t launch_decode_static(const CacheView& kc, const CacheView& vc, const
                                  int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
                                  float* out, const DecodeGeom& geom, cudaStream_t s);
 
+// Bounded-wait diagnostic (see nsn_selftest_bounded_wait).
+cudaError_t launch_bounded_wait_selftest(int32_t* status, uint32_t limit, cudaStream_t s);
+
 }  // namespace nsn

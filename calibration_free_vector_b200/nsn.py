@@ -75,6 +75,8 @@ def load():
     lib.nsn_quantize_kv.restype = c_int
     lib.nsn_quantize_kv.argtypes = [POINTER(nsn_cache), c_void_p, c_int, c_int64, c_int64, c_int64, c_int,
                                     c_void_p, c_void_p]
+    lib.nsn_selftest_bounded_wait.restype = c_int
+    lib.nsn_selftest_bounded_wait.argtypes = [c_void_p, c_int, c_void_p]
     lib.nsn_quantize_kv_ragged.restype = c_int
     lib.nsn_quantize_kv_ragged.argtypes = [POINTER(nsn_cache), c_void_p, c_int, c_int64, c_int64, c_int64, c_void_p,
                                            c_int, c_void_p, c_void_p]
@@ -227,6 +229,12 @@ def nsn_append_residual(k_cache: Cache, v_cache: Cache, k_new, v_new, cb_k, cb_v
                                     v_new.data_ptr(), _dtype_code(k_new), k_new.stride(0), k_new.stride(1),
                                     cb_k.data_ptr(), cb_v.data_ptr(), _stream_ptr(stream))
     _check(st, "nsn_append_residual")
+
+
+def nsn_selftest_bounded_wait(status, max_attempts: int = 8, stream=None) -> None:
+    """Runs the bounded-wait diagnostic; `status` is a device int32 tensor of one element."""
+    _check(load().nsn_selftest_bounded_wait(status.data_ptr(), max_attempts, _stream_ptr(stream)),
+           "nsn_selftest_bounded_wait")
 
 
 def nsn_decode_workspace_bytes(k_cache: Cache, n_q_heads: int) -> int:

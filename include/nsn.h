@@ -238,8 +238,9 @@ size_t nsn_decode_workspace_bytes(const nsn_cache* k_cache, int n_q_heads);
  *                  later calls need no clearing.  Calls sharing one workspace must not
  *                  overlap on the GPU.
  * One kernel launch: the quantized blocks of each (b, kv-head) are dealt out to
- * splits, the last split also attends the window, and the split that completes a
- * (b, kv-head, head group) last merges the partials into `out`.  Status bit 2 of
+ * splits, the last split also attends the window, and the thread block of the
+ * split that completes a (b, kv-head, head group) last merges the partials into
+ * `out`.  Status bit 2 of
  * k_cache->status is set if a copy into shared memory did not complete in time
  * (the affected outputs are then not meaningful).
  */
@@ -277,6 +278,15 @@ nsn_status nsn_decode_attention_static(const nsn_cache* k_cache, const nsn_cache
                                        int dtype, int n_q_heads, int64_t q_stride_b, int64_t q_stride_h,
                                        float softmax_scale, const float* cb_k, const float* cb_v, float* out,
                                        void* stream);
+
+/*
+ * Diagnostic of the decode's error path for a copy that never lands (the pages
+ * have no counterpart).  Launches one warp that announces 16 bytes on an mbarrier,
+ * issues no copy, and waits with the decode's bounded wait capped at max_attempts
+ * suspended attempts (1..4096, each at most about a millisecond).  The wait gives
+ * up, sets bit 2 of *status (device int32) and returns; the context stays usable.
+ */
+nsn_status nsn_selftest_bounded_wait(int32_t* status, int max_attempts, void* stream);
 
 #ifdef __cplusplus
 }
