@@ -47,18 +47,25 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # DRAM bytes (read + write) per decode_kernel launch on this workload, from one
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum; command and numbers
 # in profiles/launches-decode_b16_32k_2bit.md), valid only for the sources the
-# decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh).
+# decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh,
+# comments and whitespace removed).
 # Any later change to those files makes the figure stale; the bench then reports null.
-DECODE_TRAFFIC = {"sha256": "c5a492144be6804a0b977c1b73172ac05ee1432866c35d8a68d7c6e4ea3b772f",
+DECODE_TRAFFIC = {"sha256": "8deb421e700413a24f67a81de22c64a9e8d7a64df6e6185427734245cc29a14d",
                   "bytes_per_launch": 320970880 + 2323456}
 
 
 def decode_sources_sha256() -> str:
+    """SHA-256 of the decode kernel's sources with comments and whitespace removed
+    (a comment edit does not change the kernel the traffic figure belongs to)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for name in ("decode.cu", "nsn_common.cuh"):
-        with open(os.path.join(ROOT, "calibration_free_vector_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "calibration_free_vector_b200", "csrc", name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()
 
 

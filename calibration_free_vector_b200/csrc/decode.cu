@@ -12,15 +12,15 @@
 // Residual-window tokens are attended in the original domain.
 //
 // One kernel (decode_kernel) does the whole call:
-//   - one warp per split (a contiguous range of 128-token blocks of one (batch,
+//   - one warp per split (a contiguous range of 64-token stages of one (batch,
 //     kv-head) and a group of up to 4 query heads): rotated query, scores from the
 //     codes, online softmax, value accumulation from the codewords -> partial
 //     (m, l, acc) in the rotated domain;
 //   - the last split of a sequence also attends the residual window (original
 //     domain) -> a second partial;
-//   - the warp that finishes a (sequence, head group) last (a self-resetting
-//     counter decides) merges the partials by log-sum-exp, applies H to the
-//     rotated value sum and writes the output rows.
+//   - the thread block of the warp that finishes a (sequence, head group) last
+//     (a self-resetting counter decides) merges the partials by log-sum-exp,
+//     applies H to the rotated value sum and writes the output rows.
 // Scores are carried in log2 units (the query is pre-scaled by softmax_scale*log2 e).
 
 #include <mutex>
@@ -98,11 +98,11 @@ __device__ __forceinline__ uint32_t u4_word(const uint4& v, int i) {
 
 // ---------------------------------------------------------------------------
 // Quantized part.  One CTA of 16 warps per SM; every warp owns one split: a
-// contiguous range of 128-token blocks of one (batch, kv-head) sequence, and
-// writes its own partial (m, l, O).  The CTA shares only the two replicated
-// fp16 codebooks (staged once).  Compressed tokens stream through a per-warp
-// double-buffered ring of 64-token stages filled by cp.async, so one stage is
-// always in flight while the previous one is consumed.
+// contiguous range of 64-token stages of one (batch, kv-head) sequence, and
+// writes its own partial (m, l, O).  The CTA shares the two replicated fp16
+// codebooks (staged once) and, at the end, the merge.  Compressed tokens stream
+// through a per-warp double-buffered ring of 64-token stages filled by 1-D bulk
+// copies, so one stage is always in flight while the previous one is consumed.
 //
 // Per 16-token tile a warp computes, on the tensor cores,
 //   S^T[h][t]  = sum_k q~[h][k] u_hat[t][k]   (M = heads, N = 8 tokens, K = 16 dims)
@@ -454,9 +454,10 @@ __device__ __noinline__ void cta_merge(const float* ws, const float* ws_acc, int
 
 // One warp = one split of one (sequence, head group); GH <= 4 query heads per
 // warp (a group of 8 runs as two head groups).  A split is a contiguous range of
-// 128-token blocks; the last split of a sequence also attends the residual window.
-// The warp that completes a (sequence, head group) last merges its partials into
-// the output, so one launch does the whole decode.
+// 64-token stages (it may start or end inside a 128-token block); the last split
+// of a sequence also attends the residual window.  The CTA of the warp that
+// completes a (sequence, head group) last merges its partials into the output,
+// so one launch does the whole decode.
 //
 // Scores:  S[t][c] = sum_k u_hat[t][k] Qc[k][c]   M = 16 tokens, N = 8 columns, K = 16
 //          (columns 0-3: fp16(q~) of the GH heads, 4-7: their fp16 rounding residual),
