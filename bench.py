@@ -38,6 +38,10 @@ WORKLOAD = dict(config=3, name="decode-b16-32k-2bit", batch=16, n_kv_heads=8, n_
                 mode_k=2, mode_v=2, window=128)
 BYTES_PER_TOKEN = {1: 16 + 4, 2: 16 + 16 + 4}   # codes (+ signs) + (s1, s2) per token-head
 MEAN_BYTES_PER_BLOCK = 128 * 2
+# With double quantization s1 is a 4-bit level (0.5 B) next to fp16 alpha*s2, and a
+# block's o is 64 B of levels plus 16 B of (lo, hi) parameters.
+BYTES_PER_TOKEN_DQ = {1: 16 + 2.5, 2: 16 + 16 + 2.5}
+MEAN_BYTES_PER_BLOCK_DQ = 64 + 16
 # Kernels one decode step launches: append_kernel (K and V, flush included) and
 # decode_kernel (splits, residual window and merge).
 LAUNCHES_PER_STEP = 2
@@ -50,8 +54,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh,
 # comments and whitespace removed).
 # Any later change to those files makes the figure stale; the bench then reports null.
-DECODE_TRAFFIC = {"sha256": "8deb421e700413a24f67a81de22c64a9e8d7a64df6e6185427734245cc29a14d",
-                  "bytes_per_launch": 320970880 + 2323456}
+DECODE_TRAFFIC = {"sha256": "d185012d09b25d085472f087fae6804a393b62f07760bbafe256260b3ab4c243",
+                  "bytes_per_launch": 320946176 + 2808320}
 
 
 def decode_sources_sha256() -> str:
@@ -288,8 +292,10 @@ def run_ours(args):
 
     rk = synthetic.KVRecipe(synthetic.config_seed(3, "k") + rank_seed_offset(rank), H)
     rv = synthetic.KVRecipe(synthetic.config_seed(3, "v") + rank_seed_offset(rank), H)
-    kc = nsn.Cache(B, H, cap, W["window"], W["mode_k"], device=dev)
-    vc = nsn.Cache(B, H, cap, W["window"], W["mode_v"], device=dev)
+    kc = nsn.Cache(B, H, cap, W["window"], W["mode_k"], device=dev, double_quant=args.double_quant)
+    vc = nsn.Cache(B, H, cap, W["window"], W["mode_v"], device=dev, double_quant=args.double_quant)
+    per_token_bytes = BYTES_PER_TOKEN_DQ if args.double_quant else BYTES_PER_TOKEN
+    mean_block_bytes = MEAN_BYTES_PER_BLOCK_DQ if args.double_quant else MEAN_BYTES_PER_BLOCK
     stream = torch.cuda.current_stream()
 
     # ---- prefill (quantizer throughput is measured here) ----
@@ -373,10 +379,10 @@ def run_ours(args):
     # The (n_quant, n_window) of every step follow from the state before the timed
     # region: each append first flushes a full window into one quantized block.
     seqs = B * H
-    per_tok = BYTES_PER_TOKEN[W["mode_k"]] + BYTES_PER_TOKEN[W["mode_v"]]
+    per_tok = per_token_bytes[W["mode_k"]] + per_token_bytes[W["mode_v"]]
 
     def call_bytes(nq_s, nw_s):
-        compressed_s = seqs * (nq_s * per_tok + 2 * (nq_s // 128) * MEAN_BYTES_PER_BLOCK)
+        compressed_s = seqs * (nq_s * per_tok + 2 * (nq_s // 128) * mean_block_bytes)
         return compressed_s + seqs * 2 * nw_s * 128 * 2 + B * HQ * 128 * (2 + 4)
 
     nq_s, nw_s, step_bytes = nq_start, nw_start, []
@@ -387,7 +393,7 @@ def run_ours(args):
         step_bytes.append(call_bytes(nq_s, nw_s))
     nq, nw = int(kc.n_quant[0, 0].item()), int(kc.n_window[0, 0].item())
     assert (nq, nw) == (nq_s, nw_s), "counter schedule differs from the cache state"
-    compressed = seqs * (nq * per_tok + 2 * (nq // 128) * MEAN_BYTES_PER_BLOCK)
+    compressed = seqs * (nq * per_tok + 2 * (nq // 128) * mean_block_bytes)
     decode_bytes = float(np.mean(step_bytes))
     dec_avg_ms = float(np.mean(decode_ms))
     peaks, peak_kind = load_peaks()
@@ -446,8 +452,8 @@ def run_ours(args):
 
     # ---- quantizer roofline (ALU-bound exhaustive search) ----
     qtoken_heads = 2 * B * H * q_tokens
-    q_bytes = B * H * q_tokens * (2 * 256 + (BYTES_PER_TOKEN[W["mode_k"]] + BYTES_PER_TOKEN[W["mode_v"]])) \
-        + 2 * B * H * (q_tokens // 128) * MEAN_BYTES_PER_BLOCK
+    q_bytes = B * H * q_tokens * (2 * 256 + (per_token_bytes[W["mode_k"]] + per_token_bytes[W["mode_v"]])) \
+        + 2 * B * H * (q_tokens // 128) * mean_block_bytes
     fma_per_th = 16 * 256 * 8
     alu_peak = 148 * 128 * 1.965e9 / 1e12   # FP32 FMA lanes x max SM clock, in T FMA/s
     q_ach = qtoken_heads * fma_per_th / (quant_ms_best * 1e-3) / 1e12
@@ -466,7 +472,8 @@ def run_ours(args):
             "unit": "tokens/s",
             "n_gpus": world, "steps": K, "warmup": WU, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": W["name"], "batch": B, "seq_len": T, "n_q_heads": HQ, "n_kv_heads": H,
+            "config": {"workload": W["name"] + ("-dq" if args.double_quant else ""), "batch": B, "seq_len": T,
+                       "n_q_heads": HQ, "n_kv_heads": H, "double_quant": bool(args.double_quant),
                        "head_dim": 128, "mode_k": W["mode_k"], "mode_v": W["mode_v"], "window": W["window"],
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": f"inputs larger than L2 (compressed cache {compressed / 1e6:.0f} MB per step)"},
@@ -474,7 +481,7 @@ def run_ours(args):
             "decode_call_ms": dec_avg_ms,
             "roofline": {"kernel": "decode_kernel (one launch per decode call)", "bound": "hbm",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                         "peak_kind": peak_kind, "traffic": decode_traffic(),
+                         "peak_kind": peak_kind, "traffic": None if args.double_quant else decode_traffic(),
                          "algorithmic_bytes_per_launch": decode_bytes,
                          "frac_of_8tbs_spec": achieved / 8000.0},
             "quantize": {"workload": f"prefill {B}x{q_tokens} tokens x {H} kv-heads, K 2-bit + V 2-bit, bf16 in",
@@ -513,6 +520,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling runs)")
+    ap.add_argument("--double-quant", action="store_true",
+                    help="the same workload with double quantization (4-bit s1 and o)")
     ap.add_argument("--lite", action="store_true",
                     help="profiling run: no e2e leg, no clock soak, no CPU baseline; short summary line")
     args = ap.parse_args()

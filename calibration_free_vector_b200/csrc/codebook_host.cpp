@@ -192,3 +192,27 @@ extern "C" nsn_status nsn_build_codebook_cosine_host(uint64_t seed, int n_sample
   store_f16(cent, k * d, out);
   return NSN_OK;
 }
+
+// Double quantization of the codebook entries ([TS] Metodologia 3: the codebook
+// entries are stored in 4 bits as well): 16 uniform levels between the
+// fp16-rounded min and max of all entries, level = round-half-even((x - lo) /
+// step) clamped to 0..15, step = (hi - lo) / 15; each entry becomes the fp16
+// rounding of lo + level * step, so the quantizer and the fp16 decode read the
+// same values.
+extern "C" nsn_status nsn_codebook_4bit_host(float* codebook, int n_values) {
+  if (!codebook || n_values <= 0) return NSN_ERR_INVALID_ARG;
+  double mn = INFINITY, mx = -INFINITY;
+  for (int i = 0; i < n_values; ++i) {
+    mn = std::fmin(mn, (double)codebook[i]);
+    mx = std::fmax(mx, (double)codebook[i]);
+  }
+  const double lo = (double)__half2float(__double2half(mn));
+  const double hi = (double)__half2float(__double2half(mx));
+  const double step = (hi - lo) / 15.0;
+  for (int i = 0; i < n_values; ++i) {
+    double level = 0.0;
+    if (step > 0.0) level = std::fmin(15.0, std::fmax(0.0, std::nearbyint(((double)codebook[i] - lo) / step)));
+    codebook[i] = __half2float(__double2half(lo + level * step));
+  }
+  return NSN_OK;
+}

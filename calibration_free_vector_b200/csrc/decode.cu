@@ -178,26 +178,64 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
 
 // Lane 0 issues the bulk copies of one 64-token stage (+ the block's mean rows
 // when `with_means`) and arms the stage's barrier with the byte count.
-template <int MK, int MV>
+// With double quantization (DQ) the norms region receives alpha*s2 (fp16, 128 B)
+// followed by the 4-bit s1 levels (32 B), and the mean slot receives, from byte
+// 256 on, the K and V o levels (64 B each) and their (lo, hi) parameters (16 B
+// each); the fp16 mean rows are formed from them in shared memory.
+constexpr int DQ_LEV = 2 * D;           // o levels of K at +256, of V at +320
+constexpr int DQ_PAR = 2 * D + D;       // parameters of K at +384, of V at +400
+template <int MK, int MV, bool DQ>
 __device__ __forceinline__ void issue_stage(uint32_t dst, uint32_t mdst, uint32_t bar, const CacheView& kc,
                                            const CacheView& vc, int64_t seq, int t0, bool with_means) {
   const int64_t cap = kc.capacity;
   const int64_t tok = seq * cap + t0;
-  constexpr uint32_t CB = STAGE_TOK * 16, NB = STAGE_TOK * 4;
+  constexpr uint32_t CB = STAGE_TOK * 16;
+  constexpr uint32_t NB = DQ ? STAGE_TOK * 2 + STAGE_TOK / 2 : STAGE_TOK * 4;
+  constexpr uint32_t MB = DQ ? 2 * (D / 2) + 2 * 16 : MEAN_BYTES;
   const uint32_t bytes = CB * 2 + NB * 2 + (MK == NSN_MODE_2BIT ? CB : 0) + (MV == NSN_MODE_2BIT ? CB : 0) +
-                         (with_means ? MEAN_BYTES : 0);
+                         (with_means ? MB : 0);
   mbar_expect_tx(bar, bytes);
   bulk_g2s(dst + ST_KC, kc.codes + tok * NSUB, CB, bar);
   if constexpr (MK == NSN_MODE_2BIT) bulk_g2s(dst + ST_KS, kc.signs + tok * NSUB, CB, bar);
-  bulk_g2s(dst + ST_KN, kc.norms + tok, NB, bar);
   bulk_g2s(dst + ST_VC, vc.codes + tok * NSUB, CB, bar);
   if constexpr (MV == NSN_MODE_2BIT) bulk_g2s(dst + ST_VS, vc.signs + tok * NSUB, CB, bar);
-  bulk_g2s(dst + ST_VN, vc.norms + tok, NB, bar);
-  if (with_means) {
-    const int64_t mrow = (seq * (cap / BLK) + t0 / BLK) * D;
-    bulk_g2s(mdst, kc.means + mrow, D * 2, bar);
-    bulk_g2s(mdst + D * 2, vc.means + mrow, D * 2, bar);
+  const int64_t blk = seq * (cap / BLK) + t0 / BLK;
+  if constexpr (DQ) {
+    bulk_g2s(dst + ST_KN, reinterpret_cast<const __half*>(kc.norms) + tok, STAGE_TOK * 2, bar);
+    bulk_g2s(dst + ST_KN + STAGE_TOK * 2, kc.s1_levels + tok / 2, STAGE_TOK / 2, bar);
+    bulk_g2s(dst + ST_VN, reinterpret_cast<const __half*>(vc.norms) + tok, STAGE_TOK * 2, bar);
+    bulk_g2s(dst + ST_VN + STAGE_TOK * 2, vc.s1_levels + tok / 2, STAGE_TOK / 2, bar);
+    if (with_means) {
+      bulk_g2s(mdst + DQ_LEV, reinterpret_cast<const uint8_t*>(kc.means) + blk * (D / 2), D / 2, bar);
+      bulk_g2s(mdst + DQ_LEV + D / 2, reinterpret_cast<const uint8_t*>(vc.means) + blk * (D / 2), D / 2, bar);
+      bulk_g2s(mdst + DQ_PAR, kc.dq_params + blk * 8, 16, bar);
+      bulk_g2s(mdst + DQ_PAR + 16, vc.dq_params + blk * 8, 16, bar);
+    }
+  } else {
+    bulk_g2s(dst + ST_KN, kc.norms + tok, NB, bar);
+    bulk_g2s(dst + ST_VN, vc.norms + tok, NB, bar);
+    if (with_means) {
+      bulk_g2s(mdst, kc.means + blk * D, D * 2, bar);
+      bulk_g2s(mdst + D * 2, vc.means + blk * D, D * 2, bar);
+    }
   }
+}
+
+// (lo, step) of a 4-bit group from its fp16 (lo, hi) pair.
+__device__ __forceinline__ float2 dq_lo_step(const unsigned char* par) {
+  const float2 lh = __half22float2(*reinterpret_cast<const __half2*>(par));
+  return make_float2(lh.x, (lh.y - lh.x) * (1.0f / 15.0f));
+}
+
+// Writes the fp16 mean row of one block (128 channels, lane l: channels 4l..4l+3)
+// from its 4-bit levels into `row`.
+__device__ __forceinline__ void dq_mean_row(unsigned char* row, const unsigned char* levels, const unsigned char* par,
+                                            int lane) {
+  const float2 ls = dq_lo_step(par);
+  const uint32_t two = *reinterpret_cast<const uint16_t*>(levels + 2 * lane);
+  const float c0 = fmaf((float)(two & 15u), ls.y, ls.x), c1 = fmaf((float)((two >> 4) & 15u), ls.y, ls.x);
+  const float c2 = fmaf((float)((two >> 8) & 15u), ls.y, ls.x), c3 = fmaf((float)((two >> 12) & 15u), ls.y, ls.x);
+  *reinterpret_cast<uint2*>(row + 8 * lane) = make_uint2(pack_half2(c0, c1), pack_half2(c2, c3));
 }
 
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
@@ -466,7 +504,7 @@ __device__ __noinline__ void cta_merge(const float* ws, const float* ws_acc, int
 //          scores of token g + 8 (p >> 1) for heads 2 (p & 1), 2 (p & 1) + 1.
 // Values:  O^T[d][h] += sum_t u_hat_v[t][d] w[t][h]  M = 16 dims, N = 8 heads, K = 16 tokens;
 //          the B operand is the weight matrix moved into place with movmatrix.trans.
-template <int GH, int MK, int MV>
+template <int GH, int MK, int MV, bool DQ>
 __global__ void __launch_bounds__(32 * DEC_WARPS, 1)
 decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb, int64_t qsh,
               float qscale, const float* __restrict__ cbk_g, const float* __restrict__ cbv_g,
@@ -525,7 +563,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     mbar_init(bar0 + 8u, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     if (nstages > 0)
-      issue_stage<MK, MV>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc, seq,
+      issue_stage<MK, MV, DQ>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc, seq,
                           tok_begin, true);
   }
   __syncwarp();
@@ -536,7 +574,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
   if (active) build_q_operand<GH>(qb, qrows, qscale * INV_SQRT_D, true, lane, &sm.stage[warp][1][0]);
   if (lane == 0 && nstages > 1) {
     const int t1 = tok_begin + STAGE_TOK;
-    issue_stage<MK, MV>(st_base + STAGE_BYTES, mb_base + (uint32_t)(((t1 / BLK) & 1) * MEAN_BYTES), bar0 + 8, kc, vc,
+    issue_stage<MK, MV, DQ>(st_base + STAGE_BYTES, mb_base + (uint32_t)(((t1 / BLK) & 1) * MEAN_BYTES), bar0 + 8, kc, vc,
                         seq, t1, (t1 % BLK) == 0);
   }
 
@@ -589,9 +627,18 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     const bool block_end = ((t_stage + STAGE_TOK) % BLK) == 0 || st == nstages - 1;
     const int mbuf = (t_stage / BLK) & 1;
     const unsigned char* sb = &sm.stage[warp][buf][0];
-    const unsigned char* mb = &sm.means[warp][mbuf][0];
+    unsigned char* mb = &sm.means[warp][mbuf][0];
+    float2 k_s1 = make_float2(0.f, 0.f), v_s1 = make_float2(0.f, 0.f);  // (lo, step) of the s1 levels
+    if constexpr (DQ) {
+      k_s1 = dq_lo_step(mb + DQ_PAR);
+      v_s1 = dq_lo_step(mb + DQ_PAR + 16);
+    }
 
     if (block_start) {
+      if constexpr (DQ) {  // the fp16 o_K row, from its levels
+        dq_mean_row(mb, mb + DQ_LEV, mb + DQ_PAR + 4, lane);
+        __syncwarp();
+      }
       // (H q) . o_K of this block: the mean row as all 16 "tokens" of one score tile
       float d4[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t mrow = mb_base + (uint32_t)(mbuf * MEAN_BYTES) + (uint32_t)(lane >> 4) * 16u;
@@ -616,7 +663,8 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
         ks0 = *reinterpret_cast<const uint32_t*>(sb + ST_KS + (tt + g) * 16 + 4 * p);
         ks1 = *reinterpret_cast<const uint32_t*>(sb + ST_KS + (tt + 8 + g) * 16 + 4 * p);
       }
-      const uint32_t knw = *reinterpret_cast<const uint32_t*>(sb + ST_KN + (tt + t_l) * 4);
+      uint32_t knw = 0u, vnw = 0u;
+      if constexpr (!DQ) knw = *reinterpret_cast<const uint32_t*>(sb + ST_KN + (tt + t_l) * 4);
       const uint4 vcw = *reinterpret_cast<const uint4*>(sb + ST_VC + (tt + tok_v) * 16);
       uint32_t W0 = 0u, W1 = 0u;
       if constexpr (MV == NSN_MODE_2BIT) {
@@ -624,7 +672,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
         W0 = __byte_perm((uint32_t)vs[(tt + 2 * p) * 8 + g], (uint32_t)vs[(tt + 2 * p + 1) * 8 + g], 0x5410u);
         W1 = __byte_perm((uint32_t)vs[(tt + 8 + 2 * p) * 8 + g], (uint32_t)vs[(tt + 9 + 2 * p) * 8 + g], 0x5410u);
       }
-      const uint32_t vnw = *reinterpret_cast<const uint32_t*>(sb + ST_VN + (tt + t_l) * 4);
+      if constexpr (!DQ) vnw = *reinterpret_cast<const uint32_t*>(sb + ST_VN + (tt + t_l) * 4);
 
       // ---- scores: 8 k-steps of 16 dims in two independent accumulation chains ----
       float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
@@ -651,8 +699,18 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       const float d1 = (lo_lane ? S[1] : S[3]) + r1;
 
       // ---- scores with the NSN byproducts; online softmax (lazy re-basing) ----
-      const float2 kn = __half22float2(*reinterpret_cast<const __half2*>(&knw));
-      float2 vn = __half22float2(*reinterpret_cast<const __half2*>(&vnw));
+      float2 kn, vn;  // (s1, s2) of token t_l
+      if constexpr (DQ) {
+        const int tk = tt + t_l;
+        const uint32_t sh = 4u * (uint32_t)(tk & 1);
+        const float kl = (float)(((uint32_t)sb[ST_KN + STAGE_TOK * 2 + (tk >> 1)] >> sh) & 15u);
+        const float vl = (float)(((uint32_t)sb[ST_VN + STAGE_TOK * 2 + (tk >> 1)] >> sh) & 15u);
+        kn = make_float2(fmaf(kl, k_s1.y, k_s1.x), __half2float(reinterpret_cast<const __half*>(sb + ST_KN)[tk]));
+        vn = make_float2(fmaf(vl, v_s1.y, v_s1.x), __half2float(reinterpret_cast<const __half*>(sb + ST_VN)[tk]));
+      } else {
+        kn = __half22float2(*reinterpret_cast<const __half2*>(&knw));
+        vn = __half22float2(*reinterpret_cast<const __half2*>(&vnw));
+      }
       float sc0 = kn.x * fmaf(kn.y, d0, qo0);
       float sc1 = kn.x * fmaf(kn.y, d1, qo1);
       if (!full && t_stage + tt + t_l >= tok_end) {  // past the end: no weight, and no stale norms
@@ -695,7 +753,11 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
         c0 += __shfl_xor_sync(0xffffffffu, c0, x);
         c1 += __shfl_xor_sync(0xffffffffu, c1, x);
       }
-      const __half* ov = reinterpret_cast<const __half*>(mb + D * 2);
+      if constexpr (DQ) {  // the fp16 o_V row, from its levels (the o_K row is no longer needed)
+        dq_mean_row(mb, mb + DQ_LEV + D / 2, mb + DQ_PAR + 16 + 4, lane);
+        __syncwarp();
+      }
+      const __half* ov = reinterpret_cast<const __half*>(mb + (DQ ? 0 : D * 2));
 #pragma unroll
       for (int mm = 0; mm < 8; ++mm) {
         const float oa = __half2float(ov[16 * mm + g]);
@@ -710,7 +772,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     __syncwarp();  // every lane is done with this stage buffer (and, at a block end, its means)
     if (lane == 0 && st + 2 < nstages) {
       const int tn = t_stage + 2 * STAGE_TOK;
-      issue_stage<MK, MV>(st_base + (uint32_t)(buf * STAGE_BYTES), mb_base + (uint32_t)(((tn / BLK) & 1) * MEAN_BYTES),
+      issue_stage<MK, MV, DQ>(st_base + (uint32_t)(buf * STAGE_BYTES), mb_base + (uint32_t)(((tn / BLK) & 1) * MEAN_BYTES),
                           bar0 + 8u * buf, kc, vc, seq, tn, (tn % BLK) == 0);
     }
   }
@@ -861,18 +923,18 @@ size_t decode_workspace_bytes(int batch, int n_kv_heads, const DecodeGeom& geom)
   return (size_t)counter_words((int64_t)batch * n_kv_heads) * 4u + decode_partial_bytes(batch, n_kv_heads, geom);
 }
 
-template <int G, int MK, int MV>
+template <int G, int MK, int MV, bool DQ>
 static cudaError_t launch_t(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
                             int64_t qsb, int64_t qsh, float qscale, const float* cbk, const float* cbv, float* out,
                             unsigned int* counters, float* partials, const DecodeGeom& geom, cudaStream_t s) {
   constexpr int GH = G < 4 ? G : 4;  // heads per warp job
   const size_t smem = sizeof(DecSmem);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<GH, MK, MV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<GH, MK, MV, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   const int nwarps = kc.batch * kc.n_kv_heads * geom.nsplit_q * (G / GH);
   dim3 grid((nwarps + DEC_WARPS - 1) / DEC_WARPS);
-  decode_kernel<GH, MK, MV><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv,
+  decode_kernel<GH, MK, MV, DQ><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv,
                                                                counters, partials, out, n_q_heads, geom);
   return cudaGetLastError();
 }
@@ -881,13 +943,16 @@ template <int G>
 static cudaError_t launch_g(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
                             int64_t qsb, int64_t qsh, float qscale, const float* cbk, const float* cbv, float* out,
                             unsigned int* counters, float* partials, const DecodeGeom& geom, cudaStream_t s) {
-  if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_1BIT)
-    return launch_t<G, 1, 1>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
-  if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_2BIT)
-    return launch_t<G, 1, 2>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
-  if (kc.mode == NSN_MODE_2BIT && vc.mode == NSN_MODE_1BIT)
-    return launch_t<G, 2, 1>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
-  return launch_t<G, 2, 2>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+#define NSN_LAUNCH(MK_, MV_)                                                                                    \
+  return kc.dq ? launch_t<G, MK_, MV_, true>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters,  \
+                                             partials, geom, s)                                                       \
+               : launch_t<G, MK_, MV_, false>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, \
+                                              partials, geom, s)
+  if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_1BIT) NSN_LAUNCH(1, 1);
+  if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_2BIT) NSN_LAUNCH(1, 2);
+  if (kc.mode == NSN_MODE_2BIT && vc.mode == NSN_MODE_1BIT) NSN_LAUNCH(2, 1);
+  NSN_LAUNCH(2, 2);
+#undef NSN_LAUNCH
 }
 
 static cudaError_t launch_any(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,

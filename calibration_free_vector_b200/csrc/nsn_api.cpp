@@ -40,6 +40,9 @@ nsn_status check_cache(const nsn_cache* c) {
   if (c->window_buf && !aligned16(c->window_buf)) return NSN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(c->n_quant) & 3u) || (reinterpret_cast<uintptr_t>(c->n_window) & 3u))
     return NSN_ERR_INVALID_ARG;
+  if (c->double_quant != 0 && c->double_quant != 1) return NSN_ERR_INVALID_ARG;
+  if (c->double_quant && (!c->s1_levels || !c->dq_params || !aligned16(c->s1_levels) || !aligned16(c->dq_params)))
+    return NSN_ERR_INVALID_ARG;
   return NSN_OK;
 }
 
@@ -59,12 +62,16 @@ nsn::CacheView view(const nsn_cache* c) {
   v.n_quant = c->n_quant;
   v.n_window = c->n_window;
   v.status = c->status;
+  v.dq = c->double_quant ? 1 : 0;
+  v.s1_levels = c->double_quant ? c->s1_levels : nullptr;
+  v.dq_params = c->double_quant ? reinterpret_cast<__half*>(c->dq_params) : nullptr;
   return v;
 }
 
+// K and V caches used together must agree in shape and in double quantization.
 bool same_shape(const nsn_cache* a, const nsn_cache* b) {
   return a->batch == b->batch && a->n_kv_heads == b->n_kv_heads && a->capacity == b->capacity &&
-         a->window == b->window;
+         a->window == b->window && a->double_quant == b->double_quant;
 }
 
 }  // namespace
@@ -88,7 +95,7 @@ const char* nsn_status_string(int status) {
 const char* nsn_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
 
 nsn_status nsn_cache_buffer_sizes(int batch, int n_kv_heads, int capacity, int window, int mode,
-                                  nsn_cache_sizes* out) {
+                                  int double_quant, nsn_cache_sizes* out) {
   if (!out || batch <= 0 || n_kv_heads <= 0 || capacity <= 0 || capacity % NSN_BLOCK != 0)
     return NSN_ERR_INVALID_ARG;
   if (mode != NSN_MODE_1BIT && mode != NSN_MODE_2BIT) return NSN_ERR_INVALID_ARG;
@@ -96,8 +103,18 @@ nsn_status nsn_cache_buffer_sizes(int batch, int n_kv_heads, int capacity, int w
   const size_t seqs = (size_t)batch * n_kv_heads;
   out->codes = seqs * capacity * NSN_N_SUB;
   out->signs = mode == NSN_MODE_2BIT ? out->codes : 0;
-  out->norms = seqs * capacity * 2 * sizeof(uint16_t);
-  out->means = seqs * (capacity / NSN_BLOCK) * NSN_HEAD_DIM * sizeof(uint16_t);
+  const size_t blocks = seqs * (capacity / NSN_BLOCK);
+  if (double_quant) {
+    out->norms = seqs * capacity * sizeof(uint16_t);
+    out->means = blocks * (NSN_HEAD_DIM / 2);
+    out->s1_levels = seqs * capacity / 2;
+    out->dq_params = blocks * 8 * sizeof(uint16_t);
+  } else {
+    out->norms = seqs * capacity * 2 * sizeof(uint16_t);
+    out->means = blocks * NSN_HEAD_DIM * sizeof(uint16_t);
+    out->s1_levels = 0;
+    out->dq_params = 0;
+  }
   out->window_buf = seqs * (size_t)window * NSN_HEAD_DIM * sizeof(uint16_t);
   out->n_quant = seqs * sizeof(int32_t);
   out->n_window = seqs * sizeof(int32_t);

@@ -19,6 +19,9 @@ struct CacheView {
   int32_t* n_quant;
   int32_t* n_window;
   int32_t* status;
+  int dq;               // 1: s1 and o stored as 4-bit levels (then `norms` holds fp16 alpha*s2,
+  uint8_t* s1_levels;   //    `means` the o levels, s1_levels / dq_params the rest)
+  __half* dq_params;
 };
 
 // Decode split geometry: the quantized blocks of every (b, kv-head) are dealt

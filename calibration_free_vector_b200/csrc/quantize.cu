@@ -60,7 +60,38 @@ struct QuantSmem {
   alignas(16) float thr[BLK][NSUB + 1];  // per (token, sub-vector) threshold of the exact re-decision
   alignas(16) uint8_t code[BLK][NSUB]; // chosen codes
   alignas(16) uint32_t sgn[BLK][4];    // packed sign bits (2-bit mode)
+  // double quantization
+  alignas(16) double ofull[D];         // o of the block (fp64) until its levels are formed
+  alignas(16) double red[2][QTHREADS / 32][2];  // per-warp (min, max) of s1 and of o
+  alignas(16) double dq[2][3];         // (lo, hi, step) of s1 and of o
+  alignas(16) uint8_t lev[2][BLK];     // 4-bit levels of s1 (per token) and of o (per channel)
 };
+
+// Destination of the stored scalars of one block: either fp16 (s1, alpha*s2) pairs
+// and fp16 o, or (double quantization) fp16 alpha*s2, 4-bit s1 and o levels and the
+// block's (lo, hi) pairs.
+struct BlockOut {
+  __half2* norms;        // [n] (s1, alpha*s2)            -- plain
+  __half* means;         // [128] o                        -- plain
+  __half* s2;            // [n] alpha*s2                   -- double quantization
+  uint8_t* s1_levels;    // [64]  two levels per byte       -- double quantization
+  uint8_t* o_levels;     // [64]                            -- double quantization
+  __half* params;        // [8] (s1 lo, s1 hi, o lo, o hi, 0, 0, 0, 0) -- double quantization
+  bool dq;
+};
+
+__device__ __forceinline__ BlockOut block_out(const CacheView& c, int64_t seq, int64_t tok0, int blk) {
+  BlockOut o;
+  const int64_t bi = seq * (c.capacity / BLK) + blk;
+  o.dq = c.dq != 0;
+  o.norms = c.norms + tok0;
+  o.means = c.means + bi * D;
+  o.s2 = reinterpret_cast<__half*>(c.norms) + tok0;
+  o.s1_levels = c.s1_levels ? c.s1_levels + tok0 / 2 : nullptr;
+  o.o_levels = reinterpret_cast<uint8_t*>(c.means) + bi * (D / 2);
+  o.params = c.dq_params ? c.dq_params + bi * 8 : nullptr;
+  return o;
+}
 
 // Stages the codebook, its biases and norm bounds.  All QTHREADS threads.
 __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook) {
@@ -92,6 +123,64 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
 
 __device__ __forceinline__ double shfl_pair_sum(double x) { return x + __shfl_xor_sync(0xffffffffu, x, 1); }
 
+__device__ __forceinline__ double warp_min_d(double x) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) x = fmin(x, __shfl_xor_sync(0xffffffffu, x, m));
+  return x;
+}
+__device__ __forceinline__ double warp_max_d(double x) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) x = fmax(x, __shfl_xor_sync(0xffffffffu, x, m));
+  return x;
+}
+
+// Double quantization of a block's stored scalars ([TS] Metodologia 3): s1 over
+// the n tokens and o over the 128 channels, each as 4-bit levels of 16 uniform
+// steps between the fp16-rounded min and max of the group:
+//   lo = fp16(min), hi = fp16(max), step = (hi - lo) / 15 (fp64),
+//   level = round-half-even((x - lo) / step) clamped to 0..15 (step = 0: level 0).
+// Threads 0..127 handle s1 (token t), threads 128..255 o (channel t - 128).
+// sm.s1 and sm.ofull hold the exact fp64 values.  All QTHREADS threads.
+__device__ void store_double_quant(QuantSmem& sm, int n, const BlockOut& bo) {
+  __syncthreads();  // sm.s1 of every token is final
+  const int t = threadIdx.x, grp = t >> 7, i = t & (BLK - 1), warp = t >> 5, lane = t & 31;
+  const bool have = grp == 1 || i < n;
+  const double x = grp == 0 ? (i < n ? sm.s1[i] : 0.0) : sm.ofull[i];
+  const double mn = warp_min_d(have ? x : INFINITY), mx = warp_max_d(have ? x : -INFINITY);
+  if (lane == 0) {
+    sm.red[grp][warp & 3][0] = mn;
+    sm.red[grp][warp & 3][1] = mx;
+  }
+  __syncthreads();
+  if (t < 2) {
+    double a = INFINITY, b = -INFINITY;
+    for (int w = 0; w < 4; ++w) {
+      a = fmin(a, sm.red[t][w][0]);
+      b = fmax(b, sm.red[t][w][1]);
+    }
+    const double lo = (double)__half2float(__double2half(a));
+    const double hi = (double)__half2float(__double2half(b));
+    sm.dq[t][0] = lo;
+    sm.dq[t][1] = hi;
+    sm.dq[t][2] = (hi - lo) / 15.0;
+  }
+  __syncthreads();
+  {
+    const double lo = sm.dq[grp][0], step = sm.dq[grp][2];
+    int level = 0;
+    if (have && step > 0.0) level = (int)fmin(15.0, fmax(0.0, rint((x - lo) / step)));
+    sm.lev[grp][i] = (uint8_t)level;
+  }
+  __syncthreads();
+  if (t < 64) bo.s1_levels[t] = (uint8_t)(sm.lev[0][2 * t] | (sm.lev[0][2 * t + 1] << 4));
+  else if (t < 128) bo.o_levels[t - 64] = (uint8_t)(sm.lev[1][2 * (t - 64)] | (sm.lev[1][2 * (t - 64) + 1] << 4));
+  else if (t < 136) {
+    const int k = t - 128;
+    const double v = k == 0 ? sm.dq[0][0] : k == 1 ? sm.dq[0][1] : k == 2 ? sm.dq[1][0] : k == 3 ? sm.dq[1][1] : 0.0;
+    bo.params[k] = __double2half(v);
+  }
+}
+
 // Quantizes one block of n (1..128) tokens with QTHREADS threads: thread
 // t = 2 tk + h works on token tk, dims 64h .. 64h+63 (sub-vectors 8h .. 8h+7).
 // Rows are at src + row0 + tk*row_stride (elements).  Output pointers are
@@ -100,8 +189,8 @@ __device__ __forceinline__ double shfl_pair_sum(double x) { return x + __shfl_xo
 template <int DT, int MODE>
 __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, int64_t row0,
                                    int64_t row_stride, int n, uint8_t* __restrict__ codes,
-                                   uint8_t* __restrict__ signs, __half2* __restrict__ norms,
-                                   __half* __restrict__ means, int scale_adjust) {
+                                   uint8_t* __restrict__ signs, const CacheView& cv, int64_t seq,
+                                   int64_t tok0, int blk, int scale_adjust) {
   const int t = threadIdx.x, tk = t >> 1, h = t & 1;
   const int col = t & (D - 1), rhalf = t >> 7;  // column-sum roles: column, half of the rows
   const bool valid = tk < n;
@@ -259,7 +348,9 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   if (t < D) {
     const double dc = (sm.part[0][t] + sm.part[1][t]) / n;
     sm.o[t] = dc;  // D_c = mean_t(d_t,c rr_t)
-    means[t] = __double2half(fma(sm.big_r[t], rr_mean, dc));
+    const double o_t = fma(sm.big_r[t], rr_mean, dc);
+    if (cv.dq) sm.ofull[t] = o_t;
+    else cv.means[(seq * (cv.capacity / BLK) + blk) * D + t] = __double2half(o_t);
   }
   __syncthreads();
 
@@ -472,9 +563,12 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     if (h == 0) {
       if constexpr (MODE == NSN_MODE_2BIT)
         *reinterpret_cast<uint4*>(signs + (int64_t)tk * NSUB) = *reinterpret_cast<const uint4*>(&sm.sgn[tk][0]);
-      norms[tk] = __halves2half2(__double2half(sm.s1[tk]), __double2half(alpha * sm.s2[tk]));
+      const BlockOut bo = block_out(cv, seq, tok0, blk);
+      if (bo.dq) bo.s2[tk] = __double2half(alpha * sm.s2[tk]);
+      else bo.norms[tk] = __halves2half2(__double2half(sm.s1[tk]), __double2half(alpha * sm.s2[tk]));
     }
   }
+  if (cv.dq) store_double_quant(sm, n, block_out(cv, seq, tok0, blk));
   __syncthreads();  // shared memory is reused by the caller's next block
 }
 
@@ -516,8 +610,7 @@ quantize_prefill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int6
   const int64_t tok0 = seq * cv.capacity + (int64_t)blk * BLK;
   quantize_block_dev<DT, MODE>(sm, x, (int64_t)b * sb + (int64_t)blk * BLK * st + (int64_t)h * sh, st, n,
                                cv.codes + tok0 * NSUB, MODE == NSN_MODE_2BIT ? cv.signs + tok0 * NSUB : nullptr,
-                               cv.norms + tok0, cv.means + (seq * (cv.capacity / BLK) + blk) * D,
-                               cv.scale_adjust);
+                               cv, seq, tok0, blk, cv.scale_adjust);
 }
 
 // Prefill tail: copies tokens [q, L) of each sequence to the residual window
@@ -572,15 +665,12 @@ append_kernel(CacheView kc, CacheView vc, const void* __restrict__ k_new, const 
       const int64_t tok0 = seq * c.capacity + nq;
       const int blk = nq / BLK;
       uint8_t* sg = c.mode == NSN_MODE_2BIT ? c.signs + tok0 * NSUB : nullptr;
-      __half* mn = c.means + (seq * (c.capacity / BLK) + blk) * D;
       if (c.mode == NSN_MODE_2BIT)
         quantize_block_dev<NSN_DTYPE_F16, NSN_MODE_2BIT>(sm, c.window, seq * c.window_len * D, D, BLK,
-                                                         c.codes + tok0 * NSUB, sg, c.norms + tok0, mn,
-                                                         c.scale_adjust);
+                                                         c.codes + tok0 * NSUB, sg, c, seq, tok0, blk, c.scale_adjust);
       else
         quantize_block_dev<NSN_DTYPE_F16, NSN_MODE_1BIT>(sm, c.window, seq * c.window_len * D, D, BLK,
-                                                         c.codes + tok0 * NSUB, sg, c.norms + tok0, mn,
-                                                         c.scale_adjust);
+                                                         c.codes + tok0 * NSUB, sg, c, seq, tok0, blk, c.scale_adjust);
       nq += BLK;
       nw = 0;
     }

@@ -43,11 +43,13 @@ class nsn_cache(ctypes.Structure):
         ("mode", c_int32), ("scale_adjust", c_int32),
         ("codes", c_void_p), ("signs", c_void_p), ("norms", c_void_p), ("means", c_void_p),
         ("window_buf", c_void_p), ("n_quant", c_void_p), ("n_window", c_void_p), ("status", c_void_p),
+        ("double_quant", c_int32), ("s1_levels", c_void_p), ("dq_params", c_void_p),
     ]
 
 
 class nsn_cache_sizes(ctypes.Structure):
-    _fields_ = [(n, c_size_t) for n in ("codes", "signs", "norms", "means", "window_buf", "n_quant", "n_window")]
+    _fields_ = [(n, c_size_t) for n in ("codes", "signs", "norms", "means", "window_buf", "n_quant", "n_window",
+                                        "s1_levels", "dq_params")]
 
 
 _lib = None
@@ -66,12 +68,14 @@ def load():
     lib.nsn_status_string.argtypes = [c_int]
     lib.nsn_last_cuda_error.restype = c_char_p
     lib.nsn_cache_buffer_sizes.restype = c_int
-    lib.nsn_cache_buffer_sizes.argtypes = [c_int, c_int, c_int, c_int, c_int, POINTER(nsn_cache_sizes)]
+    lib.nsn_cache_buffer_sizes.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int, POINTER(nsn_cache_sizes)]
     lib.nsn_build_codebook_host.restype = c_int
     lib.nsn_build_codebook_host.argtypes = [c_uint64, c_int, c_int, c_int, c_int, c_int, POINTER(c_float)]
     lib.nsn_build_codebook_cosine_host.restype = c_int
     lib.nsn_build_codebook_cosine_host.argtypes = [c_uint64, c_int, c_int, c_int, c_int, c_int, c_int,
                                                    POINTER(c_float)]
+    lib.nsn_codebook_4bit_host.restype = c_int
+    lib.nsn_codebook_4bit_host.argtypes = [POINTER(c_float), c_int]
     lib.nsn_quantize_kv.restype = c_int
     lib.nsn_quantize_kv.argtypes = [POINTER(nsn_cache), c_void_p, c_int, c_int64, c_int64, c_int64, c_int,
                                     c_void_p, c_void_p]
@@ -142,9 +146,19 @@ def nsn_build_codebook_cosine_host(seed: int, n_samples: int = 65536, n_codes: i
     return out
 
 
-def nsn_cache_buffer_sizes(batch: int, n_kv_heads: int, capacity: int, window: int, mode: int) -> dict:
+def nsn_codebook_4bit_host(codebook: np.ndarray) -> np.ndarray:
+    """Copy of a float32 codebook with its entries on 16 uniform levels (see include/nsn.h)."""
+    out = np.ascontiguousarray(codebook, dtype=np.float32).copy()
+    _check(load().nsn_codebook_4bit_host(out.ctypes.data_as(POINTER(c_float)), int(out.size)),
+           "nsn_codebook_4bit_host")
+    return out
+
+
+def nsn_cache_buffer_sizes(batch: int, n_kv_heads: int, capacity: int, window: int, mode: int,
+                           double_quant: bool = False) -> dict:
     s = nsn_cache_sizes()
-    _check(load().nsn_cache_buffer_sizes(batch, n_kv_heads, capacity, window, mode, ctypes.byref(s)),
+    _check(load().nsn_cache_buffer_sizes(batch, n_kv_heads, capacity, window, mode, 1 if double_quant else 0,
+                                         ctypes.byref(s)),
            "nsn_cache_buffer_sizes")
     return {n: getattr(s, n) for n, _ in nsn_cache_sizes._fields_}
 
@@ -156,31 +170,48 @@ class Cache:
     """Device buffers of one compressed K or V cache and the matching C struct."""
 
     def __init__(self, batch: int, n_kv_heads: int, capacity: int, window: int, mode: int,
-                 scale_adjust: bool = True, device="cuda"):
+                 scale_adjust: bool = True, device="cuda", double_quant: bool = False):
         import torch
-        sizes = nsn_cache_buffer_sizes(batch, n_kv_heads, capacity, window, mode)
+        sizes = nsn_cache_buffer_sizes(batch, n_kv_heads, capacity, window, mode, double_quant)
         self.batch, self.n_kv_heads, self.capacity, self.window, self.mode = batch, n_kv_heads, capacity, window, mode
         self.scale_adjust = bool(scale_adjust)
+        self.double_quant = bool(double_quant)
         u8 = dict(dtype=torch.uint8, device=device)
+        f16 = dict(dtype=torch.float16, device=device)
+        nblk = capacity // BLOCK
         self.codes = torch.zeros((batch, n_kv_heads, capacity, N_SUB), **u8)
         self.signs = torch.zeros((batch, n_kv_heads, capacity, N_SUB), **u8) if mode == MODE_2BIT else None
-        self.norms = torch.zeros((batch, n_kv_heads, capacity, 2), dtype=torch.float16, device=device)
-        self.means = torch.zeros((batch, n_kv_heads, capacity // BLOCK, HEAD_DIM), dtype=torch.float16, device=device)
-        self.window_buf = (torch.zeros((batch, n_kv_heads, window, HEAD_DIM), dtype=torch.float16, device=device)
-                           if window > 0 else None)
+        if double_quant:
+            # norms: alpha*s2; means: 4-bit o levels; s1_levels: 4-bit s1 levels; dq_params: (lo, hi) pairs
+            self.norms = torch.zeros((batch, n_kv_heads, capacity), **f16)
+            self.means = torch.zeros((batch, n_kv_heads, nblk, HEAD_DIM // 2), **u8)
+            self.s1_levels = torch.zeros((batch, n_kv_heads, capacity // 2), **u8)
+            self.dq_params = torch.zeros((batch, n_kv_heads, nblk, 8), **f16)
+        else:
+            self.norms = torch.zeros((batch, n_kv_heads, capacity, 2), **f16)
+            self.means = torch.zeros((batch, n_kv_heads, nblk, HEAD_DIM), **f16)
+            self.s1_levels = None
+            self.dq_params = None
+        self.window_buf = torch.zeros((batch, n_kv_heads, window, HEAD_DIM), **f16) if window > 0 else None
         self.n_quant = torch.zeros((batch, n_kv_heads), dtype=torch.int32, device=device)
         self.n_window = torch.zeros((batch, n_kv_heads), dtype=torch.int32, device=device)
         self.status = torch.zeros((1,), dtype=torch.int32, device=device)
-        assert self.codes.numel() == sizes["codes"] and self.norms.numel() * 2 == sizes["norms"]
+        for name in ("codes", "norms", "means", "s1_levels", "dq_params"):
+            t = getattr(self, name)
+            assert (0 if t is None else t.numel() * t.element_size()) == sizes[name], name
         self.c = nsn_cache(
             batch, n_kv_heads, capacity, window, mode, 1 if scale_adjust else 0,
             self.codes.data_ptr(), self.signs.data_ptr() if self.signs is not None else None,
             self.norms.data_ptr(), self.means.data_ptr(),
             self.window_buf.data_ptr() if self.window_buf is not None else None,
-            self.n_quant.data_ptr(), self.n_window.data_ptr(), self.status.data_ptr())
+            self.n_quant.data_ptr(), self.n_window.data_ptr(), self.status.data_ptr(),
+            1 if double_quant else 0,
+            self.s1_levels.data_ptr() if self.s1_levels is not None else None,
+            self.dq_params.data_ptr() if self.dq_params is not None else None)
 
     def nbytes_allocated(self) -> int:
-        bufs = [self.codes, self.signs, self.norms, self.means, self.window_buf, self.n_quant, self.n_window]
+        bufs = [self.codes, self.signs, self.norms, self.means, self.window_buf, self.n_quant, self.n_window,
+                self.s1_levels, self.dq_params]
         return sum(b.numel() * b.element_size() for b in bufs if b is not None)
 
 

@@ -87,6 +87,23 @@ typedef enum { NSN_DTYPE_F32 = 0, NSN_DTYPE_BF16 = 1, NSN_DTYPE_F16 = 2 } nsn_dt
  *                                                       4 = ragged prefill length out of range
  * capacity must be a positive multiple of 128.  window must be 0 (quantize every
  * token, no append) or 128 (KIVI-style residual of one block).
+ *
+ * Double quantization (double_quant = 1; [TS] Metodologia 3: the NSN byproducts s1
+ * and o are stored in 4 bits).  s1 and o are stored as 4-bit levels of 16 uniform
+ * steps between the fp16-rounded min and max of their group (the tokens of a
+ * 128-token block for s1, the 128 channels of a block for o); level =
+ * round-half-even((x - lo) / step) clamped to 0..15, step = (hi - lo) / 15, and the
+ * value read back is lo + level * step.  The NSN itself uses the exact values.  The
+ * buffers then change to:
+ *   norms     fp16   [batch][n_kv_heads][capacity]          alpha*s2 per token
+ *   means     uint8  [batch][n_kv_heads][capacity/128][64]   o levels, channel 2c in the
+ *                                                           low nibble of byte c
+ *   s1_levels uint8  [batch][n_kv_heads][capacity/2]         s1 levels, token 2t in the
+ *                                                           low nibble of byte t
+ *   dq_params fp16   [batch][n_kv_heads][capacity/128][8]    (s1 lo, s1 hi, o lo, o hi, 0, 0,
+ *                                                           0, 0) of each block
+ * With double_quant = 0, s1_levels and dq_params are unused (may be NULL).  The K and
+ * V caches given to one append or decode call must both use it or both not.
  */
 typedef struct {
   int32_t batch;
@@ -103,11 +120,14 @@ typedef struct {
   int32_t* n_quant;
   int32_t* n_window;
   int32_t* status;
+  int32_t double_quant; /* 1: s1 and o stored in 4 bits (layout above) */
+  uint8_t* s1_levels;
+  uint16_t* dq_params;
 } nsn_cache;
 
 /* Byte sizes of the buffers of an nsn_cache with the given shape. */
 typedef struct {
-  size_t codes, signs, norms, means, window_buf, n_quant, n_window;
+  size_t codes, signs, norms, means, window_buf, n_quant, n_window, s1_levels, dq_params;
 } nsn_cache_sizes;
 
 /* Library version (major*10000 + minor*100 + patch). */
@@ -121,10 +141,11 @@ const char* nsn_last_cuda_error(void);
 
 /*
  * Fills *out with the byte size of each cache buffer.  signs is 0 in 1-bit mode,
- * window_buf is 0 when window == 0.  Returns NSN_ERR_INVALID_ARG on a bad shape.
+ * window_buf is 0 when window == 0, s1_levels and dq_params are 0 unless
+ * double_quant.  Returns NSN_ERR_INVALID_ARG on a bad shape.
  */
 nsn_status nsn_cache_buffer_sizes(int batch, int n_kv_heads, int capacity, int window, int mode,
-                                  nsn_cache_sizes* out);
+                                  int double_quant, nsn_cache_sizes* out);
 
 /*
  * Builds the codebook on the HOST (no GPU use).  [TS] Metodologia 3: k-means on
@@ -278,6 +299,16 @@ nsn_status nsn_decode_attention_static(const nsn_cache* k_cache, const nsn_cache
                                        int dtype, int n_q_heads, int64_t q_stride_b, int64_t q_stride_h,
                                        float softmax_scale, const float* cb_k, const float* cb_v, float* out,
                                        void* stream);
+
+/*
+ * Double quantization of a codebook's entries ([TS] Metodologia 3: the codebook
+ * entries are stored in 4 bits too).  In place on a HOST float array of n_values:
+ * 16 uniform levels between the fp16-rounded min and max of all entries, level =
+ * round-half-even((x - lo) / step) clamped to 0..15, step = (hi - lo) / 15; every
+ * entry becomes the fp16 rounding of lo + level * step.  The result is an ordinary
+ * codebook input for the quantizer and the decode.
+ */
+nsn_status nsn_codebook_4bit_host(float* codebook, int n_values);
 
 /*
  * Diagnostic of the decode's error path for a copy that never lands (the pages

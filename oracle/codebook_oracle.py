@@ -183,3 +183,17 @@ def build_codebook(seed: int, n_samples: int, n_codes: int, dim: int,
     """Codebook [n_codes, dim] as fp16-representable values (returned fp64)."""
     cent = kmeans(normal_samples(seed, n_samples, dim, abs_mode), n_codes, iters)
     return cent.astype(np.float16).astype(np.float64)
+
+
+def codebook_4bit(codebook: np.ndarray) -> np.ndarray:
+    """Codebook entries on 16 uniform levels between the fp16-rounded min and max
+    of all entries (double quantization of the codebook, [TS] Metodologia 3), each
+    rounded to fp16.  Same level rule as the stored scalars: round half to even,
+    clamped to 0..15."""
+    cb = np.asarray(codebook, dtype=np.float64)
+    flat = cb.reshape(-1)
+    lo = float(np.float16(flat.min()))
+    hi = float(np.float16(flat.max()))
+    step = (hi - lo) / 15.0
+    levels = np.clip(np.rint((flat - lo) / step), 0, 15) if step > 0 else np.zeros_like(flat)
+    return (lo + levels * step).astype(np.float16).astype(np.float64).reshape(cb.shape)

@@ -33,6 +33,8 @@ Readings where the pages are silent (each is listed in the design doc):
     u . u_hat <= 0), folded into the stored s2.
   * Stored s1, s2*alpha and o are rounded to fp16 (round-to-nearest-even).
   * Degenerate norms: s1 = 0 gives n1 = 0; s2 = 0 gives u = 0.
+  * Double quantization (optional): s1 and o stored in 4 bits, 16 uniform
+    levels between the fp16-rounded group min and max (`dq4`).
 
 Parity pins: every function here is pinned in tests/test_oracle_*.py against
 closed forms, a hand-derived worked example (tests/golden/), library routines
@@ -180,8 +182,29 @@ def to_f16(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
 
 
+def dq4(x) -> dict:
+    """4-bit quantization of one group of stored scalars (double quantization,
+    [TS] Metodologia 3: the NSN byproducts o and s1 are stored in 4 bits).
+
+    Reading (the pages give only the bit width): 16 uniform levels between
+    lo = fp16(min x) and hi = fp16(max x); step = (hi - lo) / 15;
+    level = clip(round-half-even((x - lo) / step), 0, 15) (step = 0 gives level 0);
+    value = lo + level * step.  Returns levels (int), lo, hi (fp64 holding fp16
+    values) and the dequantized values.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    lo = float(to_f16(x.min()))
+    hi = float(to_f16(x.max()))
+    step = (hi - lo) / 15.0
+    if step > 0.0:
+        levels = np.clip(np.rint((x - lo) / step), 0, 15).astype(np.int64)
+    else:
+        levels = np.zeros(x.shape, dtype=np.int64)
+    return {"levels": levels, "lo": lo, "hi": hi, "values": lo + levels * step}
+
+
 def quantize_block(x: np.ndarray, codebook: np.ndarray, mode: int,
-                   sub_dim: int = 8, scale_adjust: bool = True) -> dict:
+                   sub_dim: int = 8, scale_adjust: bool = True, double_quant: bool = False) -> dict:
     """Quantize one block of raw tokens x [n, d] (one batch row, one kv-head).
 
     Hadamard -> NSN -> per-sub-vector nearest codeword -> adaptive scale ->
@@ -190,6 +213,10 @@ def quantize_block(x: np.ndarray, codebook: np.ndarray, mode: int,
       s1 [n], s2 [n] (= alpha * s2, fp16-rounded), o [d] (fp16-rounded),
       gap [n, d/sub_dim] (relative top-2 distance gap of each assignment),
       u [n, d] (fp64 NSN output, for diagnostics).
+    With double_quant, s1 and o are stored in 4 bits instead (`dq4` over the
+    block's tokens and over its 128 channels); "s1" and "o" then hold the
+    dequantized values and "s1_dq" / "o_dq" the levels and (lo, hi).  The NSN,
+    the assignment and alpha use the exact values either way.
     """
     x = np.asarray(x, dtype=np.float64)
     n, d = x.shape
@@ -199,7 +226,7 @@ def quantize_block(x: np.ndarray, codebook: np.ndarray, mode: int,
     codes, signs, gap = assign(u.reshape(n * nsub, sub_dim), codebook, mode)
     u_hat = reconstruct_sub(codes, signs, codebook, mode).reshape(n, d)
     alpha = scale_factor(u, u_hat) if scale_adjust else np.ones(n)
-    return {
+    out = {
         "codes": codes.reshape(n, nsub),
         "signs": None if signs is None else signs.reshape(n, nsub),
         "s1": to_f16(s1),
@@ -208,6 +235,10 @@ def quantize_block(x: np.ndarray, codebook: np.ndarray, mode: int,
         "gap": gap.reshape(n, nsub),
         "u": u,
     }
+    if double_quant:
+        q1, qo = dq4(s1), dq4(o)
+        out.update(s1=q1["values"], o=qo["values"], s1_dq=q1, o_dq=qo)
+    return out
 
 
 def prefill_split(n_tokens: int, block: int, window: int) -> int:
@@ -227,7 +258,7 @@ def prefill_split(n_tokens: int, block: int, window: int) -> int:
 
 def quantize_sequence(x: np.ndarray, codebook: np.ndarray, mode: int,
                       block: int = 128, window: int = 128,
-                      scale_adjust: bool = True) -> dict:
+                      scale_adjust: bool = True, double_quant: bool = False) -> dict:
     """Prefill of one (batch, kv-head) sequence x [L, d].
 
     Returns codes/signs/s1/s2 per quantized token, o per block, the fp16
@@ -238,7 +269,7 @@ def quantize_sequence(x: np.ndarray, codebook: np.ndarray, mode: int,
     L, d = x.shape
     q = prefill_split(L, block, window)
     parts = [quantize_block(x[a:min(a + block, q)], codebook, mode,
-                            scale_adjust=scale_adjust)
+                            scale_adjust=scale_adjust, double_quant=double_quant)
              for a in range(0, q, block)]
     nsub = d // 8
 
@@ -257,6 +288,8 @@ def quantize_sequence(x: np.ndarray, codebook: np.ndarray, mode: int,
         "gap": cat("gap", (0, nsub)),
         "u": cat("u", (0, d)),
         "window": to_f16(x[q:]),
+        "s1_dq": [p["s1_dq"] for p in parts] if double_quant else None,
+        "o_dq": [p["o_dq"] for p in parts] if double_quant else None,
     }
 
 

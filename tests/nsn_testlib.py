@@ -58,21 +58,44 @@ def natural_to_signs(natural: np.ndarray) -> np.ndarray:
     return out
 
 
+def unpack_levels(packed: np.ndarray) -> np.ndarray:
+    """Two 4-bit levels per byte (even index in the low nibble) -> one per element."""
+    p = np.asarray(packed, dtype=np.uint8)
+    return np.stack([p & 15, p >> 4], axis=-1).reshape(*p.shape[:-1], 2 * p.shape[-1]).astype(np.int64)
+
+
 def read_cache(cache, b: int, h: int) -> dict:
-    """Stored contents of one (b, h) sequence of an nsn.Cache as numpy (oracle layout)."""
+    """Stored contents of one (b, h) sequence of an nsn.Cache as numpy (oracle layout).
+    For a double-quantized cache s1 and o are the values read back from the 4-bit
+    levels (lo + level * (hi - lo) / 15 in fp64), and the raw levels and (lo, hi)
+    pairs are returned as well."""
     nq = int(cache.n_quant[b, h].item())
     nw = int(cache.n_window[b, h].item())
+    nblk = (nq + 127) // 128
     out = {
         "n_quant": nq,
         "n_window": nw,
         "codes": cache.codes[b, h, :nq].cpu().numpy().astype(np.int64),
         "signs": None if cache.signs is None else signs_to_natural(cache.signs[b, h, :nq].cpu().numpy()),
-        "s1": cache.norms[b, h, :nq, 0].float().cpu().numpy().astype(np.float64),
-        "s2": cache.norms[b, h, :nq, 1].float().cpu().numpy().astype(np.float64),
-        "o": cache.means[b, h, :(nq + 127) // 128].float().cpu().numpy().astype(np.float64),
         "window": (cache.window_buf[b, h, :nw].float().cpu().numpy().astype(np.float64)
                    if cache.window_buf is not None else np.zeros((0, 128))),
     }
+    if getattr(cache, "double_quant", False):
+        par = cache.dq_params[b, h, :nblk].float().cpu().numpy().astype(np.float64)      # [nblk, 8]
+        s1_lev = unpack_levels(cache.s1_levels[b, h].cpu().numpy())[: nblk * 128].reshape(nblk, 128)
+        o_lev = unpack_levels(cache.means[b, h, :nblk].cpu().numpy())                   # [nblk, 128]
+        s1_step = (par[:, 1] - par[:, 0]) / 15.0
+        o_step = (par[:, 3] - par[:, 2]) / 15.0
+        out["s1"] = (par[:, 0:1] + s1_lev * s1_step[:, None]).reshape(-1)[:nq]
+        out["o"] = par[:, 2:3] + o_lev * o_step[:, None]
+        out["s2"] = cache.norms[b, h, :nq].float().cpu().numpy().astype(np.float64)
+        out["s1_levels"] = s1_lev.reshape(-1)[:nq]
+        out["o_levels"] = o_lev
+        out["params"] = par[:, :4]
+    else:
+        out["s1"] = cache.norms[b, h, :nq, 0].float().cpu().numpy().astype(np.float64)
+        out["s2"] = cache.norms[b, h, :nq, 1].float().cpu().numpy().astype(np.float64)
+        out["o"] = cache.means[b, h, :nblk].float().cpu().numpy().astype(np.float64)
     return out
 
 

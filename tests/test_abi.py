@@ -48,6 +48,13 @@ def test_buffer_sizes(lib):
     assert s["window_buf"] == 16 * 8 * 128 * 128 * 2
     s1 = nsn.nsn_cache_buffer_sizes(1, 1, 256, 0, 1)
     assert s1["signs"] == 0 and s1["window_buf"] == 0
+    d = nsn.nsn_cache_buffer_sizes(16, 8, 32896, 128, 2, double_quant=True)
+    assert d["codes"] == s["codes"] and d["signs"] == s["signs"]
+    assert d["norms"] == 16 * 8 * 32896 * 2                       # alpha*s2 only
+    assert d["means"] == 16 * 8 * (32896 // 128) * 64              # 4-bit o levels
+    assert d["s1_levels"] == 16 * 8 * 32896 // 2
+    assert d["dq_params"] == 16 * 8 * (32896 // 128) * 16
+    assert s["s1_levels"] == 0 and s["dq_params"] == 0
     with pytest.raises(nsn.NsnError):
         nsn.nsn_cache_buffer_sizes(1, 1, 100, 128, 2)   # capacity not a multiple of 128
     with pytest.raises(nsn.NsnError):
@@ -66,6 +73,14 @@ def test_host_validation_without_gpu(lib):
     assert lib.nsn_quantize_kv(ctypes.byref(c), 18, 1, 0, 1024, 128, 10, 16, None) == 1
     assert lib.nsn_quantize_kv(ctypes.byref(c), 16, 1, 0, 1020, 128, 10, 16, None) == 1
     assert lib.nsn_quantize_kv(ctypes.byref(c), 16, 1, 0, 1024, 128, 300, 16, None) == 1
+    # double quantization: its buffers are required, the flag is 0 or 1, and K / V must agree
+    dq_missing = nsn.nsn_cache(1, 1, 128, 128, 2, 1, 16, 16, 16, 16, 16, 16, 16, None, 1, None, None)
+    assert lib.nsn_quantize_kv(ctypes.byref(dq_missing), 16, 1, 0, 1024, 128, 10, 16, None) == 1
+    dq_flag = nsn.nsn_cache(1, 1, 128, 128, 2, 1, 16, 16, 16, 16, 16, 16, 16, None, 2, 16, 16)
+    assert lib.nsn_quantize_kv(ctypes.byref(dq_flag), 16, 1, 0, 1024, 128, 10, 16, None) == 1
+    dq_ok = nsn.nsn_cache(1, 2, 128, 128, 2, 1, 16, 16, 16, 16, 16, 16, 16, None, 1, 16, 16)
+    c2b = nsn.nsn_cache(1, 2, 128, 128, 2, 1, 16, 16, 16, 16, 16, 16, 16, None)
+    assert lib.nsn_append_residual(ctypes.byref(dq_ok), ctypes.byref(c2b), 16, 16, 1, 0, 128, 16, 16, None) == 1
     # ragged prefill: lengths missing or misaligned, bound over capacity, negative bound
     assert lib.nsn_quantize_kv_ragged(ctypes.byref(c), 16, 1, 0, 1024, 128, None, 10, 16, None) == 1
     assert lib.nsn_quantize_kv_ragged(ctypes.byref(c), 16, 1, 0, 1024, 128, 18, 10, 16, None) == 1
@@ -102,6 +117,16 @@ def test_host_cosine_codebook_matches_oracle(lib):
         assert np.array_equal(ours.astype(np.float64), ref)
     with pytest.raises(nsn.NsnError):
         nsn.nsn_build_codebook_cosine_host(1, 100, 256, 8, False, 3, -1)
+
+
+def test_codebook_4bit_matches_oracle(lib):
+    for abs_mode in (False, True):
+        cb = nsn.nsn_build_codebook_host(0x99, 8192, 256, 8, abs_mode, 4)
+        ours = nsn.nsn_codebook_4bit_host(cb)
+        ref = cbo.codebook_4bit(cb)
+        assert np.array_equal(ours.astype(np.float64), ref)
+        assert len(np.unique(ours)) <= 16
+        assert np.array_equal(nsn.nsn_codebook_4bit_host(ours), ours)   # already on the grid
 
 
 def test_host_codebook_full_size_properties(lib):

@@ -124,3 +124,11 @@ def test_cosine_zero_iterations_is_the_kmeans_codebook():
     a = cbo.build_codebook_cosine(9, 4096, 32, 8, True, 5, 0)
     b = cbo.build_codebook(9, 4096, 32, 8, True, 5)
     assert np.array_equal(a, b)
+
+
+def test_codebook_4bit_hand_cases():
+    # entries 0..15 are already the 16 levels; 0.5 and 2.5 round to the even level
+    cb = np.arange(16.0).reshape(2, 8)
+    assert np.array_equal(cbo.codebook_4bit(cb), cb)
+    cb2 = np.array([[0.0, 0.5, 2.5, 15.0, 1.0, 3.0, 7.0, 9.0]])
+    assert list(cbo.codebook_4bit(cb2)[0]) == [0.0, 0.0, 2.0, 15.0, 1.0, 3.0, 7.0, 9.0]

@@ -96,3 +96,41 @@ def test_output_close_to_standard_normal():
     assert np.abs(u.var(axis=0) - 1).max() < 0.15
     kurt = ((u - u.mean(0)) ** 4).mean(0) / u.var(0) ** 2
     assert np.abs(np.median(kurt) - 3.0) < 0.3
+
+
+# ---- double quantization of the stored scalars ----------------------------------
+
+def test_dq4_hand_cases():
+    r = orc.dq4(np.arange(16.0))
+    assert (r["lo"], r["hi"]) == (0.0, 15.0)
+    assert np.array_equal(r["levels"], np.arange(16)) and np.array_equal(r["values"], np.arange(16.0))
+    # round half to even on the level grid: 0.5 -> 0, 1.5 -> 2, 2.5 -> 2
+    r = orc.dq4(np.array([0.0, 0.5, 1.5, 2.5, 15.0]))
+    assert list(r["levels"]) == [0, 0, 2, 2, 15]
+    # a constant group has one level and reproduces its (fp16) value
+    r = orc.dq4(np.full(7, 0.3))
+    assert np.all(r["levels"] == 0) and np.all(r["values"] == np.float16(0.3))
+
+
+def test_dq4_error_bound_and_range():
+    rng = np.random.default_rng(4)
+    for _ in range(20):
+        x = rng.normal(size=128) * rng.uniform(0.01, 5)
+        r = orc.dq4(x)
+        step = (r["hi"] - r["lo"]) / 15
+        assert r["levels"].min() >= 0 and r["levels"].max() <= 15
+        # half a level plus the fp16 rounding of the end points
+        slack = max(abs(r["lo"] - x.min()), abs(r["hi"] - x.max()))
+        assert np.max(np.abs(r["values"] - x)) <= step / 2 + slack + 1e-15
+        # every value is exactly on the grid
+        assert np.allclose((r["values"] - r["lo"]) / step, r["levels"], atol=1e-9)
+
+
+def test_double_quant_changes_only_the_stored_scalars():
+    x = np.random.default_rng(5).normal(size=(128, 128))
+    cb = np.random.default_rng(6).normal(size=(256, 8))
+    a = orc.quantize_block(x, cb, 1)
+    b = orc.quantize_block(x, cb, 1, double_quant=True)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["s2"], b["s2"])
+    assert np.allclose(b["s1"], orc.dq4(b["s1_dq"]["values"])["values"])
+    assert np.max(np.abs(b["o"] - a["o"])) <= (b["o_dq"]["hi"] - b["o_dq"]["lo"]) / 30 + 1e-3
