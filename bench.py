@@ -54,8 +54,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh,
 # comments and whitespace removed).
 # Any later change to those files makes the figure stale; the bench then reports null.
-DECODE_TRAFFIC = {"sha256": "d185012d09b25d085472f087fae6804a393b62f07760bbafe256260b3ab4c243",
-                  "bytes_per_launch": 320946176 + 2808320}
+DECODE_TRAFFIC = {"sha256": "cf31ac75a95f8443fc28c9c52b4505962cd619fb25bfbea6c68d8f7532862f50",
+                  "bytes_per_launch": 320999808 + 2207232}
 
 
 def decode_sources_sha256() -> str:

@@ -221,6 +221,12 @@ __device__ __forceinline__ void issue_stage(uint32_t dst, uint32_t mdst, uint32_
   }
 }
 
+// A 4-bit level (the low nibble of `bits`) as a float without an int-to-float
+// conversion: 2^23 + level is exact in fp32, and subtracting 2^23 leaves the level.
+__device__ __forceinline__ float nibble_f(uint32_t bits) {
+  return __uint_as_float((bits & 15u) | 0x4B000000u) - 8388608.0f;
+}
+
 // (lo, step) of a 4-bit group from its fp16 (lo, hi) pair.
 __device__ __forceinline__ float2 dq_lo_step(const unsigned char* par) {
   const float2 lh = __half22float2(*reinterpret_cast<const __half2*>(par));
@@ -233,8 +239,8 @@ __device__ __forceinline__ void dq_mean_row(unsigned char* row, const unsigned c
                                             int lane) {
   const float2 ls = dq_lo_step(par);
   const uint32_t two = *reinterpret_cast<const uint16_t*>(levels + 2 * lane);
-  const float c0 = fmaf((float)(two & 15u), ls.y, ls.x), c1 = fmaf((float)((two >> 4) & 15u), ls.y, ls.x);
-  const float c2 = fmaf((float)((two >> 8) & 15u), ls.y, ls.x), c3 = fmaf((float)((two >> 12) & 15u), ls.y, ls.x);
+  const float c0 = fmaf(nibble_f(two), ls.y, ls.x), c1 = fmaf(nibble_f(two >> 4), ls.y, ls.x);
+  const float c2 = fmaf(nibble_f(two >> 8), ls.y, ls.x), c3 = fmaf(nibble_f(two >> 12), ls.y, ls.x);
   *reinterpret_cast<uint2*>(row + 8 * lane) = make_uint2(pack_half2(c0, c1), pack_half2(c2, c3));
 }
 
@@ -703,8 +709,8 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       if constexpr (DQ) {
         const int tk = tt + t_l;
         const uint32_t sh = 4u * (uint32_t)(tk & 1);
-        const float kl = (float)(((uint32_t)sb[ST_KN + STAGE_TOK * 2 + (tk >> 1)] >> sh) & 15u);
-        const float vl = (float)(((uint32_t)sb[ST_VN + STAGE_TOK * 2 + (tk >> 1)] >> sh) & 15u);
+        const float kl = nibble_f((uint32_t)sb[ST_KN + STAGE_TOK * 2 + (tk >> 1)] >> sh);
+        const float vl = nibble_f((uint32_t)sb[ST_VN + STAGE_TOK * 2 + (tk >> 1)] >> sh);
         kn = make_float2(fmaf(kl, k_s1.y, k_s1.x), __half2float(reinterpret_cast<const __half*>(sb + ST_KN)[tk]));
         vn = make_float2(fmaf(vl, v_s1.y, v_s1.x), __half2float(reinterpret_cast<const __half*>(sb + ST_VN)[tk]));
       } else {
