@@ -158,22 +158,24 @@ def attn_error(out: np.ndarray, ref: np.ndarray) -> float:
 # ---------------------------------------------------------------------------
 def _oracle_block(args):
     from oracle import nsn_oracle as orc
-    x, cb, mode = args
-    r = orc.quantize_block(x, cb, mode)
-    return {k: r[k] for k in ("codes", "signs", "s1", "s2", "o", "gap", "u")}
+    x, cb, mode = args[:3]
+    dq = len(args) > 3 and args[3]
+    r = orc.quantize_block(x, cb, mode, double_quant=dq)
+    keys = ("codes", "signs", "s1", "s2", "o", "gap", "u") + (("s1_dq", "o_dq") if dq else ())
+    return {k: r[k] for k in keys}
 
 
-def oracle_cache_sequence(pool, x, n_prefill, n_total, cb, mode, window=128):
+def oracle_cache_sequence(pool, x, n_prefill, n_total, cb, mode, window=128, double_quant=False):
     """Oracle cache of one sequence x [T, 128] (fp64) after a prefill of n_prefill
     tokens and appends up to n_total: (quantized dict, fp16 window rows)."""
     from oracle import nsn_oracle as orc
     q = orc.prefill_split(n_prefill, 128, window)
-    blocks = [(x[a:min(a + 128, q)], cb, mode) for a in range(0, q, 128)]
+    blocks = [(x[a:min(a + 128, q)], cb, mode, double_quant) for a in range(0, q, 128)]
     parts = list(pool.map(_oracle_block, blocks, chunksize=4)) if blocks else []
     win = list(orc.to_f16(x[q:n_prefill]))
     for t in range(n_prefill, n_total):
         if len(win) == window:
-            parts.append(_oracle_block((np.array(win), cb, mode)))
+            parts.append(_oracle_block((np.array(win), cb, mode, double_quant)))
             win = []
         win.append(orc.to_f16(x[t]))
     cat = lambda k: np.concatenate([p[k] for p in parts])  # noqa: E731

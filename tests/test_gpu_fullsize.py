@@ -32,7 +32,7 @@ def pool():
         yield ex
 
 
-def run_workload(cfg_id, steps, pool, sample_blocks=12, seed_off=0):
+def run_workload(cfg_id, steps, pool, sample_blocks=12, seed_off=0, double_quant=False):
     W = synthetic.WORKLOADS[cfg_id]
     B, H, HQ, T, mk, mv = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["seq"], W["mode_k"], W["mode_v"]
     g = HQ // H
@@ -44,7 +44,8 @@ def run_workload(cfg_id, steps, pool, sample_blocks=12, seed_off=0):
     cbk, cbv = tl.codebook(mk), tl.codebook(mv)
     dk, dv = torch.from_numpy(cbk).to(dev), torch.from_numpy(cbv).to(dev)
     cap = ((T + steps + 255) // 128) * 128
-    kc, vc = nsn.Cache(B, H, cap, 128, mk, device=dev), nsn.Cache(B, H, cap, 128, mv, device=dev)
+    kc = nsn.Cache(B, H, cap, 128, mk, device=dev, double_quant=double_quant)
+    vc = nsn.Cache(B, H, cap, 128, mv, device=dev, double_quant=double_quant)
     nsn.nsn_quantize_kv(kc, xk[:, :T], dk)
     nsn.nsn_quantize_kv(vc, xv[:, :T], dv)
     for s in range(T, T + steps):
@@ -63,26 +64,37 @@ def run_workload(cfg_id, steps, pool, sample_blocks=12, seed_off=0):
         b, h, blk = int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(n_quant0 // 128))
         for cache, x, cb, mode in ((kc, xk, cbk, mk), (vc, xv, cbv, mv)):
             xb = x[b, 128 * blk:128 * (blk + 1), h].float().cpu().numpy().astype(np.float64)
-            jobs.append((xb, cb.astype(np.float64), mode))
+            jobs.append((xb, cb.astype(np.float64), mode, double_quant))
             where.append((cache, b, h, blk))
     refs = list(pool.map(tl._oracle_block, jobs))
     for (cache, b, h, blk), ref in zip(where, refs):
         sl = slice(128 * blk, 128 * (blk + 1))
         got = {"codes": cache.codes[b, h, sl].cpu().numpy().astype(np.int64),
-               "signs": None if cache.signs is None else tl.signs_to_natural(cache.signs[b, h, sl].cpu().numpy()),
-               "s1": cache.norms[b, h, sl, 0].float().cpu().numpy().astype(np.float64),
-               "s2": cache.norms[b, h, sl, 1].float().cpu().numpy().astype(np.float64),
-               "o": cache.means[b, h, blk:blk + 1].float().cpu().numpy().astype(np.float64)}
-        ref = dict(ref, o=ref["o"][None])
-        tl.compare_codes(got, ref, ref["u"])
-        tl.compare_norms_means(got, ref, (got["codes"] != ref["codes"]).any(axis=1))
+               "signs": None if cache.signs is None else tl.signs_to_natural(cache.signs[b, h, sl].cpu().numpy())}
+        s2 = cache.norms[b, h, sl] if double_quant else cache.norms[b, h, sl, 1]
+        tl.compare_codes(dict(got, s2=s2.float().cpu().numpy().astype(np.float64)), ref, ref["u"])
+        if double_quant:
+            par = cache.dq_params[b, h, blk, :4].float().cpu().numpy().astype(np.float64)
+            q1, qo = ref["s1_dq"], ref["o_dq"]
+            assert np.array_equal(par, [q1["lo"], q1["hi"], qo["lo"], qo["hi"]])
+            s1_lev = tl.unpack_levels(cache.s1_levels[b, h, 64 * blk:64 * (blk + 1)].cpu().numpy())
+            o_lev = tl.unpack_levels(cache.means[b, h, blk].cpu().numpy())
+            for g_, r_ in ((s1_lev, q1["levels"]), (o_lev, qo["levels"])):
+                assert (np.abs(g_ - r_) <= 1).all() and (g_ != r_).sum() <= 2
+        else:
+            got.update(s1=cache.norms[b, h, sl, 0].float().cpu().numpy().astype(np.float64),
+                       s2=cache.norms[b, h, sl, 1].float().cpu().numpy().astype(np.float64),
+                       o=cache.means[b, h, blk:blk + 1].float().cpu().numpy().astype(np.float64))
+            ref = dict(ref, o=ref["o"][None])
+            tl.compare_norms_means(got, ref, (got["codes"] != ref["codes"]).any(axis=1))
 
     # ---- one sequence end to end ----
     b, h = int(rng.integers(B)), int(rng.integers(H))
     seqs = []
     for x, cb, mode in ((xk, cbk, mk), (xv, cbv, mv)):
         xs = x[b, :, h].float().cpu().numpy().astype(np.float64)
-        seqs.append(tl.oracle_cache_sequence(pool, xs, T, T + steps, cb.astype(np.float64), mode))
+        seqs.append(tl.oracle_cache_sequence(pool, xs, T, T + steps, cb.astype(np.float64), mode,
+                                             double_quant=double_quant))
     (kq, kw), (vq, vw) = seqs
     got_k = tl.read_cache(kc, b, h)
     assert got_k["n_quant"] == kq["codes"].shape[0] and got_k["n_window"] == kw.shape[0]
@@ -107,3 +119,8 @@ def test_fullsize_extreme_compression_layer(pool):
 def test_fullsize_long_context(pool):
     # batch 4, 128k-token prefill, 2-bit K / 1-bit V, 16 decode steps
     run_workload(5, 16, pool)
+
+
+def test_fullsize_decode_throughput_layer_double_quant(pool):
+    # the same layer with s1 and o stored in 4 bits (bench.py --double-quant)
+    run_workload(3, 1, pool, double_quant=True)
