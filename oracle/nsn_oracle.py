@@ -35,6 +35,8 @@ Readings where the pages are silent (each is listed in the design doc):
   * Degenerate norms: s1 = 0 gives n1 = 0; s2 = 0 gives u = 0.
   * Double quantization (optional): s1 and o stored in 4 bits, 16 uniform
     levels between the fp16-rounded group min and max (`dq4`).
+  * Pre-RoPE keys (optional): rotate-half pairing (i, i + d/2), angle
+    pos * theta_i, key position = index in the sequence (`apply_rope`).
 
 Parity pins: every function here is pinned in tests/test_oracle_*.py against
 closed forms, a hand-derived worked example (tests/golden/), library routines
@@ -340,6 +342,61 @@ def decode_attention(q_group: np.ndarray, kq: dict, vq: dict, k_window: np.ndarr
     vals = np.concatenate([v_hat, np.asarray(v_window, np.float64)], axis=0)
     if keys.shape[0] == 0:
         raise ValueError("attention over zero tokens")
+    return attention(q_group, keys, vals, scale)
+
+
+# ---------------------------------------------------------------------------
+# Rotary position embedding of the keys -- [TS] Metodologia 4: NSN is applied to
+# the keys BEFORE the rotary position embedding, so the cache holds pre-RoPE keys
+# and attention rotates each dequantized key at its own position.
+# Readings (the pages name RoPE only): the Llama "rotate-half" pairing, dim i with
+# dim i + d/2 at angle pos * theta_i; theta_i = base^(-2i/d) for the standard
+# table; the position of a cached key is its index in the sequence (quantized
+# tokens first, then the window); the query arrives already rotated.
+# ---------------------------------------------------------------------------
+def rope_inv_freq(d: int, base: float) -> np.ndarray:
+    """theta_i = base^(-2i/d), i < d/2 (fp64)."""
+    i = np.arange(d // 2, dtype=np.float64)
+    return np.power(float(base), -2.0 * i / d)
+
+
+def apply_rope(x: np.ndarray, positions, inv_freq) -> np.ndarray:
+    """Rows x [n, d] rotated at their positions [n] (rotate-half pairing).
+
+    For i < d/2, angle a = pos * theta_i:
+      out[i]       = x[i] cos a - x[i + d/2] sin a
+      out[i + d/2] = x[i + d/2] cos a + x[i] sin a
+    """
+    x = np.asarray(x, dtype=np.float64)
+    n, d = x.shape
+    half = d // 2
+    theta = np.asarray(inv_freq, dtype=np.float64)
+    if theta.shape != (half,):
+        raise ValueError("inv_freq must hold d/2 frequencies")
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * theta[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    lo, hi = x[:, :half], x[:, half:]
+    return np.concatenate([lo * c - hi * s, hi * c + lo * s], axis=1)
+
+
+def decode_attention_rope(q_group: np.ndarray, kq: dict, vq: dict, k_window: np.ndarray,
+                          v_window: np.ndarray, codebook_k, codebook_v, mode_k: int,
+                          mode_v: int, scale: float, inv_freq, block: int = 128) -> np.ndarray:
+    """Decode attention over pre-RoPE keys ([TS] Metodologia 4).
+
+    Every key -- dequantized tokens at positions 0 .. n_quant-1, then the window
+    at n_quant .. -- is rotated at its position before the scores; q_group is
+    the already-rotated query.  Values are not rotated.
+    """
+    k_hat = dequantize(kq["codes"], kq["signs"], kq["s1"], kq["s2"], kq["o"],
+                       codebook_k, mode_k, block)
+    v_hat = dequantize(vq["codes"], vq["signs"], vq["s1"], vq["s2"], vq["o"],
+                       codebook_v, mode_v, block)
+    keys = np.concatenate([k_hat, np.asarray(k_window, np.float64)], axis=0)
+    vals = np.concatenate([v_hat, np.asarray(v_window, np.float64)], axis=0)
+    if keys.shape[0] == 0:
+        raise ValueError("attention over zero tokens")
+    keys = apply_rope(keys, np.arange(keys.shape[0]), inv_freq)
     return attention(q_group, keys, vals, scale)
 
 
