@@ -184,25 +184,38 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
 // each); the fp16 mean rows are formed from them in shared memory.
 constexpr int DQ_LEV = 2 * D;           // o levels of K at +256, of V at +320
 constexpr int DQ_PAR = 2 * D + D;       // parameters of K at +384, of V at +400
-template <int MK, int MV, bool DQ>
+// With RGH > 0 (pre-RoPE keys) the K logits of the stage were computed by
+// rope_scores_kernel: the stage's 64 x RGH fp32 logits (from `rsrc`, this warp's
+// (sequence, head group) row of them) take the place of the K codes, and the K
+// signs and norms are not copied.
+template <int MK, int MV, bool DQ, int RGH = 0>
 __device__ __forceinline__ void issue_stage(uint32_t dst, uint32_t mdst, uint32_t bar, const CacheView& kc,
-                                           const CacheView& vc, int64_t seq, int t0, bool with_means) {
+                                           const CacheView& vc, int64_t seq, int t0, bool with_means,
+                                           const float* rsrc = nullptr) {
   const int64_t cap = kc.capacity;
   const int64_t tok = seq * cap + t0;
   constexpr uint32_t CB = STAGE_TOK * 16;
   constexpr uint32_t NB = DQ ? STAGE_TOK * 2 + STAGE_TOK / 2 : STAGE_TOK * 4;
   constexpr uint32_t MB = DQ ? 2 * (D / 2) + 2 * 16 : MEAN_BYTES;
-  const uint32_t bytes = CB * 2 + NB * 2 + (MK == NSN_MODE_2BIT ? CB : 0) + (MV == NSN_MODE_2BIT ? CB : 0) +
-                         (with_means ? MB : 0);
+  constexpr uint32_t RB = STAGE_TOK * RGH * 4;
+  static_assert(RB <= ST_KS - ST_KC, "the stage's logits fit the K code area");
+  constexpr uint32_t KB = RGH > 0 ? RB : CB + NB + (MK == NSN_MODE_2BIT ? CB : 0);
+  const uint32_t bytes = KB + CB + NB + (MV == NSN_MODE_2BIT ? CB : 0) + (with_means ? MB : 0);
   mbar_expect_tx(bar, bytes);
-  bulk_g2s(dst + ST_KC, kc.codes + tok * NSUB, CB, bar);
-  if constexpr (MK == NSN_MODE_2BIT) bulk_g2s(dst + ST_KS, kc.signs + tok * NSUB, CB, bar);
+  if constexpr (RGH > 0) {
+    bulk_g2s(dst + ST_KC, rsrc + (int64_t)t0 * RGH, RB, bar);
+  } else {
+    bulk_g2s(dst + ST_KC, kc.codes + tok * NSUB, CB, bar);
+    if constexpr (MK == NSN_MODE_2BIT) bulk_g2s(dst + ST_KS, kc.signs + tok * NSUB, CB, bar);
+  }
   bulk_g2s(dst + ST_VC, vc.codes + tok * NSUB, CB, bar);
   if constexpr (MV == NSN_MODE_2BIT) bulk_g2s(dst + ST_VS, vc.signs + tok * NSUB, CB, bar);
   const int64_t blk = seq * (cap / BLK) + t0 / BLK;
   if constexpr (DQ) {
-    bulk_g2s(dst + ST_KN, reinterpret_cast<const __half*>(kc.norms) + tok, STAGE_TOK * 2, bar);
-    bulk_g2s(dst + ST_KN + STAGE_TOK * 2, kc.s1_levels + tok / 2, STAGE_TOK / 2, bar);
+    if constexpr (RGH == 0) {
+      bulk_g2s(dst + ST_KN, reinterpret_cast<const __half*>(kc.norms) + tok, STAGE_TOK * 2, bar);
+      bulk_g2s(dst + ST_KN + STAGE_TOK * 2, kc.s1_levels + tok / 2, STAGE_TOK / 2, bar);
+    }
     bulk_g2s(dst + ST_VN, reinterpret_cast<const __half*>(vc.norms) + tok, STAGE_TOK * 2, bar);
     bulk_g2s(dst + ST_VN + STAGE_TOK * 2, vc.s1_levels + tok / 2, STAGE_TOK / 2, bar);
     if (with_means) {
@@ -212,7 +225,7 @@ __device__ __forceinline__ void issue_stage(uint32_t dst, uint32_t mdst, uint32_
       bulk_g2s(mdst + DQ_PAR + 16, vc.dq_params + blk * 8, 16, bar);
     }
   } else {
-    bulk_g2s(dst + ST_KN, kc.norms + tok, NB, bar);
+    if constexpr (RGH == 0) bulk_g2s(dst + ST_KN, kc.norms + tok, NB, bar);
     bulk_g2s(dst + ST_VN, vc.norms + tok, NB, bar);
     if (with_means) {
       bulk_g2s(mdst, kc.means + blk * D, D * 2, bar);
@@ -510,12 +523,15 @@ __device__ __noinline__ void cta_merge(const float* ws, const float* ws_acc, int
 //          scores of token g + 8 (p >> 1) for heads 2 (p & 1), 2 (p & 1) + 1.
 // Values:  O^T[d][h] += sum_t u_hat_v[t][d] w[t][h]  M = 16 dims, N = 8 heads, K = 16 tokens;
 //          the B operand is the weight matrix moved into place with movmatrix.trans.
-template <int GH, int MK, int MV, bool DQ>
+// RP (pre-RoPE keys): the K logits of every quantized and window token come
+// precomputed from rope_scores_kernel (`rscores`, rs_cap tokens per (sequence,
+// head group)); the kernel then reads neither the query nor the K cache.
+template <int GH, int MK, int MV, bool DQ, bool RP = false>
 __global__ void __launch_bounds__(32 * DEC_WARPS, 1)
 decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb, int64_t qsh,
               float qscale, const float* __restrict__ cbk_g, const float* __restrict__ cbv_g,
               unsigned int* __restrict__ counters, float* __restrict__ ws, float* __restrict__ out, int n_q_heads,
-              DecodeGeom geom) {
+              DecodeGeom geom, const float* __restrict__ rscores, int rs_cap) {
   static_assert(GH == 1 || GH == 2 || GH == 4, "1, 2 or 4 heads per warp");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
@@ -535,6 +551,8 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
   const int64_t P = (int64_t)nseq * (nsplit + 1);
   float* ws_acc = ws + acc_offset(P, G);
   const int64_t q_off = (int64_t)b * qsb + (int64_t)(hk * G + hbase) * qsh;
+  const float* rsrc = RP ? rscores + ((int64_t)(seq * ngroups + hg) * rs_cap) * GH : nullptr;
+  constexpr int RGH = RP ? GH : 0;
 
   // The query rows are requested first, before the codebook staging and the bulk
   // copies, so that they do not queue behind the copies of every warp.
@@ -544,7 +562,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
   // copy flies, issues its second copy, and only then does the CTA store the
   // codebooks and meet at the one barrier.
   float qrows[GH][4];
-  if (active) load_q_rows<GH>(qrows, q, dtype, q_off, qsh, lane);
+  if (!RP && active) load_q_rows<GH>(qrows, q, dtype, q_off, qsh, lane);
   static_assert(32 * DEC_WARPS == 2 * NCODES, "one codeword per thread");
   const int cb_c = tid & (NCODES - 1);
   const bool cb_isv = tid >= NCODES;
@@ -569,19 +587,19 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     mbar_init(bar0 + 8u, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     if (nstages > 0)
-      issue_stage<MK, MV, DQ>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc, seq,
-                          tok_begin, true);
+      issue_stage<MK, MV, DQ, RGH>(st_base, mb_base + (uint32_t)(((tok_begin / BLK) & 1) * MEAN_BYTES), bar0, kc, vc,
+                                   seq, tok_begin, true, rsrc);
   }
   __syncwarp();
 
   // ---- query operand (B of the score product), built while stage 0 flies, in
   // the second stage buffer, which is filled only afterwards ----
   uint32_t qb[8][2];
-  if (active) build_q_operand<GH>(qb, qrows, qscale * INV_SQRT_D, true, lane, &sm.stage[warp][1][0]);
+  if (!RP && active) build_q_operand<GH>(qb, qrows, qscale * INV_SQRT_D, true, lane, &sm.stage[warp][1][0]);
   if (lane == 0 && nstages > 1) {
     const int t1 = tok_begin + STAGE_TOK;
-    issue_stage<MK, MV, DQ>(st_base + STAGE_BYTES, mb_base + (uint32_t)(((t1 / BLK) & 1) * MEAN_BYTES), bar0 + 8, kc, vc,
-                        seq, t1, (t1 % BLK) == 0);
+    issue_stage<MK, MV, DQ, RGH>(st_base + STAGE_BYTES, mb_base + (uint32_t)(((t1 / BLK) & 1) * MEAN_BYTES), bar0 + 8,
+                                 kc, vc, seq, t1, (t1 % BLK) == 0, rsrc);
   }
 
   // ---- stage the replicated fp16 codebooks (whole CTA, once) ----
@@ -640,7 +658,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       v_s1 = dq_lo_step(mb + DQ_PAR + 16);
     }
 
-    if (block_start) {
+    if (!RP && block_start) {
       if constexpr (DQ) {  // the fp16 o_K row, from its levels
         dq_mean_row(mb, mb + DQ_LEV, mb + DQ_PAR + 4, lane);
         __syncwarp();
@@ -663,14 +681,15 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     const bool full = t_stage + STAGE_TOK <= tok_end;  // every token of the stage is valid
     for (int tile = 0; tile < ntile; ++tile) {
       const int tt = 16 * tile;  // token offset inside the stage
-      const uint4 kcw = *reinterpret_cast<const uint4*>(sb + ST_KC + (tt + tok_a) * 16);
+      uint4 kcw = make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (!RP) kcw = *reinterpret_cast<const uint4*>(sb + ST_KC + (tt + tok_a) * 16);
       uint32_t ks0 = 0u, ks1 = 0u;
-      if constexpr (MK == NSN_MODE_2BIT) {
+      if constexpr (!RP && MK == NSN_MODE_2BIT) {
         ks0 = *reinterpret_cast<const uint32_t*>(sb + ST_KS + (tt + g) * 16 + 4 * p);
         ks1 = *reinterpret_cast<const uint32_t*>(sb + ST_KS + (tt + 8 + g) * 16 + 4 * p);
       }
       uint32_t knw = 0u, vnw = 0u;
-      if constexpr (!DQ) knw = *reinterpret_cast<const uint32_t*>(sb + ST_KN + (tt + t_l) * 4);
+      if constexpr (!DQ && !RP) knw = *reinterpret_cast<const uint32_t*>(sb + ST_KN + (tt + t_l) * 4);
       const uint4 vcw = *reinterpret_cast<const uint4*>(sb + ST_VC + (tt + tok_v) * 16);
       uint32_t W0 = 0u, W1 = 0u;
       if constexpr (MV == NSN_MODE_2BIT) {
@@ -683,7 +702,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       // ---- scores: 8 k-steps of 16 dims in two independent accumulation chains ----
       float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < (RP ? 0 : 8); ++j) {
         const uint32_t code = __byte_perm(u4_word(kcw, j >> 1), 0u, (j & 1) ? sel_k1 : sel_k0);
         uint32_t aa[4];
         ldsm_x4(cbk_base + code * 128u, aa);
@@ -705,20 +724,29 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       const float d1 = (lo_lane ? S[1] : S[3]) + r1;
 
       // ---- scores with the NSN byproducts; online softmax (lazy re-basing) ----
-      float2 kn, vn;  // (s1, s2) of token t_l
+      float2 kn = make_float2(0.f, 0.f), vn;  // (s1, s2) of token t_l
       if constexpr (DQ) {
         const int tk = tt + t_l;
         const uint32_t sh = 4u * (uint32_t)(tk & 1);
-        const float kl = nibble_f((uint32_t)sb[ST_KN + STAGE_TOK * 2 + (tk >> 1)] >> sh);
+        if constexpr (!RP) {
+          const float kl = nibble_f((uint32_t)sb[ST_KN + STAGE_TOK * 2 + (tk >> 1)] >> sh);
+          kn = make_float2(fmaf(kl, k_s1.y, k_s1.x), __half2float(reinterpret_cast<const __half*>(sb + ST_KN)[tk]));
+        }
         const float vl = nibble_f((uint32_t)sb[ST_VN + STAGE_TOK * 2 + (tk >> 1)] >> sh);
-        kn = make_float2(fmaf(kl, k_s1.y, k_s1.x), __half2float(reinterpret_cast<const __half*>(sb + ST_KN)[tk]));
         vn = make_float2(fmaf(vl, v_s1.y, v_s1.x), __half2float(reinterpret_cast<const __half*>(sb + ST_VN)[tk]));
       } else {
         kn = __half22float2(*reinterpret_cast<const __half2*>(&knw));
         vn = __half22float2(*reinterpret_cast<const __half2*>(&vnw));
       }
-      float sc0 = kn.x * fmaf(kn.y, d0, qo0);
-      float sc1 = kn.x * fmaf(kn.y, d1, qo1);
+      float sc0, sc1;
+      if constexpr (RP) {  // padding heads (h >= GH) carry a running max of +1e30: any finite value will do
+        const float* lg = reinterpret_cast<const float*>(sb + ST_KC) + (tt + t_l) * GH;
+        sc0 = h0 < GH ? lg[h0] : 0.f;
+        sc1 = h0 + 1 < GH ? lg[h0 + 1] : 0.f;
+      } else {
+        sc0 = kn.x * fmaf(kn.y, d0, qo0);
+        sc1 = kn.x * fmaf(kn.y, d1, qo1);
+      }
       if (!full && t_stage + tt + t_l >= tok_end) {  // past the end: no weight, and no stale norms
         sc0 = sc1 = NEG_BIG;
         vn = make_float2(0.f, 0.f);
@@ -778,8 +806,9 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     __syncwarp();  // every lane is done with this stage buffer (and, at a block end, its means)
     if (lane == 0 && st + 2 < nstages) {
       const int tn = t_stage + 2 * STAGE_TOK;
-      issue_stage<MK, MV, DQ>(st_base + (uint32_t)(buf * STAGE_BYTES), mb_base + (uint32_t)(((tn / BLK) & 1) * MEAN_BYTES),
-                          bar0 + 8u * buf, kc, vc, seq, tn, (tn % BLK) == 0);
+      issue_stage<MK, MV, DQ, RGH>(st_base + (uint32_t)(buf * STAGE_BYTES),
+                                   mb_base + (uint32_t)(((tn / BLK) & 1) * MEAN_BYTES), bar0 + 8u * buf, kc, vc, seq, tn,
+                                   (tn % BLK) == 0, rsrc);
     }
   }
   if (active) store_partial<GH>(sx, ws, ws_acc, p0 + split, G, hbase, lane);
@@ -794,9 +823,11 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       const __half* kw0 = kc.window + seq * kc.window_len * D;
       const __half* vw0 = vc.window + seq * vc.window_len * D;
       issue_window_chunk(st_base, bar0, kw0, vw0, min(WCHUNK, nw), lane);
-      float wrows[GH][4];  // reloaded: keeping the first rows alive would cost registers in the main loop
-      load_q_rows<GH>(wrows, q, dtype, q_off, qsh, lane);
-      build_q_operand<GH>(qb, wrows, qscale, false, lane, &sm.stage[warp][1][0]);
+      if constexpr (!RP) {
+        float wrows[GH][4];  // reloaded: keeping the first rows alive would cost registers in the main loop
+        load_q_rows<GH>(wrows, q, dtype, q_off, qsh, lane);
+        build_q_operand<GH>(qb, wrows, qscale, false, lane, &sm.stage[warp][1][0]);
+      }
       if (nch > 1) issue_window_chunk(st_base + STAGE_BYTES, bar0 + 8u, kw0 + WCHUNK * D, vw0 + WCHUNK * D,
                                       min(WCHUNK, nw - WCHUNK), lane);
       const int wr = lane & 7;  // ldmatrix row (token) of this lane; rows 8-15 repeat rows 0-7
@@ -813,20 +844,27 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
         const uint32_t kbuf = st_base + (uint32_t)(buf * STAGE_BYTES);
         const uint32_t vbuf = kbuf + (uint32_t)WC_V;
         const uint32_t rowoff = (uint32_t)(min(wr, rows - 1) * WROWB);
-        float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
+        float sc0, sc1;
+        if constexpr (RP) {  // logits of window slot w at position n_quant + w
+          const float* lg = rsrc + (int64_t)(nq + c * WCHUNK + min(t_l, rows - 1)) * GH;
+          sc0 = h0 < GH ? lg[h0] : 0.f;
+          sc1 = h0 + 1 < GH ? lg[h0 + 1] : 0.f;
+        } else {
+          float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint32_t aa[4];
-          ldsm_x4(kbuf + rowoff + (uint32_t)(32 * j + 16 * (lane >> 4)), aa);
-          if (j & 1) mma_full(S2, aa, qb[j][0], qb[j][1]);
-          else mma_full(S, aa, qb[j][0], qb[j][1]);
+          for (int j = 0; j < 8; ++j) {
+            uint32_t aa[4];
+            ldsm_x4(kbuf + rowoff + (uint32_t)(32 * j + 16 * (lane >> 4)), aa);
+            if (j & 1) mma_full(S2, aa, qb[j][0], qb[j][1]);
+            else mma_full(S, aa, qb[j][0], qb[j][1]);
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) S[i] += S2[i];
+          const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[2] : S[0], 2);
+          const float r1 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[3] : S[1], 2);
+          sc0 = (lo_lane ? S[0] : S[2]) + r0;
+          sc1 = (lo_lane ? S[1] : S[3]) + r1;
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) S[i] += S2[i];
-        const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[2] : S[0], 2);
-        const float r1 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[3] : S[1], 2);
-        float sc0 = (lo_lane ? S[0] : S[2]) + r0;
-        float sc1 = (lo_lane ? S[1] : S[3]) + r1;
         if (t_l >= rows) sc0 = sc1 = NEG_BIG;  // tokens 8-15 of the tile and rows past the window
         float unused0 = 0.f, unused1 = 0.f;
         lazy_update(sx, sc0, sc1, unused0, unused1);
@@ -886,6 +924,302 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
 }
 
 // ---------------------------------------------------------------------------
+// Pre-RoPE keys: the K logits ([TS] Metodologia 4 -- NSN is applied to the keys
+// before the rotary position embedding, so the cache holds pre-RoPE keys and each
+// is rotated at its own position when it is attended).  For key t of a (batch,
+// kv-head) at position pos (its index in the sequence: quantized tokens first,
+// then the window) and query head h of one head group:
+//   quantized:  logit = qscale * s1_t * q_h . R_pos(s2_t H u_hat_t + H o_b)
+//   window:     logit = qscale * q_h . R_pos(k_t)        (k_t the stored fp16 row)
+// with H the orthonormal Hadamard matrix and R_pos the rotate-half rotation of
+// dims (i, i + 64) by pos * theta_i.  The logits (log2 units) go to a workspace
+// array that decode_kernel<..., RP = true> reads in place of its K path.
+//
+// Per 16-token tile a warp forms H u_hat on the tensor cores.  With dim
+// k = 16a + b, H_128 = H_8 (x) H_16, so output k-step a' accumulates k-step a of
+// u_hat times H_8[a'][a] H_16: the B operand is always +H_16 or -H_16 (4 constant
+// registers each) and the sum is exact up to fp32 accumulation.  On the
+// accumulator fragments the lane holds dims i and i + 64 of the same tokens in the
+// same register slot, so the NSN affine terms and the rotation run in fp32 in
+// registers; the rotated key is split into fp16 hi + lo and multiplied by the
+// fp16 hi + lo query (the m16n8k16 A-from-accumulator layout needs no shuffle).
+// (cos, sin)(pos theta_i) = (cos, sin)(pos0 theta_i) * (cos, sin)(r theta_i),
+// pos0 the 64-token stage start (per warp, angle reduced in fp64) and r < 64 from
+// a CTA table.
+// ---------------------------------------------------------------------------
+constexpr int RS_WARPS = 8;
+constexpr int RS_OFF_ROW = STAGE_TOK + 8;  // float2 per table row: 64 + padding, so 8 lanes of a
+                                           // 16-byte fetch on two rows hit different banks
+struct RsSmem {
+  alignas(128) uint4 cbk[NCODES][8];                    // replicated fp16 K codebook (as in decode_kernel)
+  alignas(16) float2 off[STAGE_TOK][RS_OFF_ROW];        // (cos, sin)(r theta_i), r < 64, i < 64
+  alignas(128) unsigned char wk[RS_WARPS][8 * QS_ROW];  // per warp: query staging, then H o_b and the stage base
+};
+static_assert(8 * QS_ROW >= D * 4 + (D / 2) * 8, "H o_b and the base angles fit the staging area");
+
+// (cos a, sin a) with a reduced to [-pi, pi] in fp64 first.
+__device__ __forceinline__ float2 rope_cs(double a) {
+  const double two_pi = 6.283185307179586;
+  const double r = a - two_pi * rint(a * (1.0 / two_pi));
+  float sn, cs;
+  sincosf((float)r, &sn, &cs);
+  return make_float2(cs, sn);
+}
+
+template <int GH, int MK, bool DQ>
+__global__ void __launch_bounds__(32 * RS_WARPS, 2)
+rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int32_t* __restrict__ v_nwindow,
+                   const void* __restrict__ q, int dtype, int64_t qsb, int64_t qsh, float qscale,
+                   const float* __restrict__ inv_freq, const float* __restrict__ cbk_g, float* __restrict__ rscores,
+                   int rs_cap, int G, int nchunk) {
+  static_assert(GH == 1 || GH == 2 || GH == 4, "1, 2 or 4 heads per warp");
+  static_assert(32 * RS_WARPS == NCODES, "one codeword per thread");
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  RsSmem& sm = *reinterpret_cast<RsSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, p = lane & 3;
+  {
+    const uint4 row = cb_row_f16(cbk_g, tid);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) sm.cbk[tid][(r + tid) & 7] = row;
+    for (int e = tid; e < STAGE_TOK * (D / 2); e += 32 * RS_WARPS) {
+      const int r = e / (D / 2), i = e % (D / 2);
+      sm.off[r][i] = rope_cs((double)r * (double)__ldg(inv_freq + i));
+    }
+  }
+  __syncthreads();  // the only CTA barrier
+
+  const int ngroups = G / GH;
+  const int nseq = kc.batch * kc.n_kv_heads;
+  const int gw = blockIdx.x * RS_WARPS + warp;
+  if (gw >= nseq * ngroups * nchunk) return;
+  const int chunk = gw % nchunk;
+  const int hg = (gw / nchunk) % ngroups;
+  const int64_t seq = (gw / nchunk) / ngroups;
+  const int b = (int)(seq / kc.n_kv_heads), hk = (int)(seq % kc.n_kv_heads);
+  // the same token counts as decode_kernel
+  const int nq = min(min(kc.n_quant[seq], v_nquant[seq]), kc.capacity);
+  const int nw = (kc.window_len > 0) ? max(0, min(min(kc.n_window[seq], v_nwindow[seq]), kc.window_len)) : 0;
+  const int nst_q = (nq + STAGE_TOK - 1) / STAGE_TOK;
+  const int nst = nst_q + (nw + STAGE_TOK - 1) / STAGE_TOK;
+  const int spc = (nst + nchunk - 1) / nchunk;
+  const int st_first = chunk * spc, st_last = min(nst, st_first + spc);
+  if (st_first >= st_last) return;
+  float* rdst = rscores + ((int64_t)(seq * ngroups + hg) * rs_cap) * GH;
+
+  // query operand, original domain (fp16 hi rows 0-3, residual rows 4-7)
+  unsigned char* wk = &sm.wk[warp][0];
+  uint32_t qb[8][2];
+  {
+    float qrows[GH][4];
+    load_q_rows<GH>(qrows, q, dtype, (int64_t)b * qsb + (int64_t)(hk * G + hg * GH) * qsh, qsh, lane);
+    build_q_operand<GH>(qb, qrows, qscale, false, lane, wk);
+  }
+  float* hob = reinterpret_cast<float*>(wk);                // H o_b of the current block (128 fp32)
+  float2* base = reinterpret_cast<float2*>(wk + D * 4);     // (cos, sin)(pos0 theta_i), 64
+
+  // +-H_16 as the B operand: column n = g + 8 nt, rows 2p, 2p+1 | 2p+8, 2p+9
+  uint32_t Hp[2][2], Hn[2][2];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const int n = g + 8 * nt;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int k0 = 2 * p + 8 * r;
+      const uint32_t e0 = (__popc(k0 & n) & 1) ? 0xBC00u : 0x3C00u;
+      const uint32_t e1 = (__popc((k0 + 1) & n) & 1) ? 0xBC00u : 0x3C00u;
+      Hp[nt][r] = e0 | (e1 << 16);
+      Hn[nt][r] = Hp[nt][r] ^ 0x80008000u;
+    }
+  }
+  const uint32_t cbk_base = smem_addr(&sm.cbk[0][0]) + (uint32_t)(lane & 7) * 16u;
+  const int tok_a = (lane & 7) + 8 * ((lane >> 3) & 1);
+  const uint32_t sel_k0 = 0x4440u | (uint32_t)(lane >> 4);
+  const uint32_t sel_k1 = 0x4440u | (uint32_t)(2 + (lane >> 4));
+  const bool lo_lane = p < 2;
+  const int t_l = g + (lo_lane ? 0 : 8);
+  const int h0 = 2 * (p & 1);
+  const int64_t cap = kc.capacity;
+  int cur_blk = -1;
+
+  for (int st = st_first; st < st_last; ++st) {
+    const bool win = st >= nst_q;
+    const int pos0 = win ? nq + (st - nst_q) * STAGE_TOK : st * STAGE_TOK;
+    const int pend = win ? nq + nw : nq;  // positions below this are keys
+    __syncwarp();  // the previous stage is done with `base` and `hob`
+    {
+      const float2 th = __ldg(reinterpret_cast<const float2*>(inv_freq) + lane);
+      base[2 * lane] = rope_cs((double)pos0 * (double)th.x);
+      base[2 * lane + 1] = rope_cs((double)pos0 * (double)th.y);
+    }
+    float2 s1ls = make_float2(0.f, 0.f);  // (lo, step) of the block's s1 levels
+    if (!win) {
+      const int64_t blk = seq * (cap / BLK) + pos0 / BLK;
+      if constexpr (DQ) s1ls = dq_lo_step(reinterpret_cast<const unsigned char*>(kc.dq_params + blk * 8));
+      if (pos0 / BLK != cur_blk) {
+        cur_blk = pos0 / BLK;
+        float v[4];
+        if constexpr (DQ) {
+          const float2 ls = dq_lo_step(reinterpret_cast<const unsigned char*>(kc.dq_params + blk * 8 + 2));
+          const uint32_t two = reinterpret_cast<const uint16_t*>(kc.means)[blk * (D / 4) + lane];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)  // o is stored as the fp16 rounding of its level's value
+            v[i] = __half2float(__float2half_rn(fmaf(nibble_f(two >> (4 * i)), ls.y, ls.x)));
+        } else {
+          const uint2 r = __ldg(reinterpret_cast<const uint2*>(kc.means + blk * D) + lane);
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
+          const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
+          v[0] = a.x; v[1] = a.y; v[2] = c.x; v[3] = c.y;
+        }
+        fwht128_warp(v, lane);
+        *reinterpret_cast<float4*>(hob + 4 * lane) =
+            make_float4(v[0] * INV_SQRT_D, v[1] * INV_SQRT_D, v[2] * INV_SQRT_D, v[3] * INV_SQRT_D);
+      }
+    }
+    __syncwarp();
+
+    for (int m = 0; m < STAGE_TOK / 16; ++m) {
+      const int tt = pos0 + 16 * m;  // position of the tile's first token
+      if (tt >= pend) break;
+      float s1r[2] = {1.f, 1.f}, s2r[2] = {1.f, 1.f};  // rows g, g + 8
+      uint32_t A[8][4];
+      if (!win) {
+        const int64_t tq = seq * cap + tt;
+        const uint4 kcw = __ldg(reinterpret_cast<const uint4*>(kc.codes + (tq + tok_a) * NSUB));
+        uint32_t ks0 = 0u, ks1 = 0u;
+        if constexpr (MK == NSN_MODE_2BIT) {
+          ks0 = __ldg(reinterpret_cast<const uint32_t*>(kc.signs + (tq + g) * NSUB) + p);
+          ks1 = __ldg(reinterpret_cast<const uint32_t*>(kc.signs + (tq + 8 + g) * NSUB) + p);
+        }
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int64_t tk = tq + g + 8 * rr;
+          if constexpr (DQ) {
+            s2r[rr] = __half2float(reinterpret_cast<const __half*>(kc.norms)[tk]);
+            const uint32_t lv = (uint32_t)__ldg(kc.s1_levels + tk / 2) >> (4 * (uint32_t)(tk & 1));
+            s1r[rr] = fmaf(nibble_f(lv), s1ls.y, s1ls.x);
+          } else {
+            const float2 n2 = __half22float2(kc.norms[tk]);
+            s1r[rr] = n2.x;
+            s2r[rr] = n2.y;
+          }
+        }
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          const uint32_t code = __byte_perm(u4_word(kcw, a >> 1), 0u, (a & 1) ? sel_k1 : sel_k0);
+          ldsm_x4(cbk_base + code * 128u, A[a]);
+          if constexpr (MK == NSN_MODE_2BIT) {
+            A[a][0] = apply_signs(A[a][0], ks0, 2 * a);
+            A[a][1] = apply_signs(A[a][1], ks1, 2 * a);
+            A[a][2] = apply_signs(A[a][2], ks0, 2 * a + 1);
+            A[a][3] = apply_signs(A[a][3], ks1, 2 * a + 1);
+          }
+        }
+      }
+      const int r_off = 16 * m + g;  // offset-table rows of this lane's tokens: r_off, r_off + 8
+      float S[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ap = 0; ap < 4; ++ap) {
+        // y[h][nt][r]: dim 16 (ap + 4h) + 8 nt + 2p + (r & 1) of token row g + 8 (r >> 1)
+        float y[2][2][4];
+        if (!win) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int r = 0; r < 4; ++r) y[h][nt][r] = 0.f;
+#pragma unroll
+          for (int a = 0; a < 8; ++a) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const bool neg = (__popc((ap + 4 * h) & a) & 1) != 0;  // H_8[ap + 4h][a]
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt)
+                mma_full(y[h][nt], A[a], neg ? Hn[nt][0] : Hp[nt][0], neg ? Hn[nt][1] : Hp[nt][1]);
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              const float2 o2 = *reinterpret_cast<const float2*>(hob + 16 * (ap + 4 * h) + 8 * nt + 2 * p);
+#pragma unroll
+              for (int r = 0; r < 4; ++r)
+                y[h][nt][r] = fmaf(s2r[r >> 1] * INV_SQRT_D, y[h][nt][r], (r & 1) ? o2.y : o2.x);
+            }
+        } else {
+          const __half* wrow = kc.window + seq * (int64_t)kc.window_len * D;
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const int w = min(tt - nq + g + 8 * rr, nw - 1);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt) {
+                const float2 kv = __half22float2(
+                    *reinterpret_cast<const __half2*>(wrow + (int64_t)w * D + 16 * (ap + 4 * h) + 8 * nt + 2 * p));
+                y[h][nt][2 * rr] = kv.x;
+                y[h][nt][2 * rr + 1] = kv.y;
+              }
+          }
+        }
+        // rotate dims (i, i + 64), i = 16 ap + 8 nt + 2p + e, at this lane's two token positions
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int i0 = 16 * ap + 8 * nt + 2 * p;
+          const float4 bb = *reinterpret_cast<const float4*>(base + i0);
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const float4 oo = *reinterpret_cast<const float4*>(&sm.off[r_off + 8 * rr][i0]);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float bc = e ? bb.z : bb.x, bs = e ? bb.w : bb.y;
+              const float oc = e ? oo.z : oo.x, os = e ? oo.w : oo.y;
+              const float c = fmaf(bc, oc, -bs * os), sn = fmaf(bs, oc, bc * os);
+              const float lo = y[0][nt][2 * rr + e], hi = y[1][nt][2 * rr + e];
+              y[0][nt][2 * rr + e] = fmaf(lo, c, -hi * sn);
+              y[1][nt][2 * rr + e] = fmaf(hi, c, lo * sn);
+            }
+          }
+        }
+        // fp16 hi + lo of the rotated key (k-steps ap and ap + 4) times the query
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t ahi[4], alo[4];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              const float x0 = y[h][nt][2 * rr], x1 = y[h][nt][2 * rr + 1];
+              const __half2 hh = __floats2half2_rn(x0, x1);
+              const float2 hf = __half22float2(hh);
+              ahi[2 * nt + rr] = *reinterpret_cast<const uint32_t*>(&hh);
+              alo[2 * nt + rr] = pack_half2(x0 - hf.x, x1 - hf.y);
+            }
+          mma_full(S, ahi, qb[ap + 4 * h][0], qb[ap + 4 * h][1]);
+          mma_full(S, alo, qb[ap + 4 * h][0], qb[ap + 4 * h][1]);
+        }
+      }
+      // hi + lo query columns -> (token t_l, heads h0, h0 + 1)
+      const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[2] : S[0], 2);
+      const float r1 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[3] : S[1], 2);
+      const float s1 = lo_lane ? s1r[0] : s1r[1];
+      const float sc0 = s1 * ((lo_lane ? S[0] : S[2]) + r0);
+      const float sc1 = s1 * ((lo_lane ? S[1] : S[3]) + r1);
+      const int pos = tt + t_l;
+      if (pos < pend) {
+        float* dst = rdst + (int64_t)pos * GH;
+        if constexpr (GH == 1) {
+          if (h0 == 0) dst[0] = sc0;
+        } else {
+          if (h0 + 1 < GH) *reinterpret_cast<float2*>(dst + h0) = make_float2(sc0, sc1);
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 static int sm_count() {
@@ -941,7 +1275,7 @@ static cudaError_t launch_t(const CacheView& kc, const CacheView& vc, const void
   const int nwarps = kc.batch * kc.n_kv_heads * geom.nsplit_q * (G / GH);
   dim3 grid((nwarps + DEC_WARPS - 1) / DEC_WARPS);
   decode_kernel<GH, MK, MV, DQ><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv,
-                                                               counters, partials, out, n_q_heads, geom);
+                                                               counters, partials, out, n_q_heads, geom, nullptr, 0);
   return cudaGetLastError();
 }
 
@@ -980,6 +1314,86 @@ cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* 
   unsigned int* counters = static_cast<unsigned int*>(ws);
   float* partials = static_cast<float*>(ws) + counter_words((int64_t)kc.batch * kc.n_kv_heads);
   return launch_any(kc, vc, q, dtype, n_q_heads, qsb, qsh, softmax_scale, cbk, cbv, out, counters, partials, geom, s);
+}
+
+// ---- pre-RoPE keys: logits kernel, then decode_kernel<..., RP = true> ----
+// Workspace: the decode workspace, then (256-byte aligned) the logits, rs_cap
+// tokens per (sequence, head group) of GH fp32 each.
+static int rope_rs_cap(int capacity, int window_len) {
+  return ((capacity + window_len + STAGE_TOK - 1) / STAGE_TOK) * STAGE_TOK;
+}
+static size_t rope_scores_offset(int batch, int n_kv_heads, const DecodeGeom& geom) {
+  return (decode_workspace_bytes(batch, n_kv_heads, geom) + 255u) / 256u * 256u;
+}
+size_t decode_rope_workspace_bytes(int batch, int n_kv_heads, int capacity, int window_len, const DecodeGeom& geom) {
+  return rope_scores_offset(batch, n_kv_heads, geom) +
+         (size_t)batch * n_kv_heads * geom.g * (size_t)rope_rs_cap(capacity, window_len) * sizeof(float);
+}
+
+template <int G, int MK, int MV, bool DQ>
+static cudaError_t launch_rope_t(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                                 int64_t qsb, int64_t qsh, float qscale, const float* inv_freq, const float* cbk,
+                                 const float* cbv, float* out, void* ws, const DecodeGeom& geom, cudaStream_t s) {
+  constexpr int GH = G < 4 ? G : 4;
+  const int nseq = kc.batch * kc.n_kv_heads;
+  const int rs_cap = rope_rs_cap(kc.capacity, kc.window_len);
+  float* rscores = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) +
+                                            rope_scores_offset(kc.batch, kc.n_kv_heads, geom));
+  // logits: jobs of contiguous 64-token stages per (sequence, head group), about
+  // two resident 8-warp CTAs per SM, twice over
+  const int jobs_per_chunk = nseq * (G / GH);
+  const int max_chunks = rs_cap / STAGE_TOK;
+  int nchunk = (sm_count() * 2 * RS_WARPS * 2 + jobs_per_chunk - 1) / jobs_per_chunk;
+  if (nchunk > max_chunks) nchunk = max_chunks;
+  if (nchunk < 1) nchunk = 1;
+  const size_t smem_a = sizeof(RsSmem);
+  cudaError_t e = cudaFuncSetAttribute(rope_scores_kernel<GH, MK, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem_a);
+  if (e != cudaSuccess) return e;
+  const int64_t nw_a = (int64_t)jobs_per_chunk * nchunk;
+  rope_scores_kernel<GH, MK, DQ><<<(unsigned)((nw_a + RS_WARPS - 1) / RS_WARPS), 32 * RS_WARPS, smem_a, s>>>(
+      kc, vc.n_quant, vc.n_window, q, dtype, qsb, qsh, qscale, inv_freq, cbk, rscores, rs_cap, G, nchunk);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // decode over the logits (the K cache is not read: one instantiation for both K modes)
+  const size_t smem = sizeof(DecSmem);
+  e = cudaFuncSetAttribute(decode_kernel<GH, NSN_MODE_2BIT, MV, DQ, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  unsigned int* counters = static_cast<unsigned int*>(ws);
+  float* partials = static_cast<float*>(ws) + counter_words((int64_t)nseq);
+  const int nwarps = nseq * geom.nsplit_q * (G / GH);
+  decode_kernel<GH, NSN_MODE_2BIT, MV, DQ, true><<<(nwarps + DEC_WARPS - 1) / DEC_WARPS, 32 * DEC_WARPS, smem, s>>>(
+      kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, counters, partials, out, n_q_heads, geom, rscores, rs_cap);
+  return cudaGetLastError();
+}
+
+template <int G>
+static cudaError_t launch_rope_g(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                                 int64_t qsb, int64_t qsh, float qscale, const float* inv_freq, const float* cbk,
+                                 const float* cbv, float* out, void* ws, const DecodeGeom& geom, cudaStream_t s) {
+#define NSN_LAUNCH_R(MK_, MV_)                                                                                      \
+  return kc.dq ? launch_rope_t<G, MK_, MV_, true>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, inv_freq, cbk, cbv, \
+                                                  out, ws, geom, s)                                                  \
+               : launch_rope_t<G, MK_, MV_, false>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, inv_freq, cbk, cbv, \
+                                                   out, ws, geom, s)
+  if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_1BIT) NSN_LAUNCH_R(1, 1);
+  if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_2BIT) NSN_LAUNCH_R(1, 2);
+  if (kc.mode == NSN_MODE_2BIT && vc.mode == NSN_MODE_1BIT) NSN_LAUNCH_R(2, 1);
+  NSN_LAUNCH_R(2, 2);
+#undef NSN_LAUNCH_R
+}
+
+cudaError_t launch_decode_rope(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                               int64_t qsb, int64_t qsh, float softmax_scale, const float* inv_freq, const float* cbk,
+                               const float* cbv, float* out, void* ws, const DecodeGeom& geom, cudaStream_t s) {
+  const float qscale = softmax_scale * LOG2E;
+  switch (geom.g) {
+    case 1: return launch_rope_g<1>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, inv_freq, cbk, cbv, out, ws, geom, s);
+    case 2: return launch_rope_g<2>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, inv_freq, cbk, cbv, out, ws, geom, s);
+    case 4: return launch_rope_g<4>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, inv_freq, cbk, cbv, out, ws, geom, s);
+    default: return launch_rope_g<8>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, inv_freq, cbk, cbv, out, ws, geom, s);
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -4,6 +4,7 @@ fallback.  torch is used for device memory and streams only.
 
 Functions keep the C names: nsn_build_codebook_host, nsn_quantize_kv,
 nsn_append_residual, nsn_decode_workspace_bytes, nsn_decode_attention,
+nsn_decode_rope_workspace_bytes, nsn_decode_attention_rope,
 nsn_cache_buffer_sizes.  `Cache` allocates the buffers of one nsn_cache with
 torch and fills the C struct.
 """
@@ -93,6 +94,12 @@ def load():
     lib.nsn_decode_attention.argtypes = [POINTER(nsn_cache), POINTER(nsn_cache), c_void_p, c_int, c_int, c_int64,
                                          c_int64, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                          c_void_p]
+    lib.nsn_decode_rope_workspace_bytes.restype = c_size_t
+    lib.nsn_decode_rope_workspace_bytes.argtypes = [POINTER(nsn_cache), c_int]
+    lib.nsn_decode_attention_rope.restype = c_int
+    lib.nsn_decode_attention_rope.argtypes = [POINTER(nsn_cache), POINTER(nsn_cache), c_void_p, c_int, c_int,
+                                              c_int64, c_int64, c_float, c_void_p, c_void_p, c_void_p, c_void_p,
+                                              c_void_p, c_size_t, c_void_p]
     lib.nsn_decode_attention_static.restype = c_int
     lib.nsn_decode_attention_static.argtypes = [POINTER(nsn_cache), POINTER(nsn_cache), c_void_p, c_int, c_int,
                                                 c_int64, c_int64, c_float, c_void_p, c_void_p, c_void_p, c_void_p]
@@ -294,6 +301,39 @@ def nsn_decode_attention(k_cache: Cache, v_cache: Cache, q, softmax_scale: float
                                      cb_k.data_ptr(), cb_v.data_ptr(), out.data_ptr(), workspace.data_ptr(),
                                      workspace.numel(), _stream_ptr(stream))
     _check(st, "nsn_decode_attention")
+
+
+def nsn_decode_rope_workspace_bytes(k_cache: Cache, n_q_heads: int) -> int:
+    return int(load().nsn_decode_rope_workspace_bytes(ctypes.byref(k_cache.c), n_q_heads))
+
+
+def decode_rope_workspace(k_cache: Cache, n_q_heads: int, device="cuda"):
+    import torch
+    n = nsn_decode_rope_workspace_bytes(k_cache, n_q_heads)
+    if n == 0:
+        raise ValueError("invalid cache or head count for decode")
+    return torch.zeros((n,), dtype=torch.uint8, device=device)
+
+
+def nsn_decode_attention_rope(k_cache: Cache, v_cache: Cache, q, softmax_scale: float, inv_freq, cb_k, cb_v, out,
+                              workspace, stream=None) -> None:
+    """Decode attention over pre-RoPE keys: every cached key is rotated at its
+    position (quantized token t at t, window slot w at n_quant + w) with the
+    rotate-half pairing (i, i + 64) and angle pos * inv_freq[i]; q [B, H_q, 128]
+    is the already-rotated query; inv_freq a device float32 tensor of 64."""
+    if q.dim() != 3 or q.shape[-1] != HEAD_DIM or q.stride(-1) != 1:
+        raise ValueError("q must be [B, H_q, 128] with a contiguous last dimension")
+    import torch
+    if out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must be a contiguous float32 tensor shaped like q")
+    if inv_freq.dtype != torch.float32 or inv_freq.numel() != HEAD_DIM // 2 or not inv_freq.is_contiguous():
+        raise ValueError("inv_freq must be a contiguous float32 tensor of 64")
+    st = load().nsn_decode_attention_rope(ctypes.byref(k_cache.c), ctypes.byref(v_cache.c), q.data_ptr(),
+                                          _dtype_code(q), q.shape[1], q.stride(0), q.stride(1),
+                                          float(softmax_scale), inv_freq.data_ptr(), cb_k.data_ptr(),
+                                          cb_v.data_ptr(), out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                          _stream_ptr(stream))
+    _check(st, "nsn_decode_attention_rope")
 
 
 def nsn_decode_attention_static(k_cache: Cache, v_cache: Cache, q, softmax_scale: float, cb_k, cb_v, out,

@@ -272,6 +272,35 @@ nsn_status nsn_decode_attention(const nsn_cache* k_cache, const nsn_cache* v_cac
                                 void* stream);
 
 /*
+ * Pre-RoPE keys ([TS] Metodologia 4: NSN is applied to the keys BEFORE the rotary
+ * position embedding).  The K cache then holds pre-RoPE keys -- both the quantized
+ * part and the fp16 window, filled by the same nsn_quantize_kv* / append calls --
+ * and the decode rotates every key at its position before the score:
+ *   score(q_h, key t) = softmax_scale * q_h . R_pos(t) k_hat_t,
+ *   pos(t) = t for quantized token t, n_quant + w for window slot w,
+ *   R_pos rotates each pair of dims (i, i + 64), i < 64 ("rotate-half" pairing), by
+ *   the angle pos * inv_freq[i]:  (x_i, x_{i+64}) -> (x_i c - x_{i+64} s, x_{i+64} c + x_i s).
+ * q is the already-rotated query (the caller applies RoPE to it at its own position).
+ * Values are not rotated.  Arguments as nsn_decode_attention, plus
+ *   inv_freq       device float[64], 16-byte aligned: theta_i (e.g. base^(-2i/128);
+ *                  any table, so scaled-RoPE variants work).  Angles are formed as
+ *                  pos * theta_i in fp64 and reduced to [-pi, pi] before sin/cos.
+ *   workspace      >= nsn_decode_rope_workspace_bytes() bytes, same zero-fill rule as
+ *                  nsn_decode_attention (its leading part is that workspace; the K
+ *                  logits follow: batch * n_q_heads * (capacity + window) fp32).
+ * Two kernel launches: the K logits of every key (the rotated key is formed in
+ * registers from the compressed cache: H u_hat on the tensor cores, the NSN terms and
+ * the rotation in fp32), then the decode over those logits and the V cache.
+ * Errors as nsn_decode_attention (NSN_ERR_WORKSPACE if ws_bytes is too small).
+ */
+size_t nsn_decode_rope_workspace_bytes(const nsn_cache* k_cache, int n_q_heads);
+nsn_status nsn_decode_attention_rope(const nsn_cache* k_cache, const nsn_cache* v_cache,
+                                     const void* q, int dtype, int n_q_heads, int64_t q_stride_b,
+                                     int64_t q_stride_h, float softmax_scale, const float* inv_freq,
+                                     const float* cb_k, const float* cb_v, float* out,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Allocation-free variant of nsn_decode_attention.  The pages have no counterpart:
  * this entry point exists for callers that cannot allocate device memory when they
  * decode -- code running inside an allocator or memory-pool callback, frameworks

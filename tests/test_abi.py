@@ -97,6 +97,19 @@ def test_host_validation_without_gpu(lib):
                                     16, None) == 3
     need = lib.nsn_decode_workspace_bytes(ctypes.byref(c2), 8)
     assert need > 0
+    # pre-RoPE decode: frequency table required, the same head rules, the larger workspace
+    need_r = lib.nsn_decode_rope_workspace_bytes(ctypes.byref(c2), 8)
+    assert need_r >= need + 1 * 8 * (128 + 128) * 4
+    assert lib.nsn_decode_attention_rope(ctypes.byref(c2), ctypes.byref(c2), 16, 1, 8, 0, 128, 0.1, None, 16, 16,
+                                         16, 16, need_r, None) == 1
+    assert lib.nsn_decode_attention_rope(ctypes.byref(c2), ctypes.byref(c2), 16, 1, 8, 0, 128, 0.1, 8, 16, 16,
+                                         16, 16, need_r, None) == 1   # inv_freq not 16-byte aligned
+    assert lib.nsn_decode_attention_rope(ctypes.byref(c2), ctypes.byref(c2), 16, 1, 3, 0, 128, 0.1, 16, 16, 16,
+                                         16, 16, need_r, None) == 1
+    assert lib.nsn_decode_attention_rope(ctypes.byref(c2), ctypes.byref(c2), 16, 1, 32, 0, 128, 0.1, 16, 16, 16,
+                                         16, 16, need_r, None) == 2
+    assert lib.nsn_decode_attention_rope(ctypes.byref(c2), ctypes.byref(c2), 16, 1, 8, 0, 128, 0.1, 16, 16, 16,
+                                         16, 16, need, None) == 3
     # append: window 0 caches cannot append; shapes must agree
     c0 = nsn.nsn_cache(1, 2, 128, 0, 2, 1, 16, 16, 16, 16, None, 16, 16, None)
     assert lib.nsn_append_residual(ctypes.byref(c0), ctypes.byref(c0), 16, 16, 1, 0, 128, 16, 16, None) == 2
