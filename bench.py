@@ -166,10 +166,16 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (test infrastructure; the only other place bench runs oracle/)
 # ---------------------------------------------------------------------------
-def oracle_decode_sample(budget_s: float, seed: int = 0):
-    """Times the oracle's decode attention for sampled (b, kv-head) sequences of
-    the workload shape (random compressed contents, 2-bit K/V, full window).
-    Returns (seconds per (b, kv-head), sequences timed, threads)."""
+def rope_theta() -> np.ndarray:
+    """RoPE frequencies of the Llama-3-8B shape: theta_i = 500000^(-2i/128), fp32."""
+    return (500000.0 ** (-2.0 * np.arange(64) / 128.0)).astype(np.float32)
+
+
+def oracle_decode_sample(budget_s: float, seed: int = 0, rope: bool = False):
+    """Times the oracle's decode attention (pre-RoPE keys with `rope`) for sampled
+    (b, kv-head) sequences of the workload shape (random compressed contents,
+    2-bit K/V, full window).  Returns (seconds per (b, kv-head), sequences timed,
+    threads)."""
     from calibration_free_vector_b200 import synthetic
     from oracle import nsn_oracle as orc
     try:
@@ -192,8 +198,13 @@ def oracle_decode_sample(budget_s: float, seed: int = 0):
                        "o": c["o"].astype(np.float64)}
         q = rs.normal(size=(g, 128))
         t0 = time.perf_counter()
-        orc.decode_attention(q, f(kc), f(vc), kc["window"].astype(np.float64), vc["window"].astype(np.float64),
-                             cbk, cbk, W["mode_k"], W["mode_v"], 1 / math.sqrt(128))
+        if rope:
+            orc.decode_attention_rope(q, f(kc), f(vc), kc["window"].astype(np.float64),
+                                      vc["window"].astype(np.float64), cbk, cbk, W["mode_k"], W["mode_v"],
+                                      1 / math.sqrt(128), rope_theta().astype(np.float64))
+        else:
+            orc.decode_attention(q, f(kc), f(vc), kc["window"].astype(np.float64), vc["window"].astype(np.float64),
+                                 cbk, cbk, W["mode_k"], W["mode_v"], 1 / math.sqrt(128))
         times.append(time.perf_counter() - t0)
         n += 1
         if time.perf_counter() - t_start > budget_s or n >= 64:
@@ -320,12 +331,19 @@ def run_ours(args):
                       for s in range(total_steps)])
     del xk, xv
     out = torch.empty((B, HQ, 128), dtype=torch.float32, device=dev)
-    ws = nsn.decode_workspace(kc, HQ, dev)
+    ws = nsn.decode_rope_workspace(kc, HQ, dev) if args.rope else nsn.decode_workspace(kc, HQ, dev)
     scale = 1.0 / math.sqrt(128)
+    theta = torch.from_numpy(rope_theta()).to(dev)
+
+    def decode_call(q_, out_):
+        if args.rope:  # pre-RoPE keys: every key rotated at its position (two launches)
+            nsn.nsn_decode_attention_rope(kc, vc, q_, scale, theta, cbk, cbv, out_, ws)
+        else:
+            nsn.nsn_decode_attention(kc, vc, q_, scale, cbk, cbv, out_, ws)
 
     def step(s):
         nsn.nsn_append_residual(kc, vc, new_k[s], new_v[s], cbk, cbv)
-        nsn.nsn_decode_attention(kc, vc, qs[s], scale, cbk, cbv, out, ws)
+        decode_call(qs[s], out)
 
     for s in range(WU):
         step(s)
@@ -356,7 +374,7 @@ def run_ours(args):
         s = WU + i
         nsn.nsn_append_residual(kc, vc, new_k[s], new_v[s], cbk, cbv)
         ev[i][0].record(stream)
-        nsn.nsn_decode_attention(kc, vc, qs[s], scale, cbk, cbv, out, ws)
+        decode_call(qs[s], out)
         ev[i][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
@@ -366,7 +384,7 @@ def run_ours(args):
     soak_end = time.perf_counter() + (0.0 if args.lite else 1.0)
     while time.perf_counter() < soak_end:
         for _ in range(20):
-            nsn.nsn_decode_attention(kc, vc, qs[WU + K - 1], scale, cbk, cbv, out, ws)
+            decode_call(qs[WU + K - 1], out)
         torch.cuda.synchronize()
     clocks = sampler.stop()
     clocks["window"] = "timed region + 1 s of the same decode call right after it"
@@ -434,7 +452,7 @@ def run_ours(args):
                 stream.wait_event(ev_out[j])
             dk, dv, dq = d_in[j]
             nsn.nsn_append_residual(kc, vc, dk, dv, cbk, cbv)
-            nsn.nsn_decode_attention(kc, vc, dq, scale, cbk, cbv, d_out[j], ws)
+            decode_call(dq, d_out[j])
             ev_done[j].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(ev_done[j])
@@ -463,7 +481,8 @@ def run_ours(args):
                           "decode_call_ms": dec_avg_ms, "decode_gbs": achieved, "quantize_ms": quant_ms_best,
                           "cache_status": int(kc.status.item()) | int(vc.status.item())}), flush=True)
     elif rank == 0:
-        cpu_t, cpu_n, cpu_threads = oracle_decode_sample(float(os.environ.get("NSN_CPU_BUDGET_S", "15")))
+        cpu_t, cpu_n, cpu_threads = oracle_decode_sample(float(os.environ.get("NSN_CPU_BUDGET_S", "15")),
+                                                         rope=args.rope)
         cpu_step = cpu_t * B * H
         cq_t, cq_n = oracle_quantize_sample(8.0)
         line = {
@@ -472,16 +491,21 @@ def run_ours(args):
             "unit": "tokens/s",
             "n_gpus": world, "steps": K, "warmup": WU, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": W["name"] + ("-dq" if args.double_quant else ""), "batch": B, "seq_len": T,
-                       "n_q_heads": HQ, "n_kv_heads": H, "double_quant": bool(args.double_quant),
+            "config": {"workload": W["name"] + ("-dq" if args.double_quant else "") + ("-prerope" if args.rope else ""),
+                       "batch": B, "seq_len": T, "n_q_heads": HQ, "n_kv_heads": H,
+                       "double_quant": bool(args.double_quant),
+                       "pre_rope_keys": bool(args.rope), **({"rope_theta_base": 500000.0} if args.rope else {}),
                        "head_dim": 128, "mode_k": W["mode_k"], "mode_v": W["mode_v"], "window": W["window"],
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": f"inputs larger than L2 (compressed cache {compressed / 1e6:.0f} MB per step)"},
             "compressed_kv_gbs": decode_bytes / (ms_per_step * 1e-3) / 1e9,
             "decode_call_ms": dec_avg_ms,
-            "roofline": {"kernel": "decode_kernel (one launch per decode call)", "bound": "hbm",
+            "roofline": {"kernel": ("rope_scores_kernel + decode_kernel (two launches per decode call; "
+                                    "the logits kernel is issue-bound)") if args.rope
+                         else "decode_kernel (one launch per decode call)", "bound": "hbm",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                         "peak_kind": peak_kind, "traffic": None if args.double_quant else decode_traffic(),
+                         "peak_kind": peak_kind,
+                         "traffic": None if (args.double_quant or args.rope) else decode_traffic(),
                          "algorithmic_bytes_per_launch": decode_bytes,
                          "frac_of_8tbs_spec": achieved / 8000.0},
             "quantize": {"workload": f"prefill {B}x{q_tokens} tokens x {H} kv-heads, K 2-bit + V 2-bit, bf16 in",
@@ -496,7 +520,7 @@ def run_ours(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "copies": "every step: its new K/V token and q from pinned host memory, its output back; "
                               "uploads of step s+1 and the download of step s-1 overlap step s"},
-            "gpu_launches": K * LAUNCHES_PER_STEP,
+            "gpu_launches": K * (LAUNCHES_PER_STEP + (1 if args.rope else 0)),
             "clocks": clocks,
             "cache_status": status,
             "cpu_baseline": {"value": B / cpu_step, "unit": "tokens/s", "cores": cpu_threads, "kind": "oracle",
@@ -522,6 +546,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling runs)")
     ap.add_argument("--double-quant", action="store_true",
                     help="the same workload with double quantization (4-bit s1 and o)")
+    ap.add_argument("--rope", action="store_true",
+                    help="the same workload with pre-RoPE keys (every key rotated at its position at decode)")
     ap.add_argument("--lite", action="store_true",
                     help="profiling run: no e2e leg, no clock soak, no CPU baseline; short summary line")
     args = ap.parse_args()

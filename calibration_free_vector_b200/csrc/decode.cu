@@ -966,6 +966,47 @@ __device__ __forceinline__ float2 rope_cs(double a) {
   return make_float2(cs, sn);
 }
 
+__device__ __forceinline__ void mma_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, {%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+__device__ __forceinline__ void mma_zero(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %10, %10, %10};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// Compressed inputs of one 16-token K tile, loaded one tile ahead.
+struct RsTileIn {
+  uint4 codes;      // code bytes of this lane's ldmatrix token
+  uint32_t ks0, ks1;  // sign words (2-bit) of tokens g, g + 8
+  uint32_t n[2];    // tokens g, g + 8: (s1, s2) fp16 pair, or (alpha*s2 fp16 | s1 level << 16) with DQ
+};
+
+template <int MK, bool DQ>
+__device__ __forceinline__ void rs_load_tile(RsTileIn& in, const CacheView& kc, int64_t tq, int tok_a, int g, int p) {
+  in.codes = __ldg(reinterpret_cast<const uint4*>(kc.codes + (tq + tok_a) * NSUB));
+  in.ks0 = in.ks1 = 0u;
+  if constexpr (MK == NSN_MODE_2BIT) {
+    in.ks0 = __ldg(reinterpret_cast<const uint32_t*>(kc.signs + (tq + g) * NSUB) + p);
+    in.ks1 = __ldg(reinterpret_cast<const uint32_t*>(kc.signs + (tq + 8 + g) * NSUB) + p);
+  }
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int64_t tk = tq + g + 8 * rr;
+    if constexpr (DQ) {
+      const uint32_t s2b = __ldg(reinterpret_cast<const unsigned short*>(kc.norms) + tk);
+      const uint32_t lv = ((uint32_t)__ldg(kc.s1_levels + tk / 2) >> (4 * (uint32_t)(tk & 1))) & 15u;
+      in.n[rr] = s2b | (lv << 16);
+    } else {
+      in.n[rr] = __ldg(reinterpret_cast<const uint32_t*>(kc.norms) + tk);
+    }
+  }
+}
+
 template <int GH, int MK, bool DQ>
 __global__ void __launch_bounds__(32 * RS_WARPS, 2)
 rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int32_t* __restrict__ v_nwindow,
@@ -1017,8 +1058,8 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
   float* hob = reinterpret_cast<float*>(wk);                // H o_b of the current block (128 fp32)
   float2* base = reinterpret_cast<float2*>(wk + D * 4);     // (cos, sin)(pos0 theta_i), 64
 
-  // +-H_16 as the B operand: column n = g + 8 nt, rows 2p, 2p+1 | 2p+8, 2p+9
-  uint32_t Hp[2][2], Hn[2][2];
+  // H_16 as the B operand: column n = g + 8 nt, rows 2p, 2p+1 | 2p+8, 2p+9
+  uint32_t Hb[2][2];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
     const int n = g + 8 * nt;
@@ -1027,8 +1068,7 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
       const int k0 = 2 * p + 8 * r;
       const uint32_t e0 = (__popc(k0 & n) & 1) ? 0xBC00u : 0x3C00u;
       const uint32_t e1 = (__popc((k0 + 1) & n) & 1) ? 0xBC00u : 0x3C00u;
-      Hp[nt][r] = e0 | (e1 << 16);
-      Hn[nt][r] = Hp[nt][r] ^ 0x80008000u;
+      Hb[nt][r] = e0 | (e1 << 16);
     }
   }
   const uint32_t cbk_base = smem_addr(&sm.cbk[0][0]) + (uint32_t)(lane & 7) * 16u;
@@ -1039,7 +1079,10 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
   const int t_l = g + (lo_lane ? 0 : 8);
   const int h0 = 2 * (p & 1);
   const int64_t cap = kc.capacity;
+  const int q_end = min(nq, st_last * STAGE_TOK);  // this job's quantized positions end here
   int cur_blk = -1;
+  RsTileIn nxt;
+  if (st_first < nst_q) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + st_first * STAGE_TOK, tok_a, g, p);
 
   for (int st = st_first; st < st_last; ++st) {
     const bool win = st >= nst_q;
@@ -1074,138 +1117,126 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
         *reinterpret_cast<float4*>(hob + 4 * lane) =
             make_float4(v[0] * INV_SQRT_D, v[1] * INV_SQRT_D, v[2] * INV_SQRT_D, v[3] * INV_SQRT_D);
       }
+    } else if (cur_blk != -2) {  // window keys: no mean term
+      cur_blk = -2;
+      *reinterpret_cast<float4*>(hob + 4 * lane) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncwarp();
 
     for (int m = 0; m < STAGE_TOK / 16; ++m) {
       const int tt = pos0 + 16 * m;  // position of the tile's first token
       if (tt >= pend) break;
-      float s1r[2] = {1.f, 1.f}, s2r[2] = {1.f, 1.f};  // rows g, g + 8
-      uint32_t A[8][4];
+      // E[a'][nt][r]: dim 16 a' + 8 nt + 2p + (r & 1) of token row g + 8 (r >> 1), before the NSN terms
+      float E[8][2][4];
+      float xs[2] = {1.f, 1.f}, s1r[2] = {1.f, 1.f};  // per row: scale of E, and s1
       if (!win) {
-        const int64_t tq = seq * cap + tt;
-        const uint4 kcw = __ldg(reinterpret_cast<const uint4*>(kc.codes + (tq + tok_a) * NSUB));
-        uint32_t ks0 = 0u, ks1 = 0u;
-        if constexpr (MK == NSN_MODE_2BIT) {
-          ks0 = __ldg(reinterpret_cast<const uint32_t*>(kc.signs + (tq + g) * NSUB) + p);
-          ks1 = __ldg(reinterpret_cast<const uint32_t*>(kc.signs + (tq + 8 + g) * NSUB) + p);
-        }
+        const RsTileIn cur = nxt;
+        if (tt + 16 < q_end) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + tt + 16, tok_a, g, p);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-          const int64_t tk = tq + g + 8 * rr;
           if constexpr (DQ) {
-            s2r[rr] = __half2float(reinterpret_cast<const __half*>(kc.norms)[tk]);
-            const uint32_t lv = (uint32_t)__ldg(kc.s1_levels + tk / 2) >> (4 * (uint32_t)(tk & 1));
-            s1r[rr] = fmaf(nibble_f(lv), s1ls.y, s1ls.x);
+            xs[rr] = __half2float(__ushort_as_half((unsigned short)(cur.n[rr] & 0xFFFFu))) * INV_SQRT_D;
+            s1r[rr] = fmaf(nibble_f(cur.n[rr] >> 16), s1ls.y, s1ls.x);
           } else {
-            const float2 n2 = __half22float2(kc.norms[tk]);
+            const float2 n2 = __half22float2(*reinterpret_cast<const __half2*>(&cur.n[rr]));
             s1r[rr] = n2.x;
-            s2r[rr] = n2.y;
+            xs[rr] = n2.y * INV_SQRT_D;
           }
         }
+        // u_hat k-step a times H_16 (independent products), then H_8 across the k-steps in fp32
 #pragma unroll
         for (int a = 0; a < 8; ++a) {
-          const uint32_t code = __byte_perm(u4_word(kcw, a >> 1), 0u, (a & 1) ? sel_k1 : sel_k0);
-          ldsm_x4(cbk_base + code * 128u, A[a]);
+          const uint32_t code = __byte_perm(u4_word(cur.codes, a >> 1), 0u, (a & 1) ? sel_k1 : sel_k0);
+          uint32_t A[4];
+          ldsm_x4(cbk_base + code * 128u, A);
           if constexpr (MK == NSN_MODE_2BIT) {
-            A[a][0] = apply_signs(A[a][0], ks0, 2 * a);
-            A[a][1] = apply_signs(A[a][1], ks1, 2 * a);
-            A[a][2] = apply_signs(A[a][2], ks0, 2 * a + 1);
-            A[a][3] = apply_signs(A[a][3], ks1, 2 * a + 1);
+            A[0] = apply_signs(A[0], cur.ks0, 2 * a);
+            A[1] = apply_signs(A[1], cur.ks1, 2 * a);
+            A[2] = apply_signs(A[2], cur.ks0, 2 * a + 1);
+            A[3] = apply_signs(A[3], cur.ks1, 2 * a + 1);
           }
+          mma_zero(E[a][0], A, Hb[0][0], Hb[0][1]);
+          mma_zero(E[a][1], A, Hb[1][0], Hb[1][1]);
         }
-      }
-      const int r_off = 16 * m + g;  // offset-table rows of this lane's tokens: r_off, r_off + 8
-      float S[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int ap = 0; ap < 4; ++ap) {
-        // y[h][nt][r]: dim 16 (ap + 4h) + 8 nt + 2p + (r & 1) of token row g + 8 (r >> 1)
-        float y[2][2][4];
-        if (!win) {
+        for (int sstep = 1; sstep < 8; sstep <<= 1)
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-              for (int r = 0; r < 4; ++r) y[h][nt][r] = 0.f;
-#pragma unroll
-          for (int a = 0; a < 8; ++a) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const bool neg = (__popc((ap + 4 * h) & a) & 1) != 0;  // H_8[ap + 4h][a]
+          for (int a = 0; a < 8; ++a)
+            if (!(a & sstep))
 #pragma unroll
               for (int nt = 0; nt < 2; ++nt)
-                mma_full(y[h][nt], A[a], neg ? Hn[nt][0] : Hp[nt][0], neg ? Hn[nt][1] : Hp[nt][1]);
-            }
-          }
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
+                for (int r = 0; r < 4; ++r) {
+                  const float u = E[a][nt][r], w = E[a + sstep][nt][r];
+                  E[a][nt][r] = u + w;
+                  E[a + sstep][nt][r] = u - w;
+                }
+      } else {
+        const __half* wrow = kc.window + seq * (int64_t)kc.window_len * D;
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int w = min(tt - nq + g + 8 * rr, nw - 1);
+#pragma unroll
+          for (int a = 0; a < 8; ++a)
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-              const float2 o2 = *reinterpret_cast<const float2*>(hob + 16 * (ap + 4 * h) + 8 * nt + 2 * p);
-#pragma unroll
-              for (int r = 0; r < 4; ++r)
-                y[h][nt][r] = fmaf(s2r[r >> 1] * INV_SQRT_D, y[h][nt][r], (r & 1) ? o2.y : o2.x);
+              const float2 kv = __half22float2(
+                  *reinterpret_cast<const __half2*>(wrow + (int64_t)w * D + 16 * a + 8 * nt + 2 * p));
+              E[a][nt][2 * rr] = kv.x;
+              E[a][nt][2 * rr + 1] = kv.y;
             }
-        } else {
-          const __half* wrow = kc.window + seq * (int64_t)kc.window_len * D;
-#pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const int w = min(tt - nq + g + 8 * rr, nw - 1);
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-              for (int nt = 0; nt < 2; ++nt) {
-                const float2 kv = __half22float2(
-                    *reinterpret_cast<const __half2*>(wrow + (int64_t)w * D + 16 * (ap + 4 * h) + 8 * nt + 2 * p));
-                y[h][nt][2 * rr] = kv.x;
-                y[h][nt][2 * rr + 1] = kv.y;
-              }
-          }
         }
-        // rotate dims (i, i + 64), i = 16 ap + 8 nt + 2p + e, at this lane's two token positions
+      }
+      // NSN terms, rotation of dims (i, i + 64), fp16 hi + lo, and the query product
+      const int r_off = 16 * m + g;  // offset-table rows of this lane's tokens: r_off, r_off + 8
+      float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ap = 0; ap < 4; ++ap)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const int i0 = 16 * ap + 8 * nt + 2 * p;
+          const float2 olo = *reinterpret_cast<const float2*>(hob + i0);
+          const float2 ohi = *reinterpret_cast<const float2*>(hob + i0 + 64);
           const float4 bb = *reinterpret_cast<const float4*>(base + i0);
+          float y0[4], y1[4];
 #pragma unroll
           for (int rr = 0; rr < 2; ++rr) {
             const float4 oo = *reinterpret_cast<const float4*>(&sm.off[r_off + 8 * rr][i0]);
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
+              const int r = 2 * rr + e;
+              const float lo = fmaf(xs[rr], E[ap][nt][r], e ? olo.y : olo.x);
+              const float hi = fmaf(xs[rr], E[ap + 4][nt][r], e ? ohi.y : ohi.x);
               const float bc = e ? bb.z : bb.x, bs = e ? bb.w : bb.y;
               const float oc = e ? oo.z : oo.x, os = e ? oo.w : oo.y;
               const float c = fmaf(bc, oc, -bs * os), sn = fmaf(bs, oc, bc * os);
-              const float lo = y[0][nt][2 * rr + e], hi = y[1][nt][2 * rr + e];
-              y[0][nt][2 * rr + e] = fmaf(lo, c, -hi * sn);
-              y[1][nt][2 * rr + e] = fmaf(hi, c, lo * sn);
+              y0[r] = fmaf(lo, c, -hi * sn);
+              y1[r] = fmaf(hi, c, lo * sn);
             }
           }
-        }
-        // fp16 hi + lo of the rotated key (k-steps ap and ap + 4) times the query
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t ahi[4], alo[4];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
+          for (int h = 0; h < 2; ++h) {
+            const float* y = h ? y1 : y0;
+            uint32_t ahi[2], alo[2];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
-              const float x0 = y[h][nt][2 * rr], x1 = y[h][nt][2 * rr + 1];
-              const __half2 hh = __floats2half2_rn(x0, x1);
+              const __half2 hh = __floats2half2_rn(y[2 * rr], y[2 * rr + 1]);
               const float2 hf = __half22float2(hh);
-              ahi[2 * nt + rr] = *reinterpret_cast<const uint32_t*>(&hh);
-              alo[2 * nt + rr] = pack_half2(x0 - hf.x, x1 - hf.y);
+              ahi[rr] = *reinterpret_cast<const uint32_t*>(&hh);
+              alo[rr] = pack_half2(y[2 * rr] - hf.x, y[2 * rr + 1] - hf.y);
             }
-          mma_full(S, ahi, qb[ap + 4 * h][0], qb[ap + 4 * h][1]);
-          mma_full(S, alo, qb[ap + 4 * h][0], qb[ap + 4 * h][1]);
+            mma_k8(S[h], ahi[0], ahi[1], qb[ap + 4 * h][nt]);
+            mma_k8(S[h], alo[0], alo[1], qb[ap + 4 * h][nt]);
+          }
         }
-      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) S[0][i] += S[1][i];
       // hi + lo query columns -> (token t_l, heads h0, h0 + 1)
-      const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[2] : S[0], 2);
-      const float r1 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[3] : S[1], 2);
+      const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[0][2] : S[0][0], 2);
+      const float r1 = __shfl_xor_sync(0xffffffffu, lo_lane ? S[0][3] : S[0][1], 2);
       const float s1 = lo_lane ? s1r[0] : s1r[1];
-      const float sc0 = s1 * ((lo_lane ? S[0] : S[2]) + r0);
-      const float sc1 = s1 * ((lo_lane ? S[1] : S[3]) + r1);
+      const float sc0 = s1 * ((lo_lane ? S[0][0] : S[0][2]) + r0);
+      const float sc1 = s1 * ((lo_lane ? S[0][1] : S[0][3]) + r1);
       const int pos = tt + t_l;
       if (pos < pend) {
         float* dst = rdst + (int64_t)pos * GH;
