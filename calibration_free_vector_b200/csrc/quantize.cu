@@ -19,13 +19,16 @@
 // offsets (outliers) out of the fp32 rounding, so u carries fp32 precision
 // relative to the token-varying part that survives the shift step.
 //
-// Nearest codeword: exhaustive fp32 search over the 256 codewords held in shared
-// memory (broadcast reads), score_k = u.c_k - ||c_k||^2/2, tracking the best and
-// second-best score (per group of 8 codewords, then inside the winning group).
-// Whenever the second best lies within the rigorous fp32 error bound of the best,
-// the sub-vector is re-decided exactly in fp64 over all codewords inside that
-// bound (ties to the lowest index).  The stored code is therefore the exact
-// nearest codeword of the fp32 u.
+// Nearest codeword: exhaustive scores score_k = u.c_k - ||c_k||^2/2 of all 256
+// codewords on the tensor cores (a token's 16 sub-vectors are the rows of one
+// m16n8k16 tile, K = the fp16 hi and lo parts of u against the fp16 codebook
+// twice, the bias as the accumulator's start), the best group of 8 codewords per
+// sub-vector, then the 8 codewords of that group rescanned in sequential fp32.
+// Whenever a rival lies within the error bounds of the best (the fp32 bound inside
+// the group, that plus a wide tensor-accumulation bound outside it), the
+// sub-vector is re-decided exactly in fp64 by a whole warp over all codewords
+// inside the bound (ties to the lowest index).  The stored code is therefore the
+// exact nearest codeword of the fp32 u.
 
 #include "nsn_common.cuh"
 #include "nsn_launch.h"
@@ -40,6 +43,28 @@ __device__ __forceinline__ double lds_f64(const double* p) {
   return r;
 }
 
+// ldmatrix / mma.sync / three-input max for the tensor-core codeword scores.
+__device__ __forceinline__ uint32_t q_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void q_ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+// d += A (16 x 16) * B (16 x 8) with both K halves of B equal to `b`
+__device__ __forceinline__ void q_mma_bb(float (&d)[4], const uint32_t (&a)[4], uint32_t b) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %8}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b));
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
+
 constexpr int QTHREADS = 2 * BLK;  // two threads per token
 constexpr int HD = D / 2;           // dims per thread
 constexpr int HSUB = NSUB / 2;      // sub-vectors per thread
@@ -47,7 +72,8 @@ constexpr int HSUB = NSUB / 2;      // sub-vectors per thread
 struct QuantSmem {
   alignas(16) float cb[NCODES][SUB];   // codebook (fp32)
   alignas(16) float bias[NCODES];      // -||c_k||^2 / 2
-  alignas(16) float cnorm[4];          // [0] = max ||c||, [1] = max ||c||^2 (rounded up)
+  alignas(16) float cnorm[4];          // [0] = max ||c||, [1] = max ||c||^2, [2] = max ||c - fp16(c)|| (rounded up)
+  alignas(16) __half cbh[NCODES][SUB]; // codebook rounded to fp16 (tensor-core operand)
   alignas(16) double rr[BLK];          // 1 / ||x_t|| (0 for a zero token)
   alignas(16) double s1[BLK];          // per-token s1 and s2 (fp64) until the final store
   alignas(16) double s2[BLK];
@@ -59,6 +85,9 @@ struct QuantSmem {
   alignas(16) float tile[BLK][D + 4];  // raw tokens, then d_t rows, then u rows; padded by 16 B
   alignas(16) float thr[BLK][NSUB + 1];  // per (token, sub-vector) threshold of the exact re-decision
   alignas(16) uint8_t code[BLK][NSUB]; // chosen codes
+  alignas(16) uint8_t grp[BLK][NSUB];  // winning (group of 8 codes, lane) of the tensor-core scores
+  alignas(16) uint16_t flag[BLK * NSUB];  // (token, sub-vector) pairs for the exact re-decision
+  int nflag;
   alignas(16) uint32_t sgn[BLK][4];    // packed sign bits (2-bit mode)
   // double quantization
   alignas(16) double ofull[D];         // o of the block (fp64) until its levels are formed
@@ -99,24 +128,39 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
   for (int i = t; i < NCODES * SUB / 4; i += blockDim.x)
     reinterpret_cast<float4*>(&sm.cb[0][0])[i] = __ldg(reinterpret_cast<const float4*>(codebook) + i);
   __syncthreads();
-  float my_max = 0.f;
+  float my_max = 0.f, my_dev = 0.f;
   for (int k = t; k < NCODES; k += blockDim.x) {
-    float s = 0.f;
+    float s = 0.f, e = 0.f;
 #pragma unroll
-    for (int i = 0; i < SUB; ++i) s = fmaf(sm.cb[k][i], sm.cb[k][i], s);
+    for (int i = 0; i < SUB; ++i) {
+      s = fmaf(sm.cb[k][i], sm.cb[k][i], s);
+      const __half c16 = __float2half_rn(sm.cb[k][i]);
+      sm.cbh[k][i] = c16;
+      const float d = sm.cb[k][i] - __half2float(c16);
+      e = fmaf(d, d, e);
+    }
     sm.bias[k] = -0.5f * s;
     my_max = fmaxf(my_max, s);
+    my_dev = fmaxf(my_dev, e);
   }
   my_max = warp_max(my_max);
-  __shared__ float red[QTHREADS / 32];
-  if ((t & 31) == 0) red[t >> 5] = my_max;
+  my_dev = warp_max(my_dev);
+  __shared__ float red[QTHREADS / 32][2];
+  if ((t & 31) == 0) {
+    red[t >> 5][0] = my_max;
+    red[t >> 5][1] = my_dev;
+  }
   __syncthreads();
   if (t == 0) {
-    float m = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    float m = 0.f, e = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+      m = fmaxf(m, red[w][0]);
+      e = fmaxf(e, red[w][1]);
+    }
     m *= 1.0001f;  // upper bound on max ||c||^2 despite the fp32 rounding above
     sm.cnorm[1] = m;
     sm.cnorm[0] = sqrtf(m) * 1.0001f;
+    sm.cnorm[2] = e > 0.f ? sqrtf(e) * 1.001f : 0.f;  // 0 for a codebook of fp16 values
   }
   __syncthreads();
 }
@@ -194,6 +238,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   const int t = threadIdx.x, tk = t >> 1, h = t & 1;
   const int col = t & (D - 1), rhalf = t >> 7;  // column-sum roles: column, half of the rows
   const bool valid = tk < n;
+  if (t == 0) sm.nflag = 0;  // read only after the barriers below
   constexpr int ESZ = (DT == NSN_DTYPE_F32) ? 4 : 2;
   constexpr int CHUNKS = D * ESZ / 16;  // 16-byte chunks per row
 
@@ -400,136 +445,207 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     if (h == 0) *reinterpret_cast<uint4*>(&sm.sgn[tk][0]) = make_uint4(sgn[0], sgn[1], sgn[2], sgn[3]);
   }
 
-  // ---- exhaustive fp32 search ------------------------------------------------
-  // score_k = u.c_k - ||c_k||^2 / 2 (maximised), one pass over the codebook for
-  // the thread's 8 sub-vectors.  Codewords are scanned in groups of CGROUP: a running
-  // max per group (one FMNMX per codeword), then the best and second-best group
-  // maxima with the best group's index.  The winning group is rescanned to find
-  // the code (lowest index on ties) and its runner-up inside the group; the
-  // overall runner-up is the larger of that and the second-best group max.
-  const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1];
+  // ---- nearest codeword: tensor-core scores, exact decision ------------------
+  // score_k = a.c_k - ||c_k||^2 / 2 (maximised) for every sub-vector a.
+  // (1) The 16 sub-vectors of a token are the 16 rows of one m16n8k16 tile with
+  //     K = [a_hi | a_lo] (the fp32 a split into two fp16 parts, exact to 2^-22)
+  //     against B = [c | c] (the codebook in fp16) and the bias as the
+  //     accumulator's start: 32 MMAs give the 256 scores of 16 sub-vectors.
+  // (2) Lane p of a quad sees codes 8n + 2p, 8n + 2p + 1 of every n-tile n: a
+  //     running max per group of 4 n-tiles (8 codes), then the best and
+  //     second-best group maxima and the best group, merged over the quad.
+  // (3) The owner lane rescans the 8 codes of the winning group in sequential
+  //     fp32 (the arithmetic of the exact path below) for the code (lowest index
+  //     on ties) and the in-group runner-up.
+  // (4) When the runner-up -- another group's tensor score or an fp32 score
+  //     inside the group -- comes within the error bounds of the best, a whole
+  //     warp re-decides the sub-vector exactly in fp64.
+  // Error bounds: the sequential fp32 score is within gamma_9 (max||c||^2 +
+  // ||a|| max||c||) of the exact one.  The tensor score's error is bounded by
+  // TC_REL (sum |a_i c_i| + |bias|) for the accumulation inside the MMA (its
+  // order and rounding are the hardware's, so the bound is taken wide: 2^-16
+  // against 17 terms of at most 2^-24 relative each), plus ||a|| ||c - fp16(c)||
+  // for a codebook that is not fp16-representable.
+  const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1], cdel = sm.cnorm[2];
   constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
-  uint32_t need = 0u;
-  // Small groups keep the unrolled body short, so the loads of the next group
-  // can be hoisted over this one's FMAs; 2 measured fastest of 1, 2, 4, 8 and 16.
-  constexpr int CGROUP = 2;
+  constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
+  const int warp = t >> 5, lane = t & 31, qg = lane >> 2, qp = lane & 3;
+  // (1) this warp's 16 tokens x 16 sub-vectors as A rows of 32 bytes (fp16 hi |
+  // lo), in the warp's own 16 tile rows (free since the column sums); the two
+  // 16-byte halves swap on every 4th row so that ldmatrix rows hit distinct banks
+  unsigned char* arow = reinterpret_cast<unsigned char*>(&sm.tile[16 * warp][0]);
   {
-    float b1[HSUB], b2[HSUB];
-    int bg[HSUB];
+    const int r0 = 16 * (lane >> 1) + HSUB * h;
 #pragma unroll
     for (int jj = 0; jj < HSUB; ++jj) {
-      b1[jj] = -INFINITY;
-      b2[jj] = -INFINITY;
-      bg[jj] = 0;
-    }
-#pragma unroll 1
-    for (int grp = 0; grp < NCODES / CGROUP; ++grp) {
-      float gm[HSUB];
+      uint32_t hw[4], lw[4];
 #pragma unroll
-      for (int jj = 0; jj < HSUB; ++jj) gm[jj] = -INFINITY;
-#pragma unroll
-      for (int kk = 0; kk < CGROUP; ++kk) {
-        const int k = CGROUP * grp + kk;
-        const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
-        const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
-        const float bk = sm.bias[k];
-#pragma unroll
-        for (int jj = 0; jj < HSUB; ++jj) {
-          float s = bk;
-          s = fmaf(v[8 * jj + 0], c0.x, s);
-          s = fmaf(v[8 * jj + 1], c0.y, s);
-          s = fmaf(v[8 * jj + 2], c0.z, s);
-          s = fmaf(v[8 * jj + 3], c0.w, s);
-          s = fmaf(v[8 * jj + 4], c1.x, s);
-          s = fmaf(v[8 * jj + 5], c1.y, s);
-          s = fmaf(v[8 * jj + 6], c1.z, s);
-          s = fmaf(v[8 * jj + 7], c1.w, s);
-          gm[jj] = fmaxf(gm[jj], s);
-        }
+      for (int i = 0; i < 4; ++i) {
+        const float x0 = valid ? v[8 * jj + 2 * i] : 0.f, x1 = valid ? v[8 * jj + 2 * i + 1] : 0.f;
+        const __half2 hh = __floats2half2_rn(x0, x1);
+        const float2 hf = __half22float2(hh);
+        hw[i] = h2_bits(hh);
+        lw[i] = h2_bits(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
       }
-#pragma unroll
-      for (int jj = 0; jj < HSUB; ++jj) {
-        const float lo = fminf(b1[jj], gm[jj]);
-        bg[jj] = (gm[jj] > b1[jj]) ? grp : bg[jj];
-        b1[jj] = fmaxf(b1[jj], gm[jj]);
-        b2[jj] = fmaxf(b2[jj], lo);
-      }
-    }
-#pragma unroll
-    for (int jj = 0; jj < HSUB; ++jj) {
-      const int j = HSUB * h + jj;
-      // rescan the winning group with the same arithmetic as above
-      float best = -INFINITY, second = -INFINITY;
-      int idx = CGROUP * bg[jj];
-#pragma unroll
-      for (int kk = 0; kk < CGROUP; ++kk) {
-        const int k = CGROUP * bg[jj] + kk;
-        const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
-        const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
-        float s = sm.bias[k];
-        s = fmaf(v[8 * jj + 0], c0.x, s);
-        s = fmaf(v[8 * jj + 1], c0.y, s);
-        s = fmaf(v[8 * jj + 2], c0.z, s);
-        s = fmaf(v[8 * jj + 3], c0.w, s);
-        s = fmaf(v[8 * jj + 4], c1.x, s);
-        s = fmaf(v[8 * jj + 5], c1.y, s);
-        s = fmaf(v[8 * jj + 6], c1.z, s);
-        s = fmaf(v[8 * jj + 7], c1.w, s);
-        const float lo = fminf(best, s);
-        idx = (s > best) ? k : idx;
-        best = fmaxf(best, s);
-        second = fmaxf(second, lo);
-      }
-      const float runner = fmaxf(b2[jj], second);
-      float na = 0.f;
-#pragma unroll
-      for (int i = 0; i < SUB; ++i) na = fmaf(v[8 * jj + i], v[8 * jj + i], na);
-      na = sqrtf(na) * 1.0001f;
-      // |fp32 score - exact score| <= gamma_9 (max||c||^2 + ||a|| max||c||) for every
-      // codeword, so a rival within twice that bound of the best may be the true best.
-      const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
-      sm.thr[tk][j] = best - margin;
-      need |= (runner >= best - margin ? 1u : 0u) << jj;
-      sm.code[tk][j] = (uint8_t)idx;
+      const int r = r0 + jj, sw = (r >> 2) & 1;
+      *reinterpret_cast<uint4*>(arow + r * 32 + 16 * sw) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(arow + r * 32 + 16 * (sw ^ 1)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
   }
+  __syncwarp();
+  // (2) scores and group maxima, one token (m-tile) at a time
+  {
+    const uint32_t abase = q_smem(arow);
+    const uint32_t cb_lane = q_smem(&sm.cbh[0][0]) + 16u * (uint32_t)lane;  // x4: n-tiles 4G .. 4G + 3
+    const int arow_l = (lane & 7) + 8 * ((lane >> 3) & 1), ahalf = lane >> 4;
+#pragma unroll 1
+    for (int mt = 0; mt < 16; ++mt) {
+      uint32_t A[4];
+      {
+        const int r = 16 * mt + arow_l;
+        q_ldsm_x4(abase + (uint32_t)(r * 32 + 16 * (ahalf ^ ((r >> 2) & 1))), A);
+      }
+      float b1[2] = {-INFINITY, -INFINITY}, b2[2] = {-INFINITY, -INFINITY};
+      int bg[2] = {0, 0};
+#pragma unroll
+      for (int G = 0; G < NCODES / 32; ++G) {
+        uint32_t B4[4];
+        q_ldsm_x4(cb_lane + 512u * (uint32_t)G, B4);
+        float gm0 = -INFINITY, gm1 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 bz = *reinterpret_cast<const float2*>(&sm.bias[8 * (4 * G + i) + 2 * qp]);
+          float d[4] = {bz.x, bz.y, bz.x, bz.y};
+          q_mma_bb(d, A, B4[i]);
+          gm0 = max3f(gm0, d[0], d[1]);
+          gm1 = max3f(gm1, d[2], d[3]);
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float gm = r ? gm1 : gm0;
+          const float lo = fminf(b1[r], gm);
+          bg[r] = (gm > b1[r]) ? G : bg[r];
+          b1[r] = fmaxf(b1[r], gm);
+          b2[r] = fmaxf(b2[r], lo);
+        }
+      }
+      // merge over the quad: best group maximum, its (group, lane), and the
+      // largest maximum of every other group
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        float x1 = b1[r], x2 = b2[r];
+        int id = 4 * bg[r] + qp;
+#pragma unroll
+        for (int m = 1; m <= 2; m <<= 1) {
+          const float y1 = __shfl_xor_sync(0xffffffffu, x1, m), y2 = __shfl_xor_sync(0xffffffffu, x2, m);
+          const int yid = __shfl_xor_sync(0xffffffffu, id, m);
+          x2 = fmaxf(fmaxf(x2, y2), fminf(x1, y1));
+          id = (y1 > x1 || (y1 == x1 && yid < id)) ? yid : id;
+          x1 = fmaxf(x1, y1);
+        }
+        if (qp == 0) {
+          const int tok = 16 * warp + mt, j = qg + 8 * r;
+          sm.grp[tok][j] = (uint8_t)id;
+          sm.thr[tok][j] = x2;  // other groups' best tensor score, until (3) overwrites it
+        }
+      }
+    }
+  }
+  __syncwarp();
+  // (3) exact-arithmetic rescan of the winning group by the owner lane
+  uint32_t need = 0u;
+#pragma unroll
+  for (int jj = 0; jj < HSUB; ++jj) {
+    const int j = HSUB * h + jj;
+    const int id = sm.grp[tk][j];
+    const float other = sm.thr[tk][j];
+    const int kbase = 32 * (id >> 2) + 2 * (id & 3);
+    float best = -INFINITY, second = -INFINITY;
+    int idx = kbase;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int k = kbase + 8 * i + e;
+        const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
+        const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
+        float sc = sm.bias[k];
+        sc = fmaf(v[8 * jj + 0], c0.x, sc);
+        sc = fmaf(v[8 * jj + 1], c0.y, sc);
+        sc = fmaf(v[8 * jj + 2], c0.z, sc);
+        sc = fmaf(v[8 * jj + 3], c0.w, sc);
+        sc = fmaf(v[8 * jj + 4], c1.x, sc);
+        sc = fmaf(v[8 * jj + 5], c1.y, sc);
+        sc = fmaf(v[8 * jj + 6], c1.z, sc);
+        sc = fmaf(v[8 * jj + 7], c1.w, sc);
+        const float lo = fminf(best, sc);
+        idx = (sc > best) ? k : idx;
+        best = fmaxf(best, sc);
+        second = fmaxf(second, lo);
+      }
+    float na = 0.f;
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) na = fmaf(v[8 * jj + i], v[8 * jj + i], na);
+    na = sqrtf(na) * 1.0001f;
+    // a rival within twice the fp32 bound of the best may be the true best; so may
+    // another group whose tensor score is within the fp32 and tensor bounds
+    const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
+    const float m_tc = (TC_REL * (1.001f * na * cmax + 0.5f * cmax2) + na * cdel) * 1.01f;
+    sm.thr[tk][j] = best - margin;
+    sm.code[tk][j] = (uint8_t)idx;
+    need |= ((second >= best - margin || other >= best - 0.5f * margin - m_tc) ? 1u : 0u) << jj;
+  }
 
-  // ---- hand u to shared memory (the tile rows are free again) ----------------
-  // From here on u is read from shared memory so that no register array stays
-  // live across the rarely taken exact path.
+  // ---- hand u to shared memory (this warp's tile rows, the A rows are read) ---
+  // From here on u is read from shared memory.
 #pragma unroll
   for (int c = 0; c < HD; c += 4)
     *reinterpret_cast<float4*>(&sm.tile[tk][HD * h + c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-
-  // ---- exact fp64 re-decision of sub-vectors with a close second -------------
-  // Candidates: codewords whose fp32 score (same operation order as the main
-  // search) reaches the threshold; winner by fp64 squared distance, ties to the
-  // lowest index.
+  if (valid) {
 #pragma unroll 1
-  for (int jj = 0; jj < HSUB; ++jj) {
-    if (!((need >> jj) & 1u)) continue;
-    const int j = HSUB * h + jj;
-    const float* a = &sm.tile[tk][8 * j];
-    const float thr = sm.thr[tk][j];
-    double bestd = INFINITY;
-    int bi = sm.code[tk][j];
-#pragma unroll 1
-    for (int k = 0; k < NCODES; ++k) {
-      float sc = sm.bias[k];
-#pragma unroll
-      for (int i = 0; i < SUB; ++i) sc = fmaf(a[i], sm.cb[k][i], sc);
-      if (sc >= thr) {
-        double dd = 0.0;
-#pragma unroll
-        for (int i = 0; i < SUB; ++i) {
-          const double e = (double)a[i] - (double)sm.cb[k][i];
-          dd = fma(e, e, dd);
-        }
-        if (dd < bestd) { bestd = dd; bi = k; }
-      }
-    }
-    sm.code[tk][j] = (uint8_t)bi;
+    for (int jj = 0; jj < HSUB; ++jj)
+      if ((need >> jj) & 1u) sm.flag[atomicAdd(&sm.nflag, 1)] = (uint16_t)(tk * NSUB + HSUB * h + jj);
   }
+  __syncthreads();
+
+  // ---- (4) exact fp64 re-decision of the flagged sub-vectors, a warp each ----
+  // Candidates: codewords whose sequential fp32 score reaches the threshold
+  // (best - twice the fp32 bound); the winner by fp64 squared distance, ties to
+  // the lowest index.
+  {
+    const int nflag = sm.nflag;
+#pragma unroll 1
+    for (int f = warp; f < nflag; f += QTHREADS / 32) {
+      const int ftk = sm.flag[f] / NSUB, fj = sm.flag[f] % NSUB;
+      const float* a = &sm.tile[ftk][8 * fj];
+      const float thr = sm.thr[ftk][fj];
+      double bestd = INFINITY;
+      int bi = NCODES;
+#pragma unroll 1
+      for (int k = lane; k < NCODES; k += 32) {
+        float sc = sm.bias[k];
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) sc = fmaf(a[i], sm.cb[k][i], sc);
+        if (sc >= thr) {
+          double dd = 0.0;
+#pragma unroll
+          for (int i = 0; i < SUB; ++i) {
+            const double e = (double)a[i] - (double)sm.cb[k][i];
+            dd = fma(e, e, dd);
+          }
+          if (dd < bestd) { bestd = dd; bi = k; }
+        }
+      }
+#pragma unroll
+      for (int m = 16; m > 0; m >>= 1) {
+        const double od = __shfl_xor_sync(0xffffffffu, bestd, m);
+        const int ob = __shfl_xor_sync(0xffffffffu, bi, m);
+        if (od < bestd || (od == bestd && ob < bi)) { bestd = od; bi = ob; }
+      }
+      if (lane == 0 && bi < NCODES) sm.code[ftk][fj] = (uint8_t)bi;
+    }
+  }
+  __syncthreads();
 
   // ---- adaptive scale: alpha = ||u||^2 / (u . u_hat) --------------------------
   double dot = 0.0, uu = 0.0;
