@@ -70,7 +70,9 @@ constexpr int HD = D / 2;           // dims per thread
 constexpr int HSUB = NSUB / 2;      // sub-vectors per thread
 
 struct QuantSmem {
-  alignas(16) float cb[NCODES][SUB];   // codebook (fp32)
+  // codebook (fp32), rows padded to 48 bytes: lanes gathering random rows (the
+  // group rescan, the adaptive scale) spread over all eight 16-byte bank groups
+  alignas(16) float cb[NCODES][SUB + 4];
   alignas(16) float bias[NCODES];      // -||c_k||^2 / 2
   alignas(16) float cnorm[4];          // [0] = max ||c||, [1] = max ||c||^2, [2] = max ||c - fp16(c)|| (rounded up)
   alignas(16) __half cbh[NCODES][SUB]; // codebook rounded to fp16 (tensor-core operand)
@@ -126,7 +128,7 @@ __device__ __forceinline__ BlockOut block_out(const CacheView& c, int64_t seq, i
 __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook) {
   const int t = threadIdx.x;
   for (int i = t; i < NCODES * SUB / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(&sm.cb[0][0])[i] = __ldg(reinterpret_cast<const float4*>(codebook) + i);
+    *reinterpret_cast<float4*>(&sm.cb[i >> 1][4 * (i & 1)]) = __ldg(reinterpret_cast<const float4*>(codebook) + i);
   __syncthreads();
   float my_max = 0.f, my_dev = 0.f;
   for (int k = t; k < NCODES; k += blockDim.x) {
@@ -511,15 +513,18 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
       for (int G = 0; G < NCODES / 32; ++G) {
         uint32_t B4[4];
         q_ldsm_x4(cb_lane + 512u * (uint32_t)G, B4);
-        float gm0 = -INFINITY, gm1 = -INFINITY;
+        float d[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 bz = *reinterpret_cast<const float2*>(&sm.bias[8 * (4 * G + i) + 2 * qp]);
-          float d[4] = {bz.x, bz.y, bz.x, bz.y};
-          q_mma_bb(d, A, B4[i]);
-          gm0 = max3f(gm0, d[0], d[1]);
-          gm1 = max3f(gm1, d[2], d[3]);
+          d[i][0] = bz.x; d[i][1] = bz.y; d[i][2] = bz.x; d[i][3] = bz.y;
+          q_mma_bb(d[i], A, B4[i]);
         }
+        // group maxima of rows g (0, 1) and g + 8 (2, 3) as shallow trees
+        const float gm0 = max3f(max3f(d[0][0], d[0][1], d[1][0]), max3f(d[1][1], d[2][0], d[2][1]),
+                                fmaxf(d[3][0], d[3][1]));
+        const float gm1 = max3f(max3f(d[0][2], d[0][3], d[1][2]), max3f(d[1][3], d[2][2], d[2][3]),
+                                fmaxf(d[3][2], d[3][3]));
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const float gm = r ? gm1 : gm0;
