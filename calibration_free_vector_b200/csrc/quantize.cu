@@ -74,6 +74,7 @@ struct QuantSmem {
   // group rescan, the adaptive scale) spread over all eight 16-byte bank groups
   alignas(16) float cb[NCODES][SUB + 4];
   alignas(16) float bias[NCODES];      // -||c_k||^2 / 2
+  alignas(16) float biasq[NCODES];     // the same, per (group G of 32 codes, quad lane p): codes 32G + 8i + 2p + e at 32G + 8p + 2i + e
   alignas(16) float cnorm[4];          // [0] = max ||c||, [1] = max ||c||^2, [2] = max ||c - fp16(c)|| (rounded up)
   alignas(16) __half cbh[NCODES][SUB]; // codebook rounded to fp16 (tensor-core operand)
   alignas(16) double rr[BLK];          // 1 / ||x_t|| (0 for a zero token)
@@ -142,6 +143,7 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
       e = fmaf(d, d, e);
     }
     sm.bias[k] = -0.5f * s;
+    sm.biasq[(k & ~31) + 8 * ((k >> 1) & 3) + 2 * ((k >> 3) & 3) + (k & 1)] = -0.5f * s;
     my_max = fmaxf(my_max, s);
     my_dev = fmaxf(my_dev, e);
   }
@@ -473,11 +475,16 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
   const int warp = t >> 5, lane = t & 31, qg = lane >> 2, qp = lane & 3;
   // (1) this warp's 16 tokens x 16 sub-vectors as A rows of 32 bytes (fp16 hi |
-  // lo), in the warp's own 16 tile rows (free since the column sums); the two
-  // 16-byte halves swap on every 4th row so that ldmatrix rows hit distinct banks
+  // lo), in the warp's own 16 tile rows (free since the column sums).  Row r of
+  // token m sits at R = 16 m + (r ^ (m & 3)) and its two 16-byte halves swap when
+  // bit 2 xor bit 3 of R is set: the 8 rows of an ldmatrix fetch and the 8 rows
+  // of a store phase (4 tokens x 2 halves of the sub-vectors) both land in 8
+  // different 16-byte bank groups.
   unsigned char* arow = reinterpret_cast<unsigned char*>(&sm.tile[16 * warp][0]);
+  auto a_phys = [](int m, int r) { return 16 * m + (r ^ (m & 3)); };
+  auto a_flip = [](int R) { return ((R >> 2) ^ (R >> 3)) & 1; };
   {
-    const int r0 = 16 * (lane >> 1) + HSUB * h;
+    const int m_own = lane >> 1;
 #pragma unroll
     for (int jj = 0; jj < HSUB; ++jj) {
       uint32_t hw[4], lw[4];
@@ -489,9 +496,9 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
         hw[i] = h2_bits(hh);
         lw[i] = h2_bits(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
       }
-      const int r = r0 + jj, sw = (r >> 2) & 1;
-      *reinterpret_cast<uint4*>(arow + r * 32 + 16 * sw) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(arow + r * 32 + 16 * (sw ^ 1)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      const int R = a_phys(m_own, HSUB * h + jj), sw = a_flip(R);
+      *reinterpret_cast<uint4*>(arow + R * 32 + 16 * sw) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(arow + R * 32 + 16 * (sw ^ 1)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
   }
   __syncwarp();
@@ -504,8 +511,8 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     for (int mt = 0; mt < 16; ++mt) {
       uint32_t A[4];
       {
-        const int r = 16 * mt + arow_l;
-        q_ldsm_x4(abase + (uint32_t)(r * 32 + 16 * (ahalf ^ ((r >> 2) & 1))), A);
+        const int R = a_phys(mt, arow_l);
+        q_ldsm_x4(abase + (uint32_t)(R * 32 + 16 * (ahalf ^ a_flip(R))), A);
       }
       float b1[2] = {-INFINITY, -INFINITY}, b2[2] = {-INFINITY, -INFINITY};
       int bg[2] = {0, 0};
@@ -514,10 +521,12 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
         uint32_t B4[4];
         q_ldsm_x4(cb_lane + 512u * (uint32_t)G, B4);
         float d[4][4];
+        const float4 bz01 = *reinterpret_cast<const float4*>(&sm.biasq[32 * G + 8 * qp]);
+        const float4 bz23 = *reinterpret_cast<const float4*>(&sm.biasq[32 * G + 8 * qp + 4]);
+        const float bzv[8] = {bz01.x, bz01.y, bz01.z, bz01.w, bz23.x, bz23.y, bz23.z, bz23.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float2 bz = *reinterpret_cast<const float2*>(&sm.bias[8 * (4 * G + i) + 2 * qp]);
-          d[i][0] = bz.x; d[i][1] = bz.y; d[i][2] = bz.x; d[i][3] = bz.y;
+          d[i][0] = bzv[2 * i]; d[i][1] = bzv[2 * i + 1]; d[i][2] = bzv[2 * i]; d[i][3] = bzv[2 * i + 1];
           q_mma_bb(d[i], A, B4[i]);
         }
         // group maxima of rows g (0, 1) and g + 8 (2, 3) as shallow trees
