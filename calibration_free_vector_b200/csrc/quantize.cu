@@ -76,7 +76,7 @@ struct QuantSmem {
   alignas(16) float bias[NCODES];      // -||c_k||^2 / 2
   alignas(16) float biasq[NCODES];     // the same, per (group G of 32 codes, quad lane p): codes 32G + 8i + 2p + e at 32G + 8p + 2i + e
   alignas(16) float cnorm[4];          // [0] = max ||c||, [1] = max ||c||^2, [2] = max ||c - fp16(c)|| (rounded up)
-  alignas(16) __half cbh[NCODES][SUB]; // codebook rounded to fp16 (tensor-core operand)
+  alignas(16) __half cbh[NCODES][SUB]; // codebook rounded to fp16, dims in the order 0 4 1 5 2 6 3 7 (tensor-core operand)
   alignas(16) double rr[BLK];          // 1 / ||x_t|| (0 for a zero token)
   alignas(16) double s1[BLK];          // per-token s1 and s2 (fp64) until the final store
   alignas(16) double s2[BLK];
@@ -138,7 +138,7 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
     for (int i = 0; i < SUB; ++i) {
       s = fmaf(sm.cb[k][i], sm.cb[k][i], s);
       const __half c16 = __float2half_rn(sm.cb[k][i]);
-      sm.cbh[k][i] = c16;
+      sm.cbh[k][i < 4 ? 2 * i : 2 * (i - 4) + 1] = c16;  // K order of the MMA: dims p, p + 4 at slots 2p, 2p + 1
       const float d = sm.cb[k][i] - __half2float(c16);
       e = fmaf(d, d, e);
     }
@@ -474,105 +474,133 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
   constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
   constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
   const int warp = t >> 5, lane = t & 31, qg = lane >> 2, qp = lane & 3;
-  // (1) this warp's 16 tokens x 16 sub-vectors as A rows of 32 bytes (fp16 hi |
-  // lo), in the warp's own 16 tile rows (free since the column sums).  Row r of
-  // token m sits at R = 16 m + (r ^ (m & 3)) and its two 16-byte halves swap when
-  // bit 2 xor bit 3 of R is set: the 8 rows of an ldmatrix fetch and the 8 rows
-  // of a store phase (4 tokens x 2 halves of the sub-vectors) both land in 8
-  // different 16-byte bank groups.
-  unsigned char* arow = reinterpret_cast<unsigned char*>(&sm.tile[16 * warp][0]);
+  // (1) this warp's 16 tokens x 16 sub-vectors as rows of 8 fp32 (the exact
+  // search operand a), in the warp's own 16 tile rows (free since the column
+  // sums).  Row r of token m sits at R = 16 m + (r ^ (m & 3)) and its two 16-byte
+  // halves (dims 0-3, 4-7) swap when bit 2 xor bit 3 of R is set: the 8 rows of
+  // an ldmatrix fetch and the 8 rows of a store phase (4 tokens x 2 halves of the
+  // sub-vectors) both land in 8 different 16-byte bank groups.  The rows stay
+  // there for the rescan, the exact path and the adaptive scale.
   auto a_phys = [](int m, int r) { return 16 * m + (r ^ (m & 3)); };
   auto a_flip = [](int R) { return ((R >> 2) ^ (R >> 3)) & 1; };
+  auto urow = [&](int tok, int j, int half) -> const float4* {
+    const unsigned char* base = reinterpret_cast<const unsigned char*>(&sm.tile[16 * (tok >> 4)][0]);
+    const int R = a_phys(tok & 15, j);
+    return reinterpret_cast<const float4*>(base + R * 32 + 16 * (half ^ a_flip(R)));
+  };
+  unsigned char* arow = reinterpret_cast<unsigned char*>(&sm.tile[16 * warp][0]);
   {
     const int m_own = lane >> 1;
 #pragma unroll
     for (int jj = 0; jj < HSUB; ++jj) {
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float x0 = valid ? v[8 * jj + 2 * i] : 0.f, x1 = valid ? v[8 * jj + 2 * i + 1] : 0.f;
-        const __half2 hh = __floats2half2_rn(x0, x1);
-        const float2 hf = __half22float2(hh);
-        hw[i] = h2_bits(hh);
-        lw[i] = h2_bits(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
-      }
       const int R = a_phys(m_own, HSUB * h + jj), sw = a_flip(R);
-      *reinterpret_cast<uint4*>(arow + R * 32 + 16 * sw) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(arow + R * 32 + 16 * (sw ^ 1)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      const float4 lo4 = valid ? make_float4(v[8 * jj], v[8 * jj + 1], v[8 * jj + 2], v[8 * jj + 3])
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 hi4 = valid ? make_float4(v[8 * jj + 4], v[8 * jj + 5], v[8 * jj + 6], v[8 * jj + 7])
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(arow + R * 32 + 16 * sw) = lo4;
+      *reinterpret_cast<float4*>(arow + R * 32 + 16 * (sw ^ 1)) = hi4;
     }
   }
   __syncwarp();
-  // (2) scores and group maxima, one token (m-tile) at a time
+  // (2) scores and group maxima, two tokens (m-tiles) at a time sharing the
+  // codebook fragments.  ldmatrix of the fp32 rows gives lane (g, p) dims p and
+  // p + 4 of rows g and g + 8; their fp16 hi and lo parts are the A fragment in
+  // the K order of the permuted fp16 codebook.
   {
     const uint32_t abase = q_smem(arow);
     const uint32_t cb_lane = q_smem(&sm.cbh[0][0]) + 16u * (uint32_t)lane;  // x4: n-tiles 4G .. 4G + 3
     const int arow_l = (lane & 7) + 8 * ((lane >> 3) & 1), ahalf = lane >> 4;
 #pragma unroll 1
-    for (int mt = 0; mt < 16; ++mt) {
-      uint32_t A[4];
-      {
-        const int R = a_phys(mt, arow_l);
-        q_ldsm_x4(abase + (uint32_t)(R * 32 + 16 * (ahalf ^ a_flip(R))), A);
+    for (int mp = 0; mp < 8; ++mp) {
+      uint32_t A[2][4];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int R = a_phys(2 * mp + q, arow_l);
+        uint32_t w[4];
+        q_ldsm_x4(abase + (uint32_t)(R * 32 + 16 * (ahalf ^ a_flip(R))), w);
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {  // row g (words 0, 2) and row g + 8 (words 1, 3)
+          const float x0 = __uint_as_float(w[rr]), x1 = __uint_as_float(w[rr + 2]);
+          const __half2 hh = __floats2half2_rn(x0, x1);
+          const float2 hf = __half22float2(hh);
+          A[q][rr] = h2_bits(hh);
+          A[q][2 + rr] = h2_bits(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
+        }
       }
-      float b1[2] = {-INFINITY, -INFINITY}, b2[2] = {-INFINITY, -INFINITY};
-      int bg[2] = {0, 0};
+      float b1[2][2], b2[2][2];
+      int bg[2][2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          b1[q][r] = -INFINITY;
+          b2[q][r] = -INFINITY;
+          bg[q][r] = 0;
+        }
 #pragma unroll
       for (int G = 0; G < NCODES / 32; ++G) {
         uint32_t B4[4];
         q_ldsm_x4(cb_lane + 512u * (uint32_t)G, B4);
-        float d[4][4];
         const float4 bz01 = *reinterpret_cast<const float4*>(&sm.biasq[32 * G + 8 * qp]);
         const float4 bz23 = *reinterpret_cast<const float4*>(&sm.biasq[32 * G + 8 * qp + 4]);
         const float bzv[8] = {bz01.x, bz01.y, bz01.z, bz01.w, bz23.x, bz23.y, bz23.z, bz23.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          d[i][0] = bzv[2 * i]; d[i][1] = bzv[2 * i + 1]; d[i][2] = bzv[2 * i]; d[i][3] = bzv[2 * i + 1];
-          q_mma_bb(d[i], A, B4[i]);
-        }
-        // group maxima of rows g (0, 1) and g + 8 (2, 3) as shallow trees
-        const float gm0 = max3f(max3f(d[0][0], d[0][1], d[1][0]), max3f(d[1][1], d[2][0], d[2][1]),
-                                fmaxf(d[3][0], d[3][1]));
-        const float gm1 = max3f(max3f(d[0][2], d[0][3], d[1][2]), max3f(d[1][3], d[2][2], d[2][3]),
-                                fmaxf(d[3][2], d[3][3]));
+        for (int q = 0; q < 2; ++q) {
+          float d[4][4];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float gm = r ? gm1 : gm0;
-          const float lo = fminf(b1[r], gm);
-          bg[r] = (gm > b1[r]) ? G : bg[r];
-          b1[r] = fmaxf(b1[r], gm);
-          b2[r] = fmaxf(b2[r], lo);
+          for (int i = 0; i < 4; ++i) {
+            d[i][0] = bzv[2 * i]; d[i][1] = bzv[2 * i + 1]; d[i][2] = bzv[2 * i]; d[i][3] = bzv[2 * i + 1];
+            q_mma_bb(d[i], A[q], B4[i]);
+          }
+          // group maxima of rows g (0, 1) and g + 8 (2, 3) as shallow trees
+          const float gm[2] = {max3f(max3f(d[0][0], d[0][1], d[1][0]), max3f(d[1][1], d[2][0], d[2][1]),
+                                     fmaxf(d[3][0], d[3][1])),
+                               max3f(max3f(d[0][2], d[0][3], d[1][2]), max3f(d[1][3], d[2][2], d[2][3]),
+                                     fmaxf(d[3][2], d[3][3]))};
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float lo = fminf(b1[q][r], gm[r]);
+            bg[q][r] = (gm[r] > b1[q][r]) ? G : bg[q][r];
+            b1[q][r] = fmaxf(b1[q][r], gm[r]);
+            b2[q][r] = fmaxf(b2[q][r], lo);
+          }
         }
       }
       // merge over the quad: best group maximum, its (group, lane), and the
       // largest maximum of every other group
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        float x1 = b1[r], x2 = b2[r];
-        int id = 4 * bg[r] + qp;
+      for (int q = 0; q < 2; ++q)
 #pragma unroll
-        for (int m = 1; m <= 2; m <<= 1) {
-          const float y1 = __shfl_xor_sync(0xffffffffu, x1, m), y2 = __shfl_xor_sync(0xffffffffu, x2, m);
-          const int yid = __shfl_xor_sync(0xffffffffu, id, m);
-          x2 = fmaxf(fmaxf(x2, y2), fminf(x1, y1));
-          id = (y1 > x1 || (y1 == x1 && yid < id)) ? yid : id;
-          x1 = fmaxf(x1, y1);
+        for (int r = 0; r < 2; ++r) {
+          float x1 = b1[q][r], x2 = b2[q][r];
+          int id = 4 * bg[q][r] + qp;
+#pragma unroll
+          for (int m = 1; m <= 2; m <<= 1) {
+            const float y1 = __shfl_xor_sync(0xffffffffu, x1, m), y2 = __shfl_xor_sync(0xffffffffu, x2, m);
+            const int yid = __shfl_xor_sync(0xffffffffu, id, m);
+            x2 = fmaxf(fmaxf(x2, y2), fminf(x1, y1));
+            id = (y1 > x1 || (y1 == x1 && yid < id)) ? yid : id;
+            x1 = fmaxf(x1, y1);
+          }
+          if (qp == 0) {
+            const int tok = 16 * warp + 2 * mp + q, j = qg + 8 * r;
+            sm.grp[tok][j] = (uint8_t)id;
+            sm.thr[tok][j] = x2;  // other groups' best tensor score, until (3) overwrites it
+          }
         }
-        if (qp == 0) {
-          const int tok = 16 * warp + mt, j = qg + 8 * r;
-          sm.grp[tok][j] = (uint8_t)id;
-          sm.thr[tok][j] = x2;  // other groups' best tensor score, until (3) overwrites it
-        }
-      }
     }
   }
   __syncwarp();
   // (3) exact-arithmetic rescan of the winning group by the owner lane
   uint32_t need = 0u;
-#pragma unroll
+#pragma unroll 2
   for (int jj = 0; jj < HSUB; ++jj) {
     const int j = HSUB * h + jj;
     const int id = sm.grp[tk][j];
     const float other = sm.thr[tk][j];
+    const float4 u0 = *urow(tk, j, 0), u1 = *urow(tk, j, 1);
+    const float a[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
     const int kbase = 32 * (id >> 2) + 2 * (id & 3);
     float best = -INFINITY, second = -INFINITY;
     int idx = kbase;
@@ -584,14 +612,14 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
         const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
         const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
         float sc = sm.bias[k];
-        sc = fmaf(v[8 * jj + 0], c0.x, sc);
-        sc = fmaf(v[8 * jj + 1], c0.y, sc);
-        sc = fmaf(v[8 * jj + 2], c0.z, sc);
-        sc = fmaf(v[8 * jj + 3], c0.w, sc);
-        sc = fmaf(v[8 * jj + 4], c1.x, sc);
-        sc = fmaf(v[8 * jj + 5], c1.y, sc);
-        sc = fmaf(v[8 * jj + 6], c1.z, sc);
-        sc = fmaf(v[8 * jj + 7], c1.w, sc);
+        sc = fmaf(a[0], c0.x, sc);
+        sc = fmaf(a[1], c0.y, sc);
+        sc = fmaf(a[2], c0.z, sc);
+        sc = fmaf(a[3], c0.w, sc);
+        sc = fmaf(a[4], c1.x, sc);
+        sc = fmaf(a[5], c1.y, sc);
+        sc = fmaf(a[6], c1.z, sc);
+        sc = fmaf(a[7], c1.w, sc);
         const float lo = fminf(best, sc);
         idx = (sc > best) ? k : idx;
         best = fmaxf(best, sc);
@@ -599,7 +627,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
       }
     float na = 0.f;
 #pragma unroll
-    for (int i = 0; i < SUB; ++i) na = fmaf(v[8 * jj + i], v[8 * jj + i], na);
+    for (int i = 0; i < SUB; ++i) na = fmaf(a[i], a[i], na);
     na = sqrtf(na) * 1.0001f;
     // a rival within twice the fp32 bound of the best may be the true best; so may
     // another group whose tensor score is within the fp32 and tensor bounds
@@ -610,11 +638,6 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     need |= ((second >= best - margin || other >= best - 0.5f * margin - m_tc) ? 1u : 0u) << jj;
   }
 
-  // ---- hand u to shared memory (this warp's tile rows, the A rows are read) ---
-  // From here on u is read from shared memory.
-#pragma unroll
-  for (int c = 0; c < HD; c += 4)
-    *reinterpret_cast<float4*>(&sm.tile[tk][HD * h + c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
   if (valid) {
 #pragma unroll 1
     for (int jj = 0; jj < HSUB; ++jj)
@@ -631,7 +654,8 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
 #pragma unroll 1
     for (int f = warp; f < nflag; f += QTHREADS / 32) {
       const int ftk = sm.flag[f] / NSUB, fj = sm.flag[f] % NSUB;
-      const float* a = &sm.tile[ftk][8 * fj];
+      const float4 fa0 = *urow(ftk, fj, 0), fa1 = *urow(ftk, fj, 1);
+      const float a[8] = {fa0.x, fa0.y, fa0.z, fa0.w, fa1.x, fa1.y, fa1.z, fa1.w};
       const float thr = sm.thr[ftk][fj];
       double bestd = INFINITY;
       int bi = NCODES;
@@ -669,8 +693,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     const int cj = sm.code[tk][j];
     const float4 q0 = *reinterpret_cast<const float4*>(&sm.cb[cj][0]);
     const float4 q1 = *reinterpret_cast<const float4*>(&sm.cb[cj][4]);
-    const float4 u0 = *reinterpret_cast<const float4*>(&sm.tile[tk][8 * j]);
-    const float4 u1 = *reinterpret_cast<const float4*>(&sm.tile[tk][8 * j + 4]);
+    const float4 u0 = *urow(tk, j, 0), u1 = *urow(tk, j, 1);
     const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
     const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
     float dj = 0.f, uj = 0.f;
