@@ -14,10 +14,10 @@ pytestmark = pytest.mark.gpu
 DT = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
 
 
-def run_prefill(batch, heads, seq, mode, dtype, window, kind="llama", seed=1, capacity=None, x=None):
+def run_prefill(batch, heads, seq, mode, dtype, window, kind="llama", seed=1, capacity=None, x=None, cb=None):
     if x is None:
         x = synthetic.KVRecipe(seed, heads, kind).tokens(batch, seq, DT[dtype], "cpu")
-    cb = tl.codebook(mode)
+    cb = tl.codebook(mode) if cb is None else cb
     cap = capacity or max(128, ((seq + 127) // 128) * 128)
     cache = nsn.Cache(batch, heads, cap, window, mode)
     nsn.nsn_quantize_kv(cache, x.cuda(), torch.from_numpy(cb).cuda())
@@ -58,6 +58,35 @@ def test_llama_shape_ragged(mode, dtype):
     # 8 kv-heads, 1061 tokens -> 1024 quantized in 8 blocks + 37 in the window.
     x, cb, cache = run_prefill(1, 8, 1061, mode, dtype, 128, seed=synthetic.config_seed(2, "k"))
     check_prefill(x, cb, cache, mode, 128)
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_codebook_not_fp16_representable(mode):
+    # The quantizer takes any fp32 codebook: its tensor-core scores use the fp16
+    # rounding of it, and the decision bound then widens by ||a|| ||c - fp16(c)||.
+    # The codes must still be the exact nearest of the fp32 codebook.
+    rng = np.random.default_rng(5 + mode)
+    cb = (tl.codebook(mode).astype(np.float64) * (1.0 + 3e-4 * rng.standard_normal((256, 8)))).astype(np.float32)
+    assert np.any(cb != cb.astype(np.float16).astype(np.float32))
+    x, cb, cache = run_prefill(1, 4, 700, mode, "bf16", 128, seed=91, cb=cb)
+    check_prefill(x, cb, cache, mode, 128)
+
+
+def test_duplicate_codeword_ties_go_to_the_lower_index():
+    # Codeword 200 repeats codeword 17 exactly: every sub-vector nearest to it is an
+    # exact tie, which the exact path resolves to the lower index, as the oracle does.
+    cb = tl.codebook(2).copy()
+    cb[200] = cb[17]
+    x, cb, cache = run_prefill(1, 2, 1000, 2, "bf16", 128, seed=93, cb=cb)
+    xf = x.float().numpy().astype(np.float64)
+    hits = 0
+    for h in range(2):
+        ref = orc.quantize_sequence(xf[0, :, h, :], cb.astype(np.float64), 2, 128, 128)
+        got = tl.read_cache(cache, 0, h)
+        assert not np.any(got["codes"] == 200) and not np.any(ref["codes"] == 200)
+        assert np.array_equal(got["codes"] == 17, ref["codes"] == 17)
+        hits += int(np.sum(ref["codes"] == 17))
+    assert hits > 0  # the tie is actually exercised
 
 
 def test_partial_last_block_no_window():
