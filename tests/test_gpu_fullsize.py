@@ -1,8 +1,9 @@
 """Parity at the full workload sizes, in the launch configuration the bench uses.
 
-For each of the decode-throughput layer (batch 16 x 32k, 2-bit K/V), the extreme
+For each of the decode-throughput layer (batch 16 x 32k, 2-bit K/V; also with
+pre-RoPE keys), the extreme
 compression layer (batch 64 x 8k, 1-bit K/V) and the long-context layer (batch 4 x
-128k, 2-bit K / 1-bit V): prefill on the GPU, append the workload's decode tokens
+128k, 2-bit K / 1-bit V; also with pre-RoPE keys): prefill on the GPU, append the workload's decode tokens
 (the first append flushes the full window), decode, then check
   * sampled prefill blocks of many (batch, kv-head) sequences element by element
     against the oracle's quantizer (blocks are independent), and
@@ -32,7 +33,12 @@ def pool():
         yield ex
 
 
-def run_workload(cfg_id, steps, pool, sample_blocks=12, seed_off=0, double_quant=False):
+def rope_theta():
+    """RoPE frequencies of the Llama-3-8B shape, theta_i = 500000^(-2i/128), as fp32."""
+    return (500000.0 ** (-2.0 * np.arange(64) / 128.0)).astype(np.float32)
+
+
+def run_workload(cfg_id, steps, pool, sample_blocks=12, seed_off=0, double_quant=False, rope=False):
     W = synthetic.WORKLOADS[cfg_id]
     B, H, HQ, T, mk, mv = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["seq"], W["mode_k"], W["mode_v"]
     g = HQ // H
@@ -52,7 +58,11 @@ def run_workload(cfg_id, steps, pool, sample_blocks=12, seed_off=0, double_quant
         nsn.nsn_append_residual(kc, vc, xk[:, s], xv[:, s], dk, dv)
     q = synthetic.queries(synthetic.config_seed(cfg_id, "q") + seed_off, B, HQ, torch.bfloat16, dev)
     out = torch.empty((B, HQ, 128), dtype=torch.float32, device=dev)
-    nsn.nsn_decode_attention(kc, vc, q, SCALE, dk, dv, out, nsn.decode_workspace(kc, HQ, dev))
+    if rope:  # the cache holds pre-RoPE keys; every key is rotated at its position
+        nsn.nsn_decode_attention_rope(kc, vc, q, SCALE, torch.from_numpy(rope_theta()).to(dev), dk, dv, out,
+                                      nsn.decode_rope_workspace(kc, HQ, dev))
+    else:
+        nsn.nsn_decode_attention(kc, vc, q, SCALE, dk, dv, out, nsn.decode_workspace(kc, HQ, dev))
     torch.cuda.synchronize()
     assert int(kc.status.item()) == 0 and int(vc.status.item()) == 0
 
@@ -100,7 +110,12 @@ def run_workload(cfg_id, steps, pool, sample_blocks=12, seed_off=0, double_quant
     assert got_k["n_quant"] == kq["codes"].shape[0] and got_k["n_window"] == kw.shape[0]
     tl.compare_codes(got_k, kq, kq["u"])
     qf = q[b, h * g:(h + 1) * g].float().cpu().numpy().astype(np.float64)
-    ref = orc.decode_attention(qf, kq, vq, kw, vw, cbk.astype(np.float64), cbv.astype(np.float64), mk, mv, SCALE)
+    if rope:
+        ref = orc.decode_attention_rope(qf, kq, vq, kw, vw, cbk.astype(np.float64), cbv.astype(np.float64), mk, mv,
+                                        SCALE, rope_theta().astype(np.float64))
+    else:
+        ref = orc.decode_attention(qf, kq, vq, kw, vw, cbk.astype(np.float64), cbv.astype(np.float64), mk, mv,
+                                   SCALE)
     err = tl.attn_error(out[b, h * g:(h + 1) * g].cpu().numpy(), ref)
     assert err <= tl.ATTN_TOL, f"workload {cfg_id}: (b={b}, h={h}) attention error {err:.3g}"
     return err
@@ -124,3 +139,13 @@ def test_fullsize_long_context(pool):
 def test_fullsize_decode_throughput_layer_double_quant(pool):
     # the same layer with s1 and o stored in 4 bits (bench.py --double-quant)
     run_workload(3, 1, pool, double_quant=True)
+
+
+def test_fullsize_decode_throughput_layer_pre_rope(pool):
+    # the same layer with pre-RoPE keys (bench.py --rope): positions up to 32k
+    run_workload(3, 1, pool, sample_blocks=2, rope=True)
+
+
+def test_fullsize_long_context_pre_rope(pool):
+    # batch 4, 128k context, pre-RoPE keys: angles up to about 1.3e5 rad at theta_0 = 1
+    run_workload(5, 16, pool, sample_blocks=2, rope=True)
