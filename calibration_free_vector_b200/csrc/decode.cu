@@ -942,20 +942,22 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
 // accumulator fragments the lane holds dims i and i + 64 of the same tokens in the
 // same register slot, so the NSN affine terms and the rotation run in fp32 in
 // registers; the rotated key is split into fp16 hi + lo and multiplied by the
-// fp16 hi + lo query (the m16n8k16 A-from-accumulator layout needs no shuffle).
-// (cos, sin)(pos theta_i) = (cos, sin)(pos0 theta_i) * (cos, sin)(r theta_i),
-// pos0 the 64-token stage start (per warp, angle reduced in fp64) and r < 64 from
-// a CTA table.
+// fp16 hi + lo query (the accumulator layout is the A layout, no shuffle).
+// Rotations compose, q . R_(pos0 + r) k = (R_(-pos0) q) . (R_r k): the query is
+// rotated back by the 64-token stage start pos0 once per stage (angles reduced in
+// fp64), and each key by its offset r < 64 from a CTA table of (cos, sin)(r theta_i).
 // ---------------------------------------------------------------------------
 constexpr int RS_WARPS = 8;
+constexpr int RS_WK_HOB = 8 * QS_ROW;             // per-warp area: query staging (8 fp16 rows) ...
+constexpr int RS_WK_BASE = RS_WK_HOB + D * 4;     // ... H o_b (128 fp32) ...
+constexpr int RS_WK_BYTES = RS_WK_BASE + (D / 2) * 8;  // ... (cos, sin)(pos0 theta_i), 64 pairs
 constexpr int RS_OFF_ROW = STAGE_TOK + 8;  // float2 per table row: 64 + padding, so 8 lanes of a
                                            // 16-byte fetch on two rows hit different banks
 struct RsSmem {
   alignas(128) uint4 cbk[NCODES][8];                    // replicated fp16 K codebook (as in decode_kernel)
   alignas(16) float2 off[STAGE_TOK][RS_OFF_ROW];        // (cos, sin)(r theta_i), r < 64, i < 64
-  alignas(128) unsigned char wk[RS_WARPS][8 * QS_ROW];  // per warp: query staging, then H o_b and the stage base
+  alignas(128) unsigned char wk[RS_WARPS][RS_WK_BYTES];  // per warp: query staging | H o_b | stage angles
 };
-static_assert(8 * QS_ROW >= D * 4 + (D / 2) * 8, "H o_b and the base angles fit the staging area");
 
 // (cos a, sin a) with a reduced to [-pi, pi] in fp64 first.
 __device__ __forceinline__ float2 rope_cs(double a) {
@@ -1047,16 +1049,13 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
   if (st_first >= st_last) return;
   float* rdst = rscores + ((int64_t)(seq * ngroups + hg) * rs_cap) * GH;
 
-  // query operand, original domain (fp16 hi rows 0-3, residual rows 4-7)
+  // query operand (original domain, fp16 hi rows 0-3, residual rows 4-7), rebuilt
+  // per stage rotated back by the stage start
   unsigned char* wk = &sm.wk[warp][0];
+  const int64_t q_off = (int64_t)b * qsb + (int64_t)(hk * G + hg * GH) * qsh;
   uint32_t qb[8][2];
-  {
-    float qrows[GH][4];
-    load_q_rows<GH>(qrows, q, dtype, (int64_t)b * qsb + (int64_t)(hk * G + hg * GH) * qsh, qsh, lane);
-    build_q_operand<GH>(qb, qrows, qscale, false, lane, wk);
-  }
-  float* hob = reinterpret_cast<float*>(wk);                // H o_b of the current block (128 fp32)
-  float2* base = reinterpret_cast<float2*>(wk + D * 4);     // (cos, sin)(pos0 theta_i), 64
+  float* hob = reinterpret_cast<float*>(wk + RS_WK_HOB);      // H o_b of the current block (128 fp32)
+  float2* base = reinterpret_cast<float2*>(wk + RS_WK_BASE);  // (cos, sin)(pos0 theta_i), 64
 
   // H_16 as the B operand: column n = g + 8 nt, rows 2p, 2p+1 | 2p+8, 2p+9
   uint32_t Hb[2][2];
@@ -1122,6 +1121,24 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
       *reinterpret_cast<float4*>(hob + 4 * lane) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncwarp();
+    // the query rotated back by the stage start: q . R_(pos0 + r) k = (R_(-pos0) q) . (R_r k)
+    {
+      float qrows[GH][4];
+      load_q_rows<GH>(qrows, q, dtype, q_off, qsh, lane);
+      const int i0 = (4 * lane) & (D / 2 - 1);  // dims 4l .. 4l+3; their pair partners sit in lane l ^ 16
+      const float4 cs01 = *reinterpret_cast<const float4*>(base + i0);
+      const float4 cs23 = *reinterpret_cast<const float4*>(base + i0 + 2);
+      const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z}, ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+      const bool upper = lane >= 16;  // dims i + 64
+#pragma unroll
+      for (int hh = 0; hh < GH; ++hh)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float mine = qrows[hh][e], other = __shfl_xor_sync(0xffffffffu, mine, 16);
+          qrows[hh][e] = fmaf(mine, cc[e], (upper ? -other : other) * ss[e]);
+        }
+      build_q_operand<GH>(qb, qrows, qscale, false, lane, wk);
+    }
 
     for (int m = 0; m < STAGE_TOK / 16; ++m) {
       const int tt = pos0 + 16 * m;  // position of the tile's first token
@@ -1197,7 +1214,6 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
           const int i0 = 16 * ap + 8 * nt + 2 * p;
           const float2 olo = *reinterpret_cast<const float2*>(hob + i0);
           const float2 ohi = *reinterpret_cast<const float2*>(hob + i0 + 64);
-          const float4 bb = *reinterpret_cast<const float4*>(base + i0);
           float y0[4], y1[4];
 #pragma unroll
           for (int rr = 0; rr < 2; ++rr) {
@@ -1207,9 +1223,7 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
               const int r = 2 * rr + e;
               const float lo = fmaf(xs[rr], E[ap][nt][r], e ? olo.y : olo.x);
               const float hi = fmaf(xs[rr], E[ap + 4][nt][r], e ? ohi.y : ohi.x);
-              const float bc = e ? bb.z : bb.x, bs = e ? bb.w : bb.y;
-              const float oc = e ? oo.z : oo.x, os = e ? oo.w : oo.y;
-              const float c = fmaf(bc, oc, -bs * os), sn = fmaf(bs, oc, bc * os);
+              const float c = e ? oo.z : oo.x, sn = e ? oo.w : oo.y;  // (cos, sin)(r theta_i)
               y0[r] = fmaf(lo, c, -hi * sn);
               y1[r] = fmaf(hi, c, lo * sn);
             }
