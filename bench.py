@@ -239,11 +239,11 @@ def run_reference(args):
     W = WORKLOAD
     per_seq = []
     for _ in range(args.warmup):
-        oracle_decode_sample(0.0, seed=99)
+        oracle_decode_sample(0.0, seed=99, rope=args.rope)
     threads = 1
     per_step_budget = min(5.0, 100.0 / max(1, args.steps))
     for s in range(args.steps):
-        t, n, threads = oracle_decode_sample(per_step_budget, seed=s)
+        t, n, threads = oracle_decode_sample(per_step_budget, seed=s, rope=args.rope)
         per_seq.append(t)
     step_s = float(np.mean(per_seq)) * W["batch"] * W["n_kv_heads"]
     value = W["batch"] / step_s
@@ -251,11 +251,14 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": W["name"], "batch": W["batch"], "seq_len": W["seq"], "n_q_heads": W["n_q_heads"],
+        "config": {"workload": W["name"] + ("-dq" if args.double_quant else "") + ("-prerope" if args.rope else ""),
+                   "batch": W["batch"], "seq_len": W["seq"], "n_q_heads": W["n_q_heads"],
                    "n_kv_heads": W["n_kv_heads"], "mode_k": W["mode_k"], "mode_v": W["mode_v"],
-                   "window": W["window"], "parallelism": "replicas"},
+                   "window": W["window"], "double_quant": bool(args.double_quant), "pre_rope_keys": bool(args.rope),
+                   "parallelism": "replicas"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"each step: oracle decode attention of >=1 sampled (batch, kv-head) "
+                         "sample": f"each step: oracle decode attention{' (pre-RoPE keys)' if args.rope else ''} "
+                                   f"of >=1 sampled (batch, kv-head) "
                                    f"sequence ({W['seq'] - 128} quantized + 128 window tokens, 4 q-heads), "
                                    f"scaled to {W['batch']}x{W['n_kv_heads']} sequences"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
