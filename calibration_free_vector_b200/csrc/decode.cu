@@ -1160,11 +1160,11 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
             xs[rr] = n2.y * INV_SQRT_D;
           }
         }
-        // u_hat k-step a times H_16 (independent products), then H_8 across the k-steps in fp32
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
+        // u_hat k-steps a and a + 4 times +-H_16: their sum and difference are the
+        // H_8 stage across bit 2 of the k-step, accumulated on the tensor cores;
+        // the stages across bits 0 and 1 follow in fp32
+        auto gather = [&](int a, uint32_t (&A)[4]) {
           const uint32_t code = __byte_perm(u4_word(cur.codes, a >> 1), 0u, (a & 1) ? sel_k1 : sel_k0);
-          uint32_t A[4];
           ldsm_x4(cbk_base + code * 128u, A);
           if constexpr (MK == NSN_MODE_2BIT) {
             A[0] = apply_signs(A[0], cur.ks0, 2 * a);
@@ -1172,11 +1172,22 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
             A[2] = apply_signs(A[2], cur.ks0, 2 * a + 1);
             A[3] = apply_signs(A[3], cur.ks1, 2 * a + 1);
           }
-          mma_zero(E[a][0], A, Hb[0][0], Hb[0][1]);
-          mma_zero(E[a][1], A, Hb[1][0], Hb[1][1]);
+        };
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          uint32_t A0[4], A1[4];
+          gather(a, A0);
+          gather(a + 4, A1);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            mma_zero(E[a][nt], A0, Hb[nt][0], Hb[nt][1]);
+            mma_full(E[a][nt], A1, Hb[nt][0], Hb[nt][1]);
+            mma_zero(E[a + 4][nt], A0, Hb[nt][0], Hb[nt][1]);
+            mma_full(E[a + 4][nt], A1, Hb[nt][0] ^ 0x80008000u, Hb[nt][1] ^ 0x80008000u);
+          }
         }
 #pragma unroll
-        for (int sstep = 1; sstep < 8; sstep <<= 1)
+        for (int sstep = 1; sstep < 4; sstep <<= 1)
 #pragma unroll
           for (int a = 0; a < 8; ++a)
             if (!(a & sstep))
