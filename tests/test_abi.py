@@ -116,6 +116,20 @@ def test_host_validation_without_gpu(lib):
     assert lib.nsn_append_residual(ctypes.byref(c), ctypes.byref(c2), 16, 16, 1, 0, 128, 16, 16, None) == 1
 
 
+@pytest.mark.parametrize("batch,heads,cap,window,hq", [(1, 2, 128, 128, 8), (4, 8, 4096, 128, 32),
+                                                        (3, 2, 1152, 0, 2), (16, 8, 32896, 128, 64)])
+def test_rope_workspace_is_decode_workspace_plus_logits(lib, batch, heads, cap, window, hq):
+    # layout (include/nsn.h): the decode workspace, then from a 256-byte boundary the
+    # K logits, batch * n_q_heads * rs_cap fp32 with rs_cap = capacity + window
+    # rounded up to 64 tokens
+    c = nsn.nsn_cache(batch, heads, cap, window, 2, 1, 16, 16, 16, 16, 16 if window else None, 16, 16, None)
+    ws = lib.nsn_decode_workspace_bytes(ctypes.byref(c), hq)
+    rope = lib.nsn_decode_rope_workspace_bytes(ctypes.byref(c), hq)
+    rs_cap = ((cap + window + 63) // 64) * 64
+    assert ws > 0
+    assert rope == ((ws + 255) // 256) * 256 + batch * hq * rs_cap * 4
+
+
 def test_host_codebook_matches_oracle(lib):
     for abs_mode in (False, True):
         ours = nsn.nsn_build_codebook_host(0x1234, 8192, 64, 8, abs_mode, 12)
