@@ -182,3 +182,54 @@ def oracle_cache_sequence(pool, x, n_prefill, n_total, cb, mode, window=128, dou
     seq = {"codes": cat("codes"), "signs": None if mode == 1 else cat("signs"), "s1": cat("s1"),
            "s2": cat("s2"), "o": np.stack([p["o"] for p in parts]), "gap": cat("gap"), "u": cat("u")}
     return seq, np.array(win).reshape(-1, 128)
+
+
+# ---------------------------------------------------------------------------
+# Shared set-up of the decode parity tests (plain and pre-RoPE keys)
+# ---------------------------------------------------------------------------
+def fill_cache(cache, contents):
+    """Writes per-(b, h) random contents into a Cache (test set-up, no math)."""
+    import torch
+    for (b, h), c in contents.items():
+        nq, nw = c["codes"].shape[0], c["window"].shape[0]
+        cache.codes[b, h, :nq] = torch.from_numpy(c["codes"])
+        if c["signs"] is not None:
+            cache.signs[b, h, :nq] = torch.from_numpy(c["signs"])
+        cache.norms[b, h, :nq, 0] = torch.from_numpy(c["s1"])
+        cache.norms[b, h, :nq, 1] = torch.from_numpy(c["s2"])
+        cache.means[b, h, :c["o"].shape[0]] = torch.from_numpy(c["o"])
+        if nw:
+            cache.window_buf[b, h, :nw] = torch.from_numpy(c["window"])
+        cache.n_quant[b, h] = nq
+        cache.n_window[b, h] = nw
+
+
+def oracle_seq(c):
+    """The same random contents in the oracle's layout (sign bits reordered)."""
+    f = lambda a: None if a is None else np.asarray(a, dtype=np.float64)  # noqa: E731
+    signs = None if c["signs"] is None else signs_to_natural(c["signs"])
+    return {"codes": c["codes"].astype(np.int64), "signs": signs, "s1": f(c["s1"]), "s2": f(c["s2"]),
+            "o": f(c["o"])}
+
+
+def oracle_pipeline(xk, xv, n_prefill, n_total, cbk, cbv, mk, mv, window):
+    """Oracle cache of one (b, h) after a prefill of n_prefill tokens and
+    appends up to n_total (flushes of the full window as fp16 blocks)."""
+    from oracle import nsn_oracle as orc
+    out = []
+    for x, cb, mode in ((xk, cbk, mk), (xv, cbv, mv)):
+        seq = orc.quantize_sequence(x[:n_prefill], cb, mode, 128, window)
+        codes, signs, s1, s2, o = [seq["codes"]], [seq["signs"]], [seq["s1"]], [seq["s2"]], [seq["o"]]
+        nq = seq["n_quant"]
+        win = list(orc.to_f16(x[nq:n_prefill]))
+        for t in range(n_prefill, n_total):
+            if len(win) == window:
+                blk = orc.quantize_block(np.array(win), cb, mode)
+                codes.append(blk["codes"]); signs.append(blk["signs"]); s1.append(blk["s1"])
+                s2.append(blk["s2"]); o.append(blk["o"][None])
+                win = []
+            win.append(orc.to_f16(x[t]))
+        out.append(({"codes": np.concatenate(codes), "signs": None if mode == 1 else np.concatenate(signs),
+                     "s1": np.concatenate(s1), "s2": np.concatenate(s2), "o": np.concatenate(o)},
+                    np.array(win).reshape(-1, 128)))
+    return out

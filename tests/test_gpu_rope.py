@@ -17,7 +17,7 @@ import torch
 from calibration_free_vector_b200 import nsn, synthetic
 from oracle import nsn_oracle as orc
 import nsn_testlib as tl
-from test_gpu_decode import fill_cache, oracle_seq, oracle_pipeline
+from nsn_testlib import fill_cache, oracle_seq, oracle_pipeline
 
 pytestmark = pytest.mark.gpu
 SCALE = 1.0 / math.sqrt(128)
