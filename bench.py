@@ -49,8 +49,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
 # DRAM bytes (read + write) per decode_kernel launch on this workload, from one
-# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum; command and numbers
-# in profiles/launches-decode_b16_32k_2bit.md), valid only for the sources the
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum of the launch list of
+# this workload, taken with --metrics and --clock-control none), valid only for the sources the
 # decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh,
 # comments and whitespace removed).
 # Any later change to those files makes the figure stale; the bench then reports null.

@@ -21,7 +21,7 @@ Sources (titles and sections of the pages that describe the method):
   [NW]  "New Quantization Technique Cuts LLM Memory Use Without Training Data",
         section "How NSNQuant Works" (the three NSN steps).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   * Hadamard is applied to every token before NSN (plain Sylvester matrix in
     natural order, no random signs).  NSN commutes with any per-token
     orthogonal map, so the order only moves o into the rotated domain.

@@ -102,3 +102,77 @@ def test_quantize_sequence_layout():
     b1 = orc.quantize_block(x[128:256], a, orc.MODE_2BIT)
     assert np.array_equal(qs["codes"][128:], b1["codes"])
     assert np.array_equal(qs["o"][1], b1["o"])
+
+
+def test_identity_codebook_over_several_blocks():
+    # Three quantization blocks (128, 128 and a partial 44 tokens), each NSN'd on
+    # its own, so every block has its own channel mean o_b.  With the exact u
+    # sub-vectors as the "codebook" and unrounded scalars, dequantize must give
+    # back every raw token, which only holds if token t reads the mean of its own
+    # block t // 128 ([TS] Metodologia 1: the byproducts s1, o, s2 reconstruct
+    # the tensor).  A per-block offset makes the blocks' means differ.
+    rng = np.random.default_rng(21)
+    d, n, blk = 128, 300, 128
+    xk = rng.standard_normal((n, d)) * 1.5
+    xv = rng.standard_normal((n, d))
+    for a in range(0, n, blk):
+        xk[a:a + blk] += rng.standard_normal(d) * 4.0
+        xv[a:a + blk] += rng.standard_normal(d) * 2.0
+
+    def identity_cache(x):
+        s1s, s2s, os_, us = [], [], [], []
+        for a in range(0, n, blk):
+            u, s1, o, s2 = orc.nsn(orc.rotate(x[a:a + blk]))
+            us.append(u)
+            s1s.append(s1)
+            s2s.append(s2)
+            os_.append(o)
+        cb = np.concatenate(us).reshape(-1, 8)
+        codes = np.arange(n * 16).reshape(n, 16)
+        return {"codes": codes, "signs": None, "s1": np.concatenate(s1s), "s2": np.concatenate(s2s),
+                "o": np.stack(os_)}, cb
+
+    kq, cbk = identity_cache(xk)
+    vq, cbv = identity_cache(xv)
+    assert kq["o"].shape == (3, d) and np.abs(kq["o"][0] - kq["o"][2]).max() > 0.1
+    for cache, cb, x in ((kq, cbk, xk), (vq, cbv, xv)):
+        xhat = orc.dequantize(cache["codes"], None, cache["s1"], cache["s2"], cache["o"], cb, orc.MODE_1BIT)
+        assert np.abs(xhat - x).max() < 1e-11
+    q = rng.standard_normal((4, d))
+    out = orc.decode_attention(q, kq, vq, np.zeros((0, d)), np.zeros((0, d)), cbk, cbv,
+                               orc.MODE_1BIT, orc.MODE_1BIT, 1 / np.sqrt(d))
+    assert np.abs(out - orc.attention(q, xk, xv, 1 / np.sqrt(d))).max() < 1e-10
+
+
+@pytest.mark.parametrize("mode", [orc.MODE_1BIT, orc.MODE_2BIT])
+def test_stored_s2_preserves_the_component_along_u(mode):
+    # [TS] Metodologia 3 (scale adjustment): the quantized vector is rescaled so
+    # that its component along the original vector is the original one.  In the
+    # original domain, with v_t = x_t - s1_t H o (the token without its block
+    # mean part, = s1 s2 H u), the reconstruction x_hat from the stored scalars
+    # must have no error along v_t: (x_hat_t - x_t) . v_t = 0 up to the fp16
+    # rounding of the stored s1, s2' and o.  Without the factor alpha the error
+    # along v_t is the full (u . u_hat - |u|^2) s2 s1^2, several percent of
+    # |v_t|^2 at these bit widths.
+    from scipy.linalg import hadamard
+
+    rng = np.random.default_rng(22)
+    d, n = 128, 128
+    x = rng.standard_normal((n, d))
+    ch = rng.choice(d, 5, replace=False)
+    x[:, ch] = 3.0 * (x[:, ch] + rng.standard_normal(5) * 4.0)
+    if mode == orc.MODE_2BIT:
+        cb = np.abs(rng.standard_normal((256, 8)))
+    else:
+        cb = rng.standard_normal((256, 8))
+    qb = orc.quantize_block(x, cb, mode)
+    xhat = orc.dequantize(qb["codes"], qb["signs"], qb["s1"], qb["s2"], qb["o"][None, :], cb, mode)
+    h = hadamard(d) / np.sqrt(d)
+    v = x - qb["s1"][:, None] * (qb["o"] @ h)[None, :]
+    along = np.einsum("td,td->t", xhat - x, v) / np.einsum("td,td->t", v, v)
+    assert np.abs(along).max() < 3e-3
+    # the same reconstruction with alpha left out errs along v_t by far more
+    raw = orc.quantize_block(x, cb, mode, scale_adjust=False)
+    xraw = orc.dequantize(raw["codes"], raw["signs"], raw["s1"], raw["s2"], raw["o"][None, :], cb, mode)
+    along_raw = np.einsum("td,td->t", xraw - x, v) / np.einsum("td,td->t", v, v)
+    assert np.median(np.abs(along_raw)) > 10 * np.abs(along).max()
