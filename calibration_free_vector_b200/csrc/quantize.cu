@@ -5,9 +5,9 @@
 // 2 (Hadamard), 3 (VQ with one global codebook, adaptive scale) and 4 (KIVI-style
 // residual that is flushed into the quantized part when full).
 //
-// One CTA of 256 threads quantizes one block of <= 128 tokens of one (batch,
-// kv-head); the adjacent lanes 2t, 2t+1 own token t (64 dims, 8 sub-vectors
-// each).  Per block:
+// One CTA of 256 threads quantizes blocks of <= 128 tokens of one (batch,
+// kv-head) at a time (a persistent loop over blocks on prefill); the adjacent
+// lanes 2t, 2t+1 own token t (64 dims, 8 sub-vectors each) during NSN.  Per block:
 //   r      = column mean of the raw tokens (fp64 sum, stored as fp32)
 //   d_t    = FWHT(x_t - r)                 fp32, in registers (exact algebra:
 //   w_t    = d_t + FWHT(r)                 FWHT is linear; FWHT(r) in fp64)
@@ -19,16 +19,25 @@
 // offsets (outliers) out of the fp32 rounding, so u carries fp32 precision
 // relative to the token-varying part that survives the shift step.
 //
-// Nearest codeword: exhaustive scores score_k = u.c_k - ||c_k||^2/2 of all 256
-// codewords on the tensor cores (a token's 16 sub-vectors are the rows of one
-// m16n8k16 tile, K = the fp16 hi and lo parts of u against the fp16 codebook
-// twice, the bias as the accumulator's start), the best group of 8 codewords per
-// sub-vector, then the 8 codewords of that group rescanned in sequential fp32.
-// Whenever a rival lies within the error bounds of the best (the fp32 bound inside
-// the group, that plus a wide tensor-accumulation bound outside it), the
-// sub-vector is re-decided exactly in fp64 by a whole warp over all codewords
-// inside the bound (ties to the lowest index).  The stored code is therefore the
-// exact nearest codeword of the fp32 u.
+// Nearest codeword, on the 5th-generation tensor cores: the 2048 sub-vectors of a
+// block form 16 tiles of 128 rows (8 tokens x 16 sub-vectors).  Per tile two
+// tcgen05.mma (M = 128, N = 256 codewords, K = 16, fp16 operands from shared
+// memory, fp32 accumulators in tensor memory) write every score
+//   score_k = a . c_k - ||c_k||^2 / 2        (a = u, or |u| in 2-bit mode)
+// The first MMA writes the bias (A = [1, 1, 0...], B = the fp16 hi and lo parts of
+// -||c_k||^2/2), the second adds K = [a_hi | a_lo] (the fp32 a split into two fp16
+// parts, exact to 2^-22) times [c | c] (the codebook in fp16).  Each TMEM lane
+// holds one sub-vector's 256 scores; a warp pair reads them back with tcgen05.ld
+// (each warp half of the columns) and keeps, with three-input max trees, the best
+// and second-best maxima of the groups of 8 codewords (the group number rides in
+// the low mantissa bits).  The 8 codewords of the winning group are then rescanned
+// in sequential fp32.  Whenever a rival lies within the error bounds of the best
+// (the fp32 bound inside the group, that plus a wide tensor-accumulation bound
+// outside it), the sub-vector is re-decided exactly in fp64 by a whole warp over
+// all codewords inside the bound (ties to the lowest index).  The stored code is
+// therefore the exact nearest codeword of the fp32 u.
+
+#include <algorithm>
 
 #include "nsn_common.cuh"
 #include "nsn_launch.h"
@@ -43,21 +52,7 @@ __device__ __forceinline__ double lds_f64(const double* p) {
   return r;
 }
 
-// ldmatrix / mma.sync / three-input max for the tensor-core codeword scores.
 __device__ __forceinline__ uint32_t q_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-__device__ __forceinline__ void q_ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
-// d += A (16 x 16) * B (16 x 8) with both K halves of B equal to `b`
-__device__ __forceinline__ void q_mma_bb(float (&d)[4], const uint32_t (&a)[4], uint32_t b) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %8}, "
-      "{%0, %1, %2, %3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b));
-}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -65,32 +60,108 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 }
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
 
+// ---------------------------------------------------------------------------
+// tcgen05 (5th-generation tensor core) helpers
+// ---------------------------------------------------------------------------
+// Shared-memory operand layout of one [rows][16] fp16 tile, K-major without
+// swizzle: 8-row x 16-byte core matrices; the two 8-element K halves of an 8-row
+// group are 128 B apart (leading byte offset), consecutive 8-row groups 256 B apart
+// (stride byte offset).
+__host__ __device__ constexpr uint32_t kmaj_off(int row, int k) {
+  return (uint32_t)((row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
+}
+// Matrix descriptor: start address, leading / stride byte offsets (16-byte units),
+// descriptor version 1 (sm_100), no swizzle.
+__device__ __forceinline__ uint64_t tc_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// Instruction descriptor of kind::f16: fp32 accumulator (bit 4), fp16 A and B,
+// both K-major, N = 256 (bits 17-22: N >> 3), M = 128 (bits 24-28: M >> 4).
+constexpr uint32_t TC_IDESC = (1u << 4) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr int TC_COLS = 256;  // tensor-memory columns of one CTA: the 256 fp32 scores of 128 rows
+
+__device__ __forceinline__ void tc_mma(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile("{.reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;}"
+               :: "r"(dtmem), "l"(adesc), "l"(bdesc), "r"(TC_IDESC), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(mbar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Bounded wait on an mbarrier phase; false after `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, int limit) {
+  for (int it = 0; it < limit; ++it) {
+    uint32_t done;
+    asm volatile("{.reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p;}"
+                 : "=r"(done) : "r"(mbar), "r"(parity) : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (one lane per thread).
+// The registers are valid only after tc_wait_ld(); tc_regs_ready() then keeps the
+// compiler from reading them before the wait.
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+               "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                 "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+                 "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                 "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_regs_ready(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                 "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
 constexpr int QTHREADS = 2 * BLK;  // two threads per token
 constexpr int HD = D / 2;           // dims per thread
 constexpr int HSUB = NSUB / 2;      // sub-vectors per thread
+constexpr int CB_ROWS = NCODES + NCODES / 8;  // codeword table rows: codeword k at k + k / 8
+__host__ __device__ constexpr int cb_row(int k) { return k + (k >> 3); }
+constexpr int MBAR_POLLS = 1 << 22;  // bounded wait for the MMAs of one tile
 
 struct QuantSmem {
-  // codebook (fp32), rows padded to 48 bytes: lanes gathering random rows (the
-  // group rescan, the adaptive scale) spread over all eight 16-byte bank groups
-  alignas(16) float cb[NCODES][SUB + 4];
-  alignas(16) float bias[NCODES];      // -||c_k||^2 / 2
-  alignas(16) float biasq[NCODES];     // the same, per (group G of 32 codes, quad lane p): codes 32G + 8i + 2p + e at 32G + 8p + 2i + e
-  alignas(16) float cnorm[4];          // [0] = max ||c||, [1] = max ||c||^2, [2] = max ||c - fp16(c)|| (rounded up)
-  alignas(16) __half cbh[NCODES][SUB]; // codebook rounded to fp16, dims in the order 0 4 1 5 2 6 3 7 (tensor-core operand)
+  // ---- operands of the tensor-core scores (staged once per CTA) ----
+  alignas(1024) unsigned char bop[NCODES * 32];   // B: codebook fp16 [c | c], K-major canonical layout
+  alignas(128) unsigned char bop2[NCODES * 16];   // B of the bias MMA: per codeword [b_hi, b_lo, 0 x 6]; K half 1 aliases K half 0
+  alignas(128) unsigned char aop2[256];           // A of the bias MMA: one core matrix of rows [1, 1, 0 ...] + a zero one
+  alignas(128) unsigned char aop[2][BLK * 32];    // A: [a_hi | a_lo] of the 128 rows of a tile (double-buffered)
+  // ---- codebook for the exact arithmetic (rows padded so that lanes of random groups spread over banks) ----
+  alignas(16) __half cbt[CB_ROWS][SUB];           // codeword k at row cb_row(k), fp16 (used when the codebook is fp16-exact)
+  alignas(16) float cbias[CB_ROWS];               // -||c_k||^2 / 2 (fp32, sequential) at row cb_row(k)
+  alignas(16) float cnorm[4];                     // [0] max ||c||, [1] max ||c||^2, [2] max ||c - fp16(c)|| (rounded up)
+  alignas(8) unsigned long long mbar;             // MMA completion barrier
+  uint32_t tmem;                                  // tensor-memory base address of this CTA
+  int nflag;
+  // ---- per block ----
   alignas(16) double rr[BLK];          // 1 / ||x_t|| (0 for a zero token)
   alignas(16) double s1[BLK];          // per-token s1 and s2 (fp64) until the final store
   alignas(16) double s2[BLK];
   alignas(16) double big_r[D];         // FWHT(r) in fp64
   alignas(16) double o[D];             // D_c = mean_t(d_t,c rr_t) (the token-varying part of o)
-  alignas(16) double part[2][D];       // per-half column partial sums
-  alignas(16) double dev_part[2];      // per-half sums of rr_t - rr_0
   alignas(16) float r[D];              // column mean of raw tokens (fp32)
-  alignas(16) float tile[BLK][D + 4];  // raw tokens, then d_t rows, then u rows; padded by 16 B
-  alignas(16) float thr[BLK][NSUB + 1];  // per (token, sub-vector) threshold of the exact re-decision
+  alignas(16) float tile[BLK][D + 4];  // raw tokens, then d_t rows, then u rows (|u| in 2-bit mode); padded by 16 B
+  union {                              // NSN column sums, then the search's warp-pair exchanges
+    struct {
+      double part[2][D];               // per-half column partial sums
+      double dev_part[2];              // per-half sums of rr_t - rr_0
+    };
+    struct {
+      float2 xch1[2][BLK];             // group maxima (best key, second) per half
+      float4 xch2[BLK];                // rescan (best, second, index) of the upper half
+    };
+  };
   alignas(16) uint8_t code[BLK][NSUB]; // chosen codes
-  alignas(16) uint8_t grp[BLK][NSUB];  // winning (group of 8 codes, lane) of the tensor-core scores
   alignas(16) uint16_t flag[BLK * NSUB];  // (token, sub-vector) pairs for the exact re-decision
-  int nflag;
   alignas(16) uint32_t sgn[BLK][4];    // packed sign bits (2-bit mode)
   // double quantization
   alignas(16) double ofull[D];         // o of the block (fp64) until its levels are formed
@@ -98,6 +169,36 @@ struct QuantSmem {
   alignas(16) double dq[2][3];         // (lo, hi, step) of s1 and of o
   alignas(16) uint8_t lev[2][BLK];     // 4-bit levels of s1 (per token) and of o (per channel)
 };
+
+// Tensor-memory allocation and the MMA barrier of one CTA (all QTHREADS threads).
+struct TcState {
+  uint32_t tmem;
+  uint32_t phase;
+};
+
+__device__ TcState tc_setup(QuantSmem& sm) {
+  const int t = threadIdx.x;
+  if (t == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(q_smem(&sm.mbar)));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if ((t >> 5) == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(q_smem(&sm.tmem)), "r"(TC_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return TcState{sm.tmem, 0u};
+}
+
+__device__ void tc_teardown(const TcState& tcs) {
+  tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tcs.tmem), "r"(TC_COLS));
+}
 
 // Destination of the stored scalars of one block: either fp16 (s1, alpha*s2) pairs
 // and fp16 o, or (double quantization) fp16 alpha*s2, 4-bit s1 and o levels and the
@@ -125,27 +226,45 @@ __device__ __forceinline__ BlockOut block_out(const CacheView& c, int64_t seq, i
   return o;
 }
 
-// Stages the codebook, its biases and norm bounds.  All QTHREADS threads.
+// Stages the codebook: the tensor-core operands (fp16 codebook, fp16 hi/lo bias,
+// the constant bias rows), the fp16 rows and fp32 biases of the exact arithmetic,
+// and the norm bounds.  All QTHREADS threads (one codeword each).
 __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook) {
   const int t = threadIdx.x;
-  for (int i = t; i < NCODES * SUB / 4; i += blockDim.x)
-    *reinterpret_cast<float4*>(&sm.cb[i >> 1][4 * (i & 1)]) = __ldg(reinterpret_cast<const float4*>(codebook) + i);
-  __syncthreads();
   float my_max = 0.f, my_dev = 0.f;
   for (int k = t; k < NCODES; k += blockDim.x) {
-    float s = 0.f, e = 0.f;
+    float c[SUB];
+    const float4 c0 = __ldg(reinterpret_cast<const float4*>(codebook + k * SUB));
+    const float4 c1 = __ldg(reinterpret_cast<const float4*>(codebook + k * SUB) + 1);
+    c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+    float ss = 0.f, e = 0.f;
+    __half ch[SUB];
 #pragma unroll
     for (int i = 0; i < SUB; ++i) {
-      s = fmaf(sm.cb[k][i], sm.cb[k][i], s);
-      const __half c16 = __float2half_rn(sm.cb[k][i]);
-      sm.cbh[k][i < 4 ? 2 * i : 2 * (i - 4) + 1] = c16;  // K order of the MMA: dims p, p + 4 at slots 2p, 2p + 1
-      const float d = sm.cb[k][i] - __half2float(c16);
-      e = fmaf(d, d, e);
+      ss = fmaf(c[i], c[i], ss);
+      ch[i] = __float2half_rn(c[i]);
+      const float dlt = c[i] - __half2float(ch[i]);
+      e = fmaf(dlt, dlt, e);
     }
-    sm.bias[k] = -0.5f * s;
-    sm.biasq[(k & ~31) + 8 * ((k >> 1) & 3) + 2 * ((k >> 3) & 3) + (k & 1)] = -0.5f * s;
-    my_max = fmaxf(my_max, s);
+    const float bias = -0.5f * ss;
+    const int row = cb_row(k);
+    *reinterpret_cast<uint4*>(&sm.cbt[row][0]) = *reinterpret_cast<const uint4*>(ch);
+    sm.cbias[row] = bias;
+    // B operand: K = 0..7 and 8..15 both hold the codeword (multiplied by a_hi and a_lo)
+    *reinterpret_cast<uint4*>(sm.bop + kmaj_off(k, 0)) = *reinterpret_cast<const uint4*>(ch);
+    *reinterpret_cast<uint4*>(sm.bop + kmaj_off(k, 8)) = *reinterpret_cast<const uint4*>(ch);
+    // bias operand: (b_hi, b_lo) with b_hi + b_lo = bias to 2^-22 relative
+    const __half bh = __float2half_rn(bias);
+    const __half bl = __float2half_rn(bias - __half2float(bh));
+    uint4 brow = make_uint4(0u, 0u, 0u, 0u);
+    brow.x = (uint32_t)__half_as_ushort(bh) | ((uint32_t)__half_as_ushort(bl) << 16);
+    *reinterpret_cast<uint4*>(sm.bop2 + (k >> 3) * 128 + (k & 7) * 16) = brow;
+    my_max = fmaxf(my_max, ss);
     my_dev = fmaxf(my_dev, e);
+  }
+  if (t < 16) {  // bias A operand: 8 rows [1, 1, 0, ...] (K half 0) and a zero core matrix (K half 1)
+    const uint32_t one2 = 0x3C003C00u;  // fp16 (1, 1)
+    *reinterpret_cast<uint4*>(sm.aop2 + 16 * t) = t < 8 ? make_uint4(one2, 0u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
   }
   my_max = warp_max(my_max);
   my_dev = warp_max(my_dev);
@@ -154,6 +273,7 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
     red[t >> 5][0] = my_max;
     red[t >> 5][1] = my_dev;
   }
+  fence_async_smem();  // operands written by the generic proxy, read by the tensor cores
   __syncthreads();
   if (t == 0) {
     float m = 0.f, e = 0.f;
@@ -167,6 +287,26 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
     sm.cnorm[2] = e > 0.f ? sqrtf(e) * 1.001f : 0.f;  // 0 for a codebook of fp16 values
   }
   __syncthreads();
+}
+
+// Codeword k as fp32: from the fp16 table when the codebook is fp16-exact (then
+// identical to the fp32 input), else from the fp32 codebook in global memory.
+__device__ __forceinline__ void codeword(const QuantSmem& sm, const float* __restrict__ cb_global, bool f16tab,
+                                         int k, float (&c)[SUB]) {
+  if (f16tab) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(&sm.cbt[cb_row(k)][0]);
+    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h[i]);
+      c[2 * i] = f.x;
+      c[2 * i + 1] = f.y;
+    }
+  } else {
+    const float4 c0 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB));
+    const float4 c1 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB) + 1);
+    c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+  }
 }
 
 __device__ __forceinline__ double shfl_pair_sum(double x) { return x + __shfl_xor_sync(0xffffffffu, x, 1); }
@@ -229,13 +369,183 @@ __device__ void store_double_quant(QuantSmem& sm, int n, const BlockOut& bo) {
   }
 }
 
+// Nearest codeword of the sub-vectors of one block (rows of sm.tile: a = u, or |u|
+// in 2-bit mode; rows of tokens past n are zero), written to sm.code.  Sub-vectors
+// whose decision lies within the error bounds are appended to sm.flag for the
+// exact re-decision.  All QTHREADS threads.
+//
+// Tile t = tokens 8t .. 8t+7: row L (TMEM lane L) = token 8t + L/16, sub-vector L%16.
+// Warp w reads TMEM lanes 32(w%4) .. 32(w%4)+31 and columns 128(w/4) .. +127, so
+// warps w and w+4 form a pair over the same rows.  Per tile:
+//   (1) thread 0 issues the bias MMA (D = b_hi + b_lo) and the score MMA
+//       (D += [a_hi | a_lo] [c | c]) and commits them to the barrier;
+//   (2) meanwhile every thread writes its half of the next tile's A rows;
+//   (3) after the barrier, each warp reads its 128 scores per row in chunks of 32
+//       and keeps the best and second-best of its 16 group maxima (group = 8
+//       consecutive codewords; the group number replaces the 5 low mantissa bits,
+//       so the maximum carries its group);
+//   (4) the pair merges its halves (both sides get the best group G and the best
+//       maximum among the other groups), thread 0 issues the next tile's MMAs,
+//       and each side rescans 4 codewords of group G in sequential fp32;
+//   (5) the lower warp merges the rescans and applies the decision bounds:
+//       the sequential fp32 score is within gamma_9 (max||c||^2 + ||a|| max||c||)
+//       of the exact one; the tensor score within 2^-16 (sum |a_i c_i| + |bias|)
+//       (accumulation order and rounding inside the MMA are the hardware's, so the
+//       bound is taken wide: 17 terms of at most 2^-24 relative error each need
+//       about 2^-19.9) plus ||a|| ||c - fp16(c)|| for a codebook that is not
+//       fp16-representable; the group number adds at most 32 ulp to a maximum.
+//       A rival inside the group within twice the fp32 bound, or another group's
+//       maximum within the fp32 plus the tensor bound, flags the sub-vector.
+__device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restrict__ cb_global, int n,
+                             int32_t* status) {
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int q = warp & 3, hf = warp >> 2;
+  const int L = 32 * q + lane;
+  const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1], cdel = sm.cnorm[2];
+  const bool f16tab = cdel == 0.f;
+  constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
+  constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
+  const uint32_t taddr = tcs.tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * hf);
+  const uint64_t db = tc_desc(q_smem(sm.bop), 128, 256);
+  const uint64_t da2 = tc_desc(q_smem(sm.aop2), 128, 0);  // every 8-row group reads the same [1, 1, 0...] rows
+  const uint64_t db2 = tc_desc(q_smem(sm.bop2), 0, 128);  // K half 1 re-reads K half 0 (times A's zero half)
+  const uint32_t mbar = q_smem(&sm.mbar);
+  const int ntiles = (n + 7) >> 3;
+
+  auto build_a = [&](int tile, float (&a)[SUB]) {
+    const int tkk = 8 * tile + (L >> 4), j = L & 15;
+    const float4 a0 = *reinterpret_cast<const float4*>(&sm.tile[tkk][SUB * j]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&sm.tile[tkk][SUB * j + 4]);
+    a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
+    a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+    uint32_t w[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const __half2 hh = __floats2half2_rn(a[2 * p], a[2 * p + 1]);
+      if (hf == 0) {
+        w[p] = h2_bits(hh);
+      } else {
+        const float2 back = __half22float2(hh);
+        w[p] = h2_bits(__floats2half2_rn(a[2 * p] - back.x, a[2 * p + 1] - back.y));
+      }
+    }
+    *reinterpret_cast<uint4*>(sm.aop[tile & 1] + kmaj_off(L, 8 * hf)) = make_uint4(w[0], w[1], w[2], w[3]);
+  };
+  auto issue = [&](int tile) {
+    tc_mma(tcs.tmem, da2, db2, 0u);
+    tc_mma(tcs.tmem, tc_desc(q_smem(sm.aop[tile & 1]), 128, 256), db, 1u);
+    tc_commit(mbar);
+  };
+
+  float a[SUB], an[SUB];
+  build_a(0, a);
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (t == 0) issue(0);
+#pragma unroll 1
+  for (int tile = 0; tile < ntiles; ++tile) {
+    if (tile + 1 < ntiles) {
+      build_a(tile + 1, an);
+      fence_async_smem();
+    }
+    if (!mbar_wait(mbar, tcs.phase, MBAR_POLLS) && lane == 0 && status) atomicOr(status, 2);
+    tcs.phase ^= 1u;
+    tc_fence_after();
+
+    // (3) best and second-best group maxima of this warp's 128 columns
+    float b1 = -INFINITY, b2 = -INFINITY;
+    uint32_t r[32];
+    tc_ld32(taddr, r);
+    tc_wait_ld();
+    tc_regs_ready(r);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t rn[32];
+      if (c < 3) tc_ld32(taddr + 32 * (c + 1), rn);
+      float key[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float m = max3f(max3f(__uint_as_float(r[8 * g]), __uint_as_float(r[8 * g + 1]), __uint_as_float(r[8 * g + 2])),
+                              max3f(__uint_as_float(r[8 * g + 3]), __uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5])),
+                              fmaxf(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7])));
+        key[g] = __uint_as_float((__float_as_uint(m) & ~31u) | (uint32_t)(16 * hf + 4 * c + g));
+      }
+      const float h01 = fmaxf(key[0], key[1]), l01 = fminf(key[0], key[1]);
+      const float h23 = fmaxf(key[2], key[3]), l23 = fminf(key[2], key[3]);
+      const float hi = fmaxf(h01, h23);
+      const float lo = max3f(l01, l23, fminf(h01, h23));
+      b2 = max3f(b2, lo, fminf(b1, hi));
+      b1 = fmaxf(b1, hi);
+      if (c < 3) {
+        tc_wait_ld();
+        tc_regs_ready(rn);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = rn[i];
+      }
+    }
+
+    // (4) merge the pair's halves; the scores are read, so the next tile may start
+    sm.xch1[hf][L] = make_float2(b1, b2);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0 && tile + 1 < ntiles) issue(tile + 1);
+    const float2 o1 = sm.xch1[hf ^ 1][L];
+    const float m1 = fmaxf(b1, o1.x);
+    const float m2 = max3f(b2, o1.y, fminf(b1, o1.x));
+    const int G = (int)(__float_as_uint(m1) & 31u);
+    float best = -INFINITY, second = -INFINITY;
+    int idx = 8 * G + 4 * hf;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int k = 8 * G + 4 * hf + i;
+      float c[SUB];
+      codeword(sm, cb_global, f16tab, k, c);
+      float sc = sm.cbias[cb_row(k)];
+#pragma unroll
+      for (int d = 0; d < SUB; ++d) sc = fmaf(a[d], c[d], sc);
+      const float lo = fminf(best, sc);
+      idx = (sc > best) ? k : idx;
+      best = fmaxf(best, sc);
+      second = fmaxf(second, lo);
+    }
+    if (hf == 1) sm.xch2[L] = make_float4(best, second, __int_as_float(idx), 0.f);
+    __syncthreads();
+
+    // (5) decision and bounds (lower warp of the pair)
+    if (hf == 0) {
+      const float4 o2 = sm.xch2[L];
+      second = max3f(second, o2.y, fminf(best, o2.x));
+      idx = (o2.x > best) ? __float_as_int(o2.z) : idx;  // the upper half holds the larger indices
+      best = fmaxf(best, o2.x);
+      float na = 0.f;
+#pragma unroll
+      for (int d = 0; d < SUB; ++d) na = fmaf(a[d], a[d], na);
+      na = sqrtf(na) * 1.0001f;
+      const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
+      const float m_tc = (TC_REL * (1.001f * na * cmax + 0.5f * cmax2) + na * cdel) * 1.01f + 1.2e-7f;
+      const float other = m2 + fabsf(m2) * 3.82e-6f;  // + 32 ulp: the group number in the low bits
+      const int tkk = 8 * tile + (L >> 4), j = L & 15;
+      sm.code[tkk][j] = (uint8_t)idx;
+      const bool need = second >= best - margin || other >= best - 0.5f * margin - m_tc;
+      if (need && tkk < n) sm.flag[atomicAdd(&sm.nflag, 1)] = (uint16_t)(tkk * NSUB + j);
+    }
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) a[i] = an[i];
+  }
+  __syncthreads();
+}
+
 // Quantizes one block of n (1..128) tokens with QTHREADS threads: thread
 // t = 2 tk + h works on token tk, dims 64h .. 64h+63 (sub-vectors 8h .. 8h+7).
 // Rows are at src + row0 + tk*row_stride (elements).  Output pointers are
 // already offset to the block's first token (codes, signs, norms) and to its
 // mean row (means).
 template <int DT, int MODE>
-__device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, int64_t row0,
+__device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __restrict__ cb_global,
+                                   const void* __restrict__ src, int64_t row0,
                                    int64_t row_stride, int n, uint8_t* __restrict__ codes,
                                    uint8_t* __restrict__ signs, const CacheView& cv, int64_t seq,
                                    int64_t tok0, int blk, int scale_adjust) {
@@ -449,226 +759,64 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
     if (h == 0) *reinterpret_cast<uint4*>(&sm.sgn[tk][0]) = make_uint4(sgn[0], sgn[1], sgn[2], sgn[3]);
   }
 
-  // ---- nearest codeword: tensor-core scores, exact decision ------------------
-  // score_k = a.c_k - ||c_k||^2 / 2 (maximised) for every sub-vector a.
-  // (1) The 16 sub-vectors of a token are the 16 rows of one m16n8k16 tile with
-  //     K = [a_hi | a_lo] (the fp32 a split into two fp16 parts, exact to 2^-22)
-  //     against B = [c | c] (the codebook in fp16) and the bias as the
-  //     accumulator's start: 32 MMAs give the 256 scores of 16 sub-vectors.
-  // (2) Lane p of a quad sees codes 8n + 2p, 8n + 2p + 1 of every n-tile n: a
-  //     running max per group of 4 n-tiles (8 codes), then the best and
-  //     second-best group maxima and the best group, merged over the quad.
-  // (3) The owner lane rescans the 8 codes of the winning group in sequential
-  //     fp32 (the arithmetic of the exact path below) for the code (lowest index
-  //     on ties) and the in-group runner-up.
-  // (4) When the runner-up -- another group's tensor score or an fp32 score
-  //     inside the group -- comes within the error bounds of the best, a whole
-  //     warp re-decides the sub-vector exactly in fp64.
-  // Error bounds: the sequential fp32 score is within gamma_9 (max||c||^2 +
-  // ||a|| max||c||) of the exact one.  The tensor score's error is bounded by
-  // TC_REL (sum |a_i c_i| + |bias|) for the accumulation inside the MMA (its
-  // order and rounding are the hardware's, so the bound is taken wide: 2^-16
-  // against 17 terms of at most 2^-24 relative each), plus ||a|| ||c - fp16(c)||
-  // for a codebook that is not fp16-representable.
-  const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1], cdel = sm.cnorm[2];
-  constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
-  constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
-  const int warp = t >> 5, lane = t & 31, qg = lane >> 2, qp = lane & 3;
-  // (1) this warp's 16 tokens x 16 sub-vectors as rows of 8 fp32 (the exact
-  // search operand a), in the warp's own 16 tile rows (free since the column
-  // sums).  Row r of token m sits at R = 16 m + (r ^ (m & 3)) and its two 16-byte
-  // halves (dims 0-3, 4-7) swap when bit 2 xor bit 3 of R is set: the 8 rows of
-  // an ldmatrix fetch and the 8 rows of a store phase (4 tokens x 2 halves of the
-  // sub-vectors) both land in 8 different 16-byte bank groups.  The rows stay
-  // there for the rescan, the exact path and the adaptive scale.
-  auto a_phys = [](int m, int r) { return 16 * m + (r ^ (m & 3)); };
-  auto a_flip = [](int R) { return ((R >> 2) ^ (R >> 3)) & 1; };
-  auto urow = [&](int tok, int j, int half) -> const float4* {
-    const unsigned char* base = reinterpret_cast<const unsigned char*>(&sm.tile[16 * (tok >> 4)][0]);
-    const int R = a_phys(tok & 15, j);
-    return reinterpret_cast<const float4*>(base + R * 32 + 16 * (half ^ a_flip(R)));
-  };
-  unsigned char* arow = reinterpret_cast<unsigned char*>(&sm.tile[16 * warp][0]);
-  {
-    const int m_own = lane >> 1;
+  // ---- u rows (|u| in 2-bit mode) to shared memory; zeros past the n tokens --
+  // The raw tile and the d_t rows are no longer read (the column sums are done).
 #pragma unroll
-    for (int jj = 0; jj < HSUB; ++jj) {
-      const int R = a_phys(m_own, HSUB * h + jj), sw = a_flip(R);
-      const float4 lo4 = valid ? make_float4(v[8 * jj], v[8 * jj + 1], v[8 * jj + 2], v[8 * jj + 3])
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 hi4 = valid ? make_float4(v[8 * jj + 4], v[8 * jj + 5], v[8 * jj + 6], v[8 * jj + 7])
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<float4*>(arow + R * 32 + 16 * sw) = lo4;
-      *reinterpret_cast<float4*>(arow + R * 32 + 16 * (sw ^ 1)) = hi4;
-    }
-  }
-  __syncwarp();
-  // (2) scores and group maxima, two tokens (m-tiles) at a time sharing the
-  // codebook fragments.  ldmatrix of the fp32 rows gives lane (g, p) dims p and
-  // p + 4 of rows g and g + 8; their fp16 hi and lo parts are the A fragment in
-  // the K order of the permuted fp16 codebook.
-  {
-    const uint32_t abase = q_smem(arow);
-    const uint32_t cb_lane = q_smem(&sm.cbh[0][0]) + 16u * (uint32_t)lane;  // x4: n-tiles 4G .. 4G + 3
-    const int arow_l = (lane & 7) + 8 * ((lane >> 3) & 1), ahalf = lane >> 4;
-#pragma unroll 1
-    for (int mp = 0; mp < 8; ++mp) {
-      uint32_t A[2][4];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int R = a_phys(2 * mp + q, arow_l);
-        uint32_t w[4];
-        q_ldsm_x4(abase + (uint32_t)(R * 32 + 16 * (ahalf ^ a_flip(R))), w);
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {  // row g (words 0, 2) and row g + 8 (words 1, 3)
-          const float x0 = __uint_as_float(w[rr]), x1 = __uint_as_float(w[rr + 2]);
-          const __half2 hh = __floats2half2_rn(x0, x1);
-          const float2 hf = __half22float2(hh);
-          A[q][rr] = h2_bits(hh);
-          A[q][2 + rr] = h2_bits(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
-        }
-      }
-      float b1[2][2], b2[2][2];
-      int bg[2][2];
-#pragma unroll
-      for (int q = 0; q < 2; ++q)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          b1[q][r] = -INFINITY;
-          b2[q][r] = -INFINITY;
-          bg[q][r] = 0;
-        }
-#pragma unroll
-      for (int G = 0; G < NCODES / 32; ++G) {
-        uint32_t B4[4];
-        q_ldsm_x4(cb_lane + 512u * (uint32_t)G, B4);
-        const float4 bz01 = *reinterpret_cast<const float4*>(&sm.biasq[32 * G + 8 * qp]);
-        const float4 bz23 = *reinterpret_cast<const float4*>(&sm.biasq[32 * G + 8 * qp + 4]);
-        const float bzv[8] = {bz01.x, bz01.y, bz01.z, bz01.w, bz23.x, bz23.y, bz23.z, bz23.w};
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float d[4][4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            d[i][0] = bzv[2 * i]; d[i][1] = bzv[2 * i + 1]; d[i][2] = bzv[2 * i]; d[i][3] = bzv[2 * i + 1];
-            q_mma_bb(d[i], A[q], B4[i]);
-          }
-          // group maxima of rows g (0, 1) and g + 8 (2, 3) as shallow trees
-          const float gm[2] = {max3f(max3f(d[0][0], d[0][1], d[1][0]), max3f(d[1][1], d[2][0], d[2][1]),
-                                     fmaxf(d[3][0], d[3][1])),
-                               max3f(max3f(d[0][2], d[0][3], d[1][2]), max3f(d[1][3], d[2][2], d[2][3]),
-                                     fmaxf(d[3][2], d[3][3]))};
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const float lo = fminf(b1[q][r], gm[r]);
-            bg[q][r] = (gm[r] > b1[q][r]) ? G : bg[q][r];
-            b1[q][r] = fmaxf(b1[q][r], gm[r]);
-            b2[q][r] = fmaxf(b2[q][r], lo);
-          }
-        }
-      }
-      // merge over the quad: best group maximum, its (group, lane), and the
-      // largest maximum of every other group
-#pragma unroll
-      for (int q = 0; q < 2; ++q)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          float x1 = b1[q][r], x2 = b2[q][r];
-          int id = 4 * bg[q][r] + qp;
-#pragma unroll
-          for (int m = 1; m <= 2; m <<= 1) {
-            const float y1 = __shfl_xor_sync(0xffffffffu, x1, m), y2 = __shfl_xor_sync(0xffffffffu, x2, m);
-            const int yid = __shfl_xor_sync(0xffffffffu, id, m);
-            x2 = fmaxf(fmaxf(x2, y2), fminf(x1, y1));
-            id = (y1 > x1 || (y1 == x1 && yid < id)) ? yid : id;
-            x1 = fmaxf(x1, y1);
-          }
-          if (qp == 0) {
-            const int tok = 16 * warp + 2 * mp + q, j = qg + 8 * r;
-            sm.grp[tok][j] = (uint8_t)id;
-            sm.thr[tok][j] = x2;  // other groups' best tensor score, until (3) overwrites it
-          }
-        }
-    }
-  }
-  __syncwarp();
-  // (3) exact-arithmetic rescan of the winning group by the owner lane
-  uint32_t need = 0u;
-#pragma unroll 2
-  for (int jj = 0; jj < HSUB; ++jj) {
-    const int j = HSUB * h + jj;
-    const int id = sm.grp[tk][j];
-    const float other = sm.thr[tk][j];
-    const float4 u0 = *urow(tk, j, 0), u1 = *urow(tk, j, 1);
-    const float a[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    const int kbase = 32 * (id >> 2) + 2 * (id & 3);
-    float best = -INFINITY, second = -INFINITY;
-    int idx = kbase;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int k = kbase + 8 * i + e;
-        const float4 c0 = *reinterpret_cast<const float4*>(&sm.cb[k][0]);
-        const float4 c1 = *reinterpret_cast<const float4*>(&sm.cb[k][4]);
-        float sc = sm.bias[k];
-        sc = fmaf(a[0], c0.x, sc);
-        sc = fmaf(a[1], c0.y, sc);
-        sc = fmaf(a[2], c0.z, sc);
-        sc = fmaf(a[3], c0.w, sc);
-        sc = fmaf(a[4], c1.x, sc);
-        sc = fmaf(a[5], c1.y, sc);
-        sc = fmaf(a[6], c1.z, sc);
-        sc = fmaf(a[7], c1.w, sc);
-        const float lo = fminf(best, sc);
-        idx = (sc > best) ? k : idx;
-        best = fmaxf(best, sc);
-        second = fmaxf(second, lo);
-      }
-    float na = 0.f;
-#pragma unroll
-    for (int i = 0; i < SUB; ++i) na = fmaf(a[i], a[i], na);
-    na = sqrtf(na) * 1.0001f;
-    // a rival within twice the fp32 bound of the best may be the true best; so may
-    // another group whose tensor score is within the fp32 and tensor bounds
-    const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
-    const float m_tc = (TC_REL * (1.001f * na * cmax + 0.5f * cmax2) + na * cdel) * 1.01f;
-    sm.thr[tk][j] = best - margin;
-    sm.code[tk][j] = (uint8_t)idx;
-    need |= ((second >= best - margin || other >= best - 0.5f * margin - m_tc) ? 1u : 0u) << jj;
-  }
-
-  if (valid) {
-#pragma unroll 1
-    for (int jj = 0; jj < HSUB; ++jj)
-      if ((need >> jj) & 1u) sm.flag[atomicAdd(&sm.nflag, 1)] = (uint16_t)(tk * NSUB + HSUB * h + jj);
-  }
+  for (int c = 0; c < HD; c += 4)
+    *reinterpret_cast<float4*>(&sm.tile[tk][HD * h + c]) =
+        valid ? make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
 
-  // ---- (4) exact fp64 re-decision of the flagged sub-vectors, a warp each ----
-  // Candidates: codewords whose sequential fp32 score reaches the threshold
-  // (best - twice the fp32 bound); the winner by fp64 squared distance, ties to
-  // the lowest index.
+  // ---- nearest codeword on the tensor cores, exact decision -----------------
+  search_block(sm, tcs, cb_global, n, cv.status);
+
+  // ---- exact fp64 re-decision of the flagged sub-vectors, a warp each --------
+  // Each lane scores its 8 codewords in sequential fp32 (bias first, one fma per
+  // dim); candidates are the codewords within twice the fp32 bound of the best of
+  // these scores; the winner by fp64 squared distance, ties to the lowest index.
   {
+    const int warp = t >> 5, lane = t & 31;
+    const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1];
+    const bool f16tab = sm.cnorm[2] == 0.f;
+    constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
     const int nflag = sm.nflag;
 #pragma unroll 1
     for (int f = warp; f < nflag; f += QTHREADS / 32) {
       const int ftk = sm.flag[f] / NSUB, fj = sm.flag[f] % NSUB;
-      const float4 fa0 = *urow(ftk, fj, 0), fa1 = *urow(ftk, fj, 1);
+      const float4 fa0 = *reinterpret_cast<const float4*>(&sm.tile[ftk][SUB * fj]);
+      const float4 fa1 = *reinterpret_cast<const float4*>(&sm.tile[ftk][SUB * fj + 4]);
       const float a[8] = {fa0.x, fa0.y, fa0.z, fa0.w, fa1.x, fa1.y, fa1.z, fa1.w};
-      const float thr = sm.thr[ftk][fj];
+      float na = 0.f;
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) na = fmaf(a[i], a[i], na);
+      na = sqrtf(na) * 1.0001f;
+      const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
+      float sc[NCODES / 32];
+      float best = -INFINITY;
+#pragma unroll
+      for (int m = 0; m < NCODES / 32; ++m) {
+        const int k = lane + 32 * m;
+        float c[SUB];
+        codeword(sm, cb_global, f16tab, k, c);
+        float x = sm.cbias[cb_row(k)];
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) x = fmaf(a[i], c[i], x);
+        sc[m] = x;
+        best = fmaxf(best, x);
+      }
+      const float thr = warp_max(best) - margin;
       double bestd = INFINITY;
       int bi = NCODES;
-#pragma unroll 1
-      for (int k = lane; k < NCODES; k += 32) {
-        float sc = sm.bias[k];
 #pragma unroll
-        for (int i = 0; i < SUB; ++i) sc = fmaf(a[i], sm.cb[k][i], sc);
-        if (sc >= thr) {
+      for (int m = 0; m < NCODES / 32; ++m) {
+        if (sc[m] >= thr) {
+          const int k = lane + 32 * m;
+          float c[SUB];
+          codeword(sm, cb_global, f16tab, k, c);
           double dd = 0.0;
 #pragma unroll
           for (int i = 0; i < SUB; ++i) {
-            const double e = (double)a[i] - (double)sm.cb[k][i];
+            const double e = (double)a[i] - (double)c[i];
             dd = fma(e, e, dd);
           }
           if (dd < bestd) { bestd = dd; bi = k; }
@@ -687,23 +835,25 @@ __device__ void quantize_block_dev(QuantSmem& sm, const void* __restrict__ src, 
 
   // ---- adaptive scale: alpha = ||u||^2 / (u . u_hat) --------------------------
   double dot = 0.0, uu = 0.0;
+  {
+    const bool f16tab = sm.cnorm[2] == 0.f;
 #pragma unroll 4
-  for (int jj = 0; jj < HSUB; ++jj) {
-    const int j = HSUB * h + jj;
-    const int cj = sm.code[tk][j];
-    const float4 q0 = *reinterpret_cast<const float4*>(&sm.cb[cj][0]);
-    const float4 q1 = *reinterpret_cast<const float4*>(&sm.cb[cj][4]);
-    const float4 u0 = *urow(tk, j, 0), u1 = *urow(tk, j, 1);
-    const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    float dj = 0.f, uj = 0.f;
+    for (int jj = 0; jj < HSUB; ++jj) {
+      const int j = HSUB * h + jj;
+      float qv[SUB];
+      codeword(sm, cb_global, f16tab, sm.code[tk][j], qv);
+      const float4 u0 = *reinterpret_cast<const float4*>(&sm.tile[tk][SUB * j]);
+      const float4 u1 = *reinterpret_cast<const float4*>(&sm.tile[tk][SUB * j + 4]);
+      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      float dj = 0.f, uj = 0.f;
 #pragma unroll
-    for (int i = 0; i < SUB; ++i) {
-      dj = fmaf(uv[i], qv[i], dj);
-      uj = fmaf(uv[i], uv[i], uj);
+      for (int i = 0; i < SUB; ++i) {
+        dj = fmaf(uv[i], qv[i], dj);
+        uj = fmaf(uv[i], uv[i], uj);
+      }
+      dot += (double)dj;
+      uu += (double)uj;
     }
-    dot += (double)dj;
-    uu += (double)uj;
   }
   // halves combined in a fixed order (low half first) so both lanes agree bit for bit
   const double dot_o = __shfl_xor_sync(0xffffffffu, dot, 1), uu_o = __shfl_xor_sync(0xffffffffu, uu, 1);
@@ -751,22 +901,33 @@ __device__ __forceinline__ PrefillSplit prefill_split(const int32_t* __restrict_
   return {L, q, bad};
 }
 
+// Persistent: CTA i takes work items i, i + gridDim.x, ... of the (block, kv-head,
+// batch) list; the tensor memory, the barrier and the staged codebook live for the
+// whole launch.
 template <int DT, int MODE>
 __global__ void __launch_bounds__(QTHREADS, 2)
 quantize_prefill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int64_t sh, int q_tokens, int n_tokens,
-                        const int32_t* __restrict__ lengths, CacheView cv, const float* __restrict__ codebook) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+                        const int32_t* __restrict__ lengths, CacheView cv, const float* __restrict__ codebook,
+                        int nblk) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw);
-  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const PrefillSplit ps = prefill_split(lengths, b, n_tokens, q_tokens, cv.window_len);
-  const int n = min(BLK, ps.q - blk * BLK);
-  if (n <= 0) return;
+  TcState tcs = tc_setup(sm);
   stage_codebook(sm, codebook);
-  const int64_t seq = (int64_t)b * cv.n_kv_heads + h;
-  const int64_t tok0 = seq * cv.capacity + (int64_t)blk * BLK;
-  quantize_block_dev<DT, MODE>(sm, x, (int64_t)b * sb + (int64_t)blk * BLK * st + (int64_t)h * sh, st, n,
-                               cv.codes + tok0 * NSUB, MODE == NSN_MODE_2BIT ? cv.signs + tok0 * NSUB : nullptr,
-                               cv, seq, tok0, blk, cv.scale_adjust);
+  const int nwork = nblk * cv.n_kv_heads * cv.batch;
+#pragma unroll 1
+  for (int w = blockIdx.x; w < nwork; w += gridDim.x) {
+    const int blk = w % nblk, h = (w / nblk) % cv.n_kv_heads, b = w / (nblk * cv.n_kv_heads);
+    const PrefillSplit ps = prefill_split(lengths, b, n_tokens, q_tokens, cv.window_len);
+    const int n = min(BLK, ps.q - blk * BLK);
+    if (n <= 0) continue;
+    const int64_t seq = (int64_t)b * cv.n_kv_heads + h;
+    const int64_t tok0 = seq * cv.capacity + (int64_t)blk * BLK;
+    quantize_block_dev<DT, MODE>(sm, tcs, codebook,
+                                 x, (int64_t)b * sb + (int64_t)blk * BLK * st + (int64_t)h * sh, st, n,
+                                 cv.codes + tok0 * NSUB, MODE == NSN_MODE_2BIT ? cv.signs + tok0 * NSUB : nullptr,
+                                 cv, seq, tok0, blk, cv.scale_adjust);
+  }
+  tc_teardown(tcs);
 }
 
 // Prefill tail: copies tokens [q, L) of each sequence to the residual window
@@ -800,7 +961,7 @@ template <int DTN>
 __global__ void __launch_bounds__(QTHREADS, 2)
 append_kernel(CacheView kc, CacheView vc, const void* __restrict__ k_new, const void* __restrict__ v_new,
               int64_t sb, int64_t sh, const float* __restrict__ cbk, const float* __restrict__ cbv) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw);
   __shared__ int state[2];
   const bool is_v = blockIdx.z == 1;
@@ -817,16 +978,19 @@ append_kernel(CacheView kc, CacheView vc, const void* __restrict__ k_new, const 
       ok = false;
       if (t == 0 && c.status) atomicOr(c.status, 1);
     } else {
-      stage_codebook(sm, is_v ? cbv : cbk);
+      const float* cb = is_v ? cbv : cbk;
+      TcState tcs = tc_setup(sm);
+      stage_codebook(sm, cb);
       const int64_t tok0 = seq * c.capacity + nq;
       const int blk = nq / BLK;
       uint8_t* sg = c.mode == NSN_MODE_2BIT ? c.signs + tok0 * NSUB : nullptr;
       if (c.mode == NSN_MODE_2BIT)
-        quantize_block_dev<NSN_DTYPE_F16, NSN_MODE_2BIT>(sm, c.window, seq * c.window_len * D, D, BLK,
+        quantize_block_dev<NSN_DTYPE_F16, NSN_MODE_2BIT>(sm, tcs, cb, c.window, seq * c.window_len * D, D, BLK,
                                                          c.codes + tok0 * NSUB, sg, c, seq, tok0, blk, c.scale_adjust);
       else
-        quantize_block_dev<NSN_DTYPE_F16, NSN_MODE_1BIT>(sm, c.window, seq * c.window_len * D, D, BLK,
+        quantize_block_dev<NSN_DTYPE_F16, NSN_MODE_1BIT>(sm, tcs, cb, c.window, seq * c.window_len * D, D, BLK,
                                                          c.codes + tok0 * NSUB, sg, c, seq, tok0, blk, c.scale_adjust);
+      tc_teardown(tcs);
       nq += BLK;
       nw = 0;
     }
@@ -858,8 +1022,12 @@ static cudaError_t launch_prefill_t(const void* x, int64_t sb, int64_t st, int64
   if (e != cudaSuccess) return e;
   const int nblk = (q_tokens + BLK - 1) / BLK;
   if (nblk > 0) {
-    dim3 grid(nblk, cv.n_kv_heads, cv.batch);
-    quantize_prefill_kernel<DT, MODE><<<grid, QTHREADS, smem, s>>>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv, cb);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long nwork = (long long)nblk * cv.n_kv_heads * cv.batch;
+    const int grid = (int)std::min<long long>(nwork, 2LL * sms);  // two resident CTAs per SM
+    quantize_prefill_kernel<DT, MODE><<<grid, QTHREADS, smem, s>>>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv, cb,
+                                                                   nblk);
   }
   return cudaGetLastError();
 }
