@@ -44,14 +44,6 @@
 
 namespace nsn {
 
-// Shared-memory fp64 load that the compiler may not merge with other loads of the
-// same address (keeps 128-entry fp64 tables from being cached in registers).
-__device__ __forceinline__ double lds_f64(const double* p) {
-  double r;
-  asm volatile("ld.shared.f64 %0, [%1];" : "=d"(r) : "r"((unsigned)__cvta_generic_to_shared(p)));
-  return r;
-}
-
 __device__ __forceinline__ uint32_t q_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
@@ -125,8 +117,6 @@ __device__ __forceinline__ void tc_regs_ready(uint32_t (&r)[32]) {
 constexpr int QTHREADS = 2 * BLK;  // two threads per token
 constexpr int HD = D / 2;           // dims per thread
 constexpr int HSUB = NSUB / 2;      // sub-vectors per thread
-constexpr int CB_ROWS = NCODES + NCODES / 8;  // codeword table rows: codeword k at k + k / 8
-__host__ __device__ constexpr int cb_row(int k) { return k + (k >> 3); }
 constexpr int MBAR_POLLS = 1 << 22;  // bounded wait for the MMAs of one tile
 
 struct QuantSmem {
@@ -135,9 +125,13 @@ struct QuantSmem {
   alignas(128) unsigned char bop2[NCODES * 16];   // B of the bias MMA: per codeword [b_hi, b_lo, 0 x 6]; K half 1 aliases K half 0
   alignas(128) unsigned char aop2[256];           // A of the bias MMA: one core matrix of rows [1, 1, 0 ...] + a zero one
   alignas(128) unsigned char aop[2][BLK * 32];    // A: [a_hi | a_lo] of the 128 rows of a tile (double-buffered)
-  // ---- codebook for the exact arithmetic (rows padded so that lanes of random groups spread over banks) ----
-  alignas(16) __half cbt[CB_ROWS][SUB];           // codeword k at row cb_row(k), fp16 (used when the codebook is fp16-exact)
-  alignas(16) float cbias[CB_ROWS];               // -||c_k||^2 / 2 (fp32, sequential) at row cb_row(k)
+  // ---- codebook for the exact arithmetic, two interleaved replicas: replica p of codeword k = 8G + j (fp16,
+  // 16 B) at byte 256 G + 32 j + 16 p, so its 16-byte bank group is 2 j + p whatever the group; its bias
+  // -||c_k||^2/2 (fp32, sequential) at word 16 G + 2 j + p of cbias.  Lanes 4p .. 4p+3 of a quarter warp
+  // read replica p and rotate the codeword order by lane, so the 8 lanes of a phase hit 8 different bank
+  // groups (codewords) and 8 different banks (biases). ----
+  alignas(16) unsigned char cbtab[NCODES * 32];
+  alignas(16) float cbias[2 * NCODES];
   alignas(16) float cnorm[4];                     // [0] max ||c||, [1] max ||c||^2, [2] max ||c - fp16(c)|| (rounded up)
   alignas(8) unsigned long long mbar;             // MMA completion barrier
   uint32_t tmem;                                  // tensor-memory base address of this CTA
@@ -146,14 +140,15 @@ struct QuantSmem {
   alignas(16) double rr[BLK];          // 1 / ||x_t|| (0 for a zero token)
   alignas(16) double s1[BLK];          // per-token s1 and s2 (fp64) until the final store
   alignas(16) double s2[BLK];
-  alignas(16) double big_r[D];         // FWHT(r) in fp64
-  alignas(16) double o[D];             // D_c = mean_t(d_t,c rr_t) (the token-varying part of o)
   alignas(16) float r[D];              // column mean of raw tokens (fp32)
   alignas(16) float tile[BLK][D + 4];  // raw tokens, then d_t rows, then u rows (|u| in 2-bit mode); padded by 16 B
   union {                              // NSN column sums, then the search's warp-pair exchanges
     struct {
       double part[2][D];               // per-half column partial sums
       double dev_part[2];              // per-half sums of rr_t - rr_0
+      double big_r[D];                 // FWHT(r) in fp64
+      float big_rf[D];                 // FWHT(r) and D_c = mean_t(d_t,c rr_t) rounded to fp32 (the constant terms of z)
+      float dcf[D];
     };
     struct {
       float2 xch1[2][BLK];             // group maxima (best key, second) per half
@@ -162,7 +157,6 @@ struct QuantSmem {
   };
   alignas(16) uint8_t code[BLK][NSUB]; // chosen codes
   alignas(16) uint16_t flag[BLK * NSUB];  // (token, sub-vector) pairs for the exact re-decision
-  alignas(16) uint32_t sgn[BLK][4];    // packed sign bits (2-bit mode)
   // double quantization
   alignas(16) double ofull[D];         // o of the block (fp64) until its levels are formed
   alignas(16) double red[2][QTHREADS / 32][2];  // per-warp (min, max) of s1 and of o
@@ -247,9 +241,10 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
       e = fmaf(dlt, dlt, e);
     }
     const float bias = -0.5f * ss;
-    const int row = cb_row(k);
-    *reinterpret_cast<uint4*>(&sm.cbt[row][0]) = *reinterpret_cast<const uint4*>(ch);
-    sm.cbias[row] = bias;
+    *reinterpret_cast<uint4*>(sm.cbtab + 32 * k) = *reinterpret_cast<const uint4*>(ch);
+    *reinterpret_cast<uint4*>(sm.cbtab + 32 * k + 16) = *reinterpret_cast<const uint4*>(ch);
+    sm.cbias[2 * k] = bias;
+    sm.cbias[2 * k + 1] = bias;
     // B operand: K = 0..7 and 8..15 both hold the codeword (multiplied by a_hi and a_lo)
     *reinterpret_cast<uint4*>(sm.bop + kmaj_off(k, 0)) = *reinterpret_cast<const uint4*>(ch);
     *reinterpret_cast<uint4*>(sm.bop + kmaj_off(k, 8)) = *reinterpret_cast<const uint4*>(ch);
@@ -289,16 +284,17 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
   __syncthreads();
 }
 
-// Codeword k as fp32: from the fp16 table when the codebook is fp16-exact (then
-// identical to the fp32 input), else from the fp32 codebook in global memory.
-__device__ __forceinline__ void codeword(const QuantSmem& sm, const float* __restrict__ cb_global, bool f16tab,
-                                         int k, float (&c)[SUB]) {
+// Codeword k (fp32) and its bias -||c_k||^2/2: replica p of the shared fp16 table
+// when the codebook is fp16-representable (then the values are the fp32 input
+// exactly), else the fp32 codebook in global memory.
+__device__ __forceinline__ float codeword(const QuantSmem& sm, const float* __restrict__ cb_global, bool f16tab,
+                                          int k, int p, float (&c)[SUB]) {
   if (f16tab) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(&sm.cbt[cb_row(k)][0]);
-    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+    const uint4 raw = *reinterpret_cast<const uint4*>(sm.cbtab + 32 * k + 16 * p);
+    const __half2* hv = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h[i]);
+      const float2 f = __half22float2(hv[i]);
       c[2 * i] = f.x;
       c[2 * i + 1] = f.y;
     }
@@ -307,6 +303,7 @@ __device__ __forceinline__ void codeword(const QuantSmem& sm, const float* __res
     const float4 c1 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB) + 1);
     c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
   }
+  return sm.cbias[2 * k + p];
 }
 
 __device__ __forceinline__ double shfl_pair_sum(double x) { return x + __shfl_xor_sync(0xffffffffu, x, 1); }
@@ -498,21 +495,32 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
     const int G = (int)(__float_as_uint(m1) & 31u);
     float best = -INFINITY, second = -INFINITY;
     int idx = 8 * G + 4 * hf;
+    {
+      // this half's 4 codewords, in an order rotated by lane (bank-conflict free);
+      // the index keeps the lowest of equal scores explicitly
+      const int rep = (lane >> 2) & 1;
+      float cw[4][SUB], sc[4];
+      int kk[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int k = 8 * G + 4 * hf + i;
-      float c[SUB];
-      codeword(sm, cb_global, f16tab, k, c);
-      float sc = sm.cbias[cb_row(k)];
+      for (int i = 0; i < 4; ++i) {
+        kk[i] = 8 * G + 4 * hf + ((i + lane) & 3);
+        sc[i] = codeword(sm, cb_global, f16tab, kk[i], rep, cw[i]);
+      }
 #pragma unroll
-      for (int d = 0; d < SUB; ++d) sc = fmaf(a[d], c[d], sc);
-      const float lo = fminf(best, sc);
-      idx = (sc > best) ? k : idx;
-      best = fmaxf(best, sc);
-      second = fmaxf(second, lo);
+      for (int d = 0; d < SUB; ++d)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sc[i] = fmaf(a[d], cw[i][d], sc[i]);
+      idx = NCODES;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = fminf(best, sc[i]);
+        idx = (sc[i] > best || (sc[i] == best && kk[i] < idx)) ? kk[i] : idx;
+        best = fmaxf(best, sc[i]);
+        second = fmaxf(second, lo);
+      }
     }
     if (hf == 1) sm.xch2[L] = make_float4(best, second, __int_as_float(idx), 0.f);
-    __syncthreads();
+    asm volatile("bar.sync %0, 64;" :: "r"(1 + q) : "memory");  // the two warps of the pair only
 
     // (5) decision and bounds (lower warp of the pair)
     if (hf == 0) {
@@ -578,21 +586,27 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   };
 
   // ---- reference r = column mean of the raw tokens ---------------------------
-  // Column `col`, rows split in two halves (two accumulators each), combined in
-  // a fixed order.
+  // r only conditions the fp32 transform (FWHT(x - r) + FWHT(r) = FWHT(x) for any
+  // r), so it is formed in fp32: the first token plus the mean deviation from it,
+  // which makes r equal the tokens exactly when they are all equal.  Column `col`,
+  // rows split in two halves (two accumulators each), combined in a fixed order.
   {
     const int lo = rhalf * (BLK / 2), hi = min(n, lo + BLK / 2);
-    double s0 = 0.0, s1 = 0.0;
+    const float x0 = raw_at(0, col);
+    float s0 = 0.f, s1 = 0.f;
     int row = lo;
     for (; row + 1 < hi; row += 2) {
-      s0 += (double)raw_at(row, col);
-      s1 += (double)raw_at(row + 1, col);
+      s0 += raw_at(row, col) - x0;
+      s1 += raw_at(row + 1, col) - x0;
     }
-    if (row < hi) s0 += (double)raw_at(row, col);
-    sm.part[rhalf][col] = s0 + s1;
+    if (row < hi) s0 += raw_at(row, col) - x0;
+    reinterpret_cast<float*>(&sm.part[0][0])[rhalf * D + col] = s0 + s1;
   }
   __syncthreads();
-  if (t < D) sm.r[t] = (float)((sm.part[0][t] + sm.part[1][t]) / n);
+  if (t < D) {
+    const float* ps = reinterpret_cast<const float*>(&sm.part[0][0]);
+    sm.r[t] = raw_at(0, t) + (ps[t] + ps[D + t]) / (float)n;
+  }
   __syncthreads();
   // FWHT(r) in fp64 by warp 0 (lane l holds elements 4l..4l+3).
   if (t < 32) {
@@ -705,8 +719,9 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   __syncthreads();
   const double rr_mean = sm.rr[0] + (sm.dev_part[0] + sm.dev_part[1]) / n;
   if (t < D) {
-    const double dc = (sm.part[0][t] + sm.part[1][t]) / n;
-    sm.o[t] = dc;  // D_c = mean_t(d_t,c rr_t)
+    const double dc = (sm.part[0][t] + sm.part[1][t]) / n;  // D_c = mean_t(d_t,c rr_t)
+    sm.big_rf[t] = (float)sm.big_r[t];
+    sm.dcf[t] = (float)dc;
     const double o_t = fma(sm.big_r[t], rr_mean, dc);
     if (cv.dq) sm.ofull[t] = o_t;
     else cv.means[(seq * (cv.capacity / BLK) + blk) * D + t] = __double2half(o_t);
@@ -714,24 +729,27 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   __syncthreads();
 
   // ---- second normalization --------------------------------------------------
-  // z_t = n1_t - o = d_t rr_t + FWHT(r) (rr_t - mean rr) - D.  The last two terms
-  // are formed in fp64 and rounded once (they are at the scale of z), then one
-  // fp32 fma per channel.
+  // z_t = n1_t - o = d_t rr_t + FWHT(r) (rr_t - mean rr) - D.  The constant part
+  // c = FWHT(r) (rr_t - mean rr) - D enters z rounded to fp32; it is formed by one
+  // fp32 fma from fp32 copies of FWHT(r), D and rr_t - mean rr (three roundings of
+  // the size of the one fp32 rounding of c), then one fp32 fma per channel.
   const double rr_t = valid ? sm.rr[tk] : 0.0;
-  const double delta = rr_t - rr_mean;
+  const float deltaf = (float)(rr_t - rr_mean);
   const float rrf = (float)rr_t;
   double zz0 = 0.0, zz1 = 0.0;
 #pragma unroll
-  for (int c = 0; c < HD; c += 2) {
+  for (int c = 0; c < HD; c += 4) {
     const int cg = HD * h + c;
-    const float c0 = (float)fma(lds_f64(&sm.big_r[cg]), delta, -lds_f64(&sm.o[cg]));
-    const float c1 = (float)fma(lds_f64(&sm.big_r[cg + 1]), delta, -lds_f64(&sm.o[cg + 1]));
-    const float z0 = fmaf(v[c], rrf, c0);
-    const float z1 = fmaf(v[c + 1], rrf, c1);
-    v[c] = z0;
-    v[c + 1] = z1;
-    zz0 = fma((double)z0, (double)z0, zz0);
-    zz1 = fma((double)z1, (double)z1, zz1);
+    const float4 br = *reinterpret_cast<const float4*>(&sm.big_rf[cg]);
+    const float4 dd = *reinterpret_cast<const float4*>(&sm.dcf[cg]);
+    const float brv[4] = {br.x, br.y, br.z, br.w}, ddv[4] = {dd.x, dd.y, dd.z, dd.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float z = fmaf(v[c + i], rrf, fmaf(brv[i], deltaf, -ddv[i]));
+      v[c + i] = z;
+      if (i & 1) zz1 = fma((double)z, (double)z, zz1);
+      else zz0 = fma((double)z, (double)z, zz0);
+    }
   }
   const double zz = shfl_pair_sum(zz0 + zz1);
   if (valid && h == 0) sm.s2[tk] = sqrt(zz) / 11.313708498984761;
@@ -756,7 +774,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) sgn[k] |= __shfl_xor_sync(0xffffffffu, sgn[k], 1);
-    if (h == 0) *reinterpret_cast<uint4*>(&sm.sgn[tk][0]) = make_uint4(sgn[0], sgn[1], sgn[2], sgn[3]);
+    if (h == 0 && valid) *reinterpret_cast<uint4*>(signs + (int64_t)tk * NSUB) = make_uint4(sgn[0], sgn[1], sgn[2], sgn[3]);
   }
 
   // ---- u rows (|u| in 2-bit mode) to shared memory; zeros past the n tokens --
@@ -777,8 +795,8 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   {
     const int warp = t >> 5, lane = t & 31;
     const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1];
-    const bool f16tab = sm.cnorm[2] == 0.f;
     constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
+    const bool f16tab = sm.cnorm[2] == 0.f;
     const int nflag = sm.nflag;
 #pragma unroll 1
     for (int f = warp; f < nflag; f += QTHREADS / 32) {
@@ -797,8 +815,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
       for (int m = 0; m < NCODES / 32; ++m) {
         const int k = lane + 32 * m;
         float c[SUB];
-        codeword(sm, cb_global, f16tab, k, c);
-        float x = sm.cbias[cb_row(k)];
+        float x = codeword(sm, cb_global, f16tab, k, (lane >> 2) & 1, c);
 #pragma unroll
         for (int i = 0; i < SUB; ++i) x = fmaf(a[i], c[i], x);
         sc[m] = x;
@@ -812,7 +829,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
         if (sc[m] >= thr) {
           const int k = lane + 32 * m;
           float c[SUB];
-          codeword(sm, cb_global, f16tab, k, c);
+          codeword(sm, cb_global, f16tab, k, (lane >> 2) & 1, c);
           double dd = 0.0;
 #pragma unroll
           for (int i = 0; i < SUB; ++i) {
@@ -841,7 +858,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
     for (int jj = 0; jj < HSUB; ++jj) {
       const int j = HSUB * h + jj;
       float qv[SUB];
-      codeword(sm, cb_global, f16tab, sm.code[tk][j], qv);
+      codeword(sm, cb_global, f16tab, sm.code[tk][j], (t >> 2) & 1, qv);
       const float4 u0 = *reinterpret_cast<const float4*>(&sm.tile[tk][SUB * j]);
       const float4 u1 = *reinterpret_cast<const float4*>(&sm.tile[tk][SUB * j + 4]);
       const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
@@ -867,8 +884,6 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
     *reinterpret_cast<uint2*>(codes + (int64_t)tk * NSUB + HSUB * h) =
         *reinterpret_cast<const uint2*>(&sm.code[tk][HSUB * h]);
     if (h == 0) {
-      if constexpr (MODE == NSN_MODE_2BIT)
-        *reinterpret_cast<uint4*>(signs + (int64_t)tk * NSUB) = *reinterpret_cast<const uint4*>(&sm.sgn[tk][0]);
       const BlockOut bo = block_out(cv, seq, tok0, blk);
       if (bo.dq) bo.s2[tk] = __double2half(alpha * sm.s2[tk]);
       else bo.norms[tk] = __halves2half2(__double2half(sm.s1[tk]), __double2half(alpha * sm.s2[tk]));
