@@ -409,12 +409,20 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
   const uint32_t mbar = q_smem(&sm.mbar);
   const int ntiles = (n + 7) >> 3;
 
-  auto build_a = [&](int tile, float (&a)[SUB]) {
+  // The A rows of a tile; the row's decision bounds are formed here too, off the
+  // critical path of the decision: margin = twice the fp32 bound, mtc = the tensor bound.
+  auto build_a = [&](int tile, float (&a)[SUB], float& margin, float& mtc) {
     const int tkk = 8 * tile + (L >> 4), j = L & 15;
     const float4 a0 = *reinterpret_cast<const float4*>(&sm.tile[tkk][SUB * j]);
     const float4 a1 = *reinterpret_cast<const float4*>(&sm.tile[tkk][SUB * j + 4]);
     a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
     a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+    float na = 0.f;
+#pragma unroll
+    for (int d = 0; d < SUB; ++d) na = fmaf(a[d], a[d], na);
+    na = sqrtf(na) * 1.0001f;
+    margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
+    mtc = (TC_REL * (1.001f * na * cmax + 0.5f * cmax2) + na * cdel) * 1.01f + 1.2e-7f;
     uint32_t w[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
@@ -434,8 +442,8 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
     tc_commit(mbar);
   };
 
-  float a[SUB], an[SUB];
-  build_a(0, a);
+  float a[SUB], an[SUB], margin, mtc, margin_n = 0.f, mtc_n = 0.f;
+  build_a(0, a, margin, mtc);
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -444,7 +452,7 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
 #pragma unroll 1
   for (int tile = 0; tile < ntiles; ++tile) {
     if (tile + 1 < ntiles) {
-      build_a(tile + 1, an);
+      build_a(tile + 1, an, margin_n, mtc_n);
       fence_async_smem();
     }
     if (!mbar_wait(mbar, tcs.phase, MBAR_POLLS) && lane == 0 && status) atomicOr(status, 2);
@@ -528,20 +536,16 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
       second = max3f(second, o2.y, fminf(best, o2.x));
       idx = (o2.x > best) ? __float_as_int(o2.z) : idx;  // the upper half holds the larger indices
       best = fmaxf(best, o2.x);
-      float na = 0.f;
-#pragma unroll
-      for (int d = 0; d < SUB; ++d) na = fmaf(a[d], a[d], na);
-      na = sqrtf(na) * 1.0001f;
-      const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
-      const float m_tc = (TC_REL * (1.001f * na * cmax + 0.5f * cmax2) + na * cdel) * 1.01f + 1.2e-7f;
       const float other = m2 + fabsf(m2) * 3.82e-6f;  // + 32 ulp: the group number in the low bits
       const int tkk = 8 * tile + (L >> 4), j = L & 15;
       sm.code[tkk][j] = (uint8_t)idx;
-      const bool need = second >= best - margin || other >= best - 0.5f * margin - m_tc;
+      const bool need = second >= best - margin || other >= best - 0.5f * margin - mtc;
       if (need && tkk < n) sm.flag[atomicAdd(&sm.nflag, 1)] = (uint16_t)(tkk * NSUB + j);
     }
 #pragma unroll
     for (int i = 0; i < SUB; ++i) a[i] = an[i];
+    margin = margin_n;
+    mtc = mtc_n;
   }
   __syncthreads();
 }
@@ -593,14 +597,16 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   {
     const int lo = rhalf * (BLK / 2), hi = min(n, lo + BLK / 2);
     const float x0 = raw_at(0, col);
-    float s0 = 0.f, s1 = 0.f;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
     int row = lo;
-    for (; row + 1 < hi; row += 2) {
+    for (; row + 3 < hi; row += 4) {
       s0 += raw_at(row, col) - x0;
       s1 += raw_at(row + 1, col) - x0;
+      s2 += raw_at(row + 2, col) - x0;
+      s3 += raw_at(row + 3, col) - x0;
     }
-    if (row < hi) s0 += raw_at(row, col) - x0;
-    reinterpret_cast<float*>(&sm.part[0][0])[rhalf * D + col] = s0 + s1;
+    for (; row < hi; ++row) s0 += raw_at(row, col) - x0;
+    reinterpret_cast<float*>(&sm.part[0][0])[rhalf * D + col] = (s0 + s1) + (s2 + s3);
   }
   __syncthreads();
   if (t < D) {
@@ -700,20 +706,22 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   {
     const double rr0 = sm.rr[0];
     const int lo = rhalf * (BLK / 2), hi = min(n, lo + BLK / 2);
-    double dev = 0.0, sd0 = 0.0, sd1 = 0.0;
+    double dev = 0.0, sd0 = 0.0, sd1 = 0.0, sd2 = 0.0, sd3 = 0.0;
     int row = lo;
-    for (; row + 1 < hi; row += 2) {
-      const double ra = sm.rr[row], rb = sm.rr[row + 1];
-      dev += (ra - rr0) + (rb - rr0);
+    for (; row + 3 < hi; row += 4) {
+      const double ra = sm.rr[row], rb = sm.rr[row + 1], rc = sm.rr[row + 2], rd = sm.rr[row + 3];
+      dev += ((ra - rr0) + (rb - rr0)) + ((rc - rr0) + (rd - rr0));
       sd0 = fma((double)sm.tile[row][col], ra, sd0);
       sd1 = fma((double)sm.tile[row + 1][col], rb, sd1);
+      sd2 = fma((double)sm.tile[row + 2][col], rc, sd2);
+      sd3 = fma((double)sm.tile[row + 3][col], rd, sd3);
     }
-    if (row < hi) {
+    for (; row < hi; ++row) {
       const double ra = sm.rr[row];
       dev += ra - rr0;
       sd0 = fma((double)sm.tile[row][col], ra, sd0);
     }
-    sm.part[rhalf][col] = sd0 + sd1;
+    sm.part[rhalf][col] = (sd0 + sd1) + (sd2 + sd3);
     if (col == 0) sm.dev_part[rhalf] = dev;
   }
   __syncthreads();

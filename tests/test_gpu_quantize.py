@@ -41,6 +41,8 @@ def check_prefill(x, cb, cache, mode, window):
             mism_rows = (got["codes"] != ref["codes"]).any(axis=1)
             tl.compare_norms_means(got, ref, mism_rows)
             assert np.array_equal(got["window"], ref["window"])
+    # near-ties are counted, not failed; they must stay rare
+    assert stats["near_ties"] <= max(2, 1e-3 * stats["n"]), stats
     return stats
 
 
