@@ -1497,28 +1497,51 @@ bool decode_static_fits(int batch, int n_kv_heads, const DecodeGeom& geom) {
          2 * (int64_t)batch * n_kv_heads <= (int64_t)NSN_DECODE_STATIC_COUNTERS;
 }
 
-// Device addresses of the two arrays for the current device.  Resolved once per
-// device (cudaGetSymbolAddress with that device current) and cached.
+// The current CUDA context (driver handle), or null.  cuCtxGetCurrent is looked
+// up through the runtime, so the library does not link the driver library.
+typedef int (*CtxGetCurrentFn)(void**);
+static void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  void* ctx = nullptr;
+  if (fn && fn(&ctx) != 0) ctx = nullptr;
+  return ctx;
+}
+
+// Device addresses of the two arrays for the current device.  Resolved with
+// cudaGetSymbolAddress (that device current) at the device's first call and cached
+// together with the CUDA context they belong to; a different context on the same
+// device (one created after cudaDeviceReset, for instance, which loads the module
+// again) resolves them anew, so a stale address is never used.
 static cudaError_t decode_static_ptrs(void** scratch, void** counters) {
   static std::mutex mu;
-  static void* ptrs[64][2] = {};
+  struct Entry { void* ctx; void* scratch; void* counters; };
+  static Entry cache[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev][0]) {
+  void* ctx = current_context();
+  Entry& en = cache[dev];
+  if (!en.scratch || !ctx || en.ctx != ctx) {
     void* p = nullptr;
     void* c = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
     e = cudaGetSymbolAddress(&c, g_decode_counters);
     if (e != cudaSuccess) return e;
-    ptrs[dev][0] = p;
-    ptrs[dev][1] = c;
+    en = Entry{current_context(), p, c};
   }
-  *scratch = ptrs[dev][0];
-  *counters = ptrs[dev][1];
+  *scratch = en.scratch;
+  *counters = en.counters;
   return cudaSuccess;
 }
 

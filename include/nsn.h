@@ -317,8 +317,14 @@ nsn_status nsn_decode_attention_rope(const nsn_cache* k_cache, const nsn_cache* 
  *   - Nothing is allocated or freed (no cudaMalloc / cudaFree / allocating library).
  *   - Returns NSN_ERR_WORKSPACE if this shape's partials need more than
  *     NSN_DECODE_SCRATCH_BYTES or 2 * batch * n_kv_heads > NSN_DECODE_STATIC_COUNTERS.
- *   - The first call on a device resolves the array's device address (with that
- *     device current) and caches it; make that first call before any stream capture.
+ *   - The first call on a device (in a given CUDA context) resolves the arrays' device
+ *     addresses (with that device current) and caches them; make that first call before
+ *     any stream capture.  With lazy module loading (the CUDA default) that first call
+ *     can also be the moment the module holding the arrays is loaded, which is when
+ *     their NSN_DECODE_SCRATCH_BYTES + 4 * NSN_DECODE_STATIC_COUNTERS bytes of device
+ *     memory are taken: a caller that reserves all device memory, or that must not
+ *     allocate at all later on, makes one warm-up call (or sets CUDA_MODULE_LOADING=EAGER)
+ *     before it does so.  Later calls allocate nothing.
  *   - All calls share the one array: two calls whose work overlaps on the GPU (e.g. on
  *     different streams without ordering between them) race on it and must not be
  *     issued.  Every partial the kernel reads is written earlier in the same call and
