@@ -29,6 +29,8 @@ Readings where the pages are silent:
     quantization block (128 tokens) of one (batch, kv-head).
   * Nearest codeword = smallest squared Euclidean distance; ties go to the
     lowest index.  2-bit mode: sign bit i = (u_i < 0), code over |u|.
+  * Cosine assignment (optional variant): the codeword of largest cosine
+    similarity p . c / ||c||, ties to the lowest index.
   * Adaptive scale: alpha = ||u||^2 / (u . u_hat) per token (alpha = 1 when
     u . u_hat <= 0), folded into the stored s2.
   * Stored s1, s2*alpha and o are rounded to fp16 (round-to-nearest-even).
@@ -137,21 +139,47 @@ def nearest_codeword(points: np.ndarray, codebook: np.ndarray):
     return idx, gap
 
 
-def assign(u_sub: np.ndarray, codebook: np.ndarray, mode: int):
+def cosine_codeword(points: np.ndarray, codebook: np.ndarray):
+    """Codeword of largest cosine similarity, ties to the lowest index.
+
+    The cosine-assignment variant of the codebook tuning ([TS] Metodologia 3: the
+    codebook is fine-tuned for the cosine distance between a vector and its
+    quantized version): code = argmax_k p . c_k / ||c_k|| (the factor 1/||p|| is the
+    same for every k; a zero codeword scores 0).  The gap is defined as for the
+    nearest codeword on the distances d_k = ||p|| - p . c_k / ||c_k||
+    (= ||p|| (1 - cos)).  Returns (index [m], relative top-2 gap [m]).
+    """
+    points = np.asarray(points, dtype=np.float64)
+    codebook = np.asarray(codebook, dtype=np.float64)
+    norms = np.sqrt(np.sum(codebook * codebook, axis=1))
+    inv = np.where(norms > 0, 1.0 / np.where(norms > 0, norms, 1.0), 0.0)
+    score = (points @ codebook.T) * inv[None, :]
+    dist = np.sqrt(np.sum(points * points, axis=1))[:, None] - score
+    idx = np.argmin(dist, axis=1)
+    srt = np.sort(dist, axis=1)
+    d1, d2 = srt[:, 0], srt[:, 1]
+    gap = np.where(d2 > 0, (d2 - d1) / np.where(d2 > 0, d2, 1.0), 0.0)
+    return idx, gap
+
+
+def assign(u_sub: np.ndarray, codebook: np.ndarray, mode: int, cosine: bool = False):
     """Code (and sign bits) of every sub-vector u_sub [m, m_dim].
 
     1-bit: code = argmin_k ||u_s - C_k||^2.
     2-bit: sign bit i = 1 iff u_i < 0; code = argmin_k || |u_s| - A_k ||^2
            over the absolute-value codebook A (entries >= 0).
+    cosine: the same with the codeword of largest cosine similarity instead of
+           the nearest one (`cosine_codeword`).
     Returns (codes [m] int, signs [m] uint8 bit-packed or None, gap [m]).
     """
     u_sub = np.asarray(u_sub, dtype=np.float64)
+    pick = cosine_codeword if cosine else nearest_codeword
     if mode == MODE_1BIT:
-        codes, gap = nearest_codeword(u_sub, codebook)
+        codes, gap = pick(u_sub, codebook)
         return codes, None, gap
     if mode == MODE_2BIT:
         neg = u_sub < 0
-        codes, gap = nearest_codeword(np.abs(u_sub), codebook)
+        codes, gap = pick(np.abs(u_sub), codebook)
         weights = (1 << np.arange(u_sub.shape[1])).astype(np.int64)
         signs = (neg.astype(np.int64) * weights[None, :]).sum(axis=1)
         return codes, signs.astype(np.uint8), gap
@@ -206,7 +234,8 @@ def dq4(x) -> dict:
 
 
 def quantize_block(x: np.ndarray, codebook: np.ndarray, mode: int,
-                   sub_dim: int = 8, scale_adjust: bool = True, double_quant: bool = False) -> dict:
+                   sub_dim: int = 8, scale_adjust: bool = True, double_quant: bool = False,
+                   cosine: bool = False) -> dict:
     """Quantize one block of raw tokens x [n, d] (one batch row, one kv-head).
 
     Hadamard -> NSN -> per-sub-vector nearest codeword -> adaptive scale ->
@@ -218,14 +247,15 @@ def quantize_block(x: np.ndarray, codebook: np.ndarray, mode: int,
     With double_quant, s1 and o are stored in 4 bits instead (`dq4` over the
     block's tokens and over its 128 channels); "s1" and "o" then hold the
     dequantized values and "s1_dq" / "o_dq" the levels and (lo, hi).  The NSN,
-    the assignment and alpha use the exact values either way.
+    the assignment and alpha use the exact values either way.  With cosine the
+    codes are the codewords of largest cosine similarity (`cosine_codeword`).
     """
     x = np.asarray(x, dtype=np.float64)
     n, d = x.shape
     nsub = d // sub_dim
     y = rotate(x)
     u, s1, o, s2 = nsn(y)
-    codes, signs, gap = assign(u.reshape(n * nsub, sub_dim), codebook, mode)
+    codes, signs, gap = assign(u.reshape(n * nsub, sub_dim), codebook, mode, cosine=cosine)
     u_hat = reconstruct_sub(codes, signs, codebook, mode).reshape(n, d)
     alpha = scale_factor(u, u_hat) if scale_adjust else np.ones(n)
     out = {
@@ -260,7 +290,7 @@ def prefill_split(n_tokens: int, block: int, window: int) -> int:
 
 def quantize_sequence(x: np.ndarray, codebook: np.ndarray, mode: int,
                       block: int = 128, window: int = 128,
-                      scale_adjust: bool = True, double_quant: bool = False) -> dict:
+                      scale_adjust: bool = True, double_quant: bool = False, cosine: bool = False) -> dict:
     """Prefill of one (batch, kv-head) sequence x [L, d].
 
     Returns codes/signs/s1/s2 per quantized token, o per block, the fp16
@@ -271,7 +301,7 @@ def quantize_sequence(x: np.ndarray, codebook: np.ndarray, mode: int,
     L, d = x.shape
     q = prefill_split(L, block, window)
     parts = [quantize_block(x[a:min(a + block, q)], codebook, mode,
-                            scale_adjust=scale_adjust, double_quant=double_quant)
+                            scale_adjust=scale_adjust, double_quant=double_quant, cosine=cosine)
              for a in range(0, q, block)]
     nsub = d // 8
 

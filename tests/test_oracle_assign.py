@@ -2,6 +2,7 @@
 adaptive scale: hand-computed cases, scipy's cdist, exhaustive search over all
 signed codewords, and the defining property of the scale factor."""
 import itertools
+import math
 
 import numpy as np
 import pytest
@@ -114,3 +115,62 @@ def test_sign_layout_conversion_roundtrip():
     one[0, 3] = 1 << 5
     st = tl.natural_to_signs(one)
     assert st[0, 11] == 1 << 4 and st.sum() == 16
+
+
+# ---------------------------------------------------------------------------
+# Cosine-assignment variant ([TS] Metodologia 3: codebook tuned for the cosine
+# distance between a vector and its quantized version)
+# ---------------------------------------------------------------------------
+def test_cosine_assignment_by_brute_force_angles():
+    # the chosen codeword has the smallest angle to the point, computed with arccos
+    rng = np.random.default_rng(31)
+    pts = rng.standard_normal((300, 8))
+    cb = rng.standard_normal((64, 8)) * rng.uniform(0.2, 3.0, (64, 1))
+    idx, _ = orc.cosine_codeword(pts, cb)
+    for i in range(pts.shape[0]):
+        ang = [math.acos(np.clip(pts[i] @ c / (np.linalg.norm(pts[i]) * np.linalg.norm(c)), -1, 1)) for c in cb]
+        assert idx[i] == int(np.argmin(ang))
+
+
+def test_cosine_assignment_ignores_codeword_lengths():
+    # rescaling codewords by positive factors changes the nearest codeword but not
+    # the cosine choice
+    rng = np.random.default_rng(32)
+    pts = np.abs(rng.standard_normal((500, 8)))
+    cb = np.abs(rng.standard_normal((256, 8)))
+    a, _ = orc.cosine_codeword(pts, cb)
+    b, _ = orc.cosine_codeword(pts, cb * rng.uniform(0.1, 10.0, (256, 1)))
+    assert np.array_equal(a, b)
+    near, _ = orc.nearest_codeword(pts, cb * rng.uniform(0.1, 10.0, (256, 1)))
+    assert (near != a).any()
+
+
+def test_cosine_equals_nearest_for_unit_vectors():
+    # for unit points and unit codewords ||p - c||^2 = 2 - 2 cos: the same choice
+    rng = np.random.default_rng(33)
+    pts = rng.standard_normal((400, 8))
+    pts /= np.linalg.norm(pts, axis=1, keepdims=True)
+    cb = rng.standard_normal((256, 8))
+    cb /= np.linalg.norm(cb, axis=1, keepdims=True)
+    assert np.array_equal(orc.cosine_codeword(pts, cb)[0], orc.nearest_codeword(pts, cb)[0])
+
+
+def test_cosine_hand_case_and_ties():
+    cb = np.array([[1.0, 0.0], [10.0, 1.0], [0.0, 0.0], [2.0, 0.0]])
+    # (3, 0.2) is nearest to (2, 0) but closest in angle to (10, 1)
+    idx, _ = orc.cosine_codeword(np.array([[3.0, 0.2]]), cb)
+    assert idx[0] == 1
+    assert orc.nearest_codeword(np.array([[3.0, 0.2]]), cb)[0][0] == 3
+    # (1, 0): codewords 0 and 3 have the same direction -> the lower index, gap 0
+    idx, gap = orc.cosine_codeword(np.array([[1.0, 0.0]]), cb)
+    assert idx[0] == 0 and gap[0] == 0.0
+
+
+def test_cosine_assign_2bit_uses_abs_and_signs():
+    rng = np.random.default_rng(34)
+    u = rng.standard_normal((50, 8))
+    A = np.abs(rng.standard_normal((256, 8)))
+    codes, signs, _ = orc.assign(u, A, orc.MODE_2BIT, cosine=True)
+    assert np.array_equal(codes, orc.cosine_codeword(np.abs(u), A)[0])
+    c1, s1, _ = orc.assign(u, A, orc.MODE_2BIT)
+    assert np.array_equal(signs, s1)
