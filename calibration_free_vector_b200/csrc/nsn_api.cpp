@@ -41,6 +41,7 @@ nsn_status check_cache(const nsn_cache* c) {
   if ((reinterpret_cast<uintptr_t>(c->n_quant) & 3u) || (reinterpret_cast<uintptr_t>(c->n_window) & 3u))
     return NSN_ERR_INVALID_ARG;
   if (c->double_quant != 0 && c->double_quant != 1) return NSN_ERR_INVALID_ARG;
+  if (c->assign != 0 && c->assign != 1) return NSN_ERR_INVALID_ARG;
   if (c->double_quant && (!c->s1_levels || !c->dq_params || !aligned16(c->s1_levels) || !aligned16(c->dq_params)))
     return NSN_ERR_INVALID_ARG;
   return NSN_OK;
@@ -63,6 +64,7 @@ nsn::CacheView view(const nsn_cache* c) {
   v.n_window = c->n_window;
   v.status = c->status;
   v.dq = c->double_quant ? 1 : 0;
+  v.assign = c->assign;
   v.s1_levels = c->double_quant ? c->s1_levels : nullptr;
   v.dq_params = c->double_quant ? reinterpret_cast<__half*>(c->dq_params) : nullptr;
   return v;

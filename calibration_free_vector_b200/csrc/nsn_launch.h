@@ -22,6 +22,7 @@ struct CacheView {
   int dq;               // 1: s1 and o stored as 4-bit levels (then `norms` holds fp16 alpha*s2,
   uint8_t* s1_levels;   //    `means` the o levels, s1_levels / dq_params the rest)
   __half* dq_params;
+  int assign;           // 0: nearest codeword, 1: largest cosine similarity
 };
 
 // Decode split geometry: the quantized blocks of every (b, kv-head) are dealt

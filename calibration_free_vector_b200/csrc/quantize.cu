@@ -118,6 +118,11 @@ constexpr int QTHREADS = 2 * BLK;  // two threads per token
 constexpr int HD = D / 2;           // dims per thread
 constexpr int HSUB = NSUB / 2;      // sub-vectors per thread
 constexpr int MBAR_POLLS = 1 << 22;  // bounded wait for the MMAs of one tile
+// Where the exact arithmetic reads codeword k and its bias: the two fp16 replicas
+// of the shared table with fp32 biases (fp16-representable codebook), the fp32
+// codebook in global memory with the fp32 biases (any other codebook), or the
+// fp32 unit codewords c_hat of the table with bias 0 (cosine assignment).
+constexpr int TAB_F16 = 0, TAB_GLOBAL = 1, TAB_COSINE = 2;
 
 struct QuantSmem {
   // ---- operands of the tensor-core scores (staged once per CTA) ----
@@ -133,6 +138,7 @@ struct QuantSmem {
   alignas(16) unsigned char cbtab[NCODES * 32];
   alignas(16) float cbias[2 * NCODES];
   alignas(16) float cnorm[4];                     // [0] max ||c||, [1] max ||c||^2, [2] max ||c - fp16(c)|| (rounded up)
+  int tab;                                        // TAB_F16, TAB_GLOBAL or TAB_COSINE
   alignas(8) unsigned long long mbar;             // MMA completion barrier
   uint32_t tmem;                                  // tensor-memory base address of this CTA
   int nflag;
@@ -223,14 +229,30 @@ __device__ __forceinline__ BlockOut block_out(const CacheView& c, int64_t seq, i
 // Stages the codebook: the tensor-core operands (fp16 codebook, fp16 hi/lo bias,
 // the constant bias rows), the fp16 rows and fp32 biases of the exact arithmetic,
 // and the norm bounds.  All QTHREADS threads (one codeword each).
-__device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook) {
+//
+// Cosine assignment (cosine = 1): the scores are a . c_hat with c_hat = c / ||c||
+// (fp64 division, rounded once to fp32; 0 for a zero codeword).  The score MMA
+// takes c_hat's fp16 high part as B, the second MMA (in place of the bias MMA)
+// adds the same A rows times its fp16 low part, the exact arithmetic reads the
+// fp32 c_hat from the table (bias 0), and the bounds are those of c_hat.
+__device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook, int cosine) {
   const int t = threadIdx.x;
   float my_max = 0.f, my_dev = 0.f;
   for (int k = t; k < NCODES; k += blockDim.x) {
     float c[SUB];
-    const float4 c0 = __ldg(reinterpret_cast<const float4*>(codebook + k * SUB));
-    const float4 c1 = __ldg(reinterpret_cast<const float4*>(codebook + k * SUB) + 1);
+    float4 c0 = __ldg(reinterpret_cast<const float4*>(codebook + k * SUB));
+    float4 c1 = __ldg(reinterpret_cast<const float4*>(codebook + k * SUB) + 1);
     c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+    if (cosine) {
+      double nn = 0.0;
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) nn = fma((double)c[i], (double)c[i], nn);
+      const double nrm = sqrt(nn);
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) c[i] = nrm > 0.0 ? (float)((double)c[i] / nrm) : 0.f;
+      c0 = make_float4(c[0], c[1], c[2], c[3]);
+      c1 = make_float4(c[4], c[5], c[6], c[7]);
+    }
     float ss = 0.f, e = 0.f;
     __half ch[SUB];
 #pragma unroll
@@ -241,18 +263,29 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
       e = fmaf(dlt, dlt, e);
     }
     const float bias = -0.5f * ss;
-    *reinterpret_cast<uint4*>(sm.cbtab + 32 * k) = *reinterpret_cast<const uint4*>(ch);
-    *reinterpret_cast<uint4*>(sm.cbtab + 32 * k + 16) = *reinterpret_cast<const uint4*>(ch);
-    sm.cbias[2 * k] = bias;
-    sm.cbias[2 * k + 1] = bias;
     // B operand: K = 0..7 and 8..15 both hold the codeword (multiplied by a_hi and a_lo)
     *reinterpret_cast<uint4*>(sm.bop + kmaj_off(k, 0)) = *reinterpret_cast<const uint4*>(ch);
     *reinterpret_cast<uint4*>(sm.bop + kmaj_off(k, 8)) = *reinterpret_cast<const uint4*>(ch);
-    // bias operand: (b_hi, b_lo) with b_hi + b_lo = bias to 2^-22 relative
-    const __half bh = __float2half_rn(bias);
-    const __half bl = __float2half_rn(bias - __half2float(bh));
     uint4 brow = make_uint4(0u, 0u, 0u, 0u);
-    brow.x = (uint32_t)__half_as_ushort(bh) | ((uint32_t)__half_as_ushort(bl) << 16);
+    if (cosine) {
+      // fp32 c_hat for the exact arithmetic; second-MMA operand: fp16(c_hat - fp16(c_hat))
+      *reinterpret_cast<float4*>(sm.cbtab + 32 * k) = c0;
+      *reinterpret_cast<float4*>(sm.cbtab + 32 * k + 16) = c1;
+      __half cl[SUB];
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) cl[i] = __float2half_rn(c[i] - __half2float(ch[i]));
+      brow = *reinterpret_cast<const uint4*>(cl);
+      e = 0.f;  // hi + lo carries c_hat to 2^-22, inside the tensor bound
+    } else {
+      *reinterpret_cast<uint4*>(sm.cbtab + 32 * k) = *reinterpret_cast<const uint4*>(ch);
+      *reinterpret_cast<uint4*>(sm.cbtab + 32 * k + 16) = *reinterpret_cast<const uint4*>(ch);
+      sm.cbias[2 * k] = bias;
+      sm.cbias[2 * k + 1] = bias;
+      // bias operand: (b_hi, b_lo) with b_hi + b_lo = bias to 2^-22 relative
+      const __half bh = __float2half_rn(bias);
+      const __half bl = __float2half_rn(bias - __half2float(bh));
+      brow.x = (uint32_t)__half_as_ushort(bh) | ((uint32_t)__half_as_ushort(bl) << 16);
+    }
     *reinterpret_cast<uint4*>(sm.bop2 + (k >> 3) * 128 + (k & 7) * 16) = brow;
     my_max = fmaxf(my_max, ss);
     my_dev = fmaxf(my_dev, e);
@@ -280,16 +313,17 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
     sm.cnorm[1] = m;
     sm.cnorm[0] = sqrtf(m) * 1.0001f;
     sm.cnorm[2] = e > 0.f ? sqrtf(e) * 1.001f : 0.f;  // 0 for a codebook of fp16 values
+    // where the exact arithmetic reads codewords (see codeword())
+    sm.tab = cosine ? TAB_COSINE : (e > 0.f ? TAB_GLOBAL : TAB_F16);
   }
   __syncthreads();
 }
 
-// Codeword k (fp32) and its bias -||c_k||^2/2: replica p of the shared fp16 table
-// when the codebook is fp16-representable (then the values are the fp32 input
-// exactly), else the fp32 codebook in global memory.
-__device__ __forceinline__ float codeword(const QuantSmem& sm, const float* __restrict__ cb_global, bool f16tab,
+// Codeword k as the scores use it (fp32) and its bias, read as sm.tab says (replica
+// p of the fp16 table when that is the source).
+__device__ __forceinline__ float codeword(const QuantSmem& sm, const float* __restrict__ cb_global, int tab,
                                           int k, int p, float (&c)[SUB]) {
-  if (f16tab) {
+  if (tab == TAB_F16) {
     const uint4 raw = *reinterpret_cast<const uint4*>(sm.cbtab + 32 * k + 16 * p);
     const __half2* hv = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
@@ -298,12 +332,25 @@ __device__ __forceinline__ float codeword(const QuantSmem& sm, const float* __re
       c[2 * i] = f.x;
       c[2 * i + 1] = f.y;
     }
-  } else {
-    const float4 c0 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB));
-    const float4 c1 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB) + 1);
-    c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+    return sm.cbias[2 * k + p];
   }
-  return sm.cbias[2 * k + p];
+  float4 c0, c1;
+  if (tab == TAB_COSINE) {
+    c0 = *reinterpret_cast<const float4*>(sm.cbtab + 32 * k);
+    c1 = *reinterpret_cast<const float4*>(sm.cbtab + 32 * k + 16);
+  } else {
+    c0 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB));
+    c1 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB) + 1);
+  }
+  c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+  return tab == TAB_COSINE ? 0.f : sm.cbias[2 * k + p];
+}
+
+// Codeword k as stored in the codebook (the reconstruction's u_hat), fp32.
+__device__ __forceinline__ void codeword_given(const QuantSmem& sm, const float* __restrict__ cb_global, int tab,
+                                               int k, int p, float (&c)[SUB]) {
+  if (tab == TAB_COSINE) tab = TAB_GLOBAL;
+  codeword(sm, cb_global, tab, k, p, c);
 }
 
 __device__ __forceinline__ double shfl_pair_sum(double x) { return x + __shfl_xor_sync(0xffffffffu, x, 1); }
@@ -399,7 +446,7 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
   const int q = warp & 3, hf = warp >> 2;
   const int L = 32 * q + lane;
   const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1], cdel = sm.cnorm[2];
-  const bool f16tab = cdel == 0.f;
+  const int tab = sm.tab;
   constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
   constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
   const uint32_t taddr = tcs.tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * hf);
@@ -437,8 +484,14 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
     *reinterpret_cast<uint4*>(sm.aop[tile & 1] + kmaj_off(L, 8 * hf)) = make_uint4(w[0], w[1], w[2], w[3]);
   };
   auto issue = [&](int tile) {
-    tc_mma(tcs.tmem, da2, db2, 0u);
-    tc_mma(tcs.tmem, tc_desc(q_smem(sm.aop[tile & 1]), 128, 256), db, 1u);
+    const uint64_t da = tc_desc(q_smem(sm.aop[tile & 1]), 128, 256);
+    if (tab == TAB_COSINE) {  // D = [a_hi | a_lo] [c_hat_hi | c_hat_hi] + [a_hi | a_lo] [c_hat_lo | c_hat_lo]
+      tc_mma(tcs.tmem, da, db, 0u);
+      tc_mma(tcs.tmem, da, db2, 1u);
+    } else {                  // D = b_hi + b_lo, then D += [a_hi | a_lo] [c | c]
+      tc_mma(tcs.tmem, da2, db2, 0u);
+      tc_mma(tcs.tmem, da, db, 1u);
+    }
     tc_commit(mbar);
   };
 
@@ -512,7 +565,7 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         kk[i] = 8 * G + 4 * hf + ((i + lane) & 3);
-        sc[i] = codeword(sm, cb_global, f16tab, kk[i], rep, cw[i]);
+        sc[i] = codeword(sm, cb_global, tab, kk[i], rep, cw[i]);
       }
 #pragma unroll
       for (int d = 0; d < SUB; ++d)
@@ -799,12 +852,13 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   // ---- exact fp64 re-decision of the flagged sub-vectors, a warp each --------
   // Each lane scores its 8 codewords in sequential fp32 (bias first, one fma per
   // dim); candidates are the codewords within twice the fp32 bound of the best of
-  // these scores; the winner by fp64 squared distance, ties to the lowest index.
+  // these scores; the winner by fp64 squared distance (cosine assignment: largest
+  // fp64 inner product with c_hat), ties to the lowest index.
   {
     const int warp = t >> 5, lane = t & 31;
     const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1];
     constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
-    const bool f16tab = sm.cnorm[2] == 0.f;
+    const int tab = sm.tab;
     const int nflag = sm.nflag;
 #pragma unroll 1
     for (int f = warp; f < nflag; f += QTHREADS / 32) {
@@ -823,7 +877,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
       for (int m = 0; m < NCODES / 32; ++m) {
         const int k = lane + 32 * m;
         float c[SUB];
-        float x = codeword(sm, cb_global, f16tab, k, (lane >> 2) & 1, c);
+        float x = codeword(sm, cb_global, tab, k, (lane >> 2) & 1, c);
 #pragma unroll
         for (int i = 0; i < SUB; ++i) x = fmaf(a[i], c[i], x);
         sc[m] = x;
@@ -837,12 +891,17 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
         if (sc[m] >= thr) {
           const int k = lane + 32 * m;
           float c[SUB];
-          codeword(sm, cb_global, f16tab, k, (lane >> 2) & 1, c);
-          double dd = 0.0;
+          codeword(sm, cb_global, tab, k, (lane >> 2) & 1, c);
+          double dd = 0.0;  // fp64 squared distance, or minus the fp64 inner product with c_hat
+          if (tab == TAB_COSINE) {
 #pragma unroll
-          for (int i = 0; i < SUB; ++i) {
-            const double e = (double)a[i] - (double)c[i];
-            dd = fma(e, e, dd);
+            for (int i = 0; i < SUB; ++i) dd = fma(-(double)a[i], (double)c[i], dd);
+          } else {
+#pragma unroll
+            for (int i = 0; i < SUB; ++i) {
+              const double e = (double)a[i] - (double)c[i];
+              dd = fma(e, e, dd);
+            }
           }
           if (dd < bestd) { bestd = dd; bi = k; }
         }
@@ -861,12 +920,12 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   // ---- adaptive scale: alpha = ||u||^2 / (u . u_hat) --------------------------
   double dot = 0.0, uu = 0.0;
   {
-    const bool f16tab = sm.cnorm[2] == 0.f;
+    const int tab = sm.tab;
 #pragma unroll 4
     for (int jj = 0; jj < HSUB; ++jj) {
       const int j = HSUB * h + jj;
       float qv[SUB];
-      codeword(sm, cb_global, f16tab, sm.code[tk][j], (t >> 2) & 1, qv);
+      codeword_given(sm, cb_global, tab, sm.code[tk][j], (t >> 2) & 1, qv);
       const float4 u0 = *reinterpret_cast<const float4*>(&sm.tile[tk][SUB * j]);
       const float4 u1 = *reinterpret_cast<const float4*>(&sm.tile[tk][SUB * j + 4]);
       const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
@@ -935,7 +994,7 @@ quantize_prefill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int6
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw);
   TcState tcs = tc_setup(sm);
-  stage_codebook(sm, codebook);
+  stage_codebook(sm, codebook, cv.assign);
   const int nwork = nblk * cv.n_kv_heads * cv.batch;
 #pragma unroll 1
   for (int w = blockIdx.x; w < nwork; w += gridDim.x) {
@@ -1003,7 +1062,7 @@ append_kernel(CacheView kc, CacheView vc, const void* __restrict__ k_new, const 
     } else {
       const float* cb = is_v ? cbv : cbk;
       TcState tcs = tc_setup(sm);
-      stage_codebook(sm, cb);
+      stage_codebook(sm, cb, c.assign);
       const int64_t tok0 = seq * c.capacity + nq;
       const int blk = nq / BLK;
       uint8_t* sg = c.mode == NSN_MODE_2BIT ? c.signs + tok0 * NSUB : nullptr;

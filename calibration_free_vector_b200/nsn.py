@@ -45,6 +45,7 @@ class nsn_cache(ctypes.Structure):
         ("codes", c_void_p), ("signs", c_void_p), ("norms", c_void_p), ("means", c_void_p),
         ("window_buf", c_void_p), ("n_quant", c_void_p), ("n_window", c_void_p), ("status", c_void_p),
         ("double_quant", c_int32), ("s1_levels", c_void_p), ("dq_params", c_void_p),
+        ("assign", c_int32),
     ]
 
 
@@ -177,12 +178,13 @@ class Cache:
     """Device buffers of one compressed K or V cache and the matching C struct."""
 
     def __init__(self, batch: int, n_kv_heads: int, capacity: int, window: int, mode: int,
-                 scale_adjust: bool = True, device="cuda", double_quant: bool = False):
+                 scale_adjust: bool = True, device="cuda", double_quant: bool = False, cosine: bool = False):
         import torch
         sizes = nsn_cache_buffer_sizes(batch, n_kv_heads, capacity, window, mode, double_quant)
         self.batch, self.n_kv_heads, self.capacity, self.window, self.mode = batch, n_kv_heads, capacity, window, mode
         self.scale_adjust = bool(scale_adjust)
         self.double_quant = bool(double_quant)
+        self.cosine = bool(cosine)  # codeword of largest cosine similarity instead of the nearest one
         u8 = dict(dtype=torch.uint8, device=device)
         f16 = dict(dtype=torch.float16, device=device)
         nblk = capacity // BLOCK
@@ -214,7 +216,8 @@ class Cache:
             self.n_quant.data_ptr(), self.n_window.data_ptr(), self.status.data_ptr(),
             1 if double_quant else 0,
             self.s1_levels.data_ptr() if self.s1_levels is not None else None,
-            self.dq_params.data_ptr() if self.dq_params is not None else None)
+            self.dq_params.data_ptr() if self.dq_params is not None else None,
+            1 if cosine else 0)
 
     def nbytes_allocated(self) -> int:
         bufs = [self.codes, self.signs, self.norms, self.means, self.window_buf, self.n_quant, self.n_window,

@@ -104,6 +104,15 @@ typedef enum { NSN_DTYPE_F32 = 0, NSN_DTYPE_BF16 = 1, NSN_DTYPE_F16 = 2 } nsn_dt
  *                                                           0, 0) of each block
  * With double_quant = 0, s1_levels and dq_params are unused (may be NULL).  The K and
  * V caches given to one append or decode call must both use it or both not.
+ *
+ * Cosine assignment (assign = 1; [TS] Metodologia 3: the codebook is fine-tuned for
+ * the cosine distance between a vector and its quantized version, [GH] Codebook
+ * tuning "--method learned"): every sub-vector a (u, or |u| in 2-bit mode) takes the
+ * codeword of largest cosine similarity, code = argmax_k a . c_k / ||c_k|| (ties to
+ * the lowest index; a zero codeword scores 0), instead of the nearest one.  The
+ * stored scalars, the adaptive scale and the decode are unchanged (they use the
+ * codebook as given).  assign applies to every quantization of the cache (prefill
+ * and flushes); the K and V caches may differ in it.
  */
 typedef struct {
   int32_t batch;
@@ -123,6 +132,8 @@ typedef struct {
   int32_t double_quant; /* 1: s1 and o stored in 4 bits (layout above) */
   uint8_t* s1_levels;
   uint16_t* dq_params;
+  int32_t assign;       /* codeword choice of the quantizer: 0 = nearest (squared Euclidean),
+                           1 = largest cosine similarity a.c/||c|| (see below) */
 } nsn_cache;
 
 /* Byte sizes of the buffers of an nsn_cache with the given shape. */

@@ -212,19 +212,20 @@ def oracle_seq(c):
             "o": f(c["o"])}
 
 
-def oracle_pipeline(xk, xv, n_prefill, n_total, cbk, cbv, mk, mv, window):
+def oracle_pipeline(xk, xv, n_prefill, n_total, cbk, cbv, mk, mv, window, cosine=False):
     """Oracle cache of one (b, h) after a prefill of n_prefill tokens and
-    appends up to n_total (flushes of the full window as fp16 blocks)."""
+    appends up to n_total (flushes of the full window as fp16 blocks); with cosine
+    the codes are the codewords of largest cosine similarity."""
     from oracle import nsn_oracle as orc
     out = []
     for x, cb, mode in ((xk, cbk, mk), (xv, cbv, mv)):
-        seq = orc.quantize_sequence(x[:n_prefill], cb, mode, 128, window)
+        seq = orc.quantize_sequence(x[:n_prefill], cb, mode, 128, window, cosine=cosine)
         codes, signs, s1, s2, o = [seq["codes"]], [seq["signs"]], [seq["s1"]], [seq["s2"]], [seq["o"]]
         nq = seq["n_quant"]
         win = list(orc.to_f16(x[nq:n_prefill]))
         for t in range(n_prefill, n_total):
             if len(win) == window:
-                blk = orc.quantize_block(np.array(win), cb, mode)
+                blk = orc.quantize_block(np.array(win), cb, mode, cosine=cosine)
                 codes.append(blk["codes"]); signs.append(blk["signs"]); s1.append(blk["s1"])
                 s2.append(blk["s2"]); o.append(blk["o"][None])
                 win = []
