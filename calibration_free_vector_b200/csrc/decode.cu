@@ -531,7 +531,7 @@ __global__ void __launch_bounds__(32 * DEC_WARPS, 1)
 decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype, int64_t qsb, int64_t qsh,
               float qscale, const float* __restrict__ cbk_g, const float* __restrict__ cbv_g,
               unsigned int* __restrict__ counters, float* __restrict__ ws, float* __restrict__ out, int n_q_heads,
-              DecodeGeom geom, const float* __restrict__ rscores, int rs_cap) {
+              DecodeGeom geom, const float* __restrict__ rscores, int rs_cap, int nw_cut, int64_t out_sb) {
   static_assert(GH == 1 || GH == 2 || GH == 4, "1, 2 or 4 heads per warp");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
@@ -569,7 +569,13 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
   const uint4 cb_row = cb_row_f16(cb_isv ? cbv_g : cbk_g, cb_c);
 
   const int nq = active ? min(min(kc.n_quant[seq], vc.n_quant[seq]), kc.capacity) : 0;
-  const int nw = (kc.window_len > 0) ? max(0, min(min(kc.n_window[seq], vc.n_window[seq]), kc.window_len)) : 0;
+  // nw_cut > 0 (chunked-prefill queries): the last nw_cut window tokens lie after
+  // this query and are not attended; status bit 8 if the query's own token is not
+  // in the window.
+  const int nw_all = (kc.window_len > 0) ? max(0, min(min(kc.n_window[seq], vc.n_window[seq]), kc.window_len)) : 0;
+  const int nw = max(0, nw_all - nw_cut);
+  if (nw_cut > 0 && active && split == 0 && hg == 0 && lane == 0 && nw_all <= nw_cut && kc.status)
+    atomicOr(kc.status, 8);
   // Splits are dealt whole 64-token stages, so a split may start or end inside
   // a 128-token block (the block's mean terms are then split between them too).
   const int nst_all = (nq + STAGE_TOK - 1) / STAGE_TOK;
@@ -919,7 +925,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     const int mseq = sm.merge_seq[m], mhg = sm.merge_hg[m];
     const int mb = mseq / kc.n_kv_heads, mhk = mseq % kc.n_kv_heads;
     cta_merge<GH>(ws, ws + acc_offset(P, G), (int64_t)mseq * (nsplit + 1), nsplit, G, mhg * GH,
-                  out + ((int64_t)mb * n_q_heads + mhk * G + mhg * GH) * D, scratch);
+                  out + (int64_t)mb * out_sb + (int64_t)(mhk * G + mhg * GH) * D, scratch);
   }
 }
 
@@ -1322,7 +1328,8 @@ size_t decode_workspace_bytes(int batch, int n_kv_heads, const DecodeGeom& geom)
 template <int G, int MK, int MV, bool DQ>
 static cudaError_t launch_t(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
                             int64_t qsb, int64_t qsh, float qscale, const float* cbk, const float* cbv, float* out,
-                            unsigned int* counters, float* partials, const DecodeGeom& geom, cudaStream_t s) {
+                            unsigned int* counters, float* partials, const DecodeGeom& geom, cudaStream_t s,
+                            int nw_cut, int64_t out_sb) {
   constexpr int GH = G < 4 ? G : 4;  // heads per warp job
   const size_t smem = sizeof(DecSmem);
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<GH, MK, MV, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1331,19 +1338,21 @@ static cudaError_t launch_t(const CacheView& kc, const CacheView& vc, const void
   const int nwarps = kc.batch * kc.n_kv_heads * geom.nsplit_q * (G / GH);
   dim3 grid((nwarps + DEC_WARPS - 1) / DEC_WARPS);
   decode_kernel<GH, MK, MV, DQ><<<grid, 32 * DEC_WARPS, smem, s>>>(kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv,
-                                                               counters, partials, out, n_q_heads, geom, nullptr, 0);
+                                                               counters, partials, out, n_q_heads, geom, nullptr, 0,
+                                                               nw_cut, out_sb);
   return cudaGetLastError();
 }
 
 template <int G>
 static cudaError_t launch_g(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
                             int64_t qsb, int64_t qsh, float qscale, const float* cbk, const float* cbv, float* out,
-                            unsigned int* counters, float* partials, const DecodeGeom& geom, cudaStream_t s) {
+                            unsigned int* counters, float* partials, const DecodeGeom& geom, cudaStream_t s,
+                            int nw_cut, int64_t out_sb) {
 #define NSN_LAUNCH(MK_, MV_)                                                                                    \
   return kc.dq ? launch_t<G, MK_, MV_, true>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters,  \
-                                             partials, geom, s)                                                       \
+                                             partials, geom, s, nw_cut, out_sb)                                       \
                : launch_t<G, MK_, MV_, false>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, \
-                                              partials, geom, s)
+                                              partials, geom, s, nw_cut, out_sb)
   if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_1BIT) NSN_LAUNCH(1, 1);
   if (kc.mode == NSN_MODE_1BIT && vc.mode == NSN_MODE_2BIT) NSN_LAUNCH(1, 2);
   if (kc.mode == NSN_MODE_2BIT && vc.mode == NSN_MODE_1BIT) NSN_LAUNCH(2, 1);
@@ -1354,14 +1363,19 @@ static cudaError_t launch_g(const CacheView& kc, const CacheView& vc, const void
 static cudaError_t launch_any(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
                               int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
                               float* out, unsigned int* counters, float* partials, const DecodeGeom& geom,
-                              cudaStream_t s) {
+                              cudaStream_t s, int nw_cut = 0, int64_t out_sb = -1) {
   const float qscale = softmax_scale * LOG2E;
+  if (out_sb < 0) out_sb = (int64_t)n_q_heads * D;
+#define NSN_G(G_) \
+  return launch_g<G_>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s, \
+                      nw_cut, out_sb)
   switch (geom.g) {
-    case 1: return launch_g<1>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
-    case 2: return launch_g<2>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
-    case 4: return launch_g<4>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
-    default: return launch_g<8>(kc, vc, q, dtype, n_q_heads, qsb, qsh, qscale, cbk, cbv, out, counters, partials, geom, s);
+    case 1: NSN_G(1);
+    case 2: NSN_G(2);
+    case 4: NSN_G(4);
+    default: NSN_G(8);
   }
+#undef NSN_G
 }
 
 cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
@@ -1370,6 +1384,27 @@ cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* 
   unsigned int* counters = static_cast<unsigned int*>(ws);
   float* partials = static_cast<float*>(ws) + counter_words((int64_t)kc.batch * kc.n_kv_heads);
   return launch_any(kc, vc, q, dtype, n_q_heads, qsb, qsh, softmax_scale, cbk, cbv, out, counters, partials, geom, s);
+}
+
+// Chunked-prefill ("extend") attention: the last n_queries tokens of every
+// sequence sit in the residual window; query i attends the quantized part and the
+// window up to its own slot.  One decode pass per query, each with the window
+// shortened by the n_queries - 1 - i tokens that follow it, all sharing the
+// workspace (stream-ordered; the merge counters return to zero after each pass).
+cudaError_t launch_extend(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                          int n_queries, int64_t qsb, int64_t qst, int64_t qsh, float softmax_scale, const float* cbk,
+                          const float* cbv, float* out, void* ws, const DecodeGeom& geom, cudaStream_t s) {
+  unsigned int* counters = static_cast<unsigned int*>(ws);
+  float* partials = static_cast<float*>(ws) + counter_words((int64_t)kc.batch * kc.n_kv_heads);
+  const int64_t esz = dtype == NSN_DTYPE_F32 ? 4 : 2;
+  const int64_t out_sb = (int64_t)n_queries * n_q_heads * D;
+  for (int i = 0; i < n_queries; ++i) {
+    const cudaError_t e = launch_any(kc, vc, static_cast<const char*>(q) + (int64_t)i * qst * esz, dtype, n_q_heads,
+                                     qsb, qsh, softmax_scale, cbk, cbv, out + (int64_t)i * n_q_heads * D, counters,
+                                     partials, geom, s, n_queries - 1 - i, out_sb);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // ---- pre-RoPE keys: logits kernel, then decode_kernel<..., RP = true> ----
@@ -1420,7 +1455,8 @@ static cudaError_t launch_rope_t(const CacheView& kc, const CacheView& vc, const
   float* partials = static_cast<float*>(ws) + counter_words((int64_t)nseq);
   const int nwarps = nseq * geom.nsplit_q * (G / GH);
   decode_kernel<GH, NSN_MODE_2BIT, MV, DQ, true><<<(nwarps + DEC_WARPS - 1) / DEC_WARPS, 32 * DEC_WARPS, smem, s>>>(
-      kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, counters, partials, out, n_q_heads, geom, rscores, rs_cap);
+      kc, vc, q, dtype, qsb, qsh, qscale, cbk, cbv, counters, partials, out, n_q_heads, geom, rscores, rs_cap, 0,
+      (int64_t)n_q_heads * D);
   return cudaGetLastError();
 }
 

@@ -213,6 +213,35 @@ nsn_status nsn_decode_attention(const nsn_cache* k_cache, const nsn_cache* v_cac
                                         static_cast<cudaStream_t>(stream)));
 }
 
+nsn_status nsn_extend_attention(const nsn_cache* k_cache, const nsn_cache* v_cache, const void* q, int dtype,
+                                int n_q_heads, int n_queries, int64_t q_stride_b, int64_t q_stride_t,
+                                int64_t q_stride_h, float softmax_scale, const float* cb_k, const float* cb_v,
+                                float* out, void* workspace, size_t ws_bytes, void* stream) {
+  nsn_status st = check_cache(k_cache);
+  if (st != NSN_OK) return st;
+  st = check_cache(v_cache);
+  if (st != NSN_OK) return st;
+  if (!same_shape(k_cache, v_cache)) return NSN_ERR_INVALID_ARG;
+  if (k_cache->window == 0) return NSN_ERR_UNSUPPORTED;
+  if (n_queries < 1 || n_queries > k_cache->window) return NSN_ERR_INVALID_ARG;
+  if (!q || !cb_k || !cb_v || !out || !workspace || !valid_dtype(dtype)) return NSN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(cb_k) || !aligned16(cb_v) || !aligned16(out) || !aligned16(workspace))
+    return NSN_ERR_INVALID_ARG;
+  if (n_q_heads <= 0 || n_q_heads % k_cache->n_kv_heads) return NSN_ERR_INVALID_ARG;
+  const int g = n_q_heads / k_cache->n_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return NSN_ERR_UNSUPPORTED;
+  const int64_t e16 = elems16(dtype);
+  if (q_stride_b < 0 || q_stride_t < 0 || q_stride_h < 0 || q_stride_b % e16 || q_stride_t % e16 ||
+      q_stride_h % e16)
+    return NSN_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return NSN_ERR_INVALID_ARG;
+  const nsn::DecodeGeom geom = nsn::decode_geometry(k_cache->batch, k_cache->capacity, n_q_heads, k_cache->n_kv_heads);
+  if (ws_bytes < nsn::decode_workspace_bytes(k_cache->batch, k_cache->n_kv_heads, geom)) return NSN_ERR_WORKSPACE;
+  return cuda_status(nsn::launch_extend(view(k_cache), view(v_cache), q, dtype, n_q_heads, n_queries, q_stride_b,
+                                        q_stride_t, q_stride_h, softmax_scale, cb_k, cb_v, out, workspace, geom,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 size_t nsn_decode_rope_workspace_bytes(const nsn_cache* k_cache, int n_q_heads) {
   if (check_cache(k_cache) != NSN_OK || n_q_heads <= 0 || n_q_heads % k_cache->n_kv_heads) return 0;
   const nsn::DecodeGeom g = nsn::decode_geometry(k_cache->batch, k_cache->capacity, n_q_heads, k_cache->n_kv_heads);

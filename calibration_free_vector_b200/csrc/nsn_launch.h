@@ -56,6 +56,11 @@ cudaError_t launch_decode(const CacheView& kc, const CacheView& vc, const void* 
                           int64_t qsb, int64_t qsh, float softmax_scale, const float* cbk, const float* cbv,
                           float* out, void* ws, const DecodeGeom& geom, cudaStream_t s);
 
+// Chunked-prefill attention of the last n_queries window tokens (causal inside the window).
+cudaError_t launch_extend(const CacheView& kc, const CacheView& vc, const void* q, int dtype, int n_q_heads,
+                          int n_queries, int64_t qsb, int64_t qst, int64_t qsh, float softmax_scale, const float* cbk,
+                          const float* cbv, float* out, void* ws, const DecodeGeom& geom, cudaStream_t s);
+
 // Pre-RoPE keys: the K logits (keys rotated at their positions by inv_freq) into
 // the workspace after the decode partials, then the decode over them.
 size_t decode_rope_workspace_bytes(int batch, int n_kv_heads, int capacity, int window_len, const DecodeGeom& geom);

@@ -95,6 +95,10 @@ def load():
     lib.nsn_decode_attention.argtypes = [POINTER(nsn_cache), POINTER(nsn_cache), c_void_p, c_int, c_int, c_int64,
                                          c_int64, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                          c_void_p]
+    lib.nsn_extend_attention.restype = c_int
+    lib.nsn_extend_attention.argtypes = [POINTER(nsn_cache), POINTER(nsn_cache), c_void_p, c_int, c_int, c_int,
+                                         c_int64, c_int64, c_int64, c_float, c_void_p, c_void_p, c_void_p, c_void_p,
+                                         c_size_t, c_void_p]
     lib.nsn_decode_rope_workspace_bytes.restype = c_size_t
     lib.nsn_decode_rope_workspace_bytes.argtypes = [POINTER(nsn_cache), c_int]
     lib.nsn_decode_attention_rope.restype = c_int
@@ -304,6 +308,23 @@ def nsn_decode_attention(k_cache: Cache, v_cache: Cache, q, softmax_scale: float
                                      cb_k.data_ptr(), cb_v.data_ptr(), out.data_ptr(), workspace.data_ptr(),
                                      workspace.numel(), _stream_ptr(stream))
     _check(st, "nsn_decode_attention")
+
+
+def nsn_extend_attention(k_cache: Cache, v_cache: Cache, q, softmax_scale: float, cb_k, cb_v, out, workspace,
+                         stream=None) -> None:
+    """Chunked-prefill attention: q [B, C, H_q, 128] (the last C tokens of every
+    sequence, all in the residual window) -> out [B, C, H_q, 128] float32; query i
+    attends the quantized part and the window up to its own token."""
+    if q.dim() != 4 or q.shape[-1] != HEAD_DIM or q.stride(-1) != 1:
+        raise ValueError("q must be [B, C, H_q, 128] with a contiguous last dimension")
+    import torch
+    if out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must be a contiguous float32 tensor shaped like q")
+    st = load().nsn_extend_attention(ctypes.byref(k_cache.c), ctypes.byref(v_cache.c), q.data_ptr(),
+                                     _dtype_code(q), q.shape[2], q.shape[1], q.stride(0), q.stride(1), q.stride(2),
+                                     float(softmax_scale), cb_k.data_ptr(), cb_v.data_ptr(), out.data_ptr(),
+                                     workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(st, "nsn_extend_attention")
 
 
 def nsn_decode_rope_workspace_bytes(k_cache: Cache, n_q_heads: int) -> int:

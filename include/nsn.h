@@ -84,7 +84,8 @@ typedef enum { NSN_DTYPE_F32 = 0, NSN_DTYPE_BF16 = 1, NSN_DTYPE_F16 = 2 } nsn_dt
  *   status   int32  [1] or NULL                         device error bits, OR-ed by kernels:
  *                                                       1 = capacity overflow on flush,
  *                                                       2 = decode copy timeout,
- *                                                       4 = ragged prefill length out of range
+ *                                                       4 = ragged prefill length out of range,
+ *                                                       8 = chunked-prefill query not in the window
  * capacity must be a positive multiple of 128.  window must be 0 (quantize every
  * token, no append) or 128 (KIVI-style residual of one block).
  *
@@ -284,6 +285,34 @@ nsn_status nsn_decode_attention(const nsn_cache* k_cache, const nsn_cache* v_cac
                                 int64_t q_stride_h, float softmax_scale, const float* cb_k,
                                 const float* cb_v, float* out, void* workspace, size_t ws_bytes,
                                 void* stream);
+
+/*
+ * Chunked-prefill ("extend") attention over the compressed cache ([TS] Metodologia 4:
+ * the quantized part and the full-precision residual window; [GH] Note on the split
+ * between them at prefill).  After a chunk of n_queries tokens has been added to the
+ * cache (they are the last n_queries tokens of every sequence and all sit in the
+ * residual window), query i of the chunk (position P - n_queries + i, P = n_quant +
+ * n_window) attends every quantized token and the window tokens up to its own:
+ *   out[b][i][h] = softmax_scale-softmax attention of q[b][i][h] over
+ *                  { k_hat_t : t < n_quant } U { window slots 0 .. n_window - n_queries + i }
+ * with the decode's arithmetic (nsn_decode_attention) for each query.
+ *   q          device, dtype, query (b, i, h) at q + b*q_stride_b + i*q_stride_t +
+ *              h*q_stride_h (elements), 128 contiguous values; all strides multiples of
+ *              16 bytes.
+ *   n_queries  1 .. window (the caches' window must be 128).
+ *   out        device float [batch][n_queries][n_q_heads][128].
+ *   workspace  as nsn_decode_attention (nsn_decode_workspace_bytes; zero-filled before
+ *              its first use), reused by every query of the chunk.
+ * Runs as n_queries passes of the decode kernel (one per query, stream-ordered), each
+ * with the window shortened by the tokens that follow its query.  A sequence whose
+ * window holds fewer than n_queries tokens sets status bit 8 (its queries then see
+ * fewer window tokens).  Errors as nsn_decode_attention; NSN_ERR_UNSUPPORTED for a
+ * cache without a window.
+ */
+nsn_status nsn_extend_attention(const nsn_cache* k_cache, const nsn_cache* v_cache, const void* q, int dtype,
+                                int n_q_heads, int n_queries, int64_t q_stride_b, int64_t q_stride_t,
+                                int64_t q_stride_h, float softmax_scale, const float* cb_k, const float* cb_v,
+                                float* out, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Pre-RoPE keys ([TS] Metodologia 4: NSN is applied to the keys BEFORE the rotary

@@ -375,6 +375,24 @@ def decode_attention(q_group: np.ndarray, kq: dict, vq: dict, k_window: np.ndarr
     return attention(q_group, keys, vals, scale)
 
 
+def extend_attention(q_chunk: np.ndarray, kq: dict, vq: dict, k_window: np.ndarray,
+                     v_window: np.ndarray, codebook_k, codebook_v, mode_k: int,
+                     mode_v: int, scale: float, block: int = 128) -> np.ndarray:
+    """Chunked-prefill attention of the last C tokens of one sequence, which all
+    sit in the residual window ([TS] Metodologia 4: quantized part + residual).
+
+    q_chunk [C, g, d]: query i (the token at window slot n_window - C + i) attends
+    every dequantized token and the window slots 0 .. n_window - C + i.  Returns
+    [C, g, d]: for each query the decode attention over that causal prefix.
+    """
+    q_chunk = np.asarray(q_chunk, dtype=np.float64)
+    C, nw = q_chunk.shape[0], np.asarray(k_window).shape[0]
+    if C > nw:
+        raise ValueError("every query of the chunk must be a window token")
+    return np.stack([decode_attention(q_chunk[i], kq, vq, k_window[:nw - C + 1 + i], v_window[:nw - C + 1 + i],
+                                      codebook_k, codebook_v, mode_k, mode_v, scale, block) for i in range(C)])
+
+
 # ---------------------------------------------------------------------------
 # Rotary position embedding of the keys -- [TS] Metodologia 4: NSN is applied to
 # the keys BEFORE the rotary position embedding, so the cache holds pre-RoPE keys

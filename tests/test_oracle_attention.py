@@ -176,3 +176,34 @@ def test_stored_s2_preserves_the_component_along_u(mode):
     xraw = orc.dequantize(raw["codes"], raw["signs"], raw["s1"], raw["s2"], raw["o"][None, :], cb, mode)
     along_raw = np.einsum("td,td->t", xraw - x, v) / np.einsum("td,td->t", v, v)
     assert np.median(np.abs(along_raw)) > 10 * np.abs(along).max()
+
+
+def test_extend_attention_is_causal_attention_over_the_cache():
+    # chunked prefill: C queries, the chunk's tokens at the end of the window.  The
+    # same result as plain softmax attention over [dequantized keys, window keys]
+    # with a causal mask on the window part; the last query is the decode of the
+    # full cache; changing window tokens after query i leaves query i unchanged.
+    rng = np.random.default_rng(23)
+    d, g, C, nw = 128, 3, 5, 9
+    cb = np.abs(rng.standard_normal((256, 8)))
+    x = rng.standard_normal((256, d))
+    kq = orc.quantize_sequence(x, cb, orc.MODE_2BIT, 128, 0)
+    vq = orc.quantize_sequence(x[::-1].copy(), cb, orc.MODE_2BIT, 128, 0)
+    kw, vw = rng.standard_normal((nw, d)), rng.standard_normal((nw, d))
+    q = rng.standard_normal((C, g, d))
+    got = orc.extend_attention(q, kq, vq, kw, vw, cb, cb, 2, 2, 0.1)
+    khat = orc.dequantize(kq["codes"], kq["signs"], kq["s1"], kq["s2"], kq["o"], cb, 2)
+    vhat = orc.dequantize(vq["codes"], vq["signs"], vq["s1"], vq["s2"], vq["o"], cb, 2)
+    keys, vals = np.concatenate([khat, kw]), np.concatenate([vhat, vw])
+    for i in range(C):
+        s = q[i] @ keys.T * 0.1
+        s[:, 256 + nw - C + 1 + i:] = -np.inf    # window slots after query i
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        assert np.abs(got[i] - p @ vals).max() < 1e-12
+    full = orc.decode_attention(q[-1], kq, vq, kw, vw, cb, cb, 2, 2, 0.1)
+    assert np.abs(got[-1] - full).max() < 1e-15
+    kw2 = kw.copy()
+    kw2[nw - C + 2:] += 5.0                      # tokens after query 0
+    again = orc.extend_attention(q, kq, vq, kw2, vw, cb, cb, 2, 2, 0.1)
+    assert np.array_equal(again[0], got[0]) and not np.allclose(again[-1], got[-1])
