@@ -586,7 +586,7 @@ def run_ours(args):
                          "ms": quant_ms_best, "gbs": q_bytes / (quant_ms_best * 1e-3) / 1e9,
                          "hbm_frac": q_bytes / (quant_ms_best * 1e-3) / 1e9 / hbm,
                          "hbm_frac_of_8tbs_spec": q_bytes / (quant_ms_best * 1e-3) / 1e9 / 8000.0,
-                         "roofline": {"kernel": "quantize_prefill_kernel", "bound": "tensor", "achieved": q_ach,
+                         "roofline": {"kernel": "quantize_prefill_ws_kernel", "bound": "tensor", "achieved": q_ach,
                                       "peak": tc_peak, "unit": "TFLOP/s", "frac": q_ach / tc_peak,
                                       "peak_kind": peak_kind,
                                       "algorithmic_flop_per_token_head": 2 * mac_per_th,

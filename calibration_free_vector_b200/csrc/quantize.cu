@@ -5,9 +5,12 @@
 // 2 (Hadamard), 3 (VQ with one global codebook, adaptive scale) and 4 (KIVI-style
 // residual that is flushed into the quantized part when full).
 //
-// One CTA of 256 threads quantizes blocks of <= 128 tokens of one (batch,
-// kv-head) at a time (a persistent loop over blocks on prefill); the adjacent
-// lanes 2t, 2t+1 own token t (64 dims, 8 sub-vectors each) during NSN.  Per block:
+// Prefill runs one persistent, warp-specialized CTA per SM (quantize_prefill_ws_kernel):
+// 8 normalizer warps run the NSN of one block of <= 128 tokens of a (batch, kv-head)
+// while two warpgroups of search warps find the codewords of the previous block.
+// Residual-window flushes run one CTA of 256 threads per block (append_kernel).
+// In NSN the adjacent lanes 2t, 2t+1 of the normalizers own token t (64 dims, 8
+// sub-vectors each).  Per block:
 //   r      = column mean of the raw tokens (fp64 sum, stored as fp32)
 //   d_t    = FWHT(x_t - r)                 fp32, in registers (exact algebra:
 //   w_t    = d_t + FWHT(r)                 FWHT is linear; FWHT(r) in fp64)
@@ -27,11 +30,11 @@
 // The first MMA writes the bias (A = [1, 1, 0...], B = the fp16 hi and lo parts of
 // -||c_k||^2/2), the second adds K = [a_hi | a_lo] (the fp32 a split into two fp16
 // parts, exact to 2^-22) times [c | c] (the codebook in fp16).  Each TMEM lane
-// holds one sub-vector's 256 scores; a warp pair reads them back with tcgen05.ld
-// (each warp half of the columns) and keeps, with three-input max trees, the best
-// and second-best maxima of the groups of 8 codewords (the group number rides in
-// the low mantissa bits).  The 8 codewords of the winning group are then rescanned
-// in sequential fp32.  Whenever a rival lies within the error bounds of the best
+// holds one sub-vector's 256 scores; its thread reads them back with tcgen05.ld and
+// keeps, with three-input max trees, the best and second-best maxima of the groups
+// of 8 codewords (the group number rides in the low mantissa bits).  The 8
+// codewords of the winning group are then rescanned in sequential fp32 from an fp32
+// copy of the codebook in shared memory.  Whenever a rival lies within the error bounds of the best
 // (the fp32 bound inside the group, that plus a wide tensor-accumulation bound
 // outside it), the sub-vector is re-decided exactly in fp64 by a whole warp over
 // all codewords inside the bound (ties to the lowest index).  The stored code is
@@ -118,36 +121,42 @@ constexpr int QTHREADS = 2 * BLK;  // two threads per token
 constexpr int HD = D / 2;           // dims per thread
 constexpr int HSUB = NSUB / 2;      // sub-vectors per thread
 constexpr int MBAR_POLLS = 1 << 22;  // bounded wait for the MMAs of one tile
-// Where the exact arithmetic reads codeword k and its bias: the two fp16 replicas
-// of the shared table with fp32 biases (fp16-representable codebook), the fp32
-// codebook in global memory with the fp32 biases (any other codebook), or the
-// fp32 unit codewords c_hat of the table with bias 0 (cosine assignment).
+// Kind of the staged codebook: fp16-representable (the tensor-core operand is exact),
+// any other (the operand is its fp16 rounding), or the unit codewords c_hat of the
+// cosine assignment (operand c_hat_hi, second operand c_hat_lo, bias 0).
 constexpr int TAB_F16 = 0, TAB_GLOBAL = 1, TAB_COSINE = 2;
 
-struct QuantSmem {
-  // ---- operands of the tensor-core scores (staged once per CTA) ----
-  alignas(1024) unsigned char bop[NCODES * 32];   // B: codebook fp16 [c | c], K-major canonical layout
+// Shared-memory state of the quantizer, in four parts so that a warp-specialized
+// CTA can keep two blocks in flight: the staged codebook (per launch), the search's
+// operands and barriers, the NSN scratch, and one block's data.
+struct QTables {
+  // ---- operands of the tensor-core scores ----
+  alignas(128) unsigned char bop[NCODES * 32];    // B: codebook fp16 [c | c], K-major canonical layout
   alignas(128) unsigned char bop2[NCODES * 16];   // B of the bias MMA: per codeword [b_hi, b_lo, 0 x 6]; K half 1 aliases K half 0
   alignas(128) unsigned char aop2[256];           // A of the bias MMA: one core matrix of rows [1, 1, 0 ...] + a zero one
-  alignas(128) unsigned char aop[2][BLK * 32];    // A: [a_hi | a_lo] of the 128 rows of a tile (double-buffered)
-  // ---- codebook for the exact arithmetic, two interleaved replicas: replica p of codeword k = 8G + j (fp16,
-  // 16 B) at byte 256 G + 32 j + 16 p, so its 16-byte bank group is 2 j + p whatever the group; its bias
-  // -||c_k||^2/2 (fp32, sequential) at word 16 G + 2 j + p of cbias.  Lanes 4p .. 4p+3 of a quarter warp
-  // read replica p and rotate the codeword order by lane, so the 8 lanes of a phase hit 8 different bank
-  // groups (codewords) and 8 different banks (biases). ----
-  alignas(16) unsigned char cbtab[NCODES * 32];
-  alignas(16) float cbias[2 * NCODES];
+  // ---- codebook for the exact arithmetic (fp32: c, or c_hat for the cosine assignment), two
+  // replicas: replica p of codeword k at floats 16 k + 8 p .. 16 k + 8 p + 7, so a 16-byte half h of it
+  // lies in bank group 4 (k & 1) + 2 p + h.  The bias -||c_k||^2/2 (fp32, sequential; 0 for the cosine
+  // assignment) in four replicas, replica r at word 4 k + r.  A search lane l reads codeword 8 G + ((i + l) & 7)
+  // from replica (l >> 2) & 1, half (l >> 1) & 1 first, and bias replica l >> 3: the 8 lanes of a phase hit
+  // 8 different bank groups, and the 32 lanes 32 different bias banks, whatever their groups G. ----
+  alignas(16) float cw[NCODES * 16];
+  alignas(16) float cbias[NCODES * 4];
   alignas(16) float cnorm[4];                     // [0] max ||c||, [1] max ||c||^2, [2] max ||c - fp16(c)|| (rounded up)
   int tab;                                        // TAB_F16, TAB_GLOBAL or TAB_COSINE
-  alignas(8) unsigned long long mbar;             // MMA completion barrier
+};
+
+struct QSearch {
+  alignas(128) unsigned char aop[2][BLK * 32];    // A: [a_hi | a_lo] of the 128 rows of a tile (double-buffered)
+  alignas(8) unsigned long long mbar[2];          // MMA completion barriers (one per tensor-memory buffer)
   uint32_t tmem;                                  // tensor-memory base address of this CTA
   int nflag;
-  // ---- per block ----
+  alignas(16) uint16_t flag[BLK * NSUB];          // (token, sub-vector) pairs for the exact re-decision
+};
+
+struct QNsn {
   alignas(16) double rr[BLK];          // 1 / ||x_t|| (0 for a zero token)
-  alignas(16) double s1[BLK];          // per-token s1 and s2 (fp64) until the final store
-  alignas(16) double s2[BLK];
   alignas(16) float r[D];              // column mean of raw tokens (fp32)
-  alignas(16) float tile[BLK][D + 4];  // raw tokens, then d_t rows, then u rows (|u| in 2-bit mode); padded by 16 B
   union {                              // NSN column sums, then the search's warp-pair exchanges
     struct {
       double part[2][D];               // per-half column partial sums
@@ -161,43 +170,78 @@ struct QuantSmem {
       float4 xch2[BLK];                // rescan (best, second, index) of the upper half
     };
   };
-  alignas(16) uint8_t code[BLK][NSUB]; // chosen codes
-  alignas(16) uint16_t flag[BLK * NSUB];  // (token, sub-vector) pairs for the exact re-decision
   // double quantization
-  alignas(16) double ofull[D];         // o of the block (fp64) until its levels are formed
   alignas(16) double red[2][QTHREADS / 32][2];  // per-warp (min, max) of s1 and of o
   alignas(16) double dq[2][3];         // (lo, hi, step) of s1 and of o
   alignas(16) uint8_t lev[2][BLK];     // 4-bit levels of s1 (per token) and of o (per channel)
 };
 
-// Tensor-memory allocation and the MMA barrier of one CTA (all QTHREADS threads).
-struct TcState {
-  uint32_t tmem;
-  uint32_t phase;
+struct QBlock {
+  alignas(16) float tile[BLK][D + 4];  // raw tokens, then d_t rows, then u rows (|u| in 2-bit mode); padded by 16 B
+  alignas(16) double s1[BLK];          // per-token s1 and s2 (fp64) until the final store
+  alignas(16) double s2[BLK];
+  alignas(16) double ofull[D];         // o of the block (fp64) until its levels are formed
+  alignas(16) uint8_t code[BLK][NSUB]; // chosen codes
 };
 
-__device__ TcState tc_setup(QuantSmem& sm) {
-  const int t = threadIdx.x;
-  if (t == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(q_smem(&sm.mbar)));
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+// One CTA, one block at a time (2 CTAs per SM): prefill flushes of the residual window.
+struct QuantSmem {
+  QTables tb;
+  QSearch se;
+  QNsn ns;
+  QBlock bk;
+};
+
+// The parts a phase works on (the warp-specialized CTA passes one of its two blocks).
+struct QRefs {
+  QTables* tb;
+  QSearch* se;
+  QNsn* ns;
+  QBlock* bk;
+};
+
+__device__ __forceinline__ QRefs refs(QuantSmem& sm) { return QRefs{&sm.tb, &sm.se, &sm.ns, &sm.bk}; }
+
+// A set of threads that synchronize among themselves: the whole CTA (id 0,
+// __syncthreads) or `n` threads on named barrier `id`; t = index within the set.
+struct Grp {
+  int id, n, t;
+  __device__ __forceinline__ void sync() const {
+    if (id == 0) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory");
   }
+};
+__device__ __forceinline__ Grp cta_grp() { return Grp{0, (int)blockDim.x, (int)threadIdx.x}; }
+
+// Tensor-memory allocation and the MMA barriers of one CTA.
+struct TcState {
+  uint32_t tmem;
+  uint32_t phase;  // parity bit per barrier
+  uint32_t ncols;
+};
+
+// Allocates `ncols` tensor-memory columns (warp 0) and initialises `nbar` MMA
+// barriers; every thread of the CTA calls it.
+__device__ TcState tc_setup(QSearch& se, uint32_t ncols, int nbar) {
+  const int t = threadIdx.x;
+  if (t < nbar) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(q_smem(&se.mbar[t])));
+  if (t == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   if ((t >> 5) == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 :: "r"(q_smem(&sm.tmem)), "r"(TC_COLS));
+                 :: "r"(q_smem(&se.tmem)), "r"(ncols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  return TcState{sm.tmem, 0u};
+  return TcState{se.tmem, 0u, ncols};
 }
 
 __device__ void tc_teardown(const TcState& tcs) {
   tc_fence_before();
   __syncthreads();
   if ((threadIdx.x >> 5) == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tcs.tmem), "r"(TC_COLS));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tcs.tmem), "r"(tcs.ncols));
 }
 
 // Destination of the stored scalars of one block: either fp16 (s1, alpha*s2) pairs
@@ -235,7 +279,7 @@ __device__ __forceinline__ BlockOut block_out(const CacheView& c, int64_t seq, i
 // takes c_hat's fp16 high part as B, the second MMA (in place of the bias MMA)
 // adds the same A rows times its fp16 low part, the exact arithmetic reads the
 // fp32 c_hat from the table (bias 0), and the bounds are those of c_hat.
-__device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook, int cosine) {
+__device__ void stage_codebook(const QRefs& q, const float* __restrict__ codebook, int cosine) {
   const int t = threadIdx.x;
   float my_max = 0.f, my_dev = 0.f;
   for (int k = t; k < NCODES; k += blockDim.x) {
@@ -264,39 +308,41 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
     }
     const float bias = -0.5f * ss;
     // B operand: K = 0..7 and 8..15 both hold the codeword (multiplied by a_hi and a_lo)
-    *reinterpret_cast<uint4*>(sm.bop + kmaj_off(k, 0)) = *reinterpret_cast<const uint4*>(ch);
-    *reinterpret_cast<uint4*>(sm.bop + kmaj_off(k, 8)) = *reinterpret_cast<const uint4*>(ch);
+    *reinterpret_cast<uint4*>(q.tb->bop + kmaj_off(k, 0)) = *reinterpret_cast<const uint4*>(ch);
+    *reinterpret_cast<uint4*>(q.tb->bop + kmaj_off(k, 8)) = *reinterpret_cast<const uint4*>(ch);
     uint4 brow = make_uint4(0u, 0u, 0u, 0u);
+    // fp32 codeword (c_hat) for the exact arithmetic, both replicas, and its bias replicas
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      *reinterpret_cast<float4*>(q.tb->cw + 16 * k + 8 * p) = c0;
+      *reinterpret_cast<float4*>(q.tb->cw + 16 * k + 8 * p + 4) = c1;
+    }
+    const float bstore = cosine ? 0.f : bias;
+    *reinterpret_cast<float4*>(q.tb->cbias + 4 * k) = make_float4(bstore, bstore, bstore, bstore);
     if (cosine) {
-      // fp32 c_hat for the exact arithmetic; second-MMA operand: fp16(c_hat - fp16(c_hat))
-      *reinterpret_cast<float4*>(sm.cbtab + 32 * k) = c0;
-      *reinterpret_cast<float4*>(sm.cbtab + 32 * k + 16) = c1;
+      // second-MMA operand: fp16(c_hat - fp16(c_hat))
       __half cl[SUB];
 #pragma unroll
       for (int i = 0; i < SUB; ++i) cl[i] = __float2half_rn(c[i] - __half2float(ch[i]));
       brow = *reinterpret_cast<const uint4*>(cl);
       e = 0.f;  // hi + lo carries c_hat to 2^-22, inside the tensor bound
     } else {
-      *reinterpret_cast<uint4*>(sm.cbtab + 32 * k) = *reinterpret_cast<const uint4*>(ch);
-      *reinterpret_cast<uint4*>(sm.cbtab + 32 * k + 16) = *reinterpret_cast<const uint4*>(ch);
-      sm.cbias[2 * k] = bias;
-      sm.cbias[2 * k + 1] = bias;
       // bias operand: (b_hi, b_lo) with b_hi + b_lo = bias to 2^-22 relative
       const __half bh = __float2half_rn(bias);
       const __half bl = __float2half_rn(bias - __half2float(bh));
       brow.x = (uint32_t)__half_as_ushort(bh) | ((uint32_t)__half_as_ushort(bl) << 16);
     }
-    *reinterpret_cast<uint4*>(sm.bop2 + (k >> 3) * 128 + (k & 7) * 16) = brow;
+    *reinterpret_cast<uint4*>(q.tb->bop2 + (k >> 3) * 128 + (k & 7) * 16) = brow;
     my_max = fmaxf(my_max, ss);
     my_dev = fmaxf(my_dev, e);
   }
   if (t < 16) {  // bias A operand: 8 rows [1, 1, 0, ...] (K half 0) and a zero core matrix (K half 1)
     const uint32_t one2 = 0x3C003C00u;  // fp16 (1, 1)
-    *reinterpret_cast<uint4*>(sm.aop2 + 16 * t) = t < 8 ? make_uint4(one2, 0u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(q.tb->aop2 + 16 * t) = t < 8 ? make_uint4(one2, 0u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
   }
   my_max = warp_max(my_max);
   my_dev = warp_max(my_dev);
-  __shared__ float red[QTHREADS / 32][2];
+  __shared__ float red[32][2];  // per-warp maxima (up to 32 warps)
   if ((t & 31) == 0) {
     red[t >> 5][0] = my_max;
     red[t >> 5][1] = my_dev;
@@ -310,47 +356,33 @@ __device__ void stage_codebook(QuantSmem& sm, const float* __restrict__ codebook
       e = fmaxf(e, red[w][1]);
     }
     m *= 1.0001f;  // upper bound on max ||c||^2 despite the fp32 rounding above
-    sm.cnorm[1] = m;
-    sm.cnorm[0] = sqrtf(m) * 1.0001f;
-    sm.cnorm[2] = e > 0.f ? sqrtf(e) * 1.001f : 0.f;  // 0 for a codebook of fp16 values
-    // where the exact arithmetic reads codewords (see codeword())
-    sm.tab = cosine ? TAB_COSINE : (e > 0.f ? TAB_GLOBAL : TAB_F16);
+    q.tb->cnorm[1] = m;
+    q.tb->cnorm[0] = sqrtf(m) * 1.0001f;
+    q.tb->cnorm[2] = e > 0.f ? sqrtf(e) * 1.001f : 0.f;  // 0 for a codebook of fp16 values
+    q.tb->tab = cosine ? TAB_COSINE : (e > 0.f ? TAB_GLOBAL : TAB_F16);
   }
   __syncthreads();
 }
 
-// Codeword k as the scores use it (fp32) and its bias, read as sm.tab says (replica
-// p of the fp16 table when that is the source).
-__device__ __forceinline__ float codeword(const QuantSmem& sm, const float* __restrict__ cb_global, int tab,
-                                          int k, int p, float (&c)[SUB]) {
-  if (tab == TAB_F16) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(sm.cbtab + 32 * k + 16 * p);
-    const __half2* hv = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(hv[i]);
-      c[2 * i] = f.x;
-      c[2 * i + 1] = f.y;
-    }
-    return sm.cbias[2 * k + p];
-  }
-  float4 c0, c1;
-  if (tab == TAB_COSINE) {
-    c0 = *reinterpret_cast<const float4*>(sm.cbtab + 32 * k);
-    c1 = *reinterpret_cast<const float4*>(sm.cbtab + 32 * k + 16);
-  } else {
-    c0 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB));
-    c1 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB) + 1);
-  }
+// Codeword k as the exact arithmetic uses it (fp32, natural order; c_hat for the cosine
+// assignment) from replica p of the table, and its bias.
+__device__ __forceinline__ float codeword(const QRefs& q, int k, int p, float (&c)[SUB]) {
+  const float4 c0 = *reinterpret_cast<const float4*>(q.tb->cw + 16 * k + 8 * p);
+  const float4 c1 = *reinterpret_cast<const float4*>(q.tb->cw + 16 * k + 8 * p + 4);
   c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
-  return tab == TAB_COSINE ? 0.f : sm.cbias[2 * k + p];
+  return q.tb->cbias[4 * k + p];
 }
 
 // Codeword k as stored in the codebook (the reconstruction's u_hat), fp32.
-__device__ __forceinline__ void codeword_given(const QuantSmem& sm, const float* __restrict__ cb_global, int tab,
+__device__ __forceinline__ void codeword_given(const QRefs& q, const float* __restrict__ cb_global, int tab,
                                                int k, int p, float (&c)[SUB]) {
-  if (tab == TAB_COSINE) tab = TAB_GLOBAL;
-  codeword(sm, cb_global, tab, k, p, c);
+  if (tab == TAB_COSINE) {
+    const float4 c0 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB));
+    const float4 c1 = __ldg(reinterpret_cast<const float4*>(cb_global + k * SUB) + 1);
+    c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+  } else {
+    codeword(q, k, p, c);
+  }
 }
 
 __device__ __forceinline__ double shfl_pair_sum(double x) { return x + __shfl_xor_sync(0xffffffffu, x, 1); }
@@ -372,50 +404,50 @@ __device__ __forceinline__ double warp_max_d(double x) {
 //   lo = fp16(min), hi = fp16(max), step = (hi - lo) / 15 (fp64),
 //   level = round-half-even((x - lo) / step) clamped to 0..15 (step = 0: level 0).
 // Threads 0..127 handle s1 (token t), threads 128..255 o (channel t - 128).
-// sm.s1 and sm.ofull hold the exact fp64 values.  All QTHREADS threads.
-__device__ void store_double_quant(QuantSmem& sm, int n, const BlockOut& bo) {
-  __syncthreads();  // sm.s1 of every token is final
-  const int t = threadIdx.x, grp = t >> 7, i = t & (BLK - 1), warp = t >> 5, lane = t & 31;
+// q.bk->s1 and q.bk->ofull hold the exact fp64 values.  All QTHREADS threads.
+__device__ void store_double_quant(const QRefs& q, const Grp& gr, int n, const BlockOut& bo) {
+  gr.sync();  // s1 of every token is final
+  const int t = gr.t, grp = t >> 7, i = t & (BLK - 1), warp = t >> 5, lane = t & 31;
   const bool have = grp == 1 || i < n;
-  const double x = grp == 0 ? (i < n ? sm.s1[i] : 0.0) : sm.ofull[i];
+  const double x = grp == 0 ? (i < n ? q.bk->s1[i] : 0.0) : q.bk->ofull[i];
   const double mn = warp_min_d(have ? x : INFINITY), mx = warp_max_d(have ? x : -INFINITY);
   if (lane == 0) {
-    sm.red[grp][warp & 3][0] = mn;
-    sm.red[grp][warp & 3][1] = mx;
+    q.ns->red[grp][warp & 3][0] = mn;
+    q.ns->red[grp][warp & 3][1] = mx;
   }
-  __syncthreads();
+  gr.sync();
   if (t < 2) {
     double a = INFINITY, b = -INFINITY;
     for (int w = 0; w < 4; ++w) {
-      a = fmin(a, sm.red[t][w][0]);
-      b = fmax(b, sm.red[t][w][1]);
+      a = fmin(a, q.ns->red[t][w][0]);
+      b = fmax(b, q.ns->red[t][w][1]);
     }
     const double lo = (double)__half2float(__double2half(a));
     const double hi = (double)__half2float(__double2half(b));
-    sm.dq[t][0] = lo;
-    sm.dq[t][1] = hi;
-    sm.dq[t][2] = (hi - lo) / 15.0;
+    q.ns->dq[t][0] = lo;
+    q.ns->dq[t][1] = hi;
+    q.ns->dq[t][2] = (hi - lo) / 15.0;
   }
-  __syncthreads();
+  gr.sync();
   {
-    const double lo = sm.dq[grp][0], step = sm.dq[grp][2];
+    const double lo = q.ns->dq[grp][0], step = q.ns->dq[grp][2];
     int level = 0;
     if (have && step > 0.0) level = (int)fmin(15.0, fmax(0.0, rint((x - lo) / step)));
-    sm.lev[grp][i] = (uint8_t)level;
+    q.ns->lev[grp][i] = (uint8_t)level;
   }
-  __syncthreads();
-  if (t < 64) bo.s1_levels[t] = (uint8_t)(sm.lev[0][2 * t] | (sm.lev[0][2 * t + 1] << 4));
-  else if (t < 128) bo.o_levels[t - 64] = (uint8_t)(sm.lev[1][2 * (t - 64)] | (sm.lev[1][2 * (t - 64) + 1] << 4));
+  gr.sync();
+  if (t < 64) bo.s1_levels[t] = (uint8_t)(q.ns->lev[0][2 * t] | (q.ns->lev[0][2 * t + 1] << 4));
+  else if (t < 128) bo.o_levels[t - 64] = (uint8_t)(q.ns->lev[1][2 * (t - 64)] | (q.ns->lev[1][2 * (t - 64) + 1] << 4));
   else if (t < 136) {
     const int k = t - 128;
-    const double v = k == 0 ? sm.dq[0][0] : k == 1 ? sm.dq[0][1] : k == 2 ? sm.dq[1][0] : k == 3 ? sm.dq[1][1] : 0.0;
+    const double v = k == 0 ? q.ns->dq[0][0] : k == 1 ? q.ns->dq[0][1] : k == 2 ? q.ns->dq[1][0] : k == 3 ? q.ns->dq[1][1] : 0.0;
     bo.params[k] = __double2half(v);
   }
 }
 
-// Nearest codeword of the sub-vectors of one block (rows of sm.tile: a = u, or |u|
-// in 2-bit mode; rows of tokens past n are zero), written to sm.code.  Sub-vectors
-// whose decision lies within the error bounds are appended to sm.flag for the
+// Nearest codeword of the sub-vectors of one block (rows of q.bk->tile: a = u, or |u|
+// in 2-bit mode; rows of tokens past n are zero), written to q.bk->code.  Sub-vectors
+// whose decision lies within the error bounds are appended to q.se->flag for the
 // exact re-decision.  All QTHREADS threads.
 //
 // Tile t = tokens 8t .. 8t+7: row L (TMEM lane L) = token 8t + L/16, sub-vector L%16.
@@ -440,28 +472,28 @@ __device__ void store_double_quant(QuantSmem& sm, int n, const BlockOut& bo) {
 //       fp16-representable; the group number adds at most 32 ulp to a maximum.
 //       A rival inside the group within twice the fp32 bound, or another group's
 //       maximum within the fp32 plus the tensor bound, flags the sub-vector.
-__device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restrict__ cb_global, int n,
+__device__ void search_block(const QRefs& q, TcState& tcs, const float* __restrict__ cb_global, int n,
                              int32_t* status) {
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int q = warp & 3, hf = warp >> 2;
-  const int L = 32 * q + lane;
-  const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1], cdel = sm.cnorm[2];
-  const int tab = sm.tab;
+  const int qd = warp & 3, hf = warp >> 2;
+  const int L = 32 * qd + lane;
+  const float cmax = q.tb->cnorm[0], cmax2 = q.tb->cnorm[1], cdel = q.tb->cnorm[2];
+  const int tab = q.tb->tab;
   constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
   constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
-  const uint32_t taddr = tcs.tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * hf);
-  const uint64_t db = tc_desc(q_smem(sm.bop), 128, 256);
-  const uint64_t da2 = tc_desc(q_smem(sm.aop2), 128, 0);  // every 8-row group reads the same [1, 1, 0...] rows
-  const uint64_t db2 = tc_desc(q_smem(sm.bop2), 0, 128);  // K half 1 re-reads K half 0 (times A's zero half)
-  const uint32_t mbar = q_smem(&sm.mbar);
+  const uint32_t taddr = tcs.tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(128 * hf);
+  const uint64_t db = tc_desc(q_smem(q.tb->bop), 128, 256);
+  const uint64_t da2 = tc_desc(q_smem(q.tb->aop2), 128, 0);  // every 8-row group reads the same [1, 1, 0...] rows
+  const uint64_t db2 = tc_desc(q_smem(q.tb->bop2), 0, 128);  // K half 1 re-reads K half 0 (times A's zero half)
+  const uint32_t mbar = q_smem(&q.se->mbar[0]);
   const int ntiles = (n + 7) >> 3;
 
   // The A rows of a tile; the row's decision bounds are formed here too, off the
   // critical path of the decision: margin = twice the fp32 bound, mtc = the tensor bound.
   auto build_a = [&](int tile, float (&a)[SUB], float& margin, float& mtc) {
     const int tkk = 8 * tile + (L >> 4), j = L & 15;
-    const float4 a0 = *reinterpret_cast<const float4*>(&sm.tile[tkk][SUB * j]);
-    const float4 a1 = *reinterpret_cast<const float4*>(&sm.tile[tkk][SUB * j + 4]);
+    const float4 a0 = *reinterpret_cast<const float4*>(&q.bk->tile[tkk][SUB * j]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&q.bk->tile[tkk][SUB * j + 4]);
     a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
     a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
     float na = 0.f;
@@ -481,10 +513,10 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
         w[p] = h2_bits(__floats2half2_rn(a[2 * p] - back.x, a[2 * p + 1] - back.y));
       }
     }
-    *reinterpret_cast<uint4*>(sm.aop[tile & 1] + kmaj_off(L, 8 * hf)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(q.se->aop[tile & 1] + kmaj_off(L, 8 * hf)) = make_uint4(w[0], w[1], w[2], w[3]);
   };
   auto issue = [&](int tile) {
-    const uint64_t da = tc_desc(q_smem(sm.aop[tile & 1]), 128, 256);
+    const uint64_t da = tc_desc(q_smem(q.se->aop[tile & 1]), 128, 256);
     if (tab == TAB_COSINE) {  // D = [a_hi | a_lo] [c_hat_hi | c_hat_hi] + [a_hi | a_lo] [c_hat_lo | c_hat_lo]
       tc_mma(tcs.tmem, da, db, 0u);
       tc_mma(tcs.tmem, da, db2, 1u);
@@ -545,12 +577,12 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
     }
 
     // (4) merge the pair's halves; the scores are read, so the next tile may start
-    sm.xch1[hf][L] = make_float2(b1, b2);
+    q.ns->xch1[hf][L] = make_float2(b1, b2);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (t == 0 && tile + 1 < ntiles) issue(tile + 1);
-    const float2 o1 = sm.xch1[hf ^ 1][L];
+    const float2 o1 = q.ns->xch1[hf ^ 1][L];
     const float m1 = fmaxf(b1, o1.x);
     const float m2 = max3f(b2, o1.y, fminf(b1, o1.x));
     const int G = (int)(__float_as_uint(m1) & 31u);
@@ -565,7 +597,7 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         kk[i] = 8 * G + 4 * hf + ((i + lane) & 3);
-        sc[i] = codeword(sm, cb_global, tab, kk[i], rep, cw[i]);
+        sc[i] = codeword(q, kk[i], rep, cw[i]);
       }
 #pragma unroll
       for (int d = 0; d < SUB; ++d)
@@ -580,20 +612,20 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
         second = fmaxf(second, lo);
       }
     }
-    if (hf == 1) sm.xch2[L] = make_float4(best, second, __int_as_float(idx), 0.f);
-    asm volatile("bar.sync %0, 64;" :: "r"(1 + q) : "memory");  // the two warps of the pair only
+    if (hf == 1) q.ns->xch2[L] = make_float4(best, second, __int_as_float(idx), 0.f);
+    asm volatile("bar.sync %0, 64;" :: "r"(1 + qd) : "memory");  // the two warps of the pair only
 
     // (5) decision and bounds (lower warp of the pair)
     if (hf == 0) {
-      const float4 o2 = sm.xch2[L];
+      const float4 o2 = q.ns->xch2[L];
       second = max3f(second, o2.y, fminf(best, o2.x));
       idx = (o2.x > best) ? __float_as_int(o2.z) : idx;  // the upper half holds the larger indices
       best = fmaxf(best, o2.x);
       const float other = m2 + fabsf(m2) * 3.82e-6f;  // + 32 ulp: the group number in the low bits
       const int tkk = 8 * tile + (L >> 4), j = L & 15;
-      sm.code[tkk][j] = (uint8_t)idx;
+      q.bk->code[tkk][j] = (uint8_t)idx;
       const bool need = second >= best - margin || other >= best - 0.5f * margin - mtc;
-      if (need && tkk < n) sm.flag[atomicAdd(&sm.nflag, 1)] = (uint16_t)(tkk * NSUB + j);
+      if (need && tkk < n) q.se->flag[atomicAdd(&q.se->nflag, 1)] = (uint16_t)(tkk * NSUB + j);
     }
 #pragma unroll
     for (int i = 0; i < SUB; ++i) a[i] = an[i];
@@ -603,40 +635,37 @@ __device__ void search_block(QuantSmem& sm, TcState& tcs, const float* __restric
   __syncthreads();
 }
 
-// Quantizes one block of n (1..128) tokens with QTHREADS threads: thread
+// NSN of one block of n (1..128) tokens by a set of 256 threads: thread
 // t = 2 tk + h works on token tk, dims 64h .. 64h+63 (sub-vectors 8h .. 8h+7).
-// Rows are at src + row0 + tk*row_stride (elements).  Output pointers are
-// already offset to the block's first token (codes, signs, norms) and to its
-// mean row (means).
+// Rows are at src + row0 + tk*row_stride (elements).  Leaves the u rows (|u| in
+// 2-bit mode; zero rows past n) in q.bk->tile, s1 and s2 (fp64) in q.bk, o in
+// q.bk->ofull (double quantization) or stored; sign bits (2-bit) are stored.
 template <int DT, int MODE>
-__device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __restrict__ cb_global,
-                                   const void* __restrict__ src, int64_t row0,
-                                   int64_t row_stride, int n, uint8_t* __restrict__ codes,
-                                   uint8_t* __restrict__ signs, const CacheView& cv, int64_t seq,
-                                   int64_t tok0, int blk, int scale_adjust) {
-  const int t = threadIdx.x, tk = t >> 1, h = t & 1;
+__device__ void nsn_phase(const QRefs& q, const Grp& gr, const void* __restrict__ src, int64_t row0,
+                          int64_t row_stride, int n, uint8_t* __restrict__ signs, const CacheView& cv, int64_t seq,
+                          int blk) {
+  const int t = gr.t, tk = t >> 1, h = t & 1;
   const int col = t & (D - 1), rhalf = t >> 7;  // column-sum roles: column, half of the rows
   const bool valid = tk < n;
-  if (t == 0) sm.nflag = 0;  // read only after the barriers below
   constexpr int ESZ = (DT == NSN_DTYPE_F32) ? 4 : 2;
   constexpr int CHUNKS = D * ESZ / 16;  // 16-byte chunks per row
 
   // ---- cooperative, coalesced load of the raw tile into shared memory --------
   {
-    char* tile_bytes = reinterpret_cast<char*>(&sm.tile[0][0]);
+    char* tile_bytes = reinterpret_cast<char*>(&q.bk->tile[0][0]);
     constexpr int ROWB = (D + 4) * 4;  // padded row stride in bytes (fits both dtypes)
-    for (int q = t; q < BLK * CHUNKS; q += QTHREADS) {
-      const int row = q / CHUNKS, ch = q % CHUNKS;
+    for (int qq = t; qq < BLK * CHUNKS; qq += gr.n) {
+      const int row = qq / CHUNKS, ch = qq % CHUNKS;
       if (row < n) {
         const char* g = static_cast<const char*>(src) + (row0 + (int64_t)row * row_stride) * ESZ + ch * 16;
         *reinterpret_cast<uint4*>(tile_bytes + row * ROWB + ch * 16) = __ldg(reinterpret_cast<const uint4*>(g));
       }
     }
   }
-  __syncthreads();
+  gr.sync();
 
   auto raw_at = [&](int row, int c) -> float {
-    const char* tb = reinterpret_cast<const char*>(&sm.tile[0][0]) + row * (D + 4) * 4;
+    const char* tb = reinterpret_cast<const char*>(&q.bk->tile[0][0]) + row * (D + 4) * 4;
     if constexpr (DT == NSN_DTYPE_F32) return reinterpret_cast<const float*>(tb)[c];
     else if constexpr (DT == NSN_DTYPE_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(tb)[c]);
     else return __half2float(reinterpret_cast<const __half*>(tb)[c]);
@@ -659,19 +688,19 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
       s3 += raw_at(row + 3, col) - x0;
     }
     for (; row < hi; ++row) s0 += raw_at(row, col) - x0;
-    reinterpret_cast<float*>(&sm.part[0][0])[rhalf * D + col] = (s0 + s1) + (s2 + s3);
+    reinterpret_cast<float*>(&q.ns->part[0][0])[rhalf * D + col] = (s0 + s1) + (s2 + s3);
   }
-  __syncthreads();
+  gr.sync();
   if (t < D) {
-    const float* ps = reinterpret_cast<const float*>(&sm.part[0][0]);
-    sm.r[t] = raw_at(0, t) + (ps[t] + ps[D + t]) / (float)n;
+    const float* ps = reinterpret_cast<const float*>(&q.ns->part[0][0]);
+    q.ns->r[t] = raw_at(0, t) + (ps[t] + ps[D + t]) / (float)n;
   }
-  __syncthreads();
+  gr.sync();
   // FWHT(r) in fp64 by warp 0 (lane l holds elements 4l..4l+3).
   if (t < 32) {
     double v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = (double)sm.r[4 * t + i];
+    for (int i = 0; i < 4; ++i) v[i] = (double)q.ns->r[4 * t + i];
     double a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
     v[0] = a0 + a2; v[2] = a0 - a2; v[1] = a1 + a3; v[3] = a1 - a3;
 #pragma unroll
@@ -684,14 +713,14 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sm.big_r[4 * t + i] = v[i];
+    for (int i = 0; i < 4; ++i) q.ns->big_r[4 * t + i] = v[i];
   }
 
   // ---- d_t = FWHT(x_t - r) over the lane pair; ||x_t||^2 from the raw values --
   float v[HD];
   double ssx0 = 0.0, ssx1 = 0.0;
   if (valid) {
-    const char* tb = reinterpret_cast<const char*>(&sm.tile[tk][0]) + HD * ESZ * h;
+    const char* tb = reinterpret_cast<const char*>(&q.bk->tile[tk][0]) + HD * ESZ * h;
     constexpr int HCHUNKS = CHUNKS / 2;
     constexpr int PER = (DT == NSN_DTYPE_F32) ? 4 : 8;
 #pragma unroll
@@ -721,7 +750,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
       }
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
-        v[PER * ch + i] = xs[i] - sm.r[HD * h + PER * ch + i];
+        v[PER * ch + i] = xs[i] - q.ns->r[HD * h + PER * ch + i];
         if (i & 1) ssx1 = fma((double)xs[i], (double)xs[i], ssx1);
         else ssx0 = fma((double)xs[i], (double)xs[i], ssx0);
       }
@@ -732,7 +761,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   }
   fwht128_pair(v, h);
   const double ssx = shfl_pair_sum(ssx0 + ssx1);
-  __syncthreads();  // raw tile fully consumed; big_r ready
+  gr.sync();  // raw tile fully consumed; big_r ready
 
   // ---- first normalization: s1 = ||H x|| / sqrt(128) = ||x|| / sqrt(128) -----
   // (H is orthonormal.)  n1_t = w_t * rr_t with w_t = FWHT(x_t) = d_t + FWHT(r)
@@ -743,66 +772,66 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
     if (valid) {
 #pragma unroll
       for (int c = 0; c < HD; c += 4)
-        *reinterpret_cast<float4*>(&sm.tile[tk][HD * h + c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+        *reinterpret_cast<float4*>(&q.bk->tile[tk][HD * h + c]) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
       if (h == 0) {
-        sm.rr[tk] = rr;
-        sm.s1[tk] = norm_x / 11.313708498984761;
+        q.ns->rr[tk] = rr;
+        q.bk->s1[tk] = norm_x / 11.313708498984761;
       }
     }
   }
-  __syncthreads();
+  gr.sync();
 
   // ---- shift: o = mean_t n1_t = FWHT(r) * mean(rr) + mean_t(d_t rr_t) --------
   // mean(rr) is accumulated as deviations from rr_0 so that equal rr give it
   // exactly (identical tokens then give z = 0 exactly, as the definition does).
   // Column `col`, rows split in two halves, combined in a fixed order.
   {
-    const double rr0 = sm.rr[0];
+    const double rr0 = q.ns->rr[0];
     const int lo = rhalf * (BLK / 2), hi = min(n, lo + BLK / 2);
     double dev = 0.0, sd0 = 0.0, sd1 = 0.0, sd2 = 0.0, sd3 = 0.0;
     int row = lo;
     for (; row + 3 < hi; row += 4) {
-      const double ra = sm.rr[row], rb = sm.rr[row + 1], rc = sm.rr[row + 2], rd = sm.rr[row + 3];
+      const double ra = q.ns->rr[row], rb = q.ns->rr[row + 1], rc = q.ns->rr[row + 2], rd = q.ns->rr[row + 3];
       dev += ((ra - rr0) + (rb - rr0)) + ((rc - rr0) + (rd - rr0));
-      sd0 = fma((double)sm.tile[row][col], ra, sd0);
-      sd1 = fma((double)sm.tile[row + 1][col], rb, sd1);
-      sd2 = fma((double)sm.tile[row + 2][col], rc, sd2);
-      sd3 = fma((double)sm.tile[row + 3][col], rd, sd3);
+      sd0 = fma((double)q.bk->tile[row][col], ra, sd0);
+      sd1 = fma((double)q.bk->tile[row + 1][col], rb, sd1);
+      sd2 = fma((double)q.bk->tile[row + 2][col], rc, sd2);
+      sd3 = fma((double)q.bk->tile[row + 3][col], rd, sd3);
     }
     for (; row < hi; ++row) {
-      const double ra = sm.rr[row];
+      const double ra = q.ns->rr[row];
       dev += ra - rr0;
-      sd0 = fma((double)sm.tile[row][col], ra, sd0);
+      sd0 = fma((double)q.bk->tile[row][col], ra, sd0);
     }
-    sm.part[rhalf][col] = (sd0 + sd1) + (sd2 + sd3);
-    if (col == 0) sm.dev_part[rhalf] = dev;
+    q.ns->part[rhalf][col] = (sd0 + sd1) + (sd2 + sd3);
+    if (col == 0) q.ns->dev_part[rhalf] = dev;
   }
-  __syncthreads();
-  const double rr_mean = sm.rr[0] + (sm.dev_part[0] + sm.dev_part[1]) / n;
+  gr.sync();
+  const double rr_mean = q.ns->rr[0] + (q.ns->dev_part[0] + q.ns->dev_part[1]) / n;
   if (t < D) {
-    const double dc = (sm.part[0][t] + sm.part[1][t]) / n;  // D_c = mean_t(d_t,c rr_t)
-    sm.big_rf[t] = (float)sm.big_r[t];
-    sm.dcf[t] = (float)dc;
-    const double o_t = fma(sm.big_r[t], rr_mean, dc);
-    if (cv.dq) sm.ofull[t] = o_t;
+    const double dc = (q.ns->part[0][t] + q.ns->part[1][t]) / n;  // D_c = mean_t(d_t,c rr_t)
+    q.ns->big_rf[t] = (float)q.ns->big_r[t];
+    q.ns->dcf[t] = (float)dc;
+    const double o_t = fma(q.ns->big_r[t], rr_mean, dc);
+    if (cv.dq) q.bk->ofull[t] = o_t;
     else cv.means[(seq * (cv.capacity / BLK) + blk) * D + t] = __double2half(o_t);
   }
-  __syncthreads();
+  gr.sync();
 
   // ---- second normalization --------------------------------------------------
   // z_t = n1_t - o = d_t rr_t + FWHT(r) (rr_t - mean rr) - D.  The constant part
   // c = FWHT(r) (rr_t - mean rr) - D enters z rounded to fp32; it is formed by one
   // fp32 fma from fp32 copies of FWHT(r), D and rr_t - mean rr (three roundings of
   // the size of the one fp32 rounding of c), then one fp32 fma per channel.
-  const double rr_t = valid ? sm.rr[tk] : 0.0;
+  const double rr_t = valid ? q.ns->rr[tk] : 0.0;
   const float deltaf = (float)(rr_t - rr_mean);
   const float rrf = (float)rr_t;
   double zz0 = 0.0, zz1 = 0.0;
 #pragma unroll
   for (int c = 0; c < HD; c += 4) {
     const int cg = HD * h + c;
-    const float4 br = *reinterpret_cast<const float4*>(&sm.big_rf[cg]);
-    const float4 dd = *reinterpret_cast<const float4*>(&sm.dcf[cg]);
+    const float4 br = *reinterpret_cast<const float4*>(&q.ns->big_rf[cg]);
+    const float4 dd = *reinterpret_cast<const float4*>(&q.ns->dcf[cg]);
     const float brv[4] = {br.x, br.y, br.z, br.w}, ddv[4] = {dd.x, dd.y, dd.z, dd.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -813,7 +842,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
     }
   }
   const double zz = shfl_pair_sum(zz0 + zz1);
-  if (valid && h == 0) sm.s2[tk] = sqrt(zz) / 11.313708498984761;
+  if (valid && h == 0) q.bk->s2[tk] = sqrt(zz) / 11.313708498984761;
   const float inv2 = (zz > 0.0) ? (float)(11.313708498984761 / sqrt(zz)) : 0.f;
 #pragma unroll
   for (int c = 0; c < HD; ++c) v[c] *= inv2;
@@ -842,29 +871,30 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   // The raw tile and the d_t rows are no longer read (the column sums are done).
 #pragma unroll
   for (int c = 0; c < HD; c += 4)
-    *reinterpret_cast<float4*>(&sm.tile[tk][HD * h + c]) =
+    *reinterpret_cast<float4*>(&q.bk->tile[tk][HD * h + c]) =
         valid ? make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
-  __syncthreads();
+  gr.sync();
+}
 
-  // ---- nearest codeword on the tensor cores, exact decision -----------------
-  search_block(sm, tcs, cb_global, n, cv.status);
-
+// Exact fp64 re-decision of the flagged sub-vectors of q.bk (q.se->flag), one
+// warp per sub-vector, by the warps of `gr`.
+__device__ void exact_phase(const QRefs& q, const Grp& gr, const float* __restrict__ cb_global) {
   // ---- exact fp64 re-decision of the flagged sub-vectors, a warp each --------
   // Each lane scores its 8 codewords in sequential fp32 (bias first, one fma per
   // dim); candidates are the codewords within twice the fp32 bound of the best of
   // these scores; the winner by fp64 squared distance (cosine assignment: largest
   // fp64 inner product with c_hat), ties to the lowest index.
   {
-    const int warp = t >> 5, lane = t & 31;
-    const float cmax = sm.cnorm[0], cmax2 = sm.cnorm[1];
+    const int warp = gr.t >> 5, lane = gr.t & 31;
+    const float cmax = q.tb->cnorm[0], cmax2 = q.tb->cnorm[1];
     constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
-    const int tab = sm.tab;
-    const int nflag = sm.nflag;
+    const int tab = q.tb->tab;
+    const int nflag = q.se->nflag;
 #pragma unroll 1
-    for (int f = warp; f < nflag; f += QTHREADS / 32) {
-      const int ftk = sm.flag[f] / NSUB, fj = sm.flag[f] % NSUB;
-      const float4 fa0 = *reinterpret_cast<const float4*>(&sm.tile[ftk][SUB * fj]);
-      const float4 fa1 = *reinterpret_cast<const float4*>(&sm.tile[ftk][SUB * fj + 4]);
+    for (int f = warp; f < nflag; f += gr.n / 32) {
+      const int ftk = q.se->flag[f] / NSUB, fj = q.se->flag[f] % NSUB;
+      const float4 fa0 = *reinterpret_cast<const float4*>(&q.bk->tile[ftk][SUB * fj]);
+      const float4 fa1 = *reinterpret_cast<const float4*>(&q.bk->tile[ftk][SUB * fj + 4]);
       const float a[8] = {fa0.x, fa0.y, fa0.z, fa0.w, fa1.x, fa1.y, fa1.z, fa1.w};
       float na = 0.f;
 #pragma unroll
@@ -877,7 +907,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
       for (int m = 0; m < NCODES / 32; ++m) {
         const int k = lane + 32 * m;
         float c[SUB];
-        float x = codeword(sm, cb_global, tab, k, (lane >> 2) & 1, c);
+        float x = codeword(q, k, (lane >> 2) & 1, c);
 #pragma unroll
         for (int i = 0; i < SUB; ++i) x = fmaf(a[i], c[i], x);
         sc[m] = x;
@@ -891,7 +921,7 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
         if (sc[m] >= thr) {
           const int k = lane + 32 * m;
           float c[SUB];
-          codeword(sm, cb_global, tab, k, (lane >> 2) & 1, c);
+          codeword(q, k, (lane >> 2) & 1, c);
           double dd = 0.0;  // fp64 squared distance, or minus the fp64 inner product with c_hat
           if (tab == TAB_COSINE) {
 #pragma unroll
@@ -912,22 +942,30 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
         const int ob = __shfl_xor_sync(0xffffffffu, bi, m);
         if (od < bestd || (od == bestd && ob < bi)) { bestd = od; bi = ob; }
       }
-      if (lane == 0 && bi < NCODES) sm.code[ftk][fj] = (uint8_t)bi;
+      if (lane == 0 && bi < NCODES) q.bk->code[ftk][fj] = (uint8_t)bi;
     }
   }
-  __syncthreads();
+  gr.sync();
+}
 
+// Adaptive scale and stores of one block of n tokens (codes final in q.bk->code)
+// by a set of 256 threads (two per token, as in nsn_phase).
+__device__ void finish_phase(const QRefs& q, const Grp& gr, const float* __restrict__ cb_global,
+                             uint8_t* __restrict__ codes, const CacheView& cv, int64_t seq, int64_t tok0, int blk,
+                             int n, int scale_adjust) {
+  const int t = gr.t, tk = t >> 1, h = t & 1;
+  const bool valid = tk < n;
   // ---- adaptive scale: alpha = ||u||^2 / (u . u_hat) --------------------------
   double dot = 0.0, uu = 0.0;
   {
-    const int tab = sm.tab;
+    const int tab = q.tb->tab;
 #pragma unroll 4
     for (int jj = 0; jj < HSUB; ++jj) {
       const int j = HSUB * h + jj;
       float qv[SUB];
-      codeword_given(sm, cb_global, tab, sm.code[tk][j], (t >> 2) & 1, qv);
-      const float4 u0 = *reinterpret_cast<const float4*>(&sm.tile[tk][SUB * j]);
-      const float4 u1 = *reinterpret_cast<const float4*>(&sm.tile[tk][SUB * j + 4]);
+      codeword_given(q, cb_global, tab, q.bk->code[tk][j], (t >> 2) & 1, qv);
+      const float4 u0 = *reinterpret_cast<const float4*>(&q.bk->tile[tk][SUB * j]);
+      const float4 u1 = *reinterpret_cast<const float4*>(&q.bk->tile[tk][SUB * j + 4]);
       const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
       float dj = 0.f, uj = 0.f;
 #pragma unroll
@@ -949,19 +987,37 @@ __device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __r
   // ---- packed stores ---------------------------------------------------------
   if (valid) {
     *reinterpret_cast<uint2*>(codes + (int64_t)tk * NSUB + HSUB * h) =
-        *reinterpret_cast<const uint2*>(&sm.code[tk][HSUB * h]);
+        *reinterpret_cast<const uint2*>(&q.bk->code[tk][HSUB * h]);
     if (h == 0) {
       const BlockOut bo = block_out(cv, seq, tok0, blk);
-      if (bo.dq) bo.s2[tk] = __double2half(alpha * sm.s2[tk]);
-      else bo.norms[tk] = __halves2half2(__double2half(sm.s1[tk]), __double2half(alpha * sm.s2[tk]));
+      if (bo.dq) bo.s2[tk] = __double2half(alpha * q.bk->s2[tk]);
+      else bo.norms[tk] = __halves2half2(__double2half(q.bk->s1[tk]), __double2half(alpha * q.bk->s2[tk]));
     }
   }
-  if (cv.dq) store_double_quant(sm, n, block_out(cv, seq, tok0, blk));
-  __syncthreads();  // shared memory is reused by the caller's next block
+  if (cv.dq) store_double_quant(q, gr, n, block_out(cv, seq, tok0, blk));
+  gr.sync();  // shared memory is reused by the caller's next block
+}
+
+// Quantizes one block of n (1..128) tokens with the whole CTA of QTHREADS threads
+// (NSN, codeword search, exact re-decision, adaptive scale and stores).  Output
+// pointers are already offset to the block's first token (codes, signs).
+template <int DT, int MODE>
+__device__ void quantize_block_dev(QuantSmem& sm, TcState& tcs, const float* __restrict__ cb_global,
+                                   const void* __restrict__ src, int64_t row0,
+                                   int64_t row_stride, int n, uint8_t* __restrict__ codes,
+                                   uint8_t* __restrict__ signs, const CacheView& cv, int64_t seq,
+                                   int64_t tok0, int blk, int scale_adjust) {
+  const QRefs q = refs(sm);
+  const Grp gr = cta_grp();
+  if (gr.t == 0) sm.se.nflag = 0;  // read only after the barriers below
+  nsn_phase<DT, MODE>(q, gr, src, row0, row_stride, n, signs, cv, seq, blk);
+  search_block(q, tcs, cb_global, n, cv.status);
+  exact_phase(q, gr, cb_global);
+  finish_phase(q, gr, cb_global, codes, cv, seq, tok0, blk, n, scale_adjust);
 }
 
 // ---------------------------------------------------------------------------
-// Prefill: grid (blocks, kv-heads, batch).
+// Prefill: which tokens of each sequence are quantized.
 // ---------------------------------------------------------------------------
 // Tokens of sequence b and its quantized prefix.  Without `lengths` every
 // sequence has the common n_tokens / q_tokens; with it, sequence b has
@@ -983,31 +1039,249 @@ __device__ __forceinline__ PrefillSplit prefill_split(const int32_t* __restrict_
   return {L, q, bad};
 }
 
-// Persistent: CTA i takes work items i, i + gridDim.x, ... of the (block, kv-head,
-// batch) list; the tensor memory, the barrier and the staged codebook live for the
-// whole launch.
-template <int DT, int MODE>
-__global__ void __launch_bounds__(QTHREADS, 2)
-quantize_prefill_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int64_t sh, int q_tokens, int n_tokens,
-                        const int32_t* __restrict__ lengths, CacheView cv, const float* __restrict__ codebook,
-                        int nblk) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw);
-  TcState tcs = tc_setup(sm);
-  stage_codebook(sm, codebook, cv.assign);
-  const int nwork = nblk * cv.n_kv_heads * cv.batch;
+
+// ---------------------------------------------------------------------------
+// Warp-specialized prefill: one persistent CTA per SM, 16 warps, two blocks in
+// flight.  Warps 0-7 (the searchers) form two warpgroups; warpgroup g searches the
+// tiles g, g + 2, ... of a block in its own 256-column tensor-memory buffer, so the
+// two warpgroups' MMA waits, score reductions and rescans overlap.  A searcher
+// thread owns one tile row (= tensor-memory lane): it builds the row's A operand,
+// one thread per warpgroup issues the MMAs, then each thread reads its row's 256
+// scores, keeps the two best group maxima, rescans the winning group's 8
+// codewords in fp32 and decides; after the block the 8 warps re-decide the
+// flagged sub-vectors.  Warps 8-15 (the normalizers) run the NSN of block j into
+// one of two block buffers while the searchers work on block j - 1, and then the
+// adaptive scale and stores of block j - 2.  Named barriers hand a block over:
+// U (u rows ready, normalizers -> searchers) and D (codes final, searchers ->
+// normalizers), one of each per buffer.
+// ---------------------------------------------------------------------------
+constexpr int WS_SWG = 2;                              // search warpgroups
+constexpr int WS_SWARPS = 4 * WS_SWG, WS_NWARPS = 8;
+constexpr int WS_THREADS = 32 * (WS_SWARPS + WS_NWARPS);
+constexpr int WS_BAR_G = 1;                            // ids 1, 2: one warpgroup of searchers
+constexpr int WS_BAR_S = 3, WS_BAR_N = 4;              // all searchers; all normalizers
+constexpr int WS_BAR_U = 5, WS_BAR_D = 7;              // ids +0 / +1 by block buffer
+constexpr uint32_t WS_TC_COLS = WS_SWG * TC_COLS;
+
+struct QuantSmemWS {
+  QTables tb;
+  QSearch se;
+  QNsn ns;
+  QBlock bk[2];
+};
+
+__device__ __forceinline__ void bar_arrive(int id, int n) { asm volatile("bar.arrive %0, %1;" :: "r"(id), "r"(n) : "memory"); }
+__device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory"); }
+
+// Search of the tiles wg, wg + 2, ... of one block by search warpgroup wg (thread
+// L = tile row = tensor-memory lane).  Bounds as in search_block.
+__device__ void search_tiles_ws(const QRefs& q, TcState& tcs, const float* __restrict__ cb_global, int n, int wg,
+                                int32_t* status) {
+  const int L = threadIdx.x & 127, wq = L >> 5, lane = L & 31;
+  const Grp g{WS_BAR_G + wg, 128, L};
+  const float cmax = q.tb->cnorm[0], cmax2 = q.tb->cnorm[1], cdel = q.tb->cnorm[2];
+  const int tab = q.tb->tab;
+  constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
+  constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
+  const uint32_t tbuf = tcs.tmem + (uint32_t)(TC_COLS * wg);
+  const uint32_t taddr = tbuf + ((uint32_t)(32 * wq) << 16);
+  const uint64_t db = tc_desc(q_smem(q.tb->bop), 128, 256);
+  const uint64_t da2 = tc_desc(q_smem(q.tb->aop2), 128, 0);
+  const uint64_t db2 = tc_desc(q_smem(q.tb->bop2), 0, 128);
+  unsigned char* ap = q.se->aop[wg];
+  const uint64_t da = tc_desc(q_smem(ap), 128, 256);
+  const uint32_t mb = q_smem(&q.se->mbar[wg]);
+  const int ntiles = (n + 7) >> 3;
+  // exact-arithmetic table reads of this lane (bank-conflict free, see QTables)
+  const int rp = (lane >> 2) & 1, hf = (lane >> 1) & 1, bq = lane >> 3;
+  const int j = L & 15;
+
 #pragma unroll 1
-  for (int w = blockIdx.x; w < nwork; w += gridDim.x) {
+  for (int tile = wg; tile < ntiles; tile += WS_SWG) {
+    const int tkk = 8 * tile + (L >> 4);
+    // ---- the row's A operand (hi and lo halves) and its decision bounds ----
+    // a[0..3] = dims 4 hf .. 4 hf + 3, a[4..7] = the other half (the order of this
+    // lane's table reads); the A operand keeps the natural order.
+    float a[SUB];
+    {
+      const float4 a0 = *reinterpret_cast<const float4*>(&q.bk->tile[tkk][SUB * j + 4 * hf]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&q.bk->tile[tkk][SUB * j + 4 - 4 * hf]);
+      a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
+      a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const __half2 hh = __floats2half2_rn(a[2 * p], a[2 * p + 1]);
+        const float2 back = __half22float2(hh);
+        hi[p] = h2_bits(hh);
+        lo[p] = h2_bits(__floats2half2_rn(a[2 * p] - back.x, a[2 * p + 1] - back.y));
+      }
+      *reinterpret_cast<uint2*>(ap + kmaj_off(L, 4 * hf)) = make_uint2(hi[0], hi[1]);
+      *reinterpret_cast<uint2*>(ap + kmaj_off(L, 4 - 4 * hf)) = make_uint2(hi[2], hi[3]);
+      *reinterpret_cast<uint2*>(ap + kmaj_off(L, 8 + 4 * hf)) = make_uint2(lo[0], lo[1]);
+      *reinterpret_cast<uint2*>(ap + kmaj_off(L, 12 - 4 * hf)) = make_uint2(lo[2], lo[3]);
+    }
+    // A rows written (generic proxy -> tensor cores) and the previous tile's scores read
+    fence_async_smem();
+    tc_fence_before();
+    g.sync();
+    tc_fence_after();
+    if (L == 0) {
+      if (tab == TAB_COSINE) {
+        tc_mma(tbuf, da, db, 0u);
+        tc_mma(tbuf, da, db2, 1u);
+      } else {
+        tc_mma(tbuf, da2, db2, 0u);
+        tc_mma(tbuf, da, db, 1u);
+      }
+      tc_commit(mb);
+    }
+    float na = 0.f;
+#pragma unroll
+    for (int d = 0; d < SUB; ++d) na = fmaf(a[d], a[d], na);
+    na = sqrtf(na) * 1.0001f;
+    const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
+    const float mtc = (TC_REL * (1.001f * na * cmax + 0.5f * cmax2) + na * cdel) * 1.01f + 1.2e-7f;
+    if (!mbar_wait(mb, (tcs.phase >> wg) & 1u, MBAR_POLLS) && lane == 0 && status) atomicOr(status, 2);
+    tcs.phase ^= 1u << wg;
+    tc_fence_after();
+
+    // ---- best and second-best of the 32 group maxima of the row's 256 scores ----
+    // (two register buffers in turn: chunk c + 1 loads while chunk c is reduced)
+    float b1 = -INFINITY, b2 = -INFINITY;
+    uint32_t rb[2][32];
+    tc_ld32(taddr, rb[0]);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint32_t (&r)[32] = rb[c & 1];
+      tc_wait_ld();
+      tc_regs_ready(r);
+      if (c < 7) tc_ld32(taddr + 32 * (c + 1), rb[(c + 1) & 1]);
+      float key[4];
+#pragma unroll
+      for (int gg = 0; gg < 4; ++gg) {
+        const float m = max3f(max3f(__uint_as_float(r[8 * gg]), __uint_as_float(r[8 * gg + 1]), __uint_as_float(r[8 * gg + 2])),
+                              max3f(__uint_as_float(r[8 * gg + 3]), __uint_as_float(r[8 * gg + 4]), __uint_as_float(r[8 * gg + 5])),
+                              fmaxf(__uint_as_float(r[8 * gg + 6]), __uint_as_float(r[8 * gg + 7])));
+        key[gg] = __uint_as_float((__float_as_uint(m) & ~31u) | (uint32_t)(4 * c + gg));
+      }
+      const float h01 = fmaxf(key[0], key[1]), l01 = fminf(key[0], key[1]);
+      const float h23 = fmaxf(key[2], key[3]), l23 = fminf(key[2], key[3]);
+      const float hi = fmaxf(h01, h23);
+      const float lo = max3f(l01, l23, fminf(h01, h23));
+      b2 = max3f(b2, lo, fminf(b1, hi));
+      b1 = fmaxf(b1, hi);
+    }
+    const int G = (int)(__float_as_uint(b1) & 31u);
+
+    // ---- the winning group's 8 codewords in sequential fp32, lane-rotated order,
+    // ties to the lowest index ----
+    float best = -INFINITY, second = -INFINITY;
+    int idx = NCODES;
+    {
+      float cw[8][SUB], sc[8];
+      int kk[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        kk[i] = 8 * G + ((i + lane) & 7);
+        const float* src = q.tb->cw + 16 * kk[i] + 8 * rp;
+        const float4 x0 = *reinterpret_cast<const float4*>(src + 4 * hf);
+        const float4 x1 = *reinterpret_cast<const float4*>(src + 4 - 4 * hf);
+        cw[i][0] = x0.x; cw[i][1] = x0.y; cw[i][2] = x0.z; cw[i][3] = x0.w;
+        cw[i][4] = x1.x; cw[i][5] = x1.y; cw[i][6] = x1.z; cw[i][7] = x1.w;
+        sc[i] = q.tb->cbias[4 * kk[i] + bq];
+      }
+#pragma unroll
+      for (int d = 0; d < SUB; ++d)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sc[i] = fmaf(a[d], cw[i][d], sc[i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float lo = fminf(best, sc[i]);
+        idx = (sc[i] > best || (sc[i] == best && kk[i] < idx)) ? kk[i] : idx;
+        best = fmaxf(best, sc[i]);
+        second = fmaxf(second, lo);
+      }
+    }
+    const float other = b2 + fabsf(b2) * 3.82e-6f;  // + 32 ulp: the group number in the low bits
+    q.bk->code[tkk][j] = (uint8_t)idx;
+    const bool need = second >= best - margin || other >= best - 0.5f * margin - mtc;
+    if (need && tkk < n) q.se->flag[atomicAdd(&q.se->nflag, 1)] = (uint16_t)(tkk * NSUB + j);
+  }
+  tc_fence_before();
+}
+
+struct WsBlock {
+  const void* src;
+  int64_t row0, seq, tok0;
+  int n, blk;
+};
+
+template <int DT, int MODE>
+__global__ void __launch_bounds__(WS_THREADS, 1)
+quantize_prefill_ws_kernel(const void* __restrict__ x, int64_t sb, int64_t st, int64_t sh, int q_tokens,
+                           int n_tokens, const int32_t* __restrict__ lengths, CacheView cv,
+                           const float* __restrict__ codebook, int nblk) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  QuantSmemWS& sm = *reinterpret_cast<QuantSmemWS*>(smem_raw);
+  TcState tcs = tc_setup(sm.se, WS_TC_COLS, WS_SWG);
+  stage_codebook(QRefs{&sm.tb, &sm.se, &sm.ns, &sm.bk[0]}, codebook, cv.assign);
+  const int nwork = nblk * cv.n_kv_heads * cv.batch;
+  auto block_at = [&](int w) {
+    WsBlock bl;
     const int blk = w % nblk, h = (w / nblk) % cv.n_kv_heads, b = w / (nblk * cv.n_kv_heads);
     const PrefillSplit ps = prefill_split(lengths, b, n_tokens, q_tokens, cv.window_len);
-    const int n = min(BLK, ps.q - blk * BLK);
-    if (n <= 0) continue;
-    const int64_t seq = (int64_t)b * cv.n_kv_heads + h;
-    const int64_t tok0 = seq * cv.capacity + (int64_t)blk * BLK;
-    quantize_block_dev<DT, MODE>(sm, tcs, codebook,
-                                 x, (int64_t)b * sb + (int64_t)blk * BLK * st + (int64_t)h * sh, st, n,
-                                 cv.codes + tok0 * NSUB, MODE == NSN_MODE_2BIT ? cv.signs + tok0 * NSUB : nullptr,
-                                 cv, seq, tok0, blk, cv.scale_adjust);
+    bl.n = min(BLK, ps.q - blk * BLK);
+    bl.blk = blk;
+    bl.seq = (int64_t)b * cv.n_kv_heads + h;
+    bl.tok0 = bl.seq * cv.capacity + (int64_t)blk * BLK;
+    bl.row0 = (int64_t)b * sb + (int64_t)blk * BLK * st + (int64_t)h * sh;
+    bl.src = x;
+    return bl;
+  };
+  const int warp = threadIdx.x >> 5;
+  if (warp < WS_SWARPS) {
+    // ---- searchers ----
+    const Grp sg{WS_BAR_S, 32 * WS_SWARPS, (int)threadIdx.x};
+    const int wg = warp >> 2;
+    int j = 0;
+#pragma unroll 1
+    for (int w = blockIdx.x; w < nwork; w += gridDim.x) {
+      const WsBlock bl = block_at(w);
+      if (bl.n <= 0) continue;
+      const QRefs q{&sm.tb, &sm.se, &sm.ns, &sm.bk[j & 1]};
+      bar_sync(WS_BAR_U + (j & 1), WS_THREADS);
+      if (sg.t == 0) sm.se.nflag = 0;
+      sg.sync();
+      search_tiles_ws(q, tcs, codebook, bl.n, wg, cv.status);
+      sg.sync();  // every code and flag of the block written
+      exact_phase(q, sg, codebook);
+      bar_arrive(WS_BAR_D + (j & 1), WS_THREADS);
+      ++j;
+    }
+  } else {
+    // ---- normalizers ----
+    const Grp ng{WS_BAR_N, 32 * WS_NWARPS, (int)threadIdx.x - 32 * WS_SWARPS};
+    WsBlock hist[2];
+    int j = 0;
+    auto finish = [&](int jj, const WsBlock& bl) {
+      bar_sync(WS_BAR_D + (jj & 1), WS_THREADS);
+      const QRefs q{&sm.tb, &sm.se, &sm.ns, &sm.bk[jj & 1]};
+      finish_phase(q, ng, codebook, cv.codes + bl.tok0 * NSUB, cv, bl.seq, bl.tok0, bl.blk, bl.n, cv.scale_adjust);
+    };
+#pragma unroll 1
+    for (int w = blockIdx.x; w < nwork; w += gridDim.x) {
+      const WsBlock bl = block_at(w);
+      if (bl.n <= 0) continue;
+      if (j >= 2) finish(j - 2, hist[j & 1]);
+      const QRefs q{&sm.tb, &sm.se, &sm.ns, &sm.bk[j & 1]};
+      nsn_phase<DT, MODE>(q, ng, bl.src, bl.row0, st, bl.n,
+                          MODE == NSN_MODE_2BIT ? cv.signs + bl.tok0 * NSUB : nullptr, cv, bl.seq, bl.blk);
+      bar_arrive(WS_BAR_U + (j & 1), WS_THREADS);
+      hist[j & 1] = bl;
+      ++j;
+    }
+    for (int jj = max(0, j - 2); jj < j; ++jj) finish(jj, hist[jj & 1]);
   }
   tc_teardown(tcs);
 }
@@ -1061,8 +1335,8 @@ append_kernel(CacheView kc, CacheView vc, const void* __restrict__ k_new, const 
       if (t == 0 && c.status) atomicOr(c.status, 1);
     } else {
       const float* cb = is_v ? cbv : cbk;
-      TcState tcs = tc_setup(sm);
-      stage_codebook(sm, cb, c.assign);
+      TcState tcs = tc_setup(sm.se, TC_COLS, 1);
+      stage_codebook(refs(sm), cb, c.assign);
       const int64_t tok0 = seq * c.capacity + nq;
       const int blk = nq / BLK;
       uint8_t* sg = c.mode == NSN_MODE_2BIT ? c.signs + tok0 * NSUB : nullptr;
@@ -1098,8 +1372,8 @@ size_t quant_smem_bytes() { return sizeof(QuantSmem); }
 template <int DT, int MODE>
 static cudaError_t launch_prefill_t(const void* x, int64_t sb, int64_t st, int64_t sh, int q_tokens, int n_tokens,
                                     const int32_t* lengths, const CacheView& cv, const float* cb, cudaStream_t s) {
-  const size_t smem = sizeof(QuantSmem);
-  cudaError_t e = cudaFuncSetAttribute(quantize_prefill_kernel<DT, MODE>,
+  const size_t smem = sizeof(QuantSmemWS);
+  cudaError_t e = cudaFuncSetAttribute(quantize_prefill_ws_kernel<DT, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int nblk = (q_tokens + BLK - 1) / BLK;
@@ -1107,9 +1381,9 @@ static cudaError_t launch_prefill_t(const void* x, int64_t sb, int64_t st, int64
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long nwork = (long long)nblk * cv.n_kv_heads * cv.batch;
-    const int grid = (int)std::min<long long>(nwork, 2LL * sms);  // two resident CTAs per SM
-    quantize_prefill_kernel<DT, MODE><<<grid, QTHREADS, smem, s>>>(x, sb, st, sh, q_tokens, n_tokens, lengths, cv, cb,
-                                                                   nblk);
+    const int grid = (int)std::min<long long>(nwork, (long long)sms);  // one persistent CTA per SM
+    quantize_prefill_ws_kernel<DT, MODE><<<grid, WS_THREADS, smem, s>>>(x, sb, st, sh, q_tokens, n_tokens, lengths,
+                                                                        cv, cb, nblk);
   }
   return cudaGetLastError();
 }
