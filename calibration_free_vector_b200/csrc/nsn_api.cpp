@@ -308,4 +308,15 @@ nsn_status nsn_selftest_bounded_wait(int32_t* status, int max_attempts, void* st
                                                        static_cast<cudaStream_t>(stream)));
 }
 
+nsn_status nsn_selftest_tensor_scores(const float* rows, int n_rows, const float* codebook, int assign,
+                                      float* scores, int32_t* status, void* stream) {
+  if (!rows || !codebook || !scores || !status || n_rows <= 0 || n_rows > 128 || (assign != 0 && assign != 1))
+    return NSN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(rows) | reinterpret_cast<uintptr_t>(codebook) |
+       reinterpret_cast<uintptr_t>(scores)) & 15u || (reinterpret_cast<uintptr_t>(status) & 3u))
+    return NSN_ERR_INVALID_ARG;
+  return cuda_status(nsn::launch_tensor_scores_selftest(rows, n_rows, codebook, assign, scores, status,
+                                                        static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -75,5 +75,8 @@ cudaError_t launch_decode_static(const CacheView& kc, const CacheView& vc, const
 
 // Bounded-wait diagnostic (see nsn_selftest_bounded_wait).
 cudaError_t launch_bounded_wait_selftest(int32_t* status, uint32_t limit, cudaStream_t s);
+// Tensor-core score diagnostic (see nsn_selftest_tensor_scores).
+cudaError_t launch_tensor_scores_selftest(const float* rows, int n, const float* codebook, int cosine, float* scores,
+                                          int32_t* status, cudaStream_t s);
 
 }  // namespace nsn

@@ -465,13 +465,28 @@ __device__ void store_double_quant(const QRefs& q, const Grp& gr, int n, const B
 //       and each side rescans 4 codewords of group G in sequential fp32;
 //   (5) the lower warp merges the rescans and applies the decision bounds:
 //       the sequential fp32 score is within gamma_9 (max||c||^2 + ||a|| max||c||)
-//       of the exact one; the tensor score within 2^-16 (sum |a_i c_i| + |bias|)
-//       (accumulation order and rounding inside the MMA are the hardware's, so the
-//       bound is taken wide: 17 terms of at most 2^-24 relative error each need
-//       about 2^-19.9) plus ||a|| ||c - fp16(c)|| for a codebook that is not
-//       fp16-representable; the group number adds at most 32 ulp to a maximum.
+//       of the exact one; the tensor score within tensor_bound() (accumulation
+//       order and rounding inside the MMA are the hardware's, so that term is taken
+//       wide: 17 terms of at most 2^-24 relative error each need about 2^-19.9);
+//       the group number adds at most 32 ulp to a maximum.
 //       A rival inside the group within twice the fp32 bound, or another group's
 //       maximum within the fp32 plus the tensor bound, flags the sub-vector.
+// Bound on |tensor score - exact score| of a row of norm na (rounded up), for a
+// codebook with max ||c|| = cmax, max ||c||^2 = cmax2 and max ||c - fp16(c)|| = cdel:
+//   2^-16 (na cmax + cmax2 / 2)   accumulation inside the MMA (taken wide: its order
+//                                  and rounding are the hardware's);
+//   + na cdel                     the fp16 operand of a codebook that is not fp16-representable;
+//   + 2^-25 sqrt(8) (cmax + na)   an fp16 lo part below the normal range (of a, and of c_hat in
+//                                  the cosine rule) is off by up to half its 2^-24 spacing, so
+//                                  hi + lo is exact to 2^-22 only relative to larger elements;
+// with 1 % and an absolute 1.2e-7 (the lo part of the bias) on top.  The raw MMA scores are
+// compared with this bound by nsn_selftest_tensor_scores.
+__device__ __forceinline__ float tensor_bound(float na, float cmax, float cmax2, float cdel) {
+  constexpr float TC_REL = 1.52587890625e-05f;        // 2^-16
+  constexpr float SUBN = 2.98023223876953125e-08f * 2.8285f;  // 2^-25 sqrt(8), rounded up
+  return (TC_REL * (1.001f * na * cmax + 0.5f * cmax2) + na * cdel + SUBN * (cmax + na)) * 1.01f + 1.2e-7f;
+}
+
 __device__ void search_block(const QRefs& q, TcState& tcs, const float* __restrict__ cb_global, int n,
                              int32_t* status) {
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -480,7 +495,6 @@ __device__ void search_block(const QRefs& q, TcState& tcs, const float* __restri
   const float cmax = q.tb->cnorm[0], cmax2 = q.tb->cnorm[1], cdel = q.tb->cnorm[2];
   const int tab = q.tb->tab;
   constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
-  constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
   const uint32_t taddr = tcs.tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(128 * hf);
   const uint64_t db = tc_desc(q_smem(q.tb->bop), 128, 256);
   const uint64_t da2 = tc_desc(q_smem(q.tb->aop2), 128, 0);  // every 8-row group reads the same [1, 1, 0...] rows
@@ -501,7 +515,7 @@ __device__ void search_block(const QRefs& q, TcState& tcs, const float* __restri
     for (int d = 0; d < SUB; ++d) na = fmaf(a[d], a[d], na);
     na = sqrtf(na) * 1.0001f;
     margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
-    mtc = (TC_REL * (1.001f * na * cmax + 0.5f * cmax2) + na * cdel) * 1.01f + 1.2e-7f;
+    mtc = tensor_bound(na, cmax, cmax2, cdel);
     uint32_t w[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
@@ -1040,6 +1054,43 @@ __device__ __forceinline__ PrefillSplit prefill_split(const int32_t* __restrict_
 }
 
 
+// Row `row` of a tile's A operand, [a_hi | a_lo] (a_hi = fp16(a), a_lo = fp16(a -
+// a_hi), so a_hi + a_lo = a to 2^-22), stored in the natural K order; a[0..3] holds
+// dims 4h .. 4h + 3 and a[4..7] the other half.
+__device__ __forceinline__ void store_a_row(unsigned char* ap, int row, const float (&a)[SUB], int h) {
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const __half2 hh = __floats2half2_rn(a[2 * p], a[2 * p + 1]);
+    const float2 back = __half22float2(hh);
+    hi[p] = h2_bits(hh);
+    lo[p] = h2_bits(__floats2half2_rn(a[2 * p] - back.x, a[2 * p + 1] - back.y));
+  }
+  *reinterpret_cast<uint2*>(ap + kmaj_off(row, 4 * h)) = make_uint2(hi[0], hi[1]);
+  *reinterpret_cast<uint2*>(ap + kmaj_off(row, 4 - 4 * h)) = make_uint2(hi[2], hi[3]);
+  *reinterpret_cast<uint2*>(ap + kmaj_off(row, 8 + 4 * h)) = make_uint2(lo[0], lo[1]);
+  *reinterpret_cast<uint2*>(ap + kmaj_off(row, 12 - 4 * h)) = make_uint2(lo[2], lo[3]);
+}
+
+// The two MMAs of one tile's 256 scores per row into the 256 tensor-memory columns
+// at `dtmem`, then the commit to `mbar`; issued by one thread.
+//   nearest codeword: D = bias + [a_hi | a_lo] [c | c]
+//   cosine rule:      D = [a_hi | a_lo] [c_hat_hi | c_hat_hi] + [a_hi | a_lo] [c_hat_lo | c_hat_lo]
+__device__ __forceinline__ void issue_scores(const QRefs& q, uint32_t dtmem, const unsigned char* ap, uint32_t mbar) {
+  const uint64_t da = tc_desc(q_smem(ap), 128, 256);
+  const uint64_t db = tc_desc(q_smem(q.tb->bop), 128, 256);
+  const uint64_t da2 = tc_desc(q_smem(q.tb->aop2), 128, 0);  // every 8-row group reads the same [1, 1, 0...] rows
+  const uint64_t db2 = tc_desc(q_smem(q.tb->bop2), 0, 128);  // K half 1 re-reads K half 0
+  if (q.tb->tab == TAB_COSINE) {
+    tc_mma(dtmem, da, db, 0u);
+    tc_mma(dtmem, da, db2, 1u);
+  } else {
+    tc_mma(dtmem, da2, db2, 0u);
+    tc_mma(dtmem, da, db, 1u);
+  }
+  tc_commit(mbar);
+}
+
 // ---------------------------------------------------------------------------
 // Warp-specialized prefill: one persistent CTA per SM, 16 warps, two blocks in
 // flight.  Warps 0-7 (the searchers) form two warpgroups; warpgroup g searches the
@@ -1080,16 +1131,10 @@ __device__ void search_tiles_ws(const QRefs& q, TcState& tcs, const float* __res
   const int L = threadIdx.x & 127, wq = L >> 5, lane = L & 31;
   const Grp g{WS_BAR_G + wg, 128, L};
   const float cmax = q.tb->cnorm[0], cmax2 = q.tb->cnorm[1], cdel = q.tb->cnorm[2];
-  const int tab = q.tb->tab;
   constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
-  constexpr float TC_REL = 1.52587890625e-05f;               // 2^-16
   const uint32_t tbuf = tcs.tmem + (uint32_t)(TC_COLS * wg);
   const uint32_t taddr = tbuf + ((uint32_t)(32 * wq) << 16);
-  const uint64_t db = tc_desc(q_smem(q.tb->bop), 128, 256);
-  const uint64_t da2 = tc_desc(q_smem(q.tb->aop2), 128, 0);
-  const uint64_t db2 = tc_desc(q_smem(q.tb->bop2), 0, 128);
   unsigned char* ap = q.se->aop[wg];
-  const uint64_t da = tc_desc(q_smem(ap), 128, 256);
   const uint32_t mb = q_smem(&q.se->mbar[wg]);
   const int ntiles = (n + 7) >> 3;
   // exact-arithmetic table reads of this lane (bank-conflict free, see QTables)
@@ -1108,40 +1153,20 @@ __device__ void search_tiles_ws(const QRefs& q, TcState& tcs, const float* __res
       const float4 a1 = *reinterpret_cast<const float4*>(&q.bk->tile[tkk][SUB * j + 4 - 4 * hf]);
       a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
       a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const __half2 hh = __floats2half2_rn(a[2 * p], a[2 * p + 1]);
-        const float2 back = __half22float2(hh);
-        hi[p] = h2_bits(hh);
-        lo[p] = h2_bits(__floats2half2_rn(a[2 * p] - back.x, a[2 * p + 1] - back.y));
-      }
-      *reinterpret_cast<uint2*>(ap + kmaj_off(L, 4 * hf)) = make_uint2(hi[0], hi[1]);
-      *reinterpret_cast<uint2*>(ap + kmaj_off(L, 4 - 4 * hf)) = make_uint2(hi[2], hi[3]);
-      *reinterpret_cast<uint2*>(ap + kmaj_off(L, 8 + 4 * hf)) = make_uint2(lo[0], lo[1]);
-      *reinterpret_cast<uint2*>(ap + kmaj_off(L, 12 - 4 * hf)) = make_uint2(lo[2], lo[3]);
+      store_a_row(ap, L, a, hf);
     }
     // A rows written (generic proxy -> tensor cores) and the previous tile's scores read
     fence_async_smem();
     tc_fence_before();
     g.sync();
     tc_fence_after();
-    if (L == 0) {
-      if (tab == TAB_COSINE) {
-        tc_mma(tbuf, da, db, 0u);
-        tc_mma(tbuf, da, db2, 1u);
-      } else {
-        tc_mma(tbuf, da2, db2, 0u);
-        tc_mma(tbuf, da, db, 1u);
-      }
-      tc_commit(mb);
-    }
+    if (L == 0) issue_scores(q, tbuf, ap, mb);
     float na = 0.f;
 #pragma unroll
     for (int d = 0; d < SUB; ++d) na = fmaf(a[d], a[d], na);
     na = sqrtf(na) * 1.0001f;
     const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
-    const float mtc = (TC_REL * (1.001f * na * cmax + 0.5f * cmax2) + na * cdel) * 1.01f + 1.2e-7f;
+    const float mtc = tensor_bound(na, cmax, cmax2, cdel);
     if (!mbar_wait(mb, (tcs.phase >> wg) & 1u, MBAR_POLLS) && lane == 0 && status) atomicOr(status, 2);
     tcs.phase ^= 1u << wg;
     tc_fence_after();
@@ -1435,6 +1460,66 @@ cudaError_t launch_append(const CacheView& kc, const CacheView& vc, const void* 
   if (dtype == NSN_DTYPE_F32) return launch_append_t<NSN_DTYPE_F32>(kc, vc, kn, vn, sb, sh, cbk, cbv, s);
   if (dtype == NSN_DTYPE_BF16) return launch_append_t<NSN_DTYPE_BF16>(kc, vc, kn, vn, sb, sh, cbk, cbv, s);
   return launch_append_t<NSN_DTYPE_F16>(kc, vc, kn, vn, sb, sh, cbk, cbv, s);
+}
+
+// ---------------------------------------------------------------------------
+// Diagnostic: the tensor-core scores of up to 128 fp32 rows against a codebook,
+// formed exactly as the prefill search forms them (codebook staging, A operand
+// rows, the two MMAs into tensor memory) and read back raw, so that their error
+// against exact arithmetic can be measured.  One CTA of 128 threads, thread =
+// row = tensor-memory lane; rows past n are zero and not written back.
+// ---------------------------------------------------------------------------
+struct TsSmem {
+  QTables tb;
+  QSearch se;
+};
+
+__global__ void __launch_bounds__(BLK, 1)
+tensor_scores_selftest_kernel(const float* __restrict__ rows, int n, const float* __restrict__ codebook, int cosine,
+                              float* __restrict__ scores, int32_t* __restrict__ status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  TsSmem& sm = *reinterpret_cast<TsSmem*>(smem_raw);
+  TcState tcs = tc_setup(sm.se, TC_COLS, 1);
+  const QRefs q{&sm.tb, &sm.se, nullptr, nullptr};
+  stage_codebook(q, codebook, cosine);
+  const int L = threadIdx.x, lane = L & 31;
+  float a[SUB];
+#pragma unroll
+  for (int d = 0; d < SUB; ++d) a[d] = L < n ? rows[(int64_t)L * SUB + d] : 0.f;
+  store_a_row(sm.se.aop[0], L, a, 0);
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (L == 0) issue_scores(q, tcs.tmem, sm.se.aop[0], q_smem(&sm.se.mbar[0]));
+  if (!mbar_wait(q_smem(&sm.se.mbar[0]), 0u, MBAR_POLLS) && lane == 0 && status) atomicOr(status, 2);
+  tc_fence_after();
+  const uint32_t taddr = tcs.tmem + ((uint32_t)(32 * (L >> 5)) << 16);
+#pragma unroll 1
+  for (int c = 0; c < NCODES / 32; ++c) {
+    uint32_t r[32];
+    tc_ld32(taddr + 32 * c, r);
+    tc_wait_ld();
+    tc_regs_ready(r);
+    if (L < n) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(scores + (int64_t)L * NCODES + 32 * c + i) =
+            make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
+                        __uint_as_float(r[i + 3]));
+    }
+  }
+  tc_teardown(tcs);
+}
+
+cudaError_t launch_tensor_scores_selftest(const float* rows, int n, const float* codebook, int cosine, float* scores,
+                                          int32_t* status, cudaStream_t s) {
+  const size_t smem = sizeof(TsSmem);
+  cudaError_t e = cudaFuncSetAttribute(tensor_scores_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  tensor_scores_selftest_kernel<<<1, BLK, smem, s>>>(rows, n, codebook, cosine, scores, status);
+  return cudaGetLastError();
 }
 
 }  // namespace nsn

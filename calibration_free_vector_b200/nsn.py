@@ -83,6 +83,8 @@ def load():
                                     c_void_p, c_void_p]
     lib.nsn_selftest_bounded_wait.restype = c_int
     lib.nsn_selftest_bounded_wait.argtypes = [c_void_p, c_int, c_void_p]
+    lib.nsn_selftest_tensor_scores.restype = c_int
+    lib.nsn_selftest_tensor_scores.argtypes = [c_void_p, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p]
     lib.nsn_quantize_kv_ragged.restype = c_int
     lib.nsn_quantize_kv_ragged.argtypes = [POINTER(nsn_cache), c_void_p, c_int, c_int64, c_int64, c_int64, c_void_p,
                                            c_int, c_void_p, c_void_p]
@@ -280,6 +282,16 @@ def nsn_selftest_bounded_wait(status, max_attempts: int = 8, stream=None) -> Non
     """Runs the bounded-wait diagnostic; `status` is a device int32 tensor of one element."""
     _check(load().nsn_selftest_bounded_wait(status.data_ptr(), max_attempts, _stream_ptr(stream)),
            "nsn_selftest_bounded_wait")
+
+
+def nsn_selftest_tensor_scores(rows, codebook, assign: int, scores, status, stream=None) -> None:
+    """Raw tensor-core scores of rows [n, 8] (n <= 128, device fp32) against the codebook
+    [256, 8] into scores [n, 256] (device fp32); status: device int32 [1]."""
+    if rows.dim() != 2 or rows.shape[1] != 8 or scores.shape != (rows.shape[0], 256):
+        raise ValueError("rows must be [n, 8] and scores [n, 256]")
+    _check(load().nsn_selftest_tensor_scores(rows.data_ptr(), rows.shape[0], codebook.data_ptr(), int(assign),
+                                             scores.data_ptr(), status.data_ptr(), _stream_ptr(stream)),
+           "nsn_selftest_tensor_scores")
 
 
 def nsn_decode_workspace_bytes(k_cache: Cache, n_q_heads: int) -> int:

@@ -397,6 +397,23 @@ nsn_status nsn_codebook_4bit_host(float* codebook, int n_values);
  */
 nsn_status nsn_selftest_bounded_wait(int32_t* status, int max_attempts, void* stream);
 
+/*
+ * Diagnostic of the quantizer's tensor-core scores ([TS] Metodologia 3: nearest
+ * codeword of one global codebook; the pages have no counterpart for the check).
+ * For n_rows (1..128) fp32 rows of 8 values (`rows`, DEVICE [n_rows][8]) and a
+ * codebook (DEVICE fp32 [256][8]) it stages the codebook, builds the A operand and
+ * runs the two tcgen05 MMAs exactly as the prefill search does, and writes the raw
+ * fp32 accumulators to `scores` (DEVICE [n_rows][256]):
+ *   assign 0: score_k = a . c_k - ||c_k||^2 / 2     (fp16 hi + lo a, fp16 c, fp16 hi + lo bias)
+ *   assign 1: score_k = a . c_hat_k                  (c_hat = c / ||c||, fp16 hi + lo on both sides)
+ * so the caller can compare them with exact arithmetic.  All pointers 16-byte
+ * aligned (status 4-byte); bit 2 of *status (device int32) is set if the MMA
+ * completion wait gave up.  Invalid arguments return NSN_ERR_INVALID_ARG before
+ * any launch.
+ */
+nsn_status nsn_selftest_tensor_scores(const float* rows, int n_rows, const float* codebook, int assign,
+                                      float* scores, int32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
