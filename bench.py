@@ -68,8 +68,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh,
 # comments and whitespace removed).
 # Any later change to those files makes the figure stale; the bench then reports null.
-DECODE_TRAFFIC = {"sha256": "ea241b89a8f2a1e6dad9d25fdcf849fe9ecc0b2c00ca6d3ef9d8527751ea33b8",
-                  "bytes_per_launch": (321008128 + 321048320) // 2 + (4360704 + 441856) // 2}
+DECODE_TRAFFIC = {"sha256": "01f3e0596579000a33f01560f218c883409f435271b18df7bd74d81fec7aec1b",
+                  "bytes_per_launch": (321052928 + 321093376) // 2 + (3606272 + 506112) // 2}
 
 
 def decode_sources_sha256() -> str:
