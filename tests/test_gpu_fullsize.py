@@ -1,6 +1,7 @@
 """Parity at the full workload sizes, in the launch configuration the bench uses.
 
-For each of the decode-throughput layer (batch 16 x 32k, 2-bit K/V; also with
+For each of the decode-throughput layer (batch 16 x 32k, 2-bit K/V, after 1 and
+after 64 decode steps; also with
 pre-RoPE keys), the extreme
 compression layer (batch 64 x 8k, 1-bit K/V) and the long-context layer (batch 4 x
 128k, 2-bit K / 1-bit V; also with pre-RoPE keys): prefill on the GPU, append the workload's decode tokens
@@ -162,3 +163,9 @@ def test_fullsize_decode_throughput_layer_pre_rope(pool):
 def test_fullsize_long_context_pre_rope(pool):
     # batch 4, 128k context, pre-RoPE keys: angles up to about 1.3e5 rad at theta_0 = 1
     run_workload(5, 16, pool, sample_blocks=2, rope=True)
+
+
+def test_fullsize_decode_throughput_layer_64_steps(pool):
+    # the state the bench times: 64 decode steps, the first append flushes the full
+    # window into the quantized part and the window then grows back to 64 tokens
+    run_workload(3, 64, pool, sample_blocks=2, seed_off=1)
