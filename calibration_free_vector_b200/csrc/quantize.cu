@@ -31,14 +31,19 @@
 // -||c_k||^2/2), the second adds K = [a_hi | a_lo] (the fp32 a split into two fp16
 // parts, exact to 2^-22) times [c | c] (the codebook in fp16).  Each TMEM lane
 // holds one sub-vector's 256 scores; its thread reads them back with tcgen05.ld and
-// keeps, with three-input max trees, the best and second-best maxima of the groups
-// of 8 codewords (the group number rides in the low mantissa bits).  The 8
-// codewords of the winning group are then rescanned in sequential fp32 from an fp32
-// copy of the codebook in shared memory.  Whenever a rival lies within the error bounds of the best
-// (the fp32 bound inside the group, that plus a wide tensor-accumulation bound
-// outside it), the sub-vector is re-decided exactly in fp64 by a whole warp over
-// all codewords inside the bound (ties to the lowest index).  The stored code is
-// therefore the exact nearest codeword of the fp32 u.
+// keeps, with three-input max trees, the best and second-best maxima of the 32
+// groups of 8 codewords (the group number rides in the low mantissa bits).
+//   Prefill: the thread also keeps the maxima of the 8 columns (position within a
+//   group) over all groups.  The best score lies in the best group G and the best
+//   column J, so it is codeword 8 G + J; every other score is below the second-best
+//   group or column maximum.  If the best beats both by more than twice the
+//   tensor-score bound the code is certain.
+//   Window flushes: the 8 codewords of the winning group are rescanned in
+//   sequential fp32 from an fp32 copy of the codebook in shared memory, and the
+//   in-group decision uses the fp32 bound.
+// Whenever a rival lies within the bounds, the sub-vector is re-decided exactly in
+// fp64 by a whole warp over all codewords inside the bound (ties to the lowest
+// index).  The stored code is therefore the exact nearest codeword of the fp32 u.
 
 #include <algorithm>
 
@@ -137,9 +142,10 @@ struct QTables {
   // ---- codebook for the exact arithmetic (fp32: c, or c_hat for the cosine assignment), two
   // replicas: replica p of codeword k at floats 16 k + 8 p .. 16 k + 8 p + 7, so a 16-byte half h of it
   // lies in bank group 4 (k & 1) + 2 p + h.  The bias -||c_k||^2/2 (fp32, sequential; 0 for the cosine
-  // assignment) in four replicas, replica r at word 4 k + r.  A search lane l reads codeword 8 G + ((i + l) & 7)
-  // from replica (l >> 2) & 1, half (l >> 1) & 1 first, and bias replica l >> 3: the 8 lanes of a phase hit
-  // 8 different bank groups, and the 32 lanes 32 different bias banks, whatever their groups G. ----
+  // assignment) in four replicas, replica r at word 4 k + r.  A lane l reading codeword 8 G + ((i + l) & 7)
+  // from replica (l >> 2) & 1, half (l >> 1) & 1 first, with bias replica l >> 3, hits with the 8 lanes of a
+  // phase 8 different bank groups, and with the 32 lanes 32 different bias banks, whatever their groups G;
+  // the exact re-decision and the adaptive scale read it, and the flush's group rescan. ----
   alignas(16) float cw[NCODES * 16];
   alignas(16) float cbias[NCODES * 4];
   alignas(16) float cnorm[4];                     // [0] max ||c||, [1] max ||c||^2, [2] max ||c - fp16(c)|| (rounded up)
@@ -1095,12 +1101,12 @@ __device__ __forceinline__ void issue_scores(const QRefs& q, uint32_t dtmem, con
 // Warp-specialized prefill: one persistent CTA per SM, 16 warps, two blocks in
 // flight.  Warps 0-7 (the searchers) form two warpgroups; warpgroup g searches the
 // tiles g, g + 2, ... of a block in its own 256-column tensor-memory buffer, so the
-// two warpgroups' MMA waits, score reductions and rescans overlap.  A searcher
-// thread owns one tile row (= tensor-memory lane): it builds the row's A operand,
-// one thread per warpgroup issues the MMAs, then each thread reads its row's 256
-// scores, keeps the two best group maxima, rescans the winning group's 8
-// codewords in fp32 and decides; after the block the 8 warps re-decide the
-// flagged sub-vectors.  Warps 8-15 (the normalizers) run the NSN of block j into
+// two warpgroups' MMA waits and score reductions overlap.  A searcher thread owns
+// one tile row (= tensor-memory lane): it builds the row's A operand, one thread
+// per warpgroup issues the MMAs, then each thread reads its row's 256 scores,
+// keeps the two best group maxima and the two best column maxima, and decides
+// (codeword 8 G + J, certified by the tensor-score bound); after the block the 8
+// warps re-decide the flagged sub-vectors.  Warps 8-15 (the normalizers) run the NSN of block j into
 // one of two block buffers while the searchers work on block j - 1, and then the
 // adaptive scale and stores of block j - 2.  Named barriers hand a block over:
 // U (u rows ready, normalizers -> searchers) and D (codes final, searchers ->
@@ -1125,28 +1131,28 @@ __device__ __forceinline__ void bar_arrive(int id, int n) { asm volatile("bar.ar
 __device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory"); }
 
 // Search of the tiles wg, wg + 2, ... of one block by search warpgroup wg (thread
-// L = tile row = tensor-memory lane).  Bounds as in search_block.
+// L = tile row = tensor-memory lane).  The tensor-score bound is tensor_bound().
 __device__ void search_tiles_ws(const QRefs& q, TcState& tcs, const float* __restrict__ cb_global, int n, int wg,
                                 int32_t* status) {
   const int L = threadIdx.x & 127, wq = L >> 5, lane = L & 31;
   const Grp g{WS_BAR_G + wg, 128, L};
   const float cmax = q.tb->cnorm[0], cmax2 = q.tb->cnorm[1], cdel = q.tb->cnorm[2];
-  constexpr float GAMMA9 = 9.0f * 5.9604645e-8f * 1.0001f;  // 9u/(1-9u), u = 2^-24
   const uint32_t tbuf = tcs.tmem + (uint32_t)(TC_COLS * wg);
   const uint32_t taddr = tbuf + ((uint32_t)(32 * wq) << 16);
   unsigned char* ap = q.se->aop[wg];
   const uint32_t mb = q_smem(&q.se->mbar[wg]);
   const int ntiles = (n + 7) >> 3;
-  // exact-arithmetic table reads of this lane (bank-conflict free, see QTables)
-  const int rp = (lane >> 2) & 1, hf = (lane >> 1) & 1, bq = lane >> 3;
+  // this lane reads its row's half hf first: the 8 lanes of a phase then hit 8
+  // different bank groups
+  const int hf = (lane >> 2) & 1;
   const int j = L & 15;
 
 #pragma unroll 1
   for (int tile = wg; tile < ntiles; tile += WS_SWG) {
     const int tkk = 8 * tile + (L >> 4);
-    // ---- the row's A operand (hi and lo halves) and its decision bounds ----
-    // a[0..3] = dims 4 hf .. 4 hf + 3, a[4..7] = the other half (the order of this
-    // lane's table reads); the A operand keeps the natural order.
+    // ---- the row's A operand (hi and lo halves) and its decision bound ----
+    // a[0..3] = dims 4 hf .. 4 hf + 3, a[4..7] = the other half; the A operand
+    // keeps the natural order.
     float a[SUB];
     {
       const float4 a0 = *reinterpret_cast<const float4*>(&q.bk->tile[tkk][SUB * j + 4 * hf]);
@@ -1165,7 +1171,6 @@ __device__ void search_tiles_ws(const QRefs& q, TcState& tcs, const float* __res
 #pragma unroll
     for (int d = 0; d < SUB; ++d) na = fmaf(a[d], a[d], na);
     na = sqrtf(na) * 1.0001f;
-    const float margin = 2.0f * GAMMA9 * (cmax2 + na * cmax) * 1.01f;
     const float mtc = tensor_bound(na, cmax, cmax2, cdel);
     if (!mbar_wait(mb, (tcs.phase >> wg) & 1u, MBAR_POLLS) && lane == 0 && status) atomicOr(status, 2);
     tcs.phase ^= 1u << wg;
@@ -1173,7 +1178,11 @@ __device__ void search_tiles_ws(const QRefs& q, TcState& tcs, const float* __res
 
     // ---- best and second-best of the 32 group maxima of the row's 256 scores ----
     // (two register buffers in turn: chunk c + 1 loads while chunk c is reduced)
+    // and the maxima of the 8 columns (index within a group) over all groups
     float b1 = -INFINITY, b2 = -INFINITY;
+    float cm[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) cm[jj] = -INFINITY;
     uint32_t rb[2][32];
     tc_ld32(taddr, rb[0]);
 #pragma unroll
@@ -1196,41 +1205,34 @@ __device__ void search_tiles_ws(const QRefs& q, TcState& tcs, const float* __res
       const float lo = max3f(l01, l23, fminf(h01, h23));
       b2 = max3f(b2, lo, fminf(b1, hi));
       b1 = fmaxf(b1, hi);
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        cm[jj] = max3f(cm[jj], __uint_as_float(r[jj]), __uint_as_float(r[8 + jj]));
+        cm[jj] = max3f(cm[jj], __uint_as_float(r[16 + jj]), __uint_as_float(r[24 + jj]));
+      }
     }
     const int G = (int)(__float_as_uint(b1) & 31u);
-
-    // ---- the winning group's 8 codewords in sequential fp32, lane-rotated order,
-    // ties to the lowest index ----
-    float best = -INFINITY, second = -INFINITY;
-    int idx = NCODES;
-    {
-      float cw[8][SUB], sc[8];
-      int kk[8];
+    // best and second-best column maximum, the column number in the low 3 bits
+    float c1 = -INFINITY, c2 = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        kk[i] = 8 * G + ((i + lane) & 7);
-        const float* src = q.tb->cw + 16 * kk[i] + 8 * rp;
-        const float4 x0 = *reinterpret_cast<const float4*>(src + 4 * hf);
-        const float4 x1 = *reinterpret_cast<const float4*>(src + 4 - 4 * hf);
-        cw[i][0] = x0.x; cw[i][1] = x0.y; cw[i][2] = x0.z; cw[i][3] = x0.w;
-        cw[i][4] = x1.x; cw[i][5] = x1.y; cw[i][6] = x1.z; cw[i][7] = x1.w;
-        sc[i] = q.tb->cbias[4 * kk[i] + bq];
-      }
-#pragma unroll
-      for (int d = 0; d < SUB; ++d)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sc[i] = fmaf(a[d], cw[i][d], sc[i]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float lo = fminf(best, sc[i]);
-        idx = (sc[i] > best || (sc[i] == best && kk[i] < idx)) ? kk[i] : idx;
-        best = fmaxf(best, sc[i]);
-        second = fmaxf(second, lo);
-      }
+    for (int jj = 0; jj < 8; ++jj) {
+      const float key = __uint_as_float((__float_as_uint(cm[jj]) & ~7u) | (uint32_t)jj);
+      c2 = fmaxf(c2, fminf(c1, key));
+      c1 = fmaxf(c1, key);
     }
-    const float other = b2 + fabsf(b2) * 3.82e-6f;  // + 32 ulp: the group number in the low bits
+    const int J = (int)(__float_as_uint(c1) & 7u);
+
+    // ---- the best tensor score lies in group G (best group maximum) and column J
+    // (best column maximum), so it is codeword 8 G + J.  Every other score is below
+    // the second-best group maximum or the second-best column maximum; if the best
+    // beats both by more than twice the tensor bound (after the key bits: 32 ulp for
+    // a group number, 8 ulp for a column number), the code is the exact nearest
+    // codeword; otherwise the sub-vector is re-decided exactly. ----
+    const int idx = 8 * G + J;
+    const float top = b1 - fabsf(b1) * 3.82e-6f;
+    const float rival = fmaxf(b2 + fabsf(b2) * 3.82e-6f, c2 + fabsf(c2) * 9.6e-7f);
     q.bk->code[tkk][j] = (uint8_t)idx;
-    const bool need = second >= best - margin || other >= best - 0.5f * margin - mtc;
+    const bool need = rival >= top - 2.0f * mtc;
     if (need && tkk < n) q.se->flag[atomicAdd(&q.se->nflag, 1)] = (uint16_t)(tkk * NSUB + j);
   }
   tc_fence_before();
