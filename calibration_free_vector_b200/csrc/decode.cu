@@ -329,14 +329,10 @@ __device__ __forceinline__ void build_q_operand(uint32_t (&qb)[8][2], const floa
       float v[4] = {rows[h < GH ? h : 0][0], rows[h < GH ? h : 0][1], rows[h < GH ? h : 0][2],
                     rows[h < GH ? h : 0][3]};
       if (rotate) fwht128_warp(v, lane);
-      float r[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v[i] *= scale;
-        r[i] = v[i] - __half2float(__float2half_rn(v[i]));
-      }
-      hi = make_uint2(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]));
-      lo = make_uint2(pack_half2(r[0], r[1]), pack_half2(r[2], r[3]));
+      for (int i = 0; i < 4; ++i) v[i] *= scale;
+      split_half2(v[0], v[1], hi.x, lo.x);
+      split_half2(v[2], v[3], hi.y, lo.y);
     }
     *reinterpret_cast<uint2*>(qs + h * QS_ROW + 8 * lane) = hi;
     *reinterpret_cast<uint2*>(qs + (h + 4) * QS_ROW + 8 * lane) = lo;
@@ -974,12 +970,6 @@ __device__ __forceinline__ float2 rope_cs(double a) {
   return make_float2(cs, sn);
 }
 
-__device__ __forceinline__ void mma_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, {%0, %1, %2, %3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(b0));
-}
-
 __device__ __forceinline__ void mma_zero(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%10, %10, %10, %10};\n"
@@ -1222,10 +1212,12 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
         }
       }
       // NSN terms, rotation of dims (i, i + 64), fp16 hi + lo, and the query product
+      // (one k16 MMA per 16 dims for the hi part and one for the lo part)
       const int r_off = 16 * m + g;  // offset-table rows of this lane's tokens: r_off, r_off + 8
       float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int ap = 0; ap < 4; ++ap)
+      for (int ap = 0; ap < 4; ++ap) {
+        uint32_t ahi[2][4], alo[2][4];  // [h][A fragment register]: rows g, g + 8 of k-halves nt = 0, 1
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const int i0 = 16 * ap + 8 * nt + 2 * p;
@@ -1248,18 +1240,16 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const float* y = h ? y1 : y0;
-            uint32_t ahi[2], alo[2];
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-              const __half2 hh = __floats2half2_rn(y[2 * rr], y[2 * rr + 1]);
-              const float2 hf = __half22float2(hh);
-              ahi[rr] = *reinterpret_cast<const uint32_t*>(&hh);
-              alo[rr] = pack_half2(y[2 * rr] - hf.x, y[2 * rr + 1] - hf.y);
-            }
-            mma_k8(S[h], ahi[0], ahi[1], qb[ap + 4 * h][nt]);
-            mma_k8(S[h], alo[0], alo[1], qb[ap + 4 * h][nt]);
+            for (int rr = 0; rr < 2; ++rr) split_half2(y[2 * rr], y[2 * rr + 1], ahi[h][2 * nt + rr], alo[h][2 * nt + rr]);
           }
         }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          mma_full(S[h], ahi[h], qb[ap + 4 * h][0], qb[ap + 4 * h][1]);
+          mma_full(S[h], alo[h], qb[ap + 4 * h][0], qb[ap + 4 * h][1]);
+        }
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) S[0][i] += S[1][i];
       // hi + lo query columns -> (token t_l, heads h0, h0 + 1)

@@ -58,6 +58,24 @@ __device__ __forceinline__ void load8<NSN_DTYPE_F16>(const void* base, int64_t e
   }
 }
 
+// y minus an fp16 value h, in fp32, by one mixed-precision fma ((-1) * h + y with
+// an fp16 multiplicand, sm_100).  When h = fp16(y) the difference is exact: it is
+// a multiple of the fp32 ulp of y and below 2^-11 |y|.
+__device__ __forceinline__ float sub_f16(float y, uint16_t h) {
+  float d;
+  asm("{\n\t.reg .b16 m1;\n\tmov.b16 m1, 0xBC00;\n\tfma.rn.f32.f16 %0, %1, m1, %2;\n\t}" : "=f"(d) : "h"(h), "f"(y));
+  return d;
+}
+
+// fp16 high and low parts of two fp32 values, each packed as a half2 (first value
+// in the low half): hi = fp16(y), lo = fp16(y - hi), so hi + lo = y to 2^-22.
+__device__ __forceinline__ void split_half2(float y0, float y1, uint32_t& hi, uint32_t& lo) {
+  const __half2 hh = __floats2half2_rn(y0, y1);
+  hi = *reinterpret_cast<const uint32_t*>(&hh);
+  const __half2 ll = __floats2half2_rn(sub_f16(y0, (uint16_t)(hi & 0xFFFFu)), sub_f16(y1, (uint16_t)(hi >> 16)));
+  lo = *reinterpret_cast<const uint32_t*>(&ll);
+}
+
 // Converts 8 values to fp16 (round to nearest even) packed in 16 bytes.
 __device__ __forceinline__ uint4 pack8_f16(const float* v) {
   uint4 r;

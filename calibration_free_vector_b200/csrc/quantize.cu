@@ -526,12 +526,10 @@ __device__ void search_block(const QRefs& q, TcState& tcs, const float* __restri
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const __half2 hh = __floats2half2_rn(a[2 * p], a[2 * p + 1]);
-      if (hf == 0) {
-        w[p] = h2_bits(hh);
-      } else {
-        const float2 back = __half22float2(hh);
-        w[p] = h2_bits(__floats2half2_rn(a[2 * p] - back.x, a[2 * p + 1] - back.y));
-      }
+      w[p] = h2_bits(hh);
+      if (hf != 0)
+        w[p] = h2_bits(__floats2half2_rn(sub_f16(a[2 * p], (uint16_t)(w[p] & 0xFFFFu)),
+                                         sub_f16(a[2 * p + 1], (uint16_t)(w[p] >> 16))));
     }
     *reinterpret_cast<uint4*>(q.se->aop[tile & 1] + kmaj_off(L, 8 * hf)) = make_uint4(w[0], w[1], w[2], w[3]);
   };
@@ -1066,12 +1064,7 @@ __device__ __forceinline__ PrefillSplit prefill_split(const int32_t* __restrict_
 __device__ __forceinline__ void store_a_row(unsigned char* ap, int row, const float (&a)[SUB], int h) {
   uint32_t hi[4], lo[4];
 #pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const __half2 hh = __floats2half2_rn(a[2 * p], a[2 * p + 1]);
-    const float2 back = __half22float2(hh);
-    hi[p] = h2_bits(hh);
-    lo[p] = h2_bits(__floats2half2_rn(a[2 * p] - back.x, a[2 * p + 1] - back.y));
-  }
+  for (int p = 0; p < 4; ++p) split_half2(a[2 * p], a[2 * p + 1], hi[p], lo[p]);
   *reinterpret_cast<uint2*>(ap + kmaj_off(row, 4 * h)) = make_uint2(hi[0], hi[1]);
   *reinterpret_cast<uint2*>(ap + kmaj_off(row, 4 - 4 * h)) = make_uint2(hi[2], hi[3]);
   *reinterpret_cast<uint2*>(ap + kmaj_off(row, 8 + 4 * h)) = make_uint2(lo[0], lo[1]);
