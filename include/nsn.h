@@ -209,9 +209,10 @@ nsn_status nsn_build_codebook_cosine_host(uint64_t seed, int n_samples, int n_co
  *              Requires Q <= capacity.
  *   codebook   device float[256*8] (signed codebook in 1-bit, absolute in 2-bit).
  * Stored values: codes/signs bit-exact to the definition: the nearest codeword of
- * the fp32 sub-vector (scores on the tensor cores, the winning group of 8 codewords
- * rescanned in fp32, and every near tie within the error bounds re-decided exactly in
- * fp64; ties to the lowest index), s1, alpha*s2 and o rounded to fp16.  Any fp32
+ * the fp32 sub-vector (scores on the tensor cores, the winner located by the best
+ * group and column maxima of the scores, and every near tie within the error bounds
+ * re-decided exactly in fp64; ties to the lowest index), s1, alpha*s2 and o rounded
+ * to fp16.  Any fp32
  * codebook works; one of fp16-representable values keeps the decision bound tightest.
  */
 nsn_status nsn_quantize_kv(nsn_cache* cache, const void* x, int dtype, int64_t stride_b,
