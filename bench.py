@@ -267,6 +267,15 @@ def oracle_quantize_check(x_blocks: np.ndarray, codebook: np.ndarray, mode: int,
     return float(np.mean(times)), len(times), n_sub, n_tie, n_bad, n_sbad
 
 
+def codes_natural(code_bytes: np.ndarray) -> np.ndarray:
+    """The cache's code records [n, 16] (the even sub-vectors' codes, then the odd
+    ones') in natural sub-vector order."""
+    out = np.empty_like(code_bytes)
+    out[:, 0::2] = code_bytes[:, :8]
+    out[:, 1::2] = code_bytes[:, 8:]
+    return out
+
+
 def signs_natural(sign_bytes: np.ndarray) -> np.ndarray:
     """The cache's sign records [n, 16] (field i = dim i of the 16 sub-vectors,
     sub-vector s at bit 15 - s) as the natural layout [n, 16] (byte s, bit i)."""
@@ -377,7 +386,7 @@ def run_ours(args):
     # the first blocks of layer 0's K prefill, for the sampled parity check against the oracle
     nchk = 0 if args.lite else 8
     chk_x = xk[0, :128 * nchk, 0].float().cpu().numpy().reshape(nchk, 128, 128)
-    chk_codes = kcs[0].codes[0, 0, :128 * nchk].cpu().numpy().reshape(nchk, 128, 16)
+    chk_codes = codes_natural(kcs[0].codes[0, 0, :128 * nchk].cpu().numpy()).reshape(nchk, 128, 16)
     chk_signs = (kcs[0].signs[0, 0, :128 * nchk].cpu().numpy().reshape(nchk, 128, 16)
                  if W["mode_k"] == 2 else None)
     del xk, xv

@@ -92,8 +92,11 @@ __device__ __forceinline__ uint32_t apply_signs(uint32_t x, uint32_t w, int s) {
   return x ^ ((w << s) & 0x80008000u);
 }
 
-__device__ __forceinline__ uint32_t u4_word(const uint4& v, int i) {
-  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+// Code of k-step j (0..7) from the 8 code bytes a lane reads: the cache stores a
+// token's codes as the even sub-vectors' (bytes 0-7) then the odd ones' (bytes
+// 8-15), and a lane whose ldmatrix row is sub-vector 2j + par reads half par.
+__device__ __forceinline__ uint32_t code_byte(const uint2& w, int j) {
+  return __byte_perm(j < 4 ? w.x : w.y, 0u, 0x4440u | (uint32_t)(j & 3));
 }
 
 // ---------------------------------------------------------------------------
@@ -620,10 +623,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
   const uint32_t cbv_base = smem_addr(&sm.cbv[0][0]) + lane_row;
   const int tok_a = (lane & 7) + 8 * ((lane >> 3) & 1);   // token of this lane's K ldmatrix row
   const int tok_v = (lane & 7) + 8 * (lane >> 4);         // token of this lane's V ldmatrix row
-  const uint32_t sel_k0 = 0x4440u | (uint32_t)(lane >> 4);
-  const uint32_t sel_k1 = 0x4440u | (uint32_t)(2 + (lane >> 4));
-  const uint32_t sel_v0 = 0x4440u | (uint32_t)((lane >> 3) & 1);
-  const uint32_t sel_v1 = 0x4440u | (uint32_t)(2 + ((lane >> 3) & 1));
+  const int kpar = lane >> 4, vpar = (lane >> 3) & 1;   // sub-vector parity of the K / V ldmatrix row
   const bool lo_lane = p < 2;                      // keeps token g (else g + 8) after the swap
   const int t_l = g + (lo_lane ? 0 : 8);           // token of this lane's two scores
   const int h0 = 2 * (p & 1);                      // its two heads: h0, h0 + 1 (within the group)
@@ -683,8 +683,8 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
     const bool full = t_stage + STAGE_TOK <= tok_end;  // every token of the stage is valid
     for (int tile = 0; tile < ntile; ++tile) {
       const int tt = 16 * tile;  // token offset inside the stage
-      uint4 kcw = make_uint4(0u, 0u, 0u, 0u);
-      if constexpr (!RP) kcw = *reinterpret_cast<const uint4*>(sb + ST_KC + (tt + tok_a) * 16);
+      uint2 kcw = make_uint2(0u, 0u);
+      if constexpr (!RP) kcw = *reinterpret_cast<const uint2*>(sb + ST_KC + (tt + tok_a) * 16 + 8 * kpar);
       uint32_t ks0 = 0u, ks1 = 0u;
       if constexpr (!RP && MK == NSN_MODE_2BIT) {
         ks0 = *reinterpret_cast<const uint32_t*>(sb + ST_KS + (tt + g) * 16 + 4 * p);
@@ -692,7 +692,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       }
       uint32_t knw = 0u, vnw = 0u;
       if constexpr (!DQ && !RP) knw = *reinterpret_cast<const uint32_t*>(sb + ST_KN + (tt + t_l) * 4);
-      const uint4 vcw = *reinterpret_cast<const uint4*>(sb + ST_VC + (tt + tok_v) * 16);
+      const uint2 vcw = *reinterpret_cast<const uint2*>(sb + ST_VC + (tt + tok_v) * 16 + 8 * vpar);
       uint32_t W0 = 0u, W1 = 0u;
       if constexpr (MV == NSN_MODE_2BIT) {
         const uint16_t* vs = reinterpret_cast<const uint16_t*>(sb + ST_VS);
@@ -705,7 +705,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < (RP ? 0 : 8); ++j) {
-        const uint32_t code = __byte_perm(u4_word(kcw, j >> 1), 0u, (j & 1) ? sel_k1 : sel_k0);
+        const uint32_t code = code_byte(kcw, j);
         uint32_t aa[4];
         ldsm_x4(cbk_base + code * 128u, aa);
         if constexpr (MK == NSN_MODE_2BIT) {
@@ -768,7 +768,7 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
       // ---- values: O^T += u_hat_v^T w ----
 #pragma unroll
       for (int mm = 0; mm < 8; ++mm) {
-        const uint32_t code = __byte_perm(u4_word(vcw, mm >> 1), 0u, (mm & 1) ? sel_v1 : sel_v0);
+        const uint32_t code = code_byte(vcw, mm);
         uint32_t aa[4];
         ldsm_x4_t(cbv_base + code * 128u, aa);
         if constexpr (MV == NSN_MODE_2BIT) {
@@ -979,14 +979,15 @@ __device__ __forceinline__ void mma_zero(float (&d)[4], const uint32_t (&a)[4], 
 
 // Compressed inputs of one 16-token K tile, loaded one tile ahead.
 struct RsTileIn {
-  uint4 codes;      // code bytes of this lane's ldmatrix token
+  uint2 codes;      // code bytes of this lane's ldmatrix row (its token, sub-vector parity)
   uint32_t ks0, ks1;  // sign words (2-bit) of tokens g, g + 8
   uint32_t n[2];    // tokens g, g + 8: (s1, s2) fp16 pair, or (alpha*s2 fp16 | s1 level << 16) with DQ
 };
 
 template <int MK, bool DQ>
-__device__ __forceinline__ void rs_load_tile(RsTileIn& in, const CacheView& kc, int64_t tq, int tok_a, int g, int p) {
-  in.codes = __ldg(reinterpret_cast<const uint4*>(kc.codes + (tq + tok_a) * NSUB));
+__device__ __forceinline__ void rs_load_tile(RsTileIn& in, const CacheView& kc, int64_t tq, int tok_a, int kpar, int g,
+                                             int p) {
+  in.codes = __ldg(reinterpret_cast<const uint2*>(kc.codes + (tq + tok_a) * NSUB + 8 * kpar));
   in.ks0 = in.ks1 = 0u;
   if constexpr (MK == NSN_MODE_2BIT) {
     in.ks0 = __ldg(reinterpret_cast<const uint32_t*>(kc.signs + (tq + g) * NSUB) + p);
@@ -1068,8 +1069,7 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
   }
   const uint32_t cbk_base = smem_addr(&sm.cbk[0][0]) + (uint32_t)(lane & 7) * 16u;
   const int tok_a = (lane & 7) + 8 * ((lane >> 3) & 1);
-  const uint32_t sel_k0 = 0x4440u | (uint32_t)(lane >> 4);
-  const uint32_t sel_k1 = 0x4440u | (uint32_t)(2 + (lane >> 4));
+  const int kpar = lane >> 4;
   const bool lo_lane = p < 2;
   const int t_l = g + (lo_lane ? 0 : 8);
   const int h0 = 2 * (p & 1);
@@ -1077,7 +1077,7 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
   const int q_end = min(nq, st_last * STAGE_TOK);  // this job's quantized positions end here
   int cur_blk = -1;
   RsTileIn nxt;
-  if (st_first < nst_q) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + st_first * STAGE_TOK, tok_a, g, p);
+  if (st_first < nst_q) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + st_first * STAGE_TOK, tok_a, kpar, g, p);
 
   for (int st = st_first; st < st_last; ++st) {
     const bool win = st >= nst_q;
@@ -1144,7 +1144,7 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
       float xs[2] = {1.f, 1.f}, s1r[2] = {1.f, 1.f};  // per row: scale of E, and s1
       if (!win) {
         const RsTileIn cur = nxt;
-        if (tt + 16 < q_end) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + tt + 16, tok_a, g, p);
+        if (tt + 16 < q_end) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + tt + 16, tok_a, kpar, g, p);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           if constexpr (DQ) {
@@ -1160,7 +1160,7 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
         // H_8 stage across bit 2 of the k-step, accumulated on the tensor cores;
         // the stages across bits 0 and 1 follow in fp32
         auto gather = [&](int a, uint32_t (&A)[4]) {
-          const uint32_t code = __byte_perm(u4_word(cur.codes, a >> 1), 0u, (a & 1) ? sel_k1 : sel_k0);
+          const uint32_t code = code_byte(cur.codes, a);
           ldsm_x4(cbk_base + code * 128u, A);
           if constexpr (MK == NSN_MODE_2BIT) {
             A[0] = apply_signs(A[0], cur.ks0, 2 * a);

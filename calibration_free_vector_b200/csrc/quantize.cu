@@ -1004,8 +1004,11 @@ __device__ void finish_phase(const QRefs& q, const Grp& gr, const float* __restr
 
   // ---- packed stores ---------------------------------------------------------
   if (valid) {
+    // stored order: the even sub-vectors' codes (h = 0), then the odd ones' (h = 1)
+    const uint4 cw = *reinterpret_cast<const uint4*>(&q.bk->code[tk][0]);
+    const uint32_t sel = h ? 0x7531u : 0x6420u;
     *reinterpret_cast<uint2*>(codes + (int64_t)tk * NSUB + HSUB * h) =
-        *reinterpret_cast<const uint2*>(&q.bk->code[tk][HSUB * h]);
+        make_uint2(__byte_perm(cw.x, cw.y, sel), __byte_perm(cw.z, cw.w, sel));
     if (h == 0) {
       const BlockOut bo = block_out(cv, seq, tok0, blk);
       if (bo.dq) bo.s2[tk] = __double2half(alpha * q.bk->s2[tk]);

@@ -69,7 +69,10 @@ typedef enum { NSN_DTYPE_F32 = 0, NSN_DTYPE_BF16 = 1, NSN_DTYPE_F16 = 2 } nsn_dt
 /*
  * Compressed cache of one tensor (K or V) of one layer.  All pointers are
  * device pointers owned by the caller.  Layout (row-major, per (b, h) contiguous):
- *   codes    uint8  [batch][n_kv_heads][capacity][16]   code of sub-vector s at byte s
+ *   codes    uint8  [batch][n_kv_heads][capacity][16]   the codes of the even sub-vectors, then
+ *                                                       of the odd ones: byte i < 8 holds the
+ *                                                       code of sub-vector 2i, byte 8+i that
+ *                                                       of sub-vector 2i+1
  *   signs    uint8  [batch][n_kv_heads][capacity][16]   2-bit mode only (NULL in 1-bit): the
  *                                                       128 sign bits of a token as eight
  *                                                       little-endian 16-bit fields; field i

@@ -30,6 +30,22 @@ def codebook(mode: int) -> np.ndarray:
     return np.loadtxt(os.path.join(GOLDEN, name)).astype(np.float32)
 
 
+def codes_to_natural(stored: np.ndarray) -> np.ndarray:
+    """Stored code records [..., 16] (the even sub-vectors' codes, then the odd
+    ones') -> the oracle's layout [..., 16] (byte s = code of sub-vector s)."""
+    stored = np.asarray(stored)
+    out = np.empty_like(stored)
+    out[..., 0::2] = stored[..., :8]
+    out[..., 1::2] = stored[..., 8:]
+    return out
+
+
+def natural_to_codes(natural: np.ndarray) -> np.ndarray:
+    """Inverse of codes_to_natural."""
+    natural = np.asarray(natural)
+    return np.concatenate([natural[..., 0::2], natural[..., 1::2]], axis=-1)
+
+
 def signs_to_natural(stored: np.ndarray) -> np.ndarray:
     """Stored sign bytes [..., 16] (eight 16-bit fields; field i bit 15-s = sign of
     dim 8s+i) -> the oracle's layout [..., 16] (byte s bit i = sign of dim 8s+i)."""
@@ -75,7 +91,7 @@ def read_cache(cache, b: int, h: int) -> dict:
     out = {
         "n_quant": nq,
         "n_window": nw,
-        "codes": cache.codes[b, h, :nq].cpu().numpy().astype(np.int64),
+        "codes": codes_to_natural(cache.codes[b, h, :nq].cpu().numpy()).astype(np.int64),
         "signs": None if cache.signs is None else signs_to_natural(cache.signs[b, h, :nq].cpu().numpy()),
         "window": (cache.window_buf[b, h, :nw].float().cpu().numpy().astype(np.float64)
                    if cache.window_buf is not None else np.zeros((0, 128))),
@@ -192,7 +208,7 @@ def fill_cache(cache, contents):
     import torch
     for (b, h), c in contents.items():
         nq, nw = c["codes"].shape[0], c["window"].shape[0]
-        cache.codes[b, h, :nq] = torch.from_numpy(c["codes"])
+        cache.codes[b, h, :nq] = torch.from_numpy(natural_to_codes(c["codes"]))
         if c["signs"] is not None:
             cache.signs[b, h, :nq] = torch.from_numpy(c["signs"])
         cache.norms[b, h, :nq, 0] = torch.from_numpy(c["s1"])

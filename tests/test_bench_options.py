@@ -1,6 +1,6 @@
 """CPU checks of bench.py's host logic: the pre-RoPE leg's frequency table is the
 oracle's closed form in fp32 and its CPU baseline runs the oracle's pre-RoPE
-decode; the sign unpacking of the sampled parity check equals the test
+decode; the code and sign unpacking of the sampled parity check equal the test
 library's; both arms print the same config object; the parity check counts a
 planted code mismatch."""
 import os
@@ -25,6 +25,15 @@ def test_rope_theta_is_the_llama3_table_in_fp32():
 def test_cpu_baseline_sample_runs_the_pre_rope_oracle():
     t, n, threads = bench.oracle_decode_sample(0.0, seed=3, rope=True)
     assert n == 1 and t > 0.0 and threads >= 1
+
+
+def test_code_records_store_even_sub_vectors_first():
+    from tests import nsn_testlib as tl
+    x = np.arange(48, dtype=np.uint8).reshape(3, 16)
+    st = tl.natural_to_codes(x)
+    assert st[0].tolist() == list(range(0, 16, 2)) + list(range(1, 16, 2))
+    np.testing.assert_array_equal(tl.codes_to_natural(st), x)
+    np.testing.assert_array_equal(bench.codes_natural(st), x)
 
 
 def test_bench_sign_unpacking_matches_the_test_library():

@@ -90,7 +90,7 @@ def run_workload(cfg_id, steps, pool, sample_blocks=12, seed_off=0, double_quant
     refs = list(pool.map(tl._oracle_block, jobs))
     for (cache, b, h, blk), ref in zip(where, refs):
         sl = slice(128 * blk, 128 * (blk + 1))
-        got = {"codes": cache.codes[b, h, sl].cpu().numpy().astype(np.int64),
+        got = {"codes": tl.codes_to_natural(cache.codes[b, h, sl].cpu().numpy()).astype(np.int64),
                "signs": None if cache.signs is None else tl.signs_to_natural(cache.signs[b, h, sl].cpu().numpy())}
         s2 = cache.norms[b, h, sl] if double_quant else cache.norms[b, h, sl, 1]
         count(tl.compare_codes(dict(got, s2=s2.float().cpu().numpy().astype(np.float64)), ref, ref["u"]))
