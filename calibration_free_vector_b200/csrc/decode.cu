@@ -52,6 +52,15 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
                : "memory");
 }
 
+// Two 8x8 matrices (row addresses from lanes 0-15): for A operands whose rows
+// 8-15 repeat rows 0-7, half the shared-memory reads of an x4.
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(addr) : "memory");
+}
+
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -666,12 +675,15 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
         __syncwarp();
       }
       // (H q) . o_K of this block: the mean row as all 16 "tokens" of one score tile
+      // (rows 8-15 repeat rows 0-7, so an x2 load gives all four A registers)
       float d4[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t mrow = mb_base + (uint32_t)(mbuf * MEAN_BYTES) + (uint32_t)(lane >> 4) * 16u;
+      const uint32_t mrow = mb_base + (uint32_t)(mbuf * MEAN_BYTES) + (uint32_t)((lane >> 3) & 1) * 16u;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         uint32_t aa[4];
-        ldsm_x4(mrow + 32u * j, aa);
+        ldsm_x2(mrow + 32u * j, aa[0], aa[2]);
+        aa[1] = aa[0];
+        aa[3] = aa[2];
         mma_full(d4, aa, qb[j][0], qb[j][1]);
       }
       const float r0 = __shfl_xor_sync(0xffffffffu, lo_lane ? d4[2] : d4[0], 2);
@@ -855,8 +867,10 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
           float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            uint32_t aa[4];
-            ldsm_x4(kbuf + rowoff + (uint32_t)(32 * j + 16 * (lane >> 4)), aa);
+            uint32_t aa[4];  // rows 8-15 repeat rows 0-7
+            ldsm_x2(kbuf + rowoff + (uint32_t)(32 * j + 16 * ((lane >> 3) & 1)), aa[0], aa[2]);
+            aa[1] = aa[0];
+            aa[3] = aa[2];
             if (j & 1) mma_full(S2, aa, qb[j][0], qb[j][1]);
             else mma_full(S, aa, qb[j][0], qb[j][1]);
           }
@@ -877,8 +891,10 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
         const uint32_t pb0 = movmatrix_t(lo_lane ? wpk : 0u);  // tokens 0-7; tokens 8-15 weigh 0
 #pragma unroll
         for (int mm = 0; mm < 8; ++mm) {
-          uint32_t aa[4];
-          ldsm_x4_t(vbuf + rowoff + (uint32_t)(32 * mm + 16 * ((lane >> 3) & 1)), aa);
+          uint32_t aa[4];  // tokens 8-15 repeat tokens 0-7 (and weigh 0)
+          ldsm_x2_t(vbuf + rowoff + (uint32_t)(32 * mm + 16 * ((lane >> 3) & 1)), aa[0], aa[1]);
+          aa[2] = aa[0];
+          aa[3] = aa[1];
           mma_full(sx.O[mm], aa, pb0, 0u);
         }
         __syncwarp();
