@@ -68,8 +68,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh,
 # comments and whitespace removed).
 # Any later change to those files makes the figure stale; the bench then reports null.
-DECODE_TRAFFIC = {"sha256": "278737980b6b300455d4ae3f71e9d62e569abe8be8a3f7e2440a3321eea7aa20",
-                  "bytes_per_launch": (320980992 + 321106432) // 2 + (3718656 + 861440) // 2}
+DECODE_TRAFFIC = {"sha256": "95dda82e613710615757f6eb9d04394d703caabccba4e3aeb718dd40737334b9",
+                  "bytes_per_launch": (320906752 + 320956928) // 2 + (3941888 + 468224) // 2}
 
 
 def decode_sources_sha256() -> str:

@@ -995,15 +995,14 @@ __device__ __forceinline__ void mma_zero(float (&d)[4], const uint32_t (&a)[4], 
 
 // Compressed inputs of one 16-token K tile, loaded one tile ahead.
 struct RsTileIn {
-  uint2 codes;      // code bytes of this lane's ldmatrix row (its token, sub-vector parity)
+  uint4 codes;      // code record of this lane's ldmatrix token (the lane uses half lane >> 4)
   uint32_t ks0, ks1;  // sign words (2-bit) of tokens g, g + 8
   uint32_t n[2];    // tokens g, g + 8: (s1, s2) fp16 pair, or (alpha*s2 fp16 | s1 level << 16) with DQ
 };
 
 template <int MK, bool DQ>
-__device__ __forceinline__ void rs_load_tile(RsTileIn& in, const CacheView& kc, int64_t tq, int tok_a, int kpar, int g,
-                                             int p) {
-  in.codes = __ldg(reinterpret_cast<const uint2*>(kc.codes + (tq + tok_a) * NSUB + 8 * kpar));
+__device__ __forceinline__ void rs_load_tile(RsTileIn& in, const CacheView& kc, int64_t tq, int tok_a, int g, int p) {
+  in.codes = __ldg(reinterpret_cast<const uint4*>(kc.codes + (tq + tok_a) * NSUB));
   in.ks0 = in.ks1 = 0u;
   if constexpr (MK == NSN_MODE_2BIT) {
     in.ks0 = __ldg(reinterpret_cast<const uint32_t*>(kc.signs + (tq + g) * NSUB) + p);
@@ -1093,7 +1092,7 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
   const int q_end = min(nq, st_last * STAGE_TOK);  // this job's quantized positions end here
   int cur_blk = -1;
   RsTileIn nxt;
-  if (st_first < nst_q) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + st_first * STAGE_TOK, tok_a, kpar, g, p);
+  if (st_first < nst_q) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + st_first * STAGE_TOK, tok_a, g, p);
 
   for (int st = st_first; st < st_last; ++st) {
     const bool win = st >= nst_q;
@@ -1160,7 +1159,7 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
       float xs[2] = {1.f, 1.f}, s1r[2] = {1.f, 1.f};  // per row: scale of E, and s1
       if (!win) {
         const RsTileIn cur = nxt;
-        if (tt + 16 < q_end) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + tt + 16, tok_a, kpar, g, p);
+        if (tt + 16 < q_end) rs_load_tile<MK, DQ>(nxt, kc, seq * cap + tt + 16, tok_a, g, p);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           if constexpr (DQ) {
@@ -1176,7 +1175,8 @@ rope_scores_kernel(CacheView kc, const int32_t* __restrict__ v_nquant, const int
         // H_8 stage across bit 2 of the k-step, accumulated on the tensor cores;
         // the stages across bits 0 and 1 follow in fp32
         auto gather = [&](int a, uint32_t (&A)[4]) {
-          const uint32_t code = code_byte(cur.codes, a);
+          // (the whole 16-byte record is loaded: an 8-byte load here costs this kernel spills)
+          const uint32_t code = code_byte(kpar ? make_uint2(cur.codes.z, cur.codes.w) : make_uint2(cur.codes.x, cur.codes.y), a);
           ldsm_x4(cbk_base + code * 128u, A);
           if constexpr (MK == NSN_MODE_2BIT) {
             A[0] = apply_signs(A[0], cur.ks0, 2 * a);
