@@ -68,8 +68,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # decode kernel is compiled from with this SHA-256 (decode.cu, nsn_common.cuh,
 # comments and whitespace removed).
 # Any later change to those files makes the figure stale; the bench then reports null.
-DECODE_TRAFFIC = {"sha256": "95dda82e613710615757f6eb9d04394d703caabccba4e3aeb718dd40737334b9",
-                  "bytes_per_launch": (320906752 + 320956928) // 2 + (3941888 + 468224) // 2}
+DECODE_TRAFFIC = {"sha256": "cd324c724a8ffcb74d40f3f35a5dbc92c074525abbfb0fa5db97801f25f3152f",
+                  "bytes_per_launch": (320936192 + 320983040) // 2 + (3968000 + 882432) // 2}
 
 
 def decode_sources_sha256() -> str:

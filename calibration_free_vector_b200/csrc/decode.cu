@@ -630,9 +630,13 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
   const uint32_t lane_row = (uint32_t)(lane & 7) * 16u;
   const uint32_t cbk_base = smem_addr(&sm.cbk[0][0]) + lane_row;
   const uint32_t cbv_base = smem_addr(&sm.cbv[0][0]) + lane_row;
-  const int tok_a = (lane & 7) + 8 * ((lane >> 3) & 1);   // token of this lane's K ldmatrix row
+  // The K and V ldmatrix rows use one lane map: lane l reads token (l & 7) + 8 (l >> 4),
+  // sub-vector parity (l >> 3) & 1, so the 8-byte code loads of a half-warp cover
+  // 128 contiguous bytes (no bank conflict).  For K this puts the matrices of rows
+  // 8-15 and of k 8-15 in the other order: the gather swaps registers 1 and 2.
+  const int tok_a = (lane & 7) + 8 * (lane >> 4);         // token of this lane's K ldmatrix row
   const int tok_v = (lane & 7) + 8 * (lane >> 4);         // token of this lane's V ldmatrix row
-  const int kpar = lane >> 4, vpar = (lane >> 3) & 1;   // sub-vector parity of the K / V ldmatrix row
+  const int kpar = (lane >> 3) & 1, vpar = kpar;       // sub-vector parity of the K / V ldmatrix row
   const bool lo_lane = p < 2;                      // keeps token g (else g + 8) after the swap
   const int t_l = g + (lo_lane ? 0 : 8);           // token of this lane's two scores
   const int h0 = 2 * (p & 1);                      // its two heads: h0, h0 + 1 (within the group)
@@ -720,6 +724,11 @@ decode_kernel(CacheView kc, CacheView vc, const void* __restrict__ q, int dtype,
         const uint32_t code = code_byte(kcw, j);
         uint32_t aa[4];
         ldsm_x4(cbk_base + code * 128u, aa);
+        {  // matrices 1 and 2 hold tokens 0-7 of k 8-15 and tokens 8-15 of k 0-7
+          const uint32_t t = aa[1];
+          aa[1] = aa[2];
+          aa[2] = t;
+        }
         if constexpr (MK == NSN_MODE_2BIT) {
           aa[0] = apply_signs(aa[0], ks0, 2 * j);
           aa[1] = apply_signs(aa[1], ks1, 2 * j);
